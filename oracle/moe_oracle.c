@@ -1,0 +1,405 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU oracle for the forward
+ * pass of a Mixture-of-Experts FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is compiled into liboracle_moe.so and
+ * is used by the test-suite, by the smoke check and by the CPU-baseline leg
+ * of the benchmark.  The CUDA library never links, includes or calls it, and
+ * it shares no code, table or header with the CUDA library.
+ *
+ * Arithmetic is IEEE double throughout.  bf16 and fp32 inputs are widened
+ * exactly to double; nothing is rounded in between.  Every loop is the plain
+ * definition: no blocking, no fusion, no reordering.
+ *
+ * Sources (page title, section / equation):
+ *  [VI]  "Mixture-of-Experts" (Vector Institute post), router section:
+ *        router score h = x W_r, softmax over experts, top-k selection,
+ *        Eq. moe-output (gates taken from the full softmax) and the
+ *        renormalised-gate variant described right after it; Eq. balance
+ *        (f_i, P_i, E * sum f_i P_i); the expert-capacity paragraph
+ *        (limit c*k*T/E, overflow dropped).
+ *  [RO]  "Fine-Tuning Mixture of Experts (MoE) Models: Router Optimization
+ *        Techniques", "What Is It?" (h = x W_g, TopK, softmax over the
+ *        selected logits, output = sum P_i E_i(x), SwiGLU expert),
+ *        "How It Works" 1 (f_i, P_i, L_aux = N sum f_i P_i) and 2 (selection
+ *        on score + b_i, gate from the unbiased score), "Why It Matters" 3
+ *        (capacity; dropped tokens bypass the layer).
+ *  [IS]  "Fine-tuning and serving MoE models" (intellisensei tutorial),
+ *        "How an MoE layer actually works" (GELU expert Linear-GELU-Linear,
+ *        fp32 router softmax, weighted index-add back to token order).
+ *  [PK]  "Mixture of Experts" tutorial (prashantkul), "The capacity factor
+ *        formula" and "Selective precision".
+ *
+ * Parity status of each function is pinned by tests (see the test-suite for
+ * the pins): brute-force top-k, library softmax/sigmoid, closed-form balance
+ * loss (1 under uniform routing, E under collapse), a second loop-over-experts
+ * formulation, and the E=1 / k=E special cases reducing to a dense FFN and to
+ * the full soft mixture.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- shapes and flags ------------------------------------------------ */
+typedef struct {
+    int32_t T;            /* tokens                                      */
+    int32_t d;            /* d_model                                     */
+    int32_t E;            /* routed experts                              */
+    int32_t d_ff;         /* hidden width of one routed expert           */
+    int32_t k;            /* experts selected per token                  */
+    int32_t xw_dtype;     /* 0: x and expert weights are fp32,
+                             1: they are bf16 (raw 16-bit patterns)      */
+    int32_t act;          /* 0: GELU expert with biases, 1: SwiGLU       */
+    int32_t score;        /* 0: softmax scores, 1: sigmoid scores        */
+    int32_t renorm;       /* softmax only: 1 renormalise gates over the
+                             selected experts, 0 keep full-softmax gates */
+    int32_t capacity;     /* tokens one expert may keep; < 0: unlimited  */
+    int32_t d_ff_shared;  /* hidden width of the shared expert; 0: none  */
+    int32_t nthreads;     /* worker threads for the per-token loops      */
+} oracle_dims;
+
+/* Widen element i of a bf16 (dtype 1) or fp32 (dtype 0) array to double.
+ * bf16 is the upper half of an fp32 pattern, so the widening is exact.   */
+static double wide(const void *base, int dtype, size_t i)
+{
+    if (dtype == 0) return (double)((const float *)base)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ---- capacity ----------------------------------------------------------
+ * [VI] expert-capacity paragraph and [PK] "The capacity factor formula":
+ * an expert keeps at most c * k * T / E assignments.  Rounded down; a
+ * non-positive factor means no limit.                                     */
+int32_t oracle_capacity(double c, int32_t k, int32_t T, int32_t E)
+{
+    if (!(c > 0.0)) return -1;
+    return (int32_t)floor(c * (double)k * (double)T / (double)E);
+}
+
+/* ---- threading helper ------------------------------------------------- */
+typedef void (*range_fn)(void *ctx, int64_t lo, int64_t hi);
+typedef struct { range_fn fn; void *ctx; int64_t lo, hi; } range_job;
+
+static void *range_thread(void *p)
+{
+    range_job *j = (range_job *)p;
+    j->fn(j->ctx, j->lo, j->hi);
+    return NULL;
+}
+
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void *ctx)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (n < nthreads) nthreads = (int)(n > 0 ? n : 1);
+    if (nthreads == 1) { fn(ctx, 0, n); return; }
+    pthread_t tid[256];
+    range_job job[256];
+    for (int i = 0; i < nthreads; ++i) {
+        job[i].fn = fn; job[i].ctx = ctx;
+        job[i].lo = n * i / nthreads; job[i].hi = n * (i + 1) / nthreads;
+        pthread_create(&tid[i], NULL, range_thread, &job[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(tid[i], NULL);
+}
+
+/* ---- router ------------------------------------------------------------
+ * For every token t:
+ *   h_e   = sum_j x[t,j] * Wr[j,e]  (+ logit_bias[e])        [VI], [RO]
+ *   softmax: p_e = exp(h_e - max h) / sum exp(h - max h)      [VI], [IS]
+ *   sigmoid: s_e = 1 / (1 + exp(-h_e))
+ *   selection key: softmax -> h_e (softmax is strictly increasing in h, so
+ *   the k largest p are the k largest h); sigmoid -> s_e; plus sel_bias[e]
+ *   when given, which steers the selection only ([RO] How It Works 2).
+ *   idx = the k experts with the largest key, largest first; equal keys are
+ *   ordered by the lower expert index.
+ *   gate: softmax & renorm=0 -> p_idx (Eq. moe-output);
+ *         softmax & renorm=1 -> p_idx / sum_{selected} p;
+ *         sigmoid            -> s_idx / sum_{selected} s (bias never enters).
+ *   pnorm_e (the per-token score whose token-mean is P_e): p_e for softmax,
+ *   s_e / sum_all s for sigmoid.
+ *   margin[t] = key of the k-th choice minus key of the (k+1)-th (HUGE_VAL
+ *   when k == E): the distance from a different selection.
+ * Outputs: idx [T,k], gate [T,k], logits [T,E] (h, or NULL), pnorm [T,E]
+ * (or NULL), margin [T] (or NULL).                                         */
+typedef struct {
+    const oracle_dims *dm;
+    const void *x; const float *Wr; const float *logit_bias; const float *sel_bias;
+    int32_t *idx; double *gate; double *logits; double *pnorm; double *margin;
+    const int32_t *tokens;      /* optional subset of tokens (NULL: all) */
+} route_ctx;
+
+static void route_range(void *vctx, int64_t lo, int64_t hi)
+{
+    route_ctx *c = (route_ctx *)vctx;
+    const oracle_dims *dm = c->dm;
+    const int E = dm->E, d = dm->d, k = dm->k;
+    double *h = (double *)malloc(sizeof(double) * E);
+    double *sc = (double *)malloc(sizeof(double) * E);   /* p or s       */
+    double *key = (double *)malloc(sizeof(double) * E);
+    int *order = (int *)malloc(sizeof(int) * E);
+    for (int64_t n = lo; n < hi; ++n) {
+        int64_t t = c->tokens ? c->tokens[n] : n;
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j)
+                acc += wide(c->x, dm->xw_dtype, (size_t)t * d + j) * (double)c->Wr[(size_t)j * E + e];
+            if (c->logit_bias) acc += (double)c->logit_bias[e];
+            h[e] = acc;
+        }
+        double norm = 0.0;
+        if (dm->score == 0) {
+            double mx = h[0];
+            for (int e = 1; e < E; ++e) if (h[e] > mx) mx = h[e];
+            for (int e = 0; e < E; ++e) { sc[e] = exp(h[e] - mx); norm += sc[e]; }
+            for (int e = 0; e < E; ++e) sc[e] /= norm;
+            for (int e = 0; e < E; ++e) key[e] = h[e];
+        } else {
+            for (int e = 0; e < E; ++e) { sc[e] = 1.0 / (1.0 + exp(-h[e])); norm += sc[e]; }
+            for (int e = 0; e < E; ++e) key[e] = sc[e];
+        }
+        if (c->sel_bias) for (int e = 0; e < E; ++e) key[e] += (double)c->sel_bias[e];
+        /* selection: insertion sort of expert ids by (key desc, id asc) */
+        for (int e = 0; e < E; ++e) {
+            int pos = e;
+            while (pos > 0 && key[order[pos - 1]] < key[e]) { order[pos] = order[pos - 1]; --pos; }
+            order[pos] = e;
+        }
+        double selsum = 0.0;
+        for (int s = 0; s < k; ++s) selsum += sc[order[s]];
+        for (int s = 0; s < k; ++s) {
+            int e = order[s];
+            c->idx[n * k + s] = e;
+            double g;
+            if (dm->score == 0 && dm->renorm == 0) g = sc[e];
+            else g = sc[e] / selsum;
+            c->gate[n * k + s] = g;
+        }
+        if (c->logits) for (int e = 0; e < E; ++e) c->logits[n * E + e] = h[e];
+        if (c->pnorm) {
+            for (int e = 0; e < E; ++e)
+                c->pnorm[n * E + e] = (dm->score == 0) ? sc[e] : sc[e] / norm;
+        }
+        if (c->margin) c->margin[n] = (k < E) ? key[order[k - 1]] - key[order[k]] : HUGE_VAL;
+    }
+    free(h); free(sc); free(key); free(order);
+}
+
+int oracle_route(const oracle_dims *dm, int64_t ntok, const int32_t *tokens,
+                 const void *x, const float *Wr, const float *logit_bias, const float *sel_bias,
+                 int32_t *idx, double *gate, double *logits, double *pnorm, double *margin)
+{
+    if (!dm || dm->k < 1 || dm->k > dm->E || dm->d < 1) return 1;
+    route_ctx c = { dm, x, Wr, logit_bias, sel_bias, idx, gate, logits, pnorm, margin, tokens };
+    parallel_for(ntok, dm->nthreads, route_range, &c);
+    return 0;
+}
+
+/* ---- counts, capacity and permutation ----------------------------------
+ * counts[e]  = number of (t, s) with idx[t,s] == e             ([RO] bincount)
+ * Visit tokens in ascending t (slots in ascending s): rank = seen[e]++;
+ * the assignment is kept when rank < capacity ([VI] capacity paragraph; the
+ * first-come order is this implementation's reading).  Dropped assignments
+ * contribute nothing ([RO] Why It Matters 3: they bypass the layer).
+ * kept[e]    = min(counts[e], capacity)
+ * offsets    = exclusive prefix sum of kept, offsets[E] = total kept rows
+ * row_of[t,s]= offsets[e] + rank if kept, else -1
+ * row_token[row] = t   (rows in (expert, token) order)                    */
+int oracle_dispatch(const oracle_dims *dm, const int32_t *idx, int32_t *counts, int32_t *kept,
+                    int32_t *offsets, int32_t *row_of, int32_t *row_token, int32_t *n_dropped)
+{
+    const int E = dm->E, k = dm->k;
+    const int64_t T = dm->T;
+    int32_t *seen = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    int32_t *rank = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * k > 0 ? T * k : 1));
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int s = 0; s < k; ++s) {
+            int e = idx[t * k + s];
+            if (e < 0 || e >= E) { free(seen); free(rank); return 1; }
+            counts[e] += 1;
+            rank[t * k + s] = seen[e]++;
+        }
+    int32_t dropped = 0;
+    for (int e = 0; e < E; ++e) {
+        kept[e] = (dm->capacity >= 0 && counts[e] > dm->capacity) ? dm->capacity : counts[e];
+        dropped += counts[e] - kept[e];
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + kept[e];
+    for (int64_t t = 0; t < T; ++t)
+        for (int s = 0; s < k; ++s) {
+            int e = idx[t * k + s];
+            int32_t r = rank[t * k + s];
+            if (dm->capacity >= 0 && r >= dm->capacity) { row_of[t * k + s] = -1; continue; }
+            int32_t row = offsets[e] + r;
+            row_of[t * k + s] = row;
+            if (row_token) row_token[row] = (int32_t)t;
+        }
+    if (n_dropped) *n_dropped = dropped;
+    free(seen); free(rank);
+    return 0;
+}
+
+/* ---- balance statistics -------------------------------------------------
+ * [VI] Eq. balance, [RO] How It Works 1, [IS] load_balancing_loss:
+ *   f_e = counts_e / (T * k)    (router decisions, before any capacity drop;
+ *                                dividing by k makes sum f = 1, so L = 1 under
+ *                                uniform routing for every k)
+ *   P_e = (1/T) sum_t pnorm[t,e]
+ *   L   = E * sum_e f_e * P_e                                              */
+int oracle_balance(const oracle_dims *dm, const int32_t *counts, const double *pnorm,
+                   double *f, double *P, double *L)
+{
+    const int E = dm->E;
+    const int64_t T = dm->T;
+    double acc = 0.0;
+    for (int e = 0; e < E; ++e) {
+        f[e] = (double)counts[e] / ((double)T * (double)dm->k);
+        double s = 0.0;
+        for (int64_t t = 0; t < T; ++t) s += pnorm[t * E + e];
+        P[e] = s / (double)T;
+        acc += f[e] * P[e];
+    }
+    *L = (double)E * acc;
+    return 0;
+}
+
+/* ---- one expert on one token -------------------------------------------
+ * GELU expert ([IS] "How an MoE layer actually works"):
+ *   a_j = sum_i W1[e,j,i] x_i + b1[e,j];  h_j = a_j * Phi(a_j)
+ *        = 0.5 a_j (1 + erf(a_j / sqrt 2))  (exact-erf GELU, nn.GELU default)
+ *   o_i = sum_j W2[e,i,j] h_j + b2[e,i]
+ * SwiGLU expert ([RO] "What Is It?"):
+ *   g_j = sum_i Wg[e,j,i] x_i;  u_j = sum_i Wu[e,j,i] x_i
+ *   h_j = g_j / (1 + exp(-g_j)) * u_j;   o_i = sum_j Wd[e,i,j] h_j
+ * Weight layouts follow nn.Linear: [out, in], stacked over experts.        */
+typedef struct {
+    const oracle_dims *dm;
+    const void *x;
+    const void *W1; const float *b1; const void *Wu; const void *W2; const float *b2;
+    const void *Wsg; const void *Wsu; const void *Wsd;
+} expert_weights;
+
+static void expert_apply_one(const expert_weights *w, int64_t t, int e, double *hbuf, double *out)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d, dt = dm->xw_dtype;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const void *Wa = shared ? w->Wsg : w->W1;
+    const void *Wb = shared ? w->Wsu : w->Wu;
+    const void *Wo = shared ? w->Wsd : w->W2;
+    const size_t ebase = shared ? 0 : (size_t)e;
+    for (int j = 0; j < dff; ++j) {
+        double a = 0.0;
+        for (int i = 0; i < d; ++i)
+            a += wide(Wa, dt, (ebase * dff + j) * d + i) * wide(w->x, dt, (size_t)t * d + i);
+        if (dm->act == 0 && !shared) {
+            if (w->b1) a += (double)w->b1[ebase * dff + j];
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else if (dm->act == 0) {
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else {
+            double u = 0.0;
+            for (int i = 0; i < d; ++i)
+                u += wide(Wb, dt, (ebase * dff + j) * d + i) * wide(w->x, dt, (size_t)t * d + i);
+            hbuf[j] = a / (1.0 + exp(-a)) * u;
+        }
+    }
+    for (int i = 0; i < d; ++i) {
+        double o = 0.0;
+        for (int j = 0; j < dff; ++j)
+            o += wide(Wo, dt, (ebase * d + i) * dff + j) * hbuf[j];
+        if (dm->act == 0 && !shared && w->b2) o += (double)w->b2[ebase * d + i];
+        out[i] = o;
+    }
+}
+
+/* out[r,:] = scale[r] * E_{expert[r]}(x[token[r],:]); expert == E selects the
+ * shared expert (GELU without biases when act == 0, SwiGLU otherwise).     */
+typedef struct {
+    expert_weights w;
+    const int32_t *token; const int32_t *expert; const double *scale; double *out;
+} apply_ctx;
+
+static void apply_range(void *vctx, int64_t lo, int64_t hi)
+{
+    apply_ctx *c = (apply_ctx *)vctx;
+    const oracle_dims *dm = c->w.dm;
+    int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    double *hbuf = (double *)malloc(sizeof(double) * (size_t)(hmax > 0 ? hmax : 1));
+    for (int64_t r = lo; r < hi; ++r) {
+        double *o = c->out + (size_t)r * dm->d;
+        expert_apply_one(&c->w, c->token[r], c->expert[r], hbuf, o);
+        double sc = c->scale ? c->scale[r] : 1.0;
+        for (int i = 0; i < dm->d; ++i) o[i] *= sc;
+    }
+    free(hbuf);
+}
+
+int oracle_expert_apply(const oracle_dims *dm, int64_t nrows, const int32_t *token,
+                        const int32_t *expert, const double *scale, const void *x,
+                        const void *W1, const float *b1, const void *Wu, const void *W2, const float *b2,
+                        const void *Wsg, const void *Wsu, const void *Wsd, double *out)
+{
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (expert[r] < 0 || expert[r] > dm->E) return 1;
+        if (expert[r] == dm->E && dm->d_ff_shared <= 0) return 1;
+    }
+    apply_ctx c = { { dm, x, W1, b1, Wu, W2, b2, Wsg, Wsu, Wsd }, token, expert, scale, out };
+    parallel_for(nrows, dm->nthreads, apply_range, &c);
+    return 0;
+}
+
+/* ---- the layer output for a list of tokens -------------------------------
+ * [VI] Eq. moe-output, [RO] "What Is It?", [IS] forward():
+ *   y_t = sum_{s : row_of[t,s] >= 0} gate[t,s] * E_{idx[t,s]}(x_t)
+ *         (+ shared expert output, weight 1, when d_ff_shared > 0)
+ * A dropped assignment (row_of < 0) adds nothing.                          */
+typedef struct {
+    expert_weights w;
+    const int32_t *tokens; const int32_t *idx; const double *gate; const int32_t *row_of;
+    double *y;
+} layer_ctx;
+
+static void layer_range(void *vctx, int64_t lo, int64_t hi)
+{
+    layer_ctx *c = (layer_ctx *)vctx;
+    const oracle_dims *dm = c->w.dm;
+    const int d = dm->d, k = dm->k;
+    int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    double *hbuf = (double *)malloc(sizeof(double) * (size_t)(hmax > 0 ? hmax : 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int64_t n = lo; n < hi; ++n) {
+        int64_t t = c->tokens[n];
+        double *y = c->y + (size_t)n * d;
+        for (int i = 0; i < d; ++i) y[i] = 0.0;
+        for (int s = 0; s < k; ++s) {
+            if (c->row_of && c->row_of[t * k + s] < 0) continue;
+            expert_apply_one(&c->w, t, c->idx[t * k + s], hbuf, o);
+            double g = c->gate[t * k + s];
+            for (int i = 0; i < d; ++i) y[i] += g * o[i];
+        }
+        if (dm->d_ff_shared > 0) {
+            expert_apply_one(&c->w, t, dm->E, hbuf, o);
+            for (int i = 0; i < d; ++i) y[i] += o[i];
+        }
+    }
+    free(hbuf); free(o);
+}
+
+int oracle_layer_tokens(const oracle_dims *dm, int64_t ntok, const int32_t *tokens,
+                        const void *x, const int32_t *idx, const double *gate, const int32_t *row_of,
+                        const void *W1, const float *b1, const void *Wu, const void *W2, const float *b2,
+                        const void *Wsg, const void *Wsu, const void *Wsd, double *y)
+{
+    layer_ctx c = { { dm, x, W1, b1, Wu, W2, b2, Wsg, Wsu, Wsd }, tokens, idx, gate, row_of, y };
+    parallel_for(ntok, dm->nthreads, layer_range, &c);
+    return 0;
+}
