@@ -1,0 +1,414 @@
+"""Benchmark of the MoE layer forward pass on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole layer forward (router, top-k, count/scan/permute, grouped
+expert FFN, combine, balance statistics) through moe_forward on one batch of
+synthetic input already resident in HBM.  The default workload is the
+Qwen3-MoE-shaped layer (T=16384, d_model=2048, 128 experts of d_ff=768, top-8,
+Zipf(1.1) expert popularity).  Under torchrun every rank runs an independent
+replica (the layer forward has no data-path exchange), so `value` is the sum
+of tokens over ranks divided by the slowest rank's time ("weak" scaling).
+
+--impl reference times the CPU oracle (fp64, host cores) on a bounded sample
+of the same workload; under torchrun only rank 0 runs it.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_49_b200 import native as nat  # noqa: E402
+from mixture_experts_layer_49_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s and % of roofline (tensor or HBM) on 1 B200"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------- util
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling around the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.1)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        power = [float(r[3]) for r in rows if re.match(r"^[0-9.]+$", r[3])]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:12]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the grouped-FFN kernels from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    if not os.path.exists(path):
+        return None
+    src = source_hash(os.path.join(ROOT, "mixture_experts_layer_49_b200", "csrc", "ffn_sm100.cu"))
+    for line in open(path):
+        m = re.match(r"\|\s*grouped_ffn\s*\|\s*(\w+)\s*\|\s*([0-9a-f]+)\s*\|\s*([0-9.eE+]+)\s*\|", line)
+        if m and m.group(1) == workload and m.group(2) == src:
+            return float(m.group(3))
+    return None
+
+
+def algorithmic_counts(wl, counts, kept):
+    """Expert FLOPs on kept rows (+ shared expert), and the layer's algorithmic
+    bytes: x, y, W_r and the weights of every expert with a kept row."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    mats = 3 if wl.act == "swiglu" else 2
+    kept_rows = int(kept.sum())
+    flops = wl.expert_flops(kept_rows)
+    touched = int((kept > 0).sum())
+    w_bytes = touched * mats * wl.d_model * wl.d_ff * esz
+    if wl.d_ff_shared:
+        w_bytes += 3 * wl.d_model * wl.d_ff_shared * esz
+    b = 2 * wl.T * wl.d_model * esz + wl.d_model * wl.E * 4 + w_bytes
+    return flops, b, kept_rows
+
+
+# ------------------------------------------------------------- CPU oracle leg
+def oracle_sample(wl, inp_host, target_s, max_tokens=None):
+    """Time the oracle (router + selection + expert FFNs in fp64) on the first
+    n tokens of the workload; n is grown until the run takes ~target_s."""
+    import oracle
+    cap = oracle.capacity(float(np.float32(wl.capacity_factor)), wl.top_k, wl.T, wl.E)
+    weights = {k: inp_host[k] for k in ("W1", "Wu", "W2", "b1", "b2", "Wsg", "Wsu", "Wsd")
+               if inp_host.get(k) is not None}
+    n = 8
+    while True:
+        dims = oracle.make_dims(n, wl.d_model, wl.E, wl.d_ff, wl.top_k, x_dtype=wl.dtype, act=wl.act,
+                                score=wl.score, renorm=wl.renorm, capacity=cap,
+                                d_ff_shared=wl.d_ff_shared)
+        x = inp_host["x"][:n]
+        t0 = time.perf_counter()
+        r = oracle.route(dims, x, inp_host["Wr"], inp_host["logit_bias"], inp_host["sel_bias"])
+        dp = oracle.dispatch(dims, r["idx"])
+        oracle.balance(dims, dp["counts"], r["pnorm"])
+        oracle.layer_tokens(dims, x, weights, r["idx"], r["gate"], dp["row_of"], np.arange(n, dtype=np.int32))
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= (max_tokens or wl.T):
+            return n, dt, dims.nthreads
+        n = min(max_tokens or wl.T, max(n * 2, int(n * target_s / max(dt, 1e-3) * 0.8)))
+
+
+def host_inputs(inp):
+    return {k: (syn.to_numpy_raw(v) if isinstance(v, torch.Tensor) else None)
+            for k, v in inp.items() if k != "workload"}
+
+
+def run_reference(args, wl, dev):
+    inp = syn.generate(wl, dev, seed=0)
+    host = host_inputs(inp)
+    del inp
+    per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    n, _, cores = oracle_sample(wl, host, per_step)
+    import oracle
+    cap = oracle.capacity(float(np.float32(wl.capacity_factor)), wl.top_k, wl.T, wl.E)
+    dims = oracle.make_dims(n, wl.d_model, wl.E, wl.d_ff, wl.top_k, x_dtype=wl.dtype, act=wl.act,
+                            score=wl.score, renorm=wl.renorm, capacity=cap, d_ff_shared=wl.d_ff_shared)
+    weights = {k: host[k] for k in ("W1", "Wu", "W2", "b1", "b2", "Wsg", "Wsu", "Wsd") if host.get(k) is not None}
+
+    def step(i):
+        lo = (i * n) % max(1, wl.T - n + 1)
+        x = np.ascontiguousarray(host["x"][lo:lo + n])
+        r = oracle.route(dims, x, host["Wr"], host["logit_bias"], host["sel_bias"])
+        dp = oracle.dispatch(dims, r["idx"])
+        oracle.balance(dims, dp["counts"], r["pnorm"])
+        oracle.layer_tokens(dims, x, weights, r["idx"], r["gate"], dp["row_of"], np.arange(n, dtype=np.int32))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = ("%d consecutive tokens of %s per step (router, top-k, dispatch, balance and expert FFNs "
+              "in fp64 for those tokens)" % (n, wl.name))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "E": wl.E, "d_ff": wl.d_ff,
+            "top_k": wl.top_k, "act": wl.act, "score": wl.score, "renorm": wl.renorm,
+            "capacity_factor": wl.capacity_factor, "d_ff_shared": wl.d_ff_shared,
+            "logit_skew": wl.logit_skew, "l2": "flushed between steps (256 MiB write)"}
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_ours(args, wl, dev, world, rank):
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inp = syn.generate(wl, dev, seed=0)
+    cfg = nat.config_from_workload(wl)
+    out = nat.Outputs(cfg, dev)
+    ws = nat.alloc_workspace(cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[dev.index])
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        nat.forward(cfg, inp, out, ws, stream)
+    torch.cuda.synchronize(dev)
+    st = nat.moe_get_device_status(ws, stream)
+    if st != nat.MOE_OK:
+        raise RuntimeError("device status after warm-up: " + nat.status_string(st))
+
+    # ---- main timed region: K whole-layer steps through moe_forward
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        nat.forward(cfg, inp, out, ws, stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(step_ms) / args.steps
+    st = nat.moe_get_device_status(ws, stream)
+    if st != nat.MOE_OK:
+        raise RuntimeError("device status after timing: " + nat.status_string(st))
+
+    # ---- per-stage timing through the staged entry points (same kernels)
+    T, d, E, k = wl.T, wl.d_model, wl.E, wl.top_k
+    dt = nat.layer_dtype(cfg)
+    psum = torch.empty((nat.router_blocks(cfg), E), dtype=torch.float32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_gate = torch.empty(T * k, dtype=torch.float32, device=dev)
+    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)
+    y_perm = torch.empty((nat.perm_rows(cfg), d), dtype=dt, device=dev)
+    stages = ["router", "permute", "grouped_ffn", "combine", "balance"]
+    stage_ms = {s: [] for s in stages}
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        evs[0].record(stream)
+        nat.moe_router_topk(cfg, inp["x"], inp["Wr"], inp["logit_bias"], inp["sel_bias"], out.idx, out.gate,
+                            None, psum, ws, stream)
+        evs[1].record(stream)
+        nat.moe_permute(cfg, inp["x"], out.idx, out.gate, out.counts, kept, offsets, row_of, row_token, row_gate,
+                        x_perm, out.n_dropped, ws, stream)
+        evs[2].record(stream)
+        nat.moe_grouped_ffn(cfg, x_perm, offsets, row_gate, inp["W1"], inp["b1"], inp["Wu"], inp["W2"], inp["b2"],
+                            inp["x"], inp["Wsg"], inp["Wsu"], inp["Wsd"], y_perm, ws, stream)
+        evs[3].record(stream)
+        nat.moe_combine(cfg, y_perm, row_of, out.y, ws, stream)
+        evs[4].record(stream)
+        nat.moe_balance_stats(cfg, out.counts, psum, out.f, out.P, out.loss, stream)
+        evs[5].record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= args.warmup:
+            for j, s in enumerate(stages):
+                stage_ms[s].append(evs[j].elapsed_time(evs[j + 1]))
+    stage_avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
+
+    # ---- end to end: pinned host x in, y + loss out, copies inside the timed region
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty_like(out.y, device="cpu").pin_memory()
+    loss_host = torch.empty(1, dtype=torch.float64).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    inp_e2e = dict(inp)
+    inp_e2e["x"] = x_dev
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        nat.forward(cfg, inp_e2e, out, ws, stream)
+        y_host.copy_(out.y, non_blocking=True)
+        loss_host.copy_(out.loss, non_blocking=True)
+        if i >= args.warmup:
+            e2e_ev[i - args.warmup][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+
+    # ---- max over ranks
+    tm = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
+    ms, e2e_ms = float(tm[0]), float(tm[1])
+
+    counts = out.counts.cpu().numpy()
+    cap = nat.capacity(cfg)
+    kept_np = np.minimum(counts, cap) if cap >= 0 else counts
+    flops, alg_bytes, kept_rows = algorithmic_counts(wl, counts, kept_np)
+    peaks, peak_src = load_peaks()
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    layer_roof_ms = max(t_tensor, t_hbm) * 1e3
+    ffn_ms = stage_avg["grouped_ffn"]
+    ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
+    traffic = recorded_traffic(wl.name)
+    result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts,
+                  flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
+                  layer_roof_ms=layer_roof_ms, ffn_tflops=ffn_tflops, traffic=traffic,
+                  loss=float(out.loss.item()), n_dropped=int(out.n_dropped.item()),
+                  bound="tensor" if t_tensor >= t_hbm else "hbm",
+                  h2d=x_host.numel() * x_host.element_size(),
+                  d2h=y_host.numel() * y_host.element_size() + 8, host_inp=None)
+    if rank == 0 and not args.no_cpu_baseline:
+        host = host_inputs(inp)
+        n, dt_cpu, cores = oracle_sample(wl, host, args.cpu_seconds)
+        result["cpu"] = {"value": n / dt_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "first %d tokens of %s: router, top-k, dispatch, balance and expert FFNs in "
+                                   "fp64 (%.1f s on the host cores)" % (n, wl.name, dt_cpu)}
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_moe", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    wl = syn.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank == 0:
+            dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+            run_reference(args, wl, dev)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    try:
+        r = run_ours(args, wl, dev, world, rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    tokens_per_s = world * wl.T / (r["ms"] * 1e-3)
+    e2e_tokens_per_s = world * wl.T / (r["e2e_ms"] * 1e-3)
+    peaks = r["peaks"]
+    tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
+    peak_tensor = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism="replicas x%d" % world),
+        "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
+        "layer_roofline": {"bound": r["bound"], "time_ms": r["layer_roof_ms"],
+                           "frac": r["layer_roof_ms"] / r["ms"], "flops": r["flops"],
+                           "alg_bytes": r["alg_bytes"], "peak_note": "burst bf16 and copy bandwidth, " + tag},
+        "roofline": {"kernel": "grouped_ffn (tcgen05 gemm1 + gemm2)", "bound": "tensor",
+                     "achieved": r["ffn_tflops"], "peak": peak_tensor, "unit": "TFLOP/s",
+                     "frac": r["ffn_tflops"] / peak_tensor, "traffic": r["traffic"], "peak_note": "burst, " + tag},
+        "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
+        "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 8 * args.steps,
+        "clocks": r["clocks"],
+        "routing": {"kept_rows": r["kept_rows"], "dropped": r["n_dropped"], "loss": r["loss"],
+                    "max_count": int(r["counts"].max()), "min_count": int(r["counts"].min()),
+                    "active_experts": int((r["counts"] > 0).sum())},
+    }
+    if "cpu" in r:
+        line["cpu_baseline"] = r["cpu"]
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of libmoe, the forward pass of a Mixture-of-Experts FFN
+ * layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources are named by page title and section):
+ *   router      h = x W_r (+ per-expert logit offset), fp32 scores:
+ *               softmax over the E experts ("Mixture-of-Experts", Vector
+ *               Institute post, router section; "Fine-tuning and serving MoE
+ *               models", How an MoE layer actually works: fp32 router softmax),
+ *               or sigmoid with a selection-only bias ("Fine-Tuning Mixture of
+ *               Experts (MoE) Models: Router Optimization Techniques", How It
+ *               Works 2, auxiliary-loss-free routing).
+ *   top-k       the k experts with the largest score (+ selection bias), gates
+ *               from the full softmax (Eq. moe-output) or renormalised over
+ *               the selected experts; sigmoid gates s_i / sum_selected s.
+ *   capacity    an expert keeps at most floor(c * k * T / E) assignments, the
+ *               earliest tokens first; the rest are dropped (contribute zero)
+ *               (Vector Institute post, expert-capacity paragraph; "Mixture of
+ *               Experts" tutorial, The capacity factor formula).
+ *   experts     GELU: W2 GELU(W1 x + b1) + b2 (Linear-GELU-Linear with biases);
+ *               SwiGLU: W_down (SiLU(W_gate x) * (W_up x)) (Router Optimization
+ *               page, What Is It?); optional always-on shared expert (weight 1).
+ *   combine     y_t = sum_s gate[t,s] * E_{idx[t,s]}(x_t) (+ shared(x_t)).
+ *   balance     f_e = counts_e / (T k), P_e = mean_t score_e(t),
+ *               L = E * sum_e f_e P_e (Eq. balance; Router Optimization page,
+ *               How It Works 1).
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers owned by the caller, except the
+ *     moe_config pointer and the out-pointers of moe_get_device_status, which
+ *     are host pointers.  The library never allocates or frees device memory;
+ *     scratch comes from the caller's workspace `ws` of `ws_bytes` bytes
+ *     (moe_workspace_size() bytes suffice for every entry point), aligned to
+ *     256 bytes.  The first 256 bytes of ws hold a device status word; zero
+ *     them once with moe_workspace_init() before first use.
+ *   - Calls are asynchronous on `stream` and never synchronise the device
+ *     (moe_get_device_status and moe_workspace_init excepted, see there).
+ *   - Arguments are checked on the host before any launch; a bad argument
+ *     returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE)
+ *     and launches nothing.  A failed launch returns MOE_ERR_CUDA.  Problems
+ *     only the device can see (an expert id out of range, a row index out of
+ *     range, a pipeline wait that ran past its time limit) are recorded in the
+ *     workspace status word and read back by moe_get_device_status.
+ *   - Layouts are row-major.  x, y and expert weights are in cfg->dtype
+ *     (bf16 or fp32); router weights, biases, gates, logits and statistics are
+ *     fp32; the loss is fp64.  Expert weights use the nn.Linear [out, in]
+ *     layout stacked over experts.
+ *   - bf16 layers run the expert GEMMs on tcgen05 tensor cores with fp32
+ *     accumulation; the hidden activation H and the gate-scaled expert
+ *     outputs are rounded to bf16, the combine accumulates in fp32 and rounds
+ *     once.  fp32 layers run everything in fp32.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, k > E, ...   */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but not built: E > 256, d % 8 != 0, ... */
+    MOE_ERR_WORKSPACE = 3,     /* ws_bytes below moe_workspace_size() or ws misaligned */
+    MOE_ERR_CUDA = 4,          /* a CUDA call failed (launch, tensor map, copy)  */
+    MOE_ERR_TIMEOUT = 5,       /* device: a pipeline wait ran past its limit     */
+    MOE_ERR_DEVICE_BOUNDS = 6  /* device: an expert id or row index out of range */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_ACT_GELU_BIAS = 0, MOE_ACT_SWIGLU = 1 } moe_act;
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+
+typedef struct {
+    int32_t T;                 /* tokens, >= 0                                    */
+    int32_t d_model;           /* >= 8 and a multiple of 8                        */
+    int32_t E;                 /* routed experts, 1..256                          */
+    int32_t d_ff;              /* routed expert hidden width, >= 8, multiple of 8 */
+    int32_t top_k;             /* 1..E                                             */
+    int32_t dtype;             /* moe_dtype of x, y and expert weights            */
+    int32_t act;               /* moe_act                                          */
+    int32_t score;             /* moe_score                                        */
+    int32_t renorm;            /* softmax: 1 renormalise gates over the top-k,
+                                  0 keep the full-softmax probabilities           */
+    float capacity_factor;     /* <= 0: no capacity limit                          */
+    int32_t d_ff_shared;       /* shared expert hidden width; 0: none; else a
+                                  multiple of 8 (same activation as the routed
+                                  experts, no biases)                              */
+} moe_config;
+
+/* Bytes of workspace every entry point below can run in (0 on a bad config). */
+MOE_API size_t moe_workspace_size(const moe_config *cfg);
+
+/* Per-expert capacity floor(capacity_factor * top_k * T / E) computed in
+ * double, or -1 when capacity_factor <= 0 (or cfg is invalid).              */
+MOE_API int32_t moe_capacity(const moe_config *cfg);
+
+/* Rows of the per-block partial score sums written by moe_router_topk
+ * (the `psum` array is [moe_router_blocks(cfg), E] fp32).                   */
+MOE_API int32_t moe_router_blocks(const moe_config *cfg);
+
+/* Rows of y_perm: T*top_k routed rows, plus T shared-expert rows when
+ * d_ff_shared > 0 (routed row r of expert e lies in [offsets[e], offsets[e+1]),
+ * shared row of token t is T*top_k + t).                                     */
+MOE_API int64_t moe_perm_rows(const moe_config *cfg);
+
+/* Zero the workspace status header (an async 256-byte memset on `stream`). */
+MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router + score + top-k + gates (see the header comment for the sources).
+ *   x          [T, d_model]  cfg->dtype
+ *   Wr         [d_model, E]  fp32
+ *   logit_bias [E] fp32 or NULL: added to every logit (enters scores and
+ *              selection, i.e. a router Linear with bias)
+ *   sel_bias   [E] fp32 or NULL: added to the score for the selection only
+ *              (softmax: to the logit; sigmoid: to sigmoid(logit)); gates and
+ *              statistics never see it
+ *   idx        [T, top_k] int32 out: chosen experts, best first; equal keys
+ *              go to the lower expert id
+ *   gate       [T, top_k] fp32 out
+ *   logits_out [T, E] fp32 out or NULL: h (with logit_bias)
+ *   psum       [moe_router_blocks(cfg), E] fp32 out: per-block sums over the
+ *              block's tokens of the score whose token-mean is P_e (softmax
+ *              probability, or sigmoid normalised over all E experts)        */
+MOE_API moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr,
+                           const float *logit_bias, const float *sel_bias,
+                           int32_t *idx, float *gate, float *logits_out, float *psum,
+                           void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Counting, capacity and permutation into expert-contiguous order, stable by
+ * token id within each expert (rows in (expert, token) order).
+ *   x          [T, d_model] cfg->dtype;  idx [T, top_k] int32;  gate [T, top_k] fp32
+ *   counts     [E] int32 out: assignments per expert before capacity
+ *   kept       [E] int32 out: min(counts, capacity)
+ *   offsets    [E+1] int32 out: exclusive prefix sum of kept
+ *   row_of     [T, top_k] int32 out: row of each assignment, -1 when dropped
+ *   row_token  [T*top_k] int32 out: token of each row (first offsets[E] valid)
+ *   row_gate   [T*top_k] fp32 out: gate of each row
+ *   x_perm     [T*top_k, d_model] cfg->dtype out: x rows in row order
+ *   n_dropped  device int32 out (may be NULL): assignments dropped by capacity
+ * An expert id outside [0, E) is recorded as MOE_ERR_DEVICE_BOUNDS and the
+ * assignment is treated as dropped.                                          */
+MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *idx,
+                       const float *gate, int32_t *counts, int32_t *kept, int32_t *offsets,
+                       int32_t *row_of, int32_t *row_token, float *row_gate, void *x_perm,
+                       int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* All experts as one grouped GEMM pair.  For every expert e and every row r
+ * in [offsets[e], offsets[e+1]):
+ *   GELU:   y_perm[r] = row_gate[r] * (W2[e] GELU(W1[e] x_perm[r] + b1[e]) + b2[e])
+ *   SwiGLU: y_perm[r] = row_gate[r] * (W2[e] (SiLU(W1[e] x_perm[r]) * (Wu[e] x_perm[r])))
+ * and, with a shared expert, for every token t:
+ *   y_perm[T*top_k + t] = Wsh_d (act(Wsh_g x[t]) [* (Wsh_u x[t])])
+ *   W1  [E, d_ff, d_model] (GELU W1 or SwiGLU W_gate);  Wu [E, d_ff, d_model]
+ *       (SwiGLU W_up; NULL for GELU);  W2 [E, d_model, d_ff] (W2 / W_down)
+ *   b1  [E, d_ff] fp32, b2 [E, d_model] fp32 (GELU; either may be NULL)
+ *   x, Wsh_g [d_ff_shared, d_model], Wsh_u (SwiGLU), Wsh_d [d_model, d_ff_shared]:
+ *       shared expert (NULL when d_ff_shared == 0)
+ *   y_perm [moe_perm_rows(cfg), d_model] cfg->dtype out; rows past offsets[E]
+ *       and before the shared rows are left untouched.                      */
+MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                           const float *row_gate, const void *W1, const float *b1,
+                           const void *Wu, const void *W2, const float *b2,
+                           const void *x, const void *Wsh_g, const void *Wsh_u,
+                           const void *Wsh_d, void *y_perm,
+                           void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* y[t] = sum over s with row_of[t,s] >= 0 of y_perm[row_of[t,s]]  (+ the
+ * shared row T*top_k + t), accumulated in fp32 in slot order and rounded once.
+ *   y_perm [moe_perm_rows(cfg), d_model], row_of [T, top_k], y [T, d_model].
+ * A row index >= T*top_k is recorded as MOE_ERR_DEVICE_BOUNDS and skipped. */
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *row_of,
+                       void *y, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* f_e = counts_e / (T*top_k), P_e = (sum_b psum[b,e]) / T (fp64 sums),
+ * loss = E * sum_e f_e P_e (fp64).  f, P [E] fp32 out; loss device fp64 out. */
+MOE_API moe_status moe_balance_stats(const moe_config *cfg, const int32_t *counts, const float *psum,
+                             float *f, float *P, double *loss, moe_stream_t stream);
+
+/* The whole layer on one stream: router, permute, grouped FFN, combine,
+ * balance statistics.  Inputs as above; outputs:
+ *   y [T, d_model] cfg->dtype; idx, gate [T, top_k]; counts [E] int32;
+ *   f, P [E] fp32; loss device fp64; logits_out [T, E] fp32 or NULL;
+ *   n_dropped device int32 or NULL.
+ * Everything else lives in ws (moe_workspace_size(cfg) bytes).             */
+MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr,
+                       const float *logit_bias, const float *sel_bias,
+                       const void *W1, const float *b1, const void *Wu, const void *W2,
+                       const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d,
+                       void *y, int32_t *idx, float *gate, int32_t *counts, float *f, float *P,
+                       double *loss, float *logits_out, int32_t *n_dropped,
+                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronise `stream`, read the workspace status word into *status_out
+ * (a moe_status) and clear it.  Returns MOE_ERR_CUDA if the read fails.   */
+MOE_API moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out);
+
+/* Static text for a status code. */
+MOE_API const char *moe_status_string(moe_status s);
+
+/* Text describing the last host-side failure on the calling thread (which
+ * check failed, or the CUDA error string); "" if none.  Owned by the library. */
+MOE_API const char *moe_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,133 @@
+// combine_balance.cu -- weighted combine back to token order, and the
+// balance-loss statistics.
+//
+// Combine: y_t = sum over the selected experts of gate * E_i(x_t) ("Mixture-
+// of-Experts" post, Eq. moe-output; "Fine-tuning and serving MoE models", the
+// index-add of the gated expert outputs).  The gates are already applied by
+// the grouped GEMM epilogue, so this is a gather-sum of k rows per token (plus
+// the shared expert's row), in slot order with fp32 accumulation: the result
+// does not depend on scheduling.  A dropped assignment (row -1) adds nothing.
+//
+// Balance: f_e = counts_e / (T k), P_e = mean over tokens of the normalised
+// score, L = E sum f_e P_e (Vector Institute post, Eq. balance; Router
+// Optimization page, How It Works 1).  The per-block partial sums written by
+// the router are added in block order in double precision.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+template <typename TY>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void add(const uint4 &v, float *acc) {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float *acc) {
+        uint4 v;
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        return v;
+    }
+};
+template <>
+struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void add(const uint4 &v, float *acc) {
+        acc[0] += __uint_as_float(v.x); acc[1] += __uint_as_float(v.y);
+        acc[2] += __uint_as_float(v.z); acc[3] += __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float *acc) {
+        return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
+                          __float_as_uint(acc[2]), __float_as_uint(acc[3]));
+    }
+};
+
+constexpr int kCombThreads = 256;
+
+// One warp per token (grid-stride); lanes stride over 16-byte column vectors.
+template <typename TY>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
+    using V = Vec16<TY>;
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (kCombThreads / 32);
+    const int nvec = a.d / V::N;
+    const uint4 *yp = static_cast<const uint4 *>(a.y_perm);
+    uint4 *y = static_cast<uint4 *>(a.y);
+    for (int t = blockIdx.x * (kCombThreads / 32) + (threadIdx.x >> 5); t < a.T; t += nwarps) {
+        int my_row = -1;
+        if (lane < a.k) {
+            my_row = a.row_of[(size_t)t * a.k + lane];
+            if (my_row >= a.rows_routed) {
+                record_error(a.status, MOE_ERR_DEVICE_BOUNDS, t);
+                my_row = -1;
+            }
+        }
+        const int64_t shared_row = a.rows_routed + t;
+        for (int v = lane; v < nvec; v += 32) {
+            float acc[V::N];
+#pragma unroll
+            for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+#pragma unroll 4
+            for (int s = 0; s < a.k; ++s) {
+                const int r = __shfl_sync(0xffffffffu, my_row, s);
+                if (r >= 0) V::add(__ldg(yp + (size_t)r * nvec + v), acc);
+            }
+            if (a.has_shared) V::add(__ldg(yp + (size_t)shared_row * nvec + v), acc);
+            y[(size_t)t * nvec + v] = V::pack(acc);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) balance_kernel(BalanceArgs a) {
+    __shared__ double red[256];
+    const int e = threadIdx.x;
+    double contrib = 0.0;
+    if (e < a.E) {
+        double s = 0.0;
+        for (int b = 0; b < a.nblk; ++b) s += (double)a.psum[(size_t)b * a.E + e];
+        const double P = s / (double)a.T;
+        const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
+        a.f[e] = (float)f;
+        a.P[e] = (float)P;
+        contrib = f * P;
+    }
+    red[e] = contrib;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (e < o) red[e] += red[e + o];
+        __syncthreads();
+    }
+    if (e == 0) *a.loss = (double)a.E * red[0];
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st) {
+    if (a.T == 0) return cudaSuccess;
+    const int warps_per_block = kCombThreads / 32;
+    int blocks = (a.T + warps_per_block - 1) / warps_per_block;
+    const int cap = a.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (bf16) combine_kernel<__nv_bfloat16><<<blocks, kCombThreads, 0, st>>>(a);
+    else combine_kernel<float><<<blocks, kCombThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st) {
+    balance_kernel<<<1, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

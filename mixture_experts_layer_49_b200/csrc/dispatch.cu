@@ -1,0 +1,199 @@
+// dispatch.cu -- per-expert counting, capacity, prefix sum and the stable
+// permutation of tokens into expert-contiguous order.
+//
+// Counts are the bincount of the chosen expert ids ("Fine-Tuning Mixture of
+// Experts (MoE) Models: Router Optimization Techniques", router module, step
+// 5).  An expert keeps at most `capacity` assignments and drops the rest
+// ("Mixture-of-Experts" post, expert-capacity paragraph); which ones are kept
+// is not fixed by the pages: this library keeps the earliest tokens.  The
+// rows are packed into one contiguous workspace per expert so the experts run
+// as one grouped GEMM (Router Optimization page, What Most Articles Miss 2).
+//
+// Three kernels, all deterministic:
+//   chunk_hist   one CTA per chunk of 64 tokens: shared-memory counts per expert
+//   chunk_scan   one CTA: per expert, exclusive scan over chunks (warp scan);
+//                counts, kept = min(counts, capacity), offsets = scan of kept
+//   permute      one CTA per chunk: the rank of (t, s) among the chunk's
+//                assignments to the same expert comes from __match_any_sync
+//                over flattened (t, s) order, so rows are stable by token id;
+//                then the kept rows of x are copied with 16-byte vectors.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kChunk = 64;        // tokens per chunk
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, int nchunks) {
+    __shared__ int cnt[256];
+    const int c = blockIdx.x;
+    for (int e = threadIdx.x; e < a.E; e += kThreads) cnt[e] = 0;
+    __syncthreads();
+    const int t0 = c * kChunk;
+    const int ntok = min(kChunk, a.T - t0);
+    const int npairs = ntok * a.k;
+    const int32_t *idx = a.idx + (size_t)t0 * a.k;
+    for (int p = threadIdx.x; p < npairs; p += kThreads) {
+        const int e = idx[p];
+        if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
+        else record_error(a.status, MOE_ERR_DEVICE_BOUNDS, t0 * a.k + p);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += kThreads) a.chunk_cnt[(size_t)e * nchunks + c] = cnt[e];
+}
+
+__global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
+    __shared__ int kept_s[256];
+    __shared__ int cnt_s[256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = warp; e < a.E; e += 32) {
+        const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
+        int32_t *dst = a.chunk_base + (size_t)e * nchunks;
+        int running = 0;
+        for (int c0 = 0; c0 < nchunks; c0 += 32) {
+            const int v = (c0 + lane < nchunks) ? src[c0 + lane] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (c0 + lane < nchunks) dst[c0 + lane] = running + incl - v;
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            cnt_s[e] = running;
+            kept_s[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int running = 0, dropped = 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < a.E ? kept_s[e] : 0;
+            const int dv = e < a.E ? cnt_s[e] - kept_s[e] : 0;
+            int incl = v, dincl = dv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                const int dn = __shfl_up_sync(0xffffffffu, dincl, o);
+                if (lane >= o) { incl += n; dincl += dn; }
+            }
+            if (e < a.E) {
+                a.offsets[e] = running + incl - v;
+                a.counts[e] = cnt_s[e];
+                a.kept[e] = v;
+            }
+            running += __shfl_sync(0xffffffffu, incl, 31);
+            dropped += __shfl_sync(0xffffffffu, dincl, 31);
+        }
+        if (lane == 0) {
+            a.offsets[a.E] = running;
+            if (a.n_dropped) *a.n_dropped = dropped;
+        }
+    }
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int nchunks) {
+    __shared__ int base[256];
+    __shared__ int offs[256];
+    __shared__ int wcnt[kWarps][256];
+    __shared__ int2 list[kChunk * 32];           // (row, token) of each pair, k <= 32
+    const int c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, k = a.k;
+    for (int e = tid; e < E; e += kThreads) {
+        base[e] = a.chunk_base[(size_t)e * nchunks + c];
+        offs[e] = a.offsets[e];
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    const int t0 = c * kChunk;
+    const int npairs = min(kChunk, a.T - t0) * k;
+    const int p_lo = warp * npairs / kWarps, p_hi = (warp + 1) * npairs / kWarps;
+    const int32_t *idx = a.idx + (size_t)t0 * k;
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    // pass 1: per-warp counts over the warp's contiguous range of pairs
+    for (int p0 = p_lo; p0 < p_hi; p0 += 32) {
+        const int p = p0 + lane;
+        const unsigned active = __ballot_sync(0xffffffffu, p < p_hi);
+        if (p < p_hi) {
+            int e = idx[p];
+            if (e < 0 || e >= E) e = -1;
+            const unsigned peers = __match_any_sync(active, e);
+            if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // exclusive scan over warps, per expert
+    for (int e = tid; e < E; e += kThreads) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) { const int v = wcnt[w][e]; wcnt[w][e] = run; run += v; }
+    }
+    __syncthreads();
+    // pass 2: final ranks, rows, drops
+    for (int p0 = p_lo; p0 < p_hi; p0 += 32) {
+        const int p = p0 + lane;
+        const unsigned active = __ballot_sync(0xffffffffu, p < p_hi);
+        int e = -1, rank = 0;
+        unsigned peers = 0;
+        if (p < p_hi) {
+            e = idx[p];
+            if (e < 0 || e >= E) e = -1;
+            peers = __match_any_sync(active, e);
+            if (e >= 0) rank = base[e] + wcnt[warp][e] + __popc(peers & lt_mask);
+        }
+        __syncwarp();
+        if (p < p_hi && e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
+        if (p < p_hi) {
+            const int t = t0 + p / k;
+            int row = -1;
+            if (e >= 0 && (a.capacity < 0 || rank < a.capacity)) {
+                row = offs[e] + rank;
+                a.row_token[row] = t;
+                a.row_gate[row] = a.gate[(size_t)t0 * k + p];
+            }
+            a.row_of[(size_t)t0 * k + p] = row;
+            list[p] = make_int2(row, t);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // copy the kept rows of x into x_perm, one warp per row, 16-byte vectors
+    const int nvec = a.d * (int)sizeof(TX) / 16;
+    const uint4 *xs = static_cast<const uint4 *>(a.x);
+    uint4 *xd = static_cast<uint4 *>(a.x_perm);
+    for (int q = warp; q < npairs; q += kWarps) {
+        const int2 rt = list[q];
+        if (rt.x < 0) continue;
+        const uint4 *src = xs + (size_t)rt.y * nvec;
+        uint4 *dst = xd + (size_t)rt.x * nvec;
+        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+}  // namespace
+
+int dispatch_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+
+cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
+    const int nchunks = dispatch_chunks(a.T);
+    if (nchunks > 0) chunk_hist_kernel<<<nchunks, kThreads, 0, st>>>(a, nchunks);
+    chunk_scan_kernel<<<1, 1024, 0, st>>>(a, nchunks);
+    if (nchunks > 0) {
+        if (bf16) permute_kernel<__nv_bfloat16><<<nchunks, kThreads, 0, st>>>(a, nchunks);
+        else permute_kernel<float><<<nchunks, kThreads, 0, st>>>(a, nchunks);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

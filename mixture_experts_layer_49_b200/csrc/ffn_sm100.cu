@@ -1,0 +1,499 @@
+// ffn_sm100.cu -- grouped expert FFN for bf16 layers on the 5th-generation
+// tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// Expert definitions: GELU expert Linear-GELU-Linear with biases ("Fine-tuning
+// and serving MoE models", How an MoE layer actually works); SwiGLU expert
+// W_down(SiLU(W_gate x) * (W_up x)) ("Fine-Tuning Mixture of Experts (MoE)
+// Models: Router Optimization Techniques", What Is It?).  Running all experts
+// in one grouped launch instead of one launch per expert is what the pages
+// recommend (Router Optimization page, What Most Articles Miss 2; serving
+// tutorial, grouped GEMM remark).
+//
+// Kernel shape (one persistent CTA per SM, 192 threads, warp-specialised):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
+//               swizzle) per stage, 4 stages, mbarrier transaction counts
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//               (M=128, N=256, K=16, fp32 accumulators in TMEM), two
+//               256-column accumulators so the epilogue of tile i overlaps
+//               the mainloop of tile i+1
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, fused activation
+//               (SwiGLU: gate and up halves of one N=256 accumulator; GELU:
+//               bias + exact-erf GELU) or fused bias + gate scale, bf16 stores
+// Tiles: groups are the routed experts (rows offsets[e]..offsets[e+1] of the
+// packed activations) plus an optional shared expert over all T tokens.  The
+// tile list is built on the device from `offsets` (no host round trip); a
+// tile may start mid-way through the packed buffer, rows past the group's end
+// are computed but never stored.  Within a group the m index runs fastest so
+// CTAs working at the same time share one weight tile through L2.
+//
+// Every mbarrier wait is bounded (a global-timer limit); a wait that runs out
+// records MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds,
+// freeing its TMEM.  No TMA multicast is used.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;                 // rows per tile (MMA M)
+constexpr int BK = 64;                  // K per stage: one 128-byte swizzle atom of bf16
+constexpr int BNB = 256;                // B rows per stage (MMA N)
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2;       // 16 KiB
+constexpr uint32_t B_BYTES = BNB * BK * 2;      // 32 KiB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 512;             // 2 accumulators x 256 fp32 columns
+constexpr int kMaxGroups = 257;
+
+enum { GM_SWIGLU = 0, GM_GELU = 1, GM_DOWN = 2 };
+
+// instruction descriptor, kind::f16: D fp32 (bit 4), A bf16 (bits 7-9),
+// B bf16 (bits 10-12), both K-major, N>>3 at bit 17, M>>4 at bit 24
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BNB >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct GemmParams {
+    const int32_t *offsets;   // [E+1]
+    const float *bias;        // [E, N_routed] or null (GELU b1 / b2)
+    const float *row_gate;    // [rows] (GM_DOWN) or null
+    __nv_bfloat16 *out;       // row stride ldo
+    int32_t *status;
+    int E, T;
+    int K_routed, K_shared;
+    int N_routed, N_shared;
+    int has_shared;
+    int ldo;
+    int64_t shared_a_row;     // first A row of the shared group
+    int64_t shared_out_row;   // first output row of the shared group
+    uint64_t timeout_ns;
+};
+
+struct SmemTail {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t accf[2];
+    uint64_t acce[2];
+    uint32_t tmem_base;
+    int abort_flag;
+    int tile_start[kMaxGroups + 1];
+    int mtiles[kMaxGroups];
+    int rows[kMaxGroups];
+    int row0[kMaxGroups];
+};
+
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemTail);
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), version 1, start address >> 4 in bits 0-13.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;                       // LBO (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;             // SBO
+    d |= (uint64_t)1 << 46;                       // descriptor version
+    d |= (uint64_t)2 << 61;                       // SWIZZLE_128B
+    return d;
+}
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.f + erff(v * 0.70710678118654752f)); }
+__device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
+
+__device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
+    uint4 pk;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&pk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(dst) = pk;
+}
+
+__device__ __forceinline__ void decode(const SmemTail &s, int G, int tile, int &g, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - s.tile_start[g];
+    mt = local % s.mtiles[g];
+    nt = local / s.mtiles[g];
+}
+
+__device__ __forceinline__ bool aborted(const SmemTail &s) {
+    return *reinterpret_cast<const volatile int *>(&s.abort_flag) != 0;
+}
+__device__ __forceinline__ void fail(SmemTail &s, const GemmParams &p, int where) {
+    record_error(p.status, MOE_ERR_TIMEOUT, where);
+    *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
+                const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    SmemTail &s = *reinterpret_cast<SmemTail *>(smem + STAGES * STAGE_BYTES);
+    const uint32_t smA = base;                          // STAGES x 16 KiB
+    const uint32_t smB = base + STAGES * A_BYTES;       // STAGES x 32 KiB
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int BNO = (MODE == GM_SWIGLU) ? 128 : 256;   // output columns per tile
+    const int G = p.E + (p.has_shared ? 1 : 0);
+
+    // ---- tile table from the device-side offsets
+    for (int g = tid; g < G; g += kThreads) {
+        const bool sh = g >= p.E;
+        const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        const int n = sh ? p.N_shared : p.N_routed;
+        const int mt = (rows + BM - 1) / BM;
+        s.rows[g] = rows;
+        s.row0[g] = sh ? 0 : p.offsets[g];
+        s.mtiles[g] = mt > 0 ? mt : 1;
+        s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
+    }
+    if (tid == 0) {
+        s.tile_start[0] = 0;
+        s.abort_flag = 0;
+        for (int i = 0; i < STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 4); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 0) {            // inclusive scan of the per-group tile counts
+        int carry = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            int v = g < G ? s.tile_start[g + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (g < G) s.tile_start[g + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    if (warp == 1) {            // TMEM: whole warp allocates, address lands in smem
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&s.tmem_base)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int total = s.tile_start[G];
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == 0) {
+        // ================= TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
+                int g, mt, nt;
+                decode(s, G, tile, g, mt, nt);
+                const bool sh = g >= p.E;
+                const int K = sh ? p.K_shared : p.K_routed;
+                const int nk = (K + BK - 1) / BK;
+                const int a_row = sh ? (int)p.shared_a_row + mt * BM : s.row0[g] + mt * BM;
+                const CUtensorMap *mA = sh ? &tmAs : &tmA;
+                const CUtensorMap *mB = sh ? &tmBs : &tmB;
+                const CUtensorMap *mB2 = sh ? &tmBs2 : &tmB2;
+                const int e = sh ? 0 : g;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail(s, p, 1); break; }
+                    const uint32_t fb = smem_u32(&s.full[stage]);
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(smA + stage * A_BYTES, mA, fb, kb * BK, a_row);
+                    if (MODE == GM_SWIGLU) {
+                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * 128, e);
+                        tma_load_3d(smB + stage * B_BYTES + B_BYTES / 2, mB2, fb, kb * BK, nt * 128, e);
+                    } else {
+                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * BNB, e);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int ab = 0;
+            uint32_t aphase = 0;
+            for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
+                int g, mt, nt;
+                decode(s, G, tile, g, mt, nt);
+                const int K = g >= p.E ? p.K_shared : p.K_routed;
+                const int nk = (K + BK - 1) / BK;
+                if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail(s, p, 2); break; }
+                tc_fence_after();
+                const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) { fail(s, p, 3); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smA + stage * A_BYTES, b0 = smB + stage * B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), (kb | k) ? 1u : 0u);
+                    mma_commit(smem_u32(&s.empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&s.accf[ab]));
+                if (++ab == 2) { ab = 0; aphase ^= 1u; }
+            }
+        }
+    } else {
+        // ================= epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        const int q = warp & 3;
+        const int r_in_tile = q * 32 + lane;
+        int ab = 0;
+        uint32_t aphase = 0;
+        for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
+            int g, mt, nt;
+            decode(s, G, tile, g, mt, nt);
+            const bool sh = g >= p.E;
+            // lane 0 waits, the warp follows its verdict (keeps the warp converged
+            // for the .sync.aligned TMEM loads)
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(smem_u32(&s.accf[ab]), aphase, p.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { if (lane == 0) fail(s, p, 4); break; }
+            __syncwarp();
+            tc_fence_after();
+            const int grow = mt * BM + r_in_tile;
+            const bool valid = grow < s.rows[g];
+            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            const int N = sh ? p.N_shared : p.N_routed;
+            const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
+            __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
+            if (MODE == GM_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float gv[32], uv[32];
+                    tmem_ld32(taddr + c * 32, gv);
+                    tmem_ld32(taddr + 128 + c * 32, uv);
+                    const int col0 = nt * 128 + c * 32;
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) h[i] = silu(gv[v * 8 + i]) * uv[v * 8 + i];
+                            if (col0 + v * 8 < N) store8(orow_ptr + col0 + v * 8, h);
+                        }
+                    }
+                }
+            } else {
+                const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+                float gscale = 1.f;
+                if (MODE == GM_DOWN && !sh && valid) gscale = p.row_gate[orow];
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float acc[32];
+                    tmem_ld32(taddr + c * 32, acc);
+                    const int col0 = nt * BNB + c * 32;
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int cb = col0 + v * 8;
+                            if (cb >= N) continue;
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float t = acc[v * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
+                                h[i] = (MODE == GM_GELU) ? gelu_erf(t) : gscale * t;
+                            }
+                            store8(orow_ptr + cb, h);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
+            if (++ab == 2) { ab = 0; aphase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// bf16 tensor [outer][mid][inner] (inner contiguous), box {64, box_mid(, 1)}.
+// rank 2 maps (A operands) ignore `outer`; rank 3 maps (expert-stacked B
+// operands) are indexed by expert in the third coordinate.
+bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
+              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    if (outer_stride_elems == 0) outer_stride_elems = mid * mid_stride_elems;
+    cuuint64_t dims[3] = {inner, mid, outer};
+    cuuint64_t strides[2] = {mid_stride_elems * 2, outer_stride_elems * 2};
+    cuuint32_t box[3] = {(cuuint32_t)BK, box_mid, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
+                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const GemmParams &p, int grid, cudaStream_t st) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    tc_grouped_gemm<MODE><<<grid, kThreads, kSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
+    if (a.T == 0) return cudaSuccess;
+    const bool swiglu = a.act == MOE_ACT_SWIGLU;
+    const bool has_sh = a.S > 0;
+    const uint64_t routed_rows = (uint64_t)a.T * a.k;
+    const uint64_t all_rows = routed_rows + (has_sh ? (uint64_t)a.T : 0);
+    const int grid = a.num_sms > 0 ? a.num_sms : 148;
+    const uint64_t timeout_ns = 2000000000ull;
+
+    // ---- GEMM 1: H = act(X W1^T [+ b1])   (A: x_perm / x, B: W1 (+Wu) / Wsg (+Wsu))
+    CUtensorMap A1, A1s, B1, B1u, B1s, B1su;
+    const uint32_t box1 = swiglu ? 128 : 256;
+    if (!make_map(&A1, 2, a.x_perm, a.d, routed_rows, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&B1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
+    if (swiglu) {
+        if (!make_map(&B1u, 3, a.Wu, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
+    } else {
+        B1u = B1;
+    }
+    if (has_sh) {
+        if (!make_map(&A1s, 2, a.x, a.d, a.T, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&B1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, box1)) return cudaErrorInvalidValue;
+        if (swiglu) {
+            if (!make_map(&B1su, 3, a.Wsu, a.d, a.S, 1, a.d, 0, box1)) return cudaErrorInvalidValue;
+        } else {
+            B1su = B1s;
+        }
+    } else {
+        A1s = A1; B1s = B1; B1su = B1u;
+    }
+    GemmParams p1{};
+    p1.offsets = a.offsets;
+    p1.bias = swiglu ? nullptr : a.b1;
+    p1.row_gate = nullptr;
+    p1.out = static_cast<__nv_bfloat16 *>(a.H);
+    p1.status = a.status;
+    p1.E = a.E; p1.T = a.T;
+    p1.K_routed = a.d; p1.K_shared = a.d;
+    p1.N_routed = a.F; p1.N_shared = a.S;
+    p1.has_shared = has_sh ? 1 : 0;
+    p1.ldo = a.hF;
+    p1.shared_a_row = 0;
+    p1.shared_out_row = a.shared_base;
+    p1.timeout_ns = timeout_ns;
+    cudaError_t err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
+                             : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
+    if (err != cudaSuccess) return err;
+
+    // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
+    CUtensorMap A2, A2s, B2m, B2s;
+    if (!make_map(&A2, 2, a.H, a.F, all_rows, 1, a.hF, 0, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&B2m, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, BNB)) return cudaErrorInvalidValue;
+    if (has_sh) {
+        if (!make_map(&A2s, 2, a.H, a.S, all_rows, 1, a.hF, 0, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&B2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, BNB)) return cudaErrorInvalidValue;
+    } else {
+        A2s = A2; B2s = B2m;
+    }
+    GemmParams p2{};
+    p2.offsets = a.offsets;
+    p2.bias = swiglu ? nullptr : a.b2;
+    p2.row_gate = a.row_gate;
+    p2.out = static_cast<__nv_bfloat16 *>(a.y_perm);
+    p2.status = a.status;
+    p2.E = a.E; p2.T = a.T;
+    p2.K_routed = a.F; p2.K_shared = a.S;
+    p2.N_routed = a.d; p2.N_shared = a.d;
+    p2.has_shared = has_sh ? 1 : 0;
+    p2.ldo = a.d;
+    p2.shared_a_row = a.shared_base;
+    p2.shared_out_row = a.shared_base;
+    p2.timeout_ns = timeout_ns;
+    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st);
+}
+
+}  // namespace moe

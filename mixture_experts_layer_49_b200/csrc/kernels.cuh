@@ -1,0 +1,84 @@
+// kernels.cuh -- argument blocks and launchers of the libmoe kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct RouterArgs {
+    const void *x;               // [T, d] bf16 or fp32
+    const float *Wr;             // [d, E]
+    const float *logit_bias;     // [E] or null
+    const float *sel_bias;       // [E] or null
+    int32_t *idx;                // [T, k]
+    float *gate;                 // [T, k]
+    float *logits_out;           // [T, E] or null
+    float *psum;                 // [router_blocks(T), E]
+    int T, d, E, k, score, renorm;
+};
+int router_blocks(int T);
+cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st);
+
+struct DispatchArgs {
+    const void *x;               // [T, d]
+    const int32_t *idx;          // [T, k]
+    const float *gate;           // [T, k]
+    int32_t *chunk_cnt;          // [E, nchunks] scratch
+    int32_t *chunk_base;         // [E, nchunks] scratch
+    int32_t *counts, *kept, *offsets;   // [E], [E], [E+1]
+    int32_t *row_of;             // [T, k]
+    int32_t *row_token;          // [T*k]
+    float *row_gate;             // [T*k]
+    void *x_perm;                // [T*k, d]
+    int32_t *n_dropped;          // device scalar or null
+    int32_t *status;             // workspace status word
+    int T, d, E, k, capacity;    // capacity < 0: unlimited
+};
+int dispatch_chunks(int T);
+cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st);
+
+// Grouped expert FFN.  Group g < E is routed expert g (rows offsets[g] ..
+// offsets[g+1] of x_perm / H / y_perm); group E is the shared expert (rows
+// 0..T-1 of x, rows shared_base.. of H / y_perm).
+struct FfnArgs {
+    const void *x_perm;          // [T*k, d]
+    const void *x;               // [T, d] (shared expert) or null
+    const int32_t *offsets;      // [E+1]
+    const float *row_gate;       // [T*k]
+    const void *W1, *Wu, *W2;    // [E, F, d], [E, F, d] or null, [E, d, F]
+    const float *b1, *b2;        // [E, F], [E, d] or null
+    const void *Wsg, *Wsu, *Wsd; // [S, d], [S, d] or null, [d, S]
+    void *H;                     // [T*k (+T), max(F, S)] scratch, row stride hF
+    void *y_perm;                // [T*k (+T), d]
+    int32_t *status;
+    int T, d, E, k, F, S, act;   // S = d_ff_shared (0: none)
+    int hF;                      // row stride of H in elements
+    int64_t shared_base;         // = T*k
+    int num_sms;
+};
+cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st);
+cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st);
+
+struct CombineArgs {
+    const void *y_perm;
+    const int32_t *row_of;
+    void *y;
+    int32_t *status;
+    int T, d, k, has_shared;
+    int64_t rows_routed;         // T*k: valid routed row indices are below it
+    int num_sms;
+};
+cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
+
+struct BalanceArgs {
+    const int32_t *counts;
+    const float *psum;
+    float *f, *P;
+    double *loss;
+    int T, E, k, nblk;
+};
+cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st);
+
+}  // namespace moe

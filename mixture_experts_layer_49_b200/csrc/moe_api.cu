@@ -1,0 +1,348 @@
+// moe_api.cu -- the extern "C" boundary of libmoe: argument checks, workspace
+// layout and the launch sequence.  See include/moe.h for the contract.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+moe_status fail(moe_status s, const char *fmt, const char *what = "") {
+    snprintf(g_detail, sizeof g_detail, fmt, what);
+    return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char *where) {
+    snprintf(g_detail, sizeof g_detail, "%s: %s", where, cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Layout {
+    size_t psum, chunk_cnt, chunk_base, kept, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
+};
+
+int64_t perm_rows(const moe_config *c) {
+    return (int64_t)c->T * c->top_k + (c->d_ff_shared > 0 ? (int64_t)c->T : 0);
+}
+
+Layout layout(const moe_config *c) {
+    Layout L{};
+    const size_t esz = c->dtype == MOE_BF16 ? 2 : 4;
+    const size_t Tk = (size_t)c->T * c->top_k;
+    const size_t rows = (size_t)perm_rows(c);
+    const size_t hF = (size_t)(c->d_ff > c->d_ff_shared ? c->d_ff : c->d_ff_shared);
+    const size_t nblk = (size_t)moe::router_blocks(c->T);
+    const size_t nch = (size_t)moe::dispatch_chunks(c->T);
+    size_t o = sizeof(moe::WsHeader);
+    L.psum = o;       o = align256(o + nblk * c->E * 4);
+    L.chunk_cnt = o;  o = align256(o + nch * c->E * 4);
+    L.chunk_base = o; o = align256(o + nch * c->E * 4);
+    L.kept = o;       o = align256(o + (size_t)c->E * 4);
+    L.offsets = o;    o = align256(o + (size_t)(c->E + 1) * 4);
+    L.row_of = o;     o = align256(o + Tk * 4);
+    L.row_token = o;  o = align256(o + Tk * 4);
+    L.row_gate = o;   o = align256(o + Tk * 4);
+    L.x_perm = o;     o = align256(o + Tk * c->d_model * esz);
+    L.H = o;          o = align256(o + rows * hF * esz);
+    L.y_perm = o;     o = align256(o + rows * c->d_model * esz);
+    L.total = o;
+    return L;
+}
+
+moe_status check_cfg(const moe_config *c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL%s");
+    if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0%s");
+    if (c->E < 1) return fail(MOE_ERR_INVALID_ARG, "E < 1%s");
+    if (c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "E > 256%s");
+    if (c->top_k < 1 || c->top_k > c->E) return fail(MOE_ERR_INVALID_ARG, "top_k outside 1..E%s");
+    if (c->top_k > 32) return fail(MOE_ERR_UNSUPPORTED, "top_k > 32%s");
+    if (c->d_model < 1 || c->d_ff < 1 || c->d_ff_shared < 0) return fail(MOE_ERR_INVALID_ARG, "non-positive width%s");
+    if (c->d_model % 8 || c->d_ff % 8 || c->d_ff_shared % 8)
+        return fail(MOE_ERR_UNSUPPORTED, "d_model, d_ff and d_ff_shared must be multiples of 8%s");
+    if (c->d_model > 65536 || c->d_ff > 65536 || c->d_ff_shared > 65536)
+        return fail(MOE_ERR_UNSUPPORTED, "widths above 65536%s");
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "bad dtype%s");
+    if (c->act != MOE_ACT_GELU_BIAS && c->act != MOE_ACT_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "bad act%s");
+    if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return fail(MOE_ERR_INVALID_ARG, "bad score%s");
+    if (c->renorm != 0 && c->renorm != 1) return fail(MOE_ERR_INVALID_ARG, "renorm must be 0 or 1%s");
+    if (!isfinite(c->capacity_factor)) return fail(MOE_ERR_INVALID_ARG, "capacity_factor not finite%s");
+    if (perm_rows(c) >= ((int64_t)1 << 31) - 256) return fail(MOE_ERR_UNSUPPORTED, "T * (top_k + 1) too large%s");
+    return MOE_OK;
+}
+
+moe_status check_ws(const moe_config *c, void *ws, size_t ws_bytes) {
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL%s");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    if (ws_bytes < layout(c).total) return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_workspace_size()%s");
+    return MOE_OK;
+}
+
+#define NEED(p) \
+    do { if (!(p)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer: %s", #p); } while (0)
+// 16-byte vector loads / TMA need 16-byte aligned rows; 4-byte arrays need 4.
+#define ALIGNED(p, a) \
+    do { if ((p) && (reinterpret_cast<uintptr_t>(p) % (a))) \
+        return fail(MOE_ERR_INVALID_ARG, "misaligned pointer: %s", #p); } while (0)
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <typename T>
+T *at(void *ws, size_t off) { return reinterpret_cast<T *>(static_cast<char *>(ws) + off); }
+
+int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
+
+moe_status check_weights(const moe_config *c, const void *W1, const void *Wu, const void *W2,
+                         const void *x, const void *Wsg, const void *Wsu, const void *Wsd) {
+    NEED(W1); NEED(W2);
+    ALIGNED(W1, 16); ALIGNED(Wu, 16); ALIGNED(W2, 16); ALIGNED(x, 16);
+    ALIGNED(Wsg, 16); ALIGNED(Wsu, 16); ALIGNED(Wsd, 16);
+    if (c->act == MOE_ACT_SWIGLU) NEED(Wu);
+    if (c->d_ff_shared > 0) {
+        NEED(x); NEED(Wsg); NEED(Wsd);
+        if (c->act == MOE_ACT_SWIGLU) NEED(Wsu);
+    }
+    return MOE_OK;
+}
+
+moe::FfnArgs ffn_args(const moe_config *c, const void *x_perm, const int32_t *offsets, const float *row_gate,
+                      const void *W1, const float *b1, const void *Wu, const void *W2, const float *b2,
+                      const void *x, const void *Wsg, const void *Wsu, const void *Wsd, void *y_perm, void *ws) {
+    const Layout L = layout(c);
+    moe::FfnArgs a{};
+    a.x_perm = x_perm; a.x = x; a.offsets = offsets; a.row_gate = row_gate;
+    a.W1 = W1; a.Wu = Wu; a.W2 = W2; a.b1 = b1; a.b2 = b2;
+    a.Wsg = Wsg; a.Wsu = Wsu; a.Wsd = Wsd;
+    a.H = at<char>(ws, L.H);
+    a.y_perm = y_perm;
+    a.status = status_word(ws);
+    a.T = c->T; a.d = c->d_model; a.E = c->E; a.k = c->top_k; a.F = c->d_ff; a.S = c->d_ff_shared;
+    a.act = c->act;
+    a.hF = c->d_ff > c->d_ff_shared ? c->d_ff : c->d_ff_shared;
+    a.shared_base = (int64_t)c->T * c->top_k;
+    a.num_sms = num_sms();
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config *cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return layout(cfg).total;
+}
+
+int32_t moe_capacity(const moe_config *cfg) {
+    if (check_cfg(cfg) != MOE_OK) return -1;
+    if (!(cfg->capacity_factor > 0.f)) return -1;
+    const double c = floor((double)cfg->capacity_factor * (double)cfg->top_k * (double)cfg->T / (double)cfg->E);
+    return c > 2147483647.0 ? 2147483647 : (int32_t)c;
+}
+
+int32_t moe_router_blocks(const moe_config *cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return moe::router_blocks(cfg->T);
+}
+
+int64_t moe_perm_rows(const moe_config *cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return perm_rows(cfg);
+}
+
+const char *moe_last_error_detail(void) { return g_detail; }
+
+moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!ws || ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace missing or < 256 bytes%s");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(moe::WsHeader), reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
+}
+
+moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                           const float *sel_bias, int32_t *idx, float *gate, float *logits_out, float *psum,
+                           void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    if (cfg->T > 0) { NEED(x); NEED(Wr); NEED(idx); NEED(gate); NEED(psum); }
+    ALIGNED(x, 16); ALIGNED(Wr, 4); ALIGNED(logit_bias, 4); ALIGNED(sel_bias, 4); ALIGNED(idx, 4);
+    ALIGNED(gate, 4); ALIGNED(logits_out, 4); ALIGNED(psum, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::RouterArgs a{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
+                      cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm};
+    cudaError_t e = moe::launch_router(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router");
+}
+
+moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *idx, const float *gate,
+                       int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of, int32_t *row_token,
+                       float *row_gate, void *x_perm, int32_t *n_dropped, void *ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(counts); NEED(kept); NEED(offsets);
+    if (cfg->T > 0) { NEED(x); NEED(idx); NEED(gate); NEED(row_of); NEED(row_token); NEED(row_gate); NEED(x_perm); }
+    ALIGNED(x, 16); ALIGNED(x_perm, 16); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(kept, 4);
+    ALIGNED(offsets, 4); ALIGNED(row_of, 4); ALIGNED(row_token, 4); ALIGNED(row_gate, 4); ALIGNED(n_dropped, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    const Layout L = layout(cfg);
+    moe::DispatchArgs a{};
+    a.x = x; a.idx = idx; a.gate = gate;
+    a.chunk_cnt = at<int32_t>(ws, L.chunk_cnt);
+    a.chunk_base = at<int32_t>(ws, L.chunk_base);
+    a.counts = counts; a.kept = kept; a.offsets = offsets;
+    a.row_of = row_of; a.row_token = row_token; a.row_gate = row_gate; a.x_perm = x_perm;
+    a.n_dropped = n_dropped;
+    a.status = status_word(ws);
+    a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.k = cfg->top_k;
+    a.capacity = moe_capacity(cfg);
+    cudaError_t e = moe::launch_dispatch(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "permute");
+}
+
+moe_status moe_grouped_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets, const float *row_gate,
+                           const void *W1, const float *b1, const void *Wu, const void *W2, const float *b2,
+                           const void *x, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y_perm,
+                           void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    if (cfg->T > 0) {
+        NEED(x_perm); NEED(offsets); NEED(row_gate); NEED(y_perm);
+        if ((s = check_weights(cfg, W1, Wu, W2, x, Wsh_g, Wsh_u, Wsh_d)) != MOE_OK) return s;
+    }
+    ALIGNED(x_perm, 16); ALIGNED(y_perm, 16); ALIGNED(offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4);
+    ALIGNED(b2, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::FfnArgs a = ffn_args(cfg, x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d, y_perm, ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cfg->dtype == MOE_BF16 ? moe::launch_ffn_bf16(a, st) : moe::launch_ffn_f32(a, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "grouped_ffn");
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *row_of, void *y, void *ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    if (cfg->T > 0) { NEED(y_perm); NEED(row_of); NEED(y); }
+    ALIGNED(y_perm, 16); ALIGNED(y, 16); ALIGNED(row_of, 4);
+    if (!ws || ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace missing%s");
+    moe::CombineArgs a{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
+                       cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
+    cudaError_t e = moe::launch_combine(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "combine");
+}
+
+moe_status moe_balance_stats(const moe_config *cfg, const int32_t *counts, const float *psum, float *f, float *P,
+                             double *loss, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    if (cfg->T > 0) NEED(psum);
+    ALIGNED(counts, 4); ALIGNED(psum, 4); ALIGNED(f, 4); ALIGNED(P, 4); ALIGNED(loss, 8);
+    moe::BalanceArgs a{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
+    cudaError_t e = moe::launch_balance(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "balance");
+}
+
+moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                       const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
+                       const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y,
+                       int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                       float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    if (cfg->T > 0) {
+        NEED(x); NEED(Wr); NEED(y); NEED(idx); NEED(gate);
+        if ((s = check_weights(cfg, W1, Wu, W2, x, Wsh_g, Wsh_u, Wsh_d)) != MOE_OK) return s;
+    }
+    ALIGNED(x, 16); ALIGNED(y, 16); ALIGNED(Wr, 4); ALIGNED(logit_bias, 4); ALIGNED(sel_bias, 4);
+    ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
+    ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    const Layout L = layout(cfg);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = cfg->dtype == MOE_BF16;
+    float *psum = at<float>(ws, L.psum);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *row_of = at<int32_t>(ws, L.row_of);
+    float *row_gate = at<float>(ws, L.row_gate);
+    void *y_perm = at<char>(ws, L.y_perm);
+    cudaError_t e;
+
+    moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
+                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm};
+    if ((e = moe::launch_router(ra, bf16, st)) != cudaSuccess) return cuda_fail(e, "router");
+
+    moe::DispatchArgs da{};
+    da.x = x; da.idx = idx; da.gate = gate;
+    da.chunk_cnt = at<int32_t>(ws, L.chunk_cnt);
+    da.chunk_base = at<int32_t>(ws, L.chunk_base);
+    da.counts = counts; da.kept = at<int32_t>(ws, L.kept); da.offsets = offsets;
+    da.row_of = row_of; da.row_token = at<int32_t>(ws, L.row_token); da.row_gate = row_gate;
+    da.x_perm = at<char>(ws, L.x_perm);
+    da.n_dropped = n_dropped;
+    da.status = status_word(ws);
+    da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
+    da.capacity = moe_capacity(cfg);
+    if ((e = moe::launch_dispatch(da, bf16, st)) != cudaSuccess) return cuda_fail(e, "permute");
+
+    moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
+                               y_perm, ws);
+    e = bf16 ? moe::launch_ffn_bf16(fa, st) : moe::launch_ffn_f32(fa, st);
+    if (e != cudaSuccess) return cuda_fail(e, "grouped_ffn");
+
+    moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
+                        cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
+    if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
+
+    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
+    if ((e = moe::launch_balance(ba, st)) != cudaSuccess) return cuda_fail(e, "balance");
+    return MOE_OK;
+}
+
+moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out) {
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL%s");
+    if (!status_out) return fail(MOE_ERR_INVALID_ARG, "status_out is NULL%s");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_get_device_status sync");
+    int32_t h[2] = {0, 0};
+    e = cudaMemcpy(h, ws, sizeof h, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_get_device_status read");
+    e = cudaMemset(ws, 0, sizeof h);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_get_device_status clear");
+    *status_out = h[0];
+    if (h[0] != 0) snprintf(g_detail, sizeof g_detail, "device status %d, detail %d", h[0], h[1]);
+    return MOE_OK;
+}
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "CUDA call failed";
+        case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case MOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

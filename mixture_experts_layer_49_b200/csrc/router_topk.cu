@@ -1,0 +1,218 @@
+// router_topk.cu -- router GEMM, fp32 scores, top-k selection and gates.
+//
+// "Mixture-of-Experts" (Vector Institute post), router section: one score per
+// expert h = x W_r, softmax over experts, top-k, gates from the full softmax
+// (Eq. moe-output) or renormalised over the selected experts.  "Fine-tuning
+// and serving MoE models", How an MoE layer actually works: the router softmax
+// runs in fp32.  "Fine-Tuning Mixture of Experts (MoE) Models: Router
+// Optimization Techniques", How It Works 2: a per-expert bias steers the
+// selection only; gates come from the unbiased scores.
+//
+// One CTA handles 32 tokens and all E (<= 256) experts.  The logits of a token
+// live in the registers of one warp (expert e on lane e % 32), so the softmax,
+// the k rounds of warp arg-max and the gates never leave registers.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kTok = 32;          // tokens per CTA
+constexpr int kThreads = 256;     // 8 warps, 4 tokens each
+constexpr int kKc = 32;           // d_model chunk staged in shared memory
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <typename TX>
+__device__ __forceinline__ void load_x_vec(const TX *src, float *dst);
+
+template <>
+__device__ __forceinline__ void load_x_vec<__nv_bfloat16>(const __nv_bfloat16 *src, float *dst) {
+    uint4 v = *reinterpret_cast<const uint4 *>(src);
+    const __nv_bfloat16 *h = reinterpret_cast<const __nv_bfloat16 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = __bfloat162float(h[i]);
+}
+template <>
+__device__ __forceinline__ void load_x_vec<float>(const float *src, float *dst) {
+    float4 v = *reinterpret_cast<const float4 *>(src);
+    dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+}
+
+template <typename TX, int EPT>
+__global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
+    constexpr int VEC = 16 / sizeof(TX);              // x elements per 16-byte load
+    constexpr int EW = EPT * 32;                      // expert slots per warp row
+    __shared__ float xs[kTok][kKc + 1];
+    __shared__ float wsm[kKc][EW];
+    __shared__ float part[kThreads / 32][EW];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * kTok;
+    const int d = a.d, E = a.E, k = a.k;
+
+    float acc[4][EPT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
+
+    const TX *x = static_cast<const TX *>(a.x);
+    for (int k0 = 0; k0 < d; k0 += kKc) {
+        // x chunk [32 tokens][32]: 16-byte vector loads (d % 8 == 0)
+        for (int v = tid; v < kTok * (kKc / VEC); v += kThreads) {
+            const int tt = v / (kKc / VEC), kv = (v % (kKc / VEC)) * VEC;
+            float vals[VEC];
+            const int t = t0 + tt;
+            if (t < a.T && k0 + kv < d) {
+                load_x_vec<TX>(x + (size_t)t * d + k0 + kv, vals);
+            } else {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) vals[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) xs[tt][kv + i] = vals[i];
+        }
+        // W_r chunk [32][E] (row-major [d, E], coalesced along E)
+        for (int v = tid; v < kKc * EW; v += kThreads) {
+            const int kk = v / EW, e = v % EW;
+            wsm[kk][e] = (k0 + kk < d && e < E) ? a.Wr[(size_t)(k0 + kk) * E + e] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kKc; ++kk) {
+            float xv[4], wv[EPT];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[i] = xs[warp * 4 + i][kk];
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) wv[j] = wsm[kk][lane + 32 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < EPT; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+
+    float psum_acc[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
+
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + warp * 4 + i;
+        if (t >= a.T) break;                         // uniform across the warp
+        float h[EPT], sc[EPT], key[EPT];
+        bool valid[EPT];
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const int e = lane + 32 * j;
+            valid[j] = e < E;
+            h[j] = acc[i][j] + ((a.logit_bias && valid[j]) ? a.logit_bias[e] : 0.f);
+        }
+        float norm;
+        if (a.score == MOE_SCORE_SOFTMAX) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) if (valid[j]) m = fmaxf(m, h[j]);
+            m = warp_max(m);
+            float z = 0.f;
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) { sc[j] = valid[j] ? expf(h[j] - m) : 0.f; z += sc[j]; }
+            norm = warp_sum(z);
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) { sc[j] = sc[j] / norm; key[j] = h[j]; }
+            norm = 1.f;                              // sc already normalised
+        } else {
+            float z = 0.f;
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) { sc[j] = valid[j] ? 1.f / (1.f + expf(-h[j])) : 0.f; z += sc[j]; }
+            norm = warp_sum(z);
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) key[j] = sc[j];
+        }
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            if (a.sel_bias && valid[j]) key[j] += a.sel_bias[lane + 32 * j];
+            psum_acc[j] += (a.score == MOE_SCORE_SOFTMAX) ? sc[j] : sc[j] / norm;
+        }
+        if (a.logits_out) {
+#pragma unroll
+            for (int j = 0; j < EPT; ++j)
+                if (valid[j]) a.logits_out[(size_t)t * E + lane + 32 * j] = h[j];
+        }
+        // k rounds of warp arg-max on (key desc, expert id asc)
+        unsigned taken = 0;
+        int my_e = -1;
+        float my_sc = 0.f;
+        for (int r = 0; r < k; ++r) {
+            float bk = -INFINITY, bs = 0.f;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) {
+                const int e = lane + 32 * j;
+                if (valid[j] && !(taken & (1u << j)) && (key[j] > bk || (key[j] == bk && e < be))) {
+                    bk = key[j]; be = e; bs = sc[j];
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+                if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; bs = os; }
+            }
+            if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
+            if (lane == r) { my_e = be; my_sc = bs; }
+        }
+        const float selsum = warp_sum(lane < k ? my_sc : 0.f);
+        if (lane < k) {
+            float g;
+            if (a.score == MOE_SCORE_SOFTMAX && !a.renorm) g = my_sc;
+            else g = my_sc / selsum;
+            a.idx[(size_t)t * k + lane] = my_e;
+            a.gate[(size_t)t * k + lane] = g;
+        }
+    }
+    // per-CTA partial sums of the normalised scores, fixed order
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) part[warp][lane + 32 * j] = psum_acc[j];
+    __syncthreads();
+    for (int e = tid; e < E; e += kThreads) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) s += part[w][e];
+        a.psum[(size_t)blockIdx.x * E + e] = s;
+    }
+}
+
+template <typename TX>
+cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
+    const int blocks = (a.T + kTok - 1) / kTok;
+    if (a.E <= 32) router_topk_kernel<TX, 1><<<blocks, kThreads, 0, st>>>(a);
+    else if (a.E <= 64) router_topk_kernel<TX, 2><<<blocks, kThreads, 0, st>>>(a);
+    else if (a.E <= 128) router_topk_kernel<TX, 4><<<blocks, kThreads, 0, st>>>(a);
+    else router_topk_kernel<TX, 8><<<blocks, kThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int router_blocks(int T) { return (T + kTok - 1) / kTok; }
+
+cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
+    if (a.T == 0) return cudaSuccess;
+    return bf16 ? launch_router_t<__nv_bfloat16>(a, st) : launch_router_t<float>(a, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+"""Thin ctypes binding of libmoe (include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+Functions keep the C names and take torch tensors that already live on the
+GPU; they pass raw device pointers and the current CUDA stream through the
+C ABI and raise MoEError on any non-OK status.  There is no fallback path:
+if the library is missing or no GPU is present, calls fail.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+c_i32 = ctypes.c_int32
+c_vp = ctypes.c_void_p
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
+    MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_BOUNDS = range(7)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ACT_GELU_BIAS, MOE_ACT_SWIGLU = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+
+EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_rows",
+           "moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
+           "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
+           "moe_status_string", "moe_last_error_detail")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status, where, detail=""):
+        self.status = status
+        super().__init__("%s: %s (%d)%s" % (where, status_string(status), status,
+                                            (" -- " + detail) if detail else ""))
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", c_i32), ("d_model", c_i32), ("E", c_i32), ("d_ff", c_i32),
+                ("top_k", c_i32), ("dtype", c_i32), ("act", c_i32), ("score", c_i32),
+                ("renorm", c_i32), ("capacity_factor", ctypes.c_float), ("d_ff_shared", c_i32)]
+
+    def __repr__(self):
+        return "MoeConfig(%s)" % ", ".join("%s=%s" % (n, getattr(self, n)) for n, _ in self._fields_)
+
+
+_lib = None
+
+
+def lib():
+    """Load libmoe.so (building it in-tree first if it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if not os.path.exists(path) or _build.stale():
+            path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.POINTER
+        L.moe_workspace_size.restype = ctypes.c_size_t
+        L.moe_workspace_size.argtypes = [P(MoeConfig)]
+        for n in ("moe_capacity", "moe_router_blocks"):
+            getattr(L, n).restype = c_i32
+            getattr(L, n).argtypes = [P(MoeConfig)]
+        L.moe_perm_rows.restype = ctypes.c_int64
+        L.moe_perm_rows.argtypes = [P(MoeConfig)]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_last_error_detail.restype = ctypes.c_char_p
+        L.moe_last_error_detail.argtypes = []
+        for n in ("moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
+                  "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status"):
+            getattr(L, n).restype = ctypes.c_int
+        L.moe_workspace_init.argtypes = [c_vp, ctypes.c_size_t, c_vp]
+        L.moe_router_topk.argtypes = [P(MoeConfig)] + [c_vp] * 9 + [ctypes.c_size_t, c_vp]
+        L.moe_permute.argtypes = [P(MoeConfig)] + [c_vp] * 12 + [ctypes.c_size_t, c_vp]
+        L.moe_grouped_ffn.argtypes = [P(MoeConfig)] + [c_vp] * 14 + [ctypes.c_size_t, c_vp]
+        L.moe_combine.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [ctypes.c_size_t, c_vp]
+        L.moe_balance_stats.argtypes = [P(MoeConfig)] + [c_vp] * 6
+        L.moe_forward.argtypes = [P(MoeConfig)] + [c_vp] * 22 + [ctypes.c_size_t, c_vp]
+        L.moe_get_device_status.argtypes = [c_vp, c_vp, P(c_i32)]
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().moe_status_string(int(s)).decode()
+
+
+def last_error_detail() -> str:
+    return lib().moe_last_error_detail().decode()
+
+
+def _check(rc, where):
+    if rc != MOE_OK:
+        raise MoEError(rc, where, last_error_detail())
+
+
+def make_config(T, d_model, E, d_ff, top_k, *, dtype="bf16", act="swiglu", score="softmax",
+                renorm=1, capacity_factor=0.0, d_ff_shared=0) -> MoeConfig:
+    return MoeConfig(T=T, d_model=d_model, E=E, d_ff=d_ff, top_k=top_k,
+                     dtype={"f32": MOE_F32, "bf16": MOE_BF16}[dtype],
+                     act={"gelu": MOE_ACT_GELU_BIAS, "swiglu": MOE_ACT_SWIGLU}[act],
+                     score={"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score],
+                     renorm=int(renorm), capacity_factor=float(capacity_factor),
+                     d_ff_shared=int(d_ff_shared))
+
+
+def config_from_workload(wl, T=None) -> MoeConfig:
+    return make_config(wl.T if T is None else T, wl.d_model, wl.E, wl.d_ff, wl.top_k,
+                       dtype=wl.dtype, act=wl.act, score=wl.score, renorm=wl.renorm,
+                       capacity_factor=wl.capacity_factor, d_ff_shared=wl.d_ff_shared)
+
+
+def _p(t):
+    """Device pointer of a CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("libmoe takes device tensors; got one on %s" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return c_vp(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_vp(stream.cuda_stream)
+
+
+def workspace_size(cfg) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg)))
+
+
+def capacity(cfg) -> int:
+    return int(lib().moe_capacity(ctypes.byref(cfg)))
+
+
+def router_blocks(cfg) -> int:
+    return int(lib().moe_router_blocks(ctypes.byref(cfg)))
+
+
+def perm_rows(cfg) -> int:
+    return int(lib().moe_perm_rows(ctypes.byref(cfg)))
+
+
+def alloc_workspace(cfg, device="cuda", stream=None) -> torch.Tensor:
+    n = workspace_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size", last_error_detail())
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream=stream)
+    return ws
+
+
+def moe_workspace_init(ws, stream=None):
+    _check(lib().moe_workspace_init(_p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_workspace_init")
+
+
+def moe_router_topk(cfg, x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum, ws, stream=None):
+    _check(lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias),
+                                 _p(idx), _p(gate), _p(logits_out), _p(psum), _p(ws), ws.numel(),
+                                 _stream(stream)), "moe_router_topk")
+
+
+def moe_permute(cfg, x, idx, gate, counts, kept, offsets, row_of, row_token, row_gate, x_perm,
+                n_dropped, ws, stream=None):
+    _check(lib().moe_permute(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(counts), _p(kept),
+                             _p(offsets), _p(row_of), _p(row_token), _p(row_gate), _p(x_perm),
+                             _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_grouped_ffn(cfg, x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
+                    y_perm, ws, stream=None):
+    _check(lib().moe_grouped_ffn(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(row_gate), _p(W1),
+                                 _p(b1), _p(Wu), _p(W2), _p(b2), _p(x), _p(Wsh_g), _p(Wsh_u),
+                                 _p(Wsh_d), _p(y_perm), _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn")
+
+
+def moe_combine(cfg, y_perm, row_of, y, ws, stream=None):
+    _check(lib().moe_combine(ctypes.byref(cfg), _p(y_perm), _p(row_of), _p(y), _p(ws), ws.numel(),
+                             _stream(stream)), "moe_combine")
+
+
+def moe_balance_stats(cfg, counts, psum, f, P, loss, stream=None):
+    _check(lib().moe_balance_stats(ctypes.byref(cfg), _p(counts), _p(psum), _p(f), _p(P), _p(loss),
+                                   _stream(stream)), "moe_balance_stats")
+
+
+def moe_forward(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh_u, Wsh_d,
+                y, idx, gate, counts, f, P, loss, logits_out, n_dropped, ws, stream=None):
+    _check(lib().moe_forward(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias), _p(W1),
+                             _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g), _p(Wsh_u), _p(Wsh_d), _p(y),
+                             _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss), _p(logits_out),
+                             _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    out = c_i32(0)
+    _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(out)),
+           "moe_get_device_status")
+    return int(out.value)
+
+
+def layer_dtype(cfg):
+    return torch.bfloat16 if cfg.dtype == MOE_BF16 else torch.float32
+
+
+class Outputs:
+    """Device output buffers of one moe_forward call (allocated once, reused)."""
+
+    def __init__(self, cfg, device="cuda", want_logits=False):
+        T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.top_k
+        self.y = torch.empty((T, d), dtype=layer_dtype(cfg), device=device)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.gate = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.counts = torch.empty(E, dtype=torch.int32, device=device)
+        self.f = torch.empty(E, dtype=torch.float32, device=device)
+        self.P = torch.empty(E, dtype=torch.float32, device=device)
+        self.loss = torch.empty(1, dtype=torch.float64, device=device)
+        self.n_dropped = torch.zeros(1, dtype=torch.int32, device=device)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=device) if want_logits else None
+
+
+def forward(cfg, inp, out: Outputs, ws, stream=None):
+    """moe_forward on a dict of device inputs (keys as in synthetic.generate)."""
+    moe_forward(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"),
+                inp["W1"], inp.get("b1"), inp.get("Wu"), inp["W2"], inp.get("b2"),
+                inp.get("Wsg"), inp.get("Wsu"), inp.get("Wsd"),
+                out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss, out.logits,
+                out.n_dropped, ws, stream)

@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/moe.h declares, and its host-side checks reject bad arguments before
+any CUDA call (none of these calls reaches a launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from mixture_experts_layer_49_b200 import native as nat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
+                 "moe_forward", "moe_balance_stats"):
+        assert name in syms
+    assert set(syms) == set(nat.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = nat.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    # nothing else is exported from the library's C namespace
+    out = os.popen("nm -D --defined-only %s" % nat._build.LIB).read()
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def cfg(**kw):
+    base = dict(T=64, d_model=128, E=8, d_ff=256, top_k=2)
+    base.update({k: kw.pop(k) for k in list(kw) if k in base})
+    return nat.make_config(base["T"], base["d_model"], base["E"], base["d_ff"], base["top_k"], **kw)
+
+
+def test_sizes_and_capacity():
+    c = cfg()
+    assert nat.workspace_size(c) > 0
+    assert nat.router_blocks(c) == 2
+    assert nat.perm_rows(c) == 128
+    assert nat.perm_rows(cfg(d_ff_shared=64)) == 128 + 64
+    assert nat.capacity(c) == -1
+    assert nat.capacity(cfg(T=8192, d_model=1024, E=16, d_ff=4096, top_k=1, capacity_factor=1.25)) == 640
+    assert nat.capacity(cfg(T=7, E=3, top_k=2, capacity_factor=1.25)) == 5
+    big = nat.workspace_size(cfg(T=1024))
+    assert big > nat.workspace_size(c)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=-1), nat.MOE_ERR_INVALID_ARG),
+    (dict(E=0), nat.MOE_ERR_INVALID_ARG),
+    (dict(E=300), nat.MOE_ERR_UNSUPPORTED),
+    (dict(top_k=0), nat.MOE_ERR_INVALID_ARG),
+    (dict(top_k=9), nat.MOE_ERR_INVALID_ARG),
+    (dict(E=64, top_k=33), nat.MOE_ERR_UNSUPPORTED),
+    (dict(d_model=100), nat.MOE_ERR_UNSUPPORTED),
+    (dict(d_ff=0), nat.MOE_ERR_INVALID_ARG),
+    (dict(d_ff_shared=12), nat.MOE_ERR_UNSUPPORTED),
+    (dict(renorm=2), nat.MOE_ERR_INVALID_ARG),
+])
+def test_bad_config_is_rejected(kw, code):
+    c = cfg(**kw)
+    assert nat.workspace_size(c) == 0
+    rc = nat.lib().moe_balance_stats(ctypes.byref(c), *([ctypes.c_void_p(256)] * 5), None)
+    assert rc == code, nat.last_error_detail()
+
+
+def fake(n=1):
+    return ctypes.c_void_p(4096 * n)
+
+
+def forward_raw(c, ws=None, ws_bytes=None, **null):
+    args = dict(x=fake(), Wr=fake(), lb=None, sb=None, W1=fake(), b1=None, Wu=fake(), W2=fake(), b2=None,
+                Wsg=None, Wsu=None, Wsd=None, y=fake(), idx=fake(), gate=fake(), counts=fake(), f=fake(),
+                P=fake(), loss=fake(), logits=None, nd=None)
+    for k in null:
+        args[k] = None
+    if ws is None:
+        ws = fake(16)
+    if ws_bytes is None:
+        ws_bytes = nat.workspace_size(c)
+    return nat.lib().moe_forward(ctypes.byref(c), *args.values(), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("missing", ["x", "Wr", "W1", "Wu", "W2", "y", "idx", "gate", "counts", "loss"])
+def test_null_pointer_is_rejected(missing):
+    assert forward_raw(cfg(), **{missing: None}) == nat.MOE_ERR_INVALID_ARG
+    assert missing.lower() in nat.last_error_detail().lower() or missing in nat.last_error_detail()
+
+
+def test_shared_expert_weights_are_required():
+    c = cfg(d_ff_shared=64)
+    assert forward_raw(c) == nat.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_checks():
+    c = cfg()
+    assert forward_raw(c, ws_bytes=nat.workspace_size(c) - 1) == nat.MOE_ERR_WORKSPACE
+    assert forward_raw(c, ws=ctypes.c_void_p(4096 + 16)) == nat.MOE_ERR_WORKSPACE
+    assert nat.lib().moe_workspace_init(None, 1024, None) == nat.MOE_ERR_WORKSPACE
+    out = ctypes.c_int32(0)
+    assert nat.lib().moe_get_device_status(None, None, ctypes.byref(out)) == nat.MOE_ERR_WORKSPACE
+
+
+def test_status_strings():
+    for s in range(7):
+        assert nat.status_string(s) != "unknown status"
+    assert nat.status_string(99) == "unknown status"
+
+
+def test_binding_refuses_host_tensors():
+    c = cfg()
+    with pytest.raises(ValueError):
+        nat.moe_combine(c, torch.zeros(4), torch.zeros(4, dtype=torch.int32), torch.zeros(4),
+                        torch.zeros(256, dtype=torch.uint8))
