@@ -96,7 +96,8 @@ def route(dims, x, Wr, logit_bias=None, sel_bias=None, tokens=None, want_logits=
     """Router + selection + gates for all tokens (or the listed ones).
 
     Returns dict(idx [n,k] int32, gate [n,k] f64, margin [n] f64,
-    pnorm [n,E] f64 (optional), logits [n,E] f64 (optional))."""
+    sel_key [n,k] f64 (selection key of each choice), pnorm [n,E] f64
+    (optional), logits [n,E] f64 (optional))."""
     lib = _load()
     x = _raw(x, "x")
     Wr = _f32(Wr)
@@ -104,14 +105,15 @@ def route(dims, x, Wr, logit_bias=None, sel_bias=None, tokens=None, want_logits=
     tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
     n = dims.T if tok is None else len(tok)
     out = dict(idx=np.empty((n, dims.k), np.int32), gate=np.empty((n, dims.k), np.float64),
-               margin=np.empty(n, np.float64))
+               margin=np.empty(n, np.float64), sel_key=np.empty((n, dims.k), np.float64))
     if want_pnorm:
         out["pnorm"] = np.empty((n, dims.E), np.float64)
     if want_logits:
         out["logits"] = np.empty((n, dims.E), np.float64)
     rc = lib.oracle_route(ctypes.byref(dims), ctypes.c_int64(n), _ptr(tok), _ptr(x), _ptr(Wr),
                           _ptr(lb), _ptr(sb), _ptr(out["idx"]), _ptr(out["gate"]),
-                          _ptr(out.get("logits")), _ptr(out.get("pnorm")), _ptr(out["margin"]))
+                          _ptr(out.get("logits")), _ptr(out.get("pnorm")), _ptr(out["margin"]),
+                          _ptr(out["sel_key"]))
     if rc:
         raise ValueError("oracle_route rejected its arguments")
     return out

@@ -126,11 +126,12 @@ static void parallel_for(int64_t n, int nthreads, range_fn fn, void *ctx)
  *   margin[t] = key of the k-th choice minus key of the (k+1)-th (HUGE_VAL
  *   when k == E): the distance from a different selection.
  * Outputs: idx [T,k], gate [T,k], logits [T,E] (h, or NULL), pnorm [T,E]
- * (or NULL), margin [T] (or NULL).                                         */
+ * (or NULL), margin [T] (or NULL), sel_key [T,k] (key of each choice, or
+ * NULL).                                                                   */
 typedef struct {
     const oracle_dims *dm;
     const void *x; const float *Wr; const float *logit_bias; const float *sel_bias;
-    int32_t *idx; double *gate; double *logits; double *pnorm; double *margin;
+    int32_t *idx; double *gate; double *logits; double *pnorm; double *margin; double *sel_key;
     const int32_t *tokens;      /* optional subset of tokens (NULL: all) */
 } route_ctx;
 
@@ -179,6 +180,7 @@ static void route_range(void *vctx, int64_t lo, int64_t hi)
             if (dm->score == 0 && dm->renorm == 0) g = sc[e];
             else g = sc[e] / selsum;
             c->gate[n * k + s] = g;
+            if (c->sel_key) c->sel_key[n * k + s] = key[e];
         }
         if (c->logits) for (int e = 0; e < E; ++e) c->logits[n * E + e] = h[e];
         if (c->pnorm) {
@@ -192,10 +194,11 @@ static void route_range(void *vctx, int64_t lo, int64_t hi)
 
 int oracle_route(const oracle_dims *dm, int64_t ntok, const int32_t *tokens,
                  const void *x, const float *Wr, const float *logit_bias, const float *sel_bias,
-                 int32_t *idx, double *gate, double *logits, double *pnorm, double *margin)
+                 int32_t *idx, double *gate, double *logits, double *pnorm, double *margin,
+                 double *sel_key)
 {
     if (!dm || dm->k < 1 || dm->k > dm->E || dm->d < 1) return 1;
-    route_ctx c = { dm, x, Wr, logit_bias, sel_bias, idx, gate, logits, pnorm, margin, tokens };
+    route_ctx c = { dm, x, Wr, logit_bias, sel_bias, idx, gate, logits, pnorm, margin, sel_key, tokens };
     parallel_for(ntok, dm->nthreads, route_range, &c);
     return 0;
 }

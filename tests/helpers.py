@@ -17,6 +17,8 @@ TOL_BF16 = 2e-2      # max|y - y_ref| / max|y_ref| for bf16 layers
 TOL_F32 = 1e-4       # the same measure for fp32 layers
 TOL_LOSS = 1e-5      # relative error of the balance loss
 TOL_GATE = 1e-5      # absolute error of an fp32 gate against the fp64 oracle
+TIE_KEY = 1e-5       # selected experts whose keys differ by less than this may
+                     # appear in either slot order (fp32 vs fp64 rounding)
 
 WEIGHT_KEYS = ("W1", "Wu", "W2", "b1", "b2", "Wsg", "Wsu", "Wsd")
 
@@ -94,3 +96,25 @@ def sample_tokens(idx, row_of, E, n_random, seed, T):
         if len(covered) == E:
             break
     return np.array(sorted(chosen), np.int32)
+
+
+def check_routing(idx, gate, ref):
+    """Selected experts bit-exact per token; slot order equal to the oracle's
+    except between choices whose oracle keys tie within TIE_KEY; gates
+    compared expert by expert.  Returns the number of tokens whose slot order
+    differs (all within ties)."""
+    idx = np.asarray(idx)
+    gate = np.asarray(gate, np.float64)
+    ridx, rgate, rkey = ref["idx"], ref["gate"], ref["sel_key"]
+    np.testing.assert_array_equal(np.sort(idx, 1), np.sort(ridx, 1))
+    swapped = np.nonzero((idx != ridx).any(1))[0]
+    for t in swapped:
+        key_of = dict(zip(ridx[t].tolist(), rkey[t].tolist()))
+        keys = np.array([key_of[e] for e in idx[t].tolist()])
+        assert np.all(np.diff(keys) <= TIE_KEY), "token %d: slot order is not a valid tie order" % t
+    oi = np.argsort(idx, 1, kind="stable")
+    ro = np.argsort(ridx, 1, kind="stable")
+    g_sorted = np.take_along_axis(gate, oi, 1)
+    r_sorted = np.take_along_axis(rgate, ro, 1)
+    assert np.max(np.abs(g_sorted - r_sorted), initial=0.0) <= TOL_GATE
+    return len(swapped)

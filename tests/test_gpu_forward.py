@@ -16,7 +16,7 @@ import oracle
 from mixture_experts_layer_49_b200 import native as nat
 from mixture_experts_layer_49_b200 import synthetic as syn
 
-from helpers import (TOL_BF16, TOL_F32, TOL_GATE, TOL_LOSS, make_case, oracle_dims, rel_err,
+from helpers import (TOL_BF16, TOL_F32, TOL_LOSS, check_routing, make_case, oracle_dims, rel_err,
                      sample_tokens, to_f64, weights_host)
 
 pytestmark = pytest.mark.gpu
@@ -41,9 +41,7 @@ def check_forward(wl, inp, host, n_sample=None, seed=0):
     dp = oracle.dispatch(dims, r["idx"])
     bal = oracle.balance(dims, dp["counts"], r["pnorm"])
 
-    idx = out.idx.cpu().numpy()
-    np.testing.assert_array_equal(idx, r["idx"])
-    assert np.max(np.abs(out.gate.cpu().numpy() - r["gate"]), initial=0.0) <= TOL_GATE
+    swapped = check_routing(out.idx.cpu().numpy(), out.gate.cpu().numpy(), r)
     np.testing.assert_array_equal(out.counts.cpu().numpy(), dp["counts"])
     assert int(out.n_dropped.item()) == dp["n_dropped"]
     assert rel_err(out.logits.cpu().numpy(), r["logits"]) < 1e-5
@@ -61,7 +59,7 @@ def check_forward(wl, inp, host, n_sample=None, seed=0):
     err = rel_err(y, y_ref)
     tol = TOL_F32 if wl.dtype == "f32" else TOL_BF16
     assert err <= tol, "max|y-y_ref|/max|y_ref| = %.3e > %.1e" % (err, tol)
-    return dict(err=err, loss=loss, loss_ref=bal["loss"], out=out, ref=r, dp=dp, tokens=tokens)
+    return dict(err=err, loss=loss, loss_ref=bal["loss"], out=out, ref=r, dp=dp, tokens=tokens, swapped=swapped)
 
 
 SMALL = [
@@ -94,8 +92,8 @@ def test_forward_full_size(name, cuda_device):
     inp, host = make_case(wl, cuda_device, seed=0)
     n_sample = None if wl.T * wl.d_model * wl.d_ff <= 256 * 128 * 256 else 48
     res = check_forward(wl, inp, host, n_sample=n_sample)
-    print("%s: max rel err %.3e, loss %.6f (ref %.6f), %d tokens checked" % (
-        name, res["err"], res["loss"], res["loss_ref"], len(res["tokens"])))
+    print("%s: max rel err %.3e, loss %.6f (ref %.6f), %d tokens checked, %d tie-swapped slot orders" % (
+        name, res["err"], res["loss"], res["loss_ref"], len(res["tokens"]), res["swapped"]))
 
 
 def test_forward_is_deterministic(cuda_device):
