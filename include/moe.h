@@ -203,6 +203,29 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        double *loss, float *logits_out, int32_t *n_dropped,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute for callers that cannot allocate device memory.  The paper has
+ * no counterpart: this entry point exists for integration only.
+ * Same computation, arguments and outputs as moe_permute, but no workspace:
+ * its scratch (per-chunk expert counts and their prefix sums) lives in a
+ * static device array inside libmoe (2 MiB + 256 bytes on every GPU that
+ * loads the library, held until the process exits).  It serves callers that
+ * cannot call cudaMalloc (a plug-in in a host framework that owns the whole
+ * device-memory budget, a latency-critical caller that cannot take
+ * cudaMalloc's implicit device synchronisation).
+ *   - Limit: E * ceil(T / 64) <= 262144 (E = 256 allows T <= 65536); beyond it
+ *     the call returns MOE_ERR_UNSUPPORTED and launches nothing.
+ *   - The first call on a device looks up the array's address with that
+ *     device current; make that first call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race.
+ *   - A bad expert id is dropped (row -1) as in moe_permute but, with no
+ *     workspace status word, not reported.
+ * Never calls cudaMalloc, cudaFree or any allocating routine.               */
+MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, const int32_t *idx,
+                                       const float *gate, int32_t *counts, int32_t *kept,
+                                       int32_t *offsets, int32_t *row_of, int32_t *row_token,
+                                       float *row_gate, void *x_perm, int32_t *n_dropped,
+                                       moe_stream_t stream);
+
 /* Synchronise `stream`, read the workspace status word into *status_out
  * (a moe_status) and clear it.  Returns MOE_ERR_CUDA if the read fails.   */
 MOE_API moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 struct RouterArgs {
@@ -80,5 +82,9 @@ struct BalanceArgs {
     int T, E, k, nblk;
 };
 cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st);
+
+// Host-side helpers shared by the entry points (moe_api.cu).
+moe_status validate_config(const moe_config *cfg);        // sets the error detail
+void set_error_detail(const char *where, const char *what);
 
 }  // namespace moe

@@ -141,6 +141,13 @@ moe::FfnArgs ffn_args(const moe_config *c, const void *x_perm, const int32_t *of
 
 }  // namespace
 
+namespace moe {
+moe_status validate_config(const moe_config *cfg) { return check_cfg(cfg); }
+void set_error_detail(const char *where, const char *what) {
+    snprintf(g_detail, sizeof g_detail, "%s: %s", where, what);
+}
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_size(const moe_config *cfg) {

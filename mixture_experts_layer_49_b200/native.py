@@ -27,7 +27,7 @@ MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_rows",
            "moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
-           "moe_status_string", "moe_last_error_detail")
+           "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -80,6 +80,8 @@ def lib():
         L.moe_balance_stats.argtypes = [P(MoeConfig)] + [c_vp] * 6
         L.moe_forward.argtypes = [P(MoeConfig)] + [c_vp] * 22 + [ctypes.c_size_t, c_vp]
         L.moe_get_device_status.argtypes = [c_vp, c_vp, P(c_i32)]
+        L.moe_permute_noalloc.restype = ctypes.c_int
+        L.moe_permute_noalloc.argtypes = [P(MoeConfig)] + [c_vp] * 11 + [c_vp]
         _lib = L
     return _lib
 
@@ -173,6 +175,16 @@ def moe_permute(cfg, x, idx, gate, counts, kept, offsets, row_of, row_token, row
     _check(lib().moe_permute(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(counts), _p(kept),
                              _p(offsets), _p(row_of), _p(row_token), _p(row_gate), _p(x_perm),
                              _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, x, idx, gate, counts, kept, offsets, row_of, row_token, row_gate, x_perm,
+                        n_dropped, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate
+    device memory (scratch lives in a fixed array inside libmoe; calls that
+    overlap on the GPU race on it; limit E * ceil(T/64) <= 262144)."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(counts), _p(kept),
+                                     _p(offsets), _p(row_of), _p(row_token), _p(row_gate), _p(x_perm),
+                                     _p(n_dropped), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_grouped_ffn(cfg, x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
