@@ -90,26 +90,43 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     }
 }
 
-__global__ void __launch_bounds__(256) balance_kernel(BalanceArgs a) {
+// 1024 threads: quarter g (= threadIdx.x / 256) of expert e (= threadIdx.x %
+// 256) adds the block rows b = g, g+4, ... in order; the four quarter sums
+// are then added in quarter order, and the loss terms f_e P_e in a fixed
+// tree.  Everything in double; the result does not depend on scheduling.
+__global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
+    __shared__ double quarter[4][256];
     __shared__ double red[256];
-    const int e = threadIdx.x;
-    double contrib = 0.0;
+    const int e = threadIdx.x & 255, g = threadIdx.x >> 8;
+    double s = 0.0;
     if (e < a.E) {
-        double s = 0.0;
-        for (int b = 0; b < a.nblk; ++b) s += (double)a.psum[(size_t)b * a.E + e];
-        const double P = s / (double)a.T;
-        const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
-        a.f[e] = (float)f;
-        a.P[e] = (float)P;
-        contrib = f * P;
+        int b = g;
+        for (; b + 12 < a.nblk; b += 16) {       // four independent loads in flight
+            const float v0 = a.psum[(size_t)b * a.E + e], v1 = a.psum[(size_t)(b + 4) * a.E + e];
+            const float v2 = a.psum[(size_t)(b + 8) * a.E + e], v3 = a.psum[(size_t)(b + 12) * a.E + e];
+            s += (double)v0; s += (double)v1; s += (double)v2; s += (double)v3;
+        }
+        for (; b < a.nblk; b += 4) s += (double)a.psum[(size_t)b * a.E + e];
     }
-    red[e] = contrib;
+    quarter[g][e] = s;
+    __syncthreads();
+    if (g == 0) {
+        double contrib = 0.0;
+        if (e < a.E) {
+            const double P = (((quarter[0][e] + quarter[1][e]) + quarter[2][e]) + quarter[3][e]) / (double)a.T;
+            const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
+            a.f[e] = (float)f;
+            a.P[e] = (float)P;
+            contrib = f * P;
+        }
+        red[e] = contrib;
+    }
     __syncthreads();
     for (int o = 128; o > 0; o >>= 1) {
-        if (e < o) red[e] += red[e + o];
+        if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
         __syncthreads();
     }
-    if (e == 0) *a.loss = (double)a.E * red[0];
+    if (threadIdx.x == 0) *a.loss = (double)a.E * red[0];
 }
 
 }  // namespace
@@ -126,7 +143,7 @@ cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st) {
 }
 
 cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st) {
-    balance_kernel<<<1, 256, 0, st>>>(a);
+    balance_kernel<<<1, 1024, 0, st>>>(a);
     return cudaGetLastError();
 }
 

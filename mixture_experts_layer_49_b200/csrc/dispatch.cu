@@ -11,9 +11,10 @@
 //
 // Three kernels, all deterministic:
 //   chunk_hist   one CTA per chunk of 64 tokens: shared-memory counts per expert
-//   chunk_scan   one CTA: per expert, exclusive scan over chunks (warp scan);
-//                counts, kept = min(counts, capacity), offsets = scan of kept
-//   permute      one CTA per chunk: the rank of (t, s) among the chunk's
+//   chunk_scan   one warp per expert: exclusive scan over chunks; counts and
+//                kept = min(counts, capacity)
+//   permute      one CTA per chunk: offsets = exclusive scan of kept (CTA 0
+//                publishes them); the rank of (t, s) among the chunk's
 //                assignments to the same expert comes from __match_any_sync
 //                over flattened (t, s) order, so rows are stable by token id;
 //                then the kept rows of x are copied with 16-byte vectors.
@@ -46,56 +47,45 @@ __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, in
     for (int e = threadIdx.x; e < a.E; e += kThreads) a.chunk_cnt[(size_t)e * nchunks + c] = cnt[e];
 }
 
+// One warp per expert: exclusive scan of the expert's per-chunk counts (each
+// lane first sums 8 consecutive chunks, then a warp scan of the lane totals),
+// the expert's total count and its kept count.  Experts are independent, so
+// the grid covers them 32 per CTA.
 __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
-    __shared__ int kept_s[256];
-    __shared__ int cnt_s[256];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int e = warp; e < a.E; e += 32) {
-        const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
-        int32_t *dst = a.chunk_base + (size_t)e * nchunks;
-        int running = 0;
-        for (int c0 = 0; c0 < nchunks; c0 += 32) {
-            const int v = (c0 + lane < nchunks) ? src[c0 + lane] : 0;
-            int incl = v;
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
+    if (e >= a.E) return;
+    const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
+    int32_t *dst = a.chunk_base + (size_t)e * nchunks;
+    int running = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 256) {
+        int v[8];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            if (c0 + lane < nchunks) dst[c0 + lane] = running + incl - v;
-            running += __shfl_sync(0xffffffffu, incl, 31);
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + lane * 8 + i;
+            v[i] = c < nchunks ? src[c] : 0;
         }
-        if (lane == 0) {
-            cnt_s[e] = running;
-            kept_s[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
+        int tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tot += v[i];
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
         }
+        int run = running + incl - tot;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + lane * 8 + i;
+            if (c < nchunks) dst[c] = run;
+            run += v[i];
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
     }
-    __syncthreads();
-    if (warp == 0) {
-        int running = 0, dropped = 0;
-        for (int e0 = 0; e0 < a.E; e0 += 32) {
-            const int e = e0 + lane;
-            const int v = e < a.E ? kept_s[e] : 0;
-            const int dv = e < a.E ? cnt_s[e] - kept_s[e] : 0;
-            int incl = v, dincl = dv;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                const int dn = __shfl_up_sync(0xffffffffu, dincl, o);
-                if (lane >= o) { incl += n; dincl += dn; }
-            }
-            if (e < a.E) {
-                a.offsets[e] = running + incl - v;
-                a.counts[e] = cnt_s[e];
-                a.kept[e] = v;
-            }
-            running += __shfl_sync(0xffffffffu, incl, 31);
-            dropped += __shfl_sync(0xffffffffu, dincl, 31);
-        }
-        if (lane == 0) {
-            a.offsets[a.E] = running;
-            if (a.n_dropped) *a.n_dropped = dropped;
-        }
+    if (lane == 0) {
+        a.counts[e] = running;
+        a.kept[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
     }
 }
 
@@ -109,9 +99,35 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int n
     const int E = a.E, k = a.k;
     for (int e = tid; e < E; e += kThreads) {
         base[e] = a.chunk_base[(size_t)e * nchunks + c];
-        offs[e] = a.offsets[e];
+        offs[e] = a.kept[e];
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    if (warp == 0) {       // expert offsets: exclusive scan of kept (every CTA; CTA 0 publishes)
+        int running = 0, dropped = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < E ? offs[e] : 0;
+            const int dv = (c == 0 && e < E) ? a.counts[e] - v : 0;
+            int incl = v, dincl = dv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                const int dn = __shfl_up_sync(0xffffffffu, dincl, o);
+                if (lane >= o) { incl += n; dincl += dn; }
+            }
+            if (e < E) {
+                offs[e] = running + incl - v;
+                if (c == 0) a.offsets[e] = running + incl - v;
+            }
+            running += __shfl_sync(0xffffffffu, incl, 31);
+            dropped += __shfl_sync(0xffffffffu, dincl, 31);
+        }
+        if (c == 0 && lane == 0) {
+            a.offsets[E] = running;
+            if (a.n_dropped) *a.n_dropped = dropped;
+        }
     }
     __syncthreads();
     const int t0 = c * kChunk;
@@ -177,8 +193,19 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int n
         if (rt.x < 0) continue;
         const uint4 *src = xs + (size_t)rt.y * nvec;
         uint4 *dst = xd + (size_t)rt.x * nvec;
-        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        int v = lane;
+        for (; v + 96 < nvec; v += 128) {          // four 16-byte loads in flight per lane
+            const uint4 r0 = __ldg(src + v), r1 = __ldg(src + v + 32);
+            const uint4 r2 = __ldg(src + v + 64), r3 = __ldg(src + v + 96);
+            dst[v] = r0; dst[v + 32] = r1; dst[v + 64] = r2; dst[v + 96] = r3;
+        }
+        for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
     }
+}
+
+__global__ void empty_offsets_kernel(DispatchArgs a) {
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.offsets[e] = 0;
+    if (threadIdx.x == 0 && a.n_dropped) *a.n_dropped = 0;
 }
 
 }  // namespace
@@ -188,8 +215,10 @@ int dispatch_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
     const int nchunks = dispatch_chunks(a.T);
     if (nchunks > 0) chunk_hist_kernel<<<nchunks, kThreads, 0, st>>>(a, nchunks);
-    chunk_scan_kernel<<<1, 1024, 0, st>>>(a, nchunks);
-    if (nchunks > 0) {
+    chunk_scan_kernel<<<(a.E + 31) / 32, 1024, 0, st>>>(a, nchunks);
+    if (nchunks == 0) {           // no tokens: every count is zero, offsets all zero
+        empty_offsets_kernel<<<1, 256, 0, st>>>(a);
+    } else {
         if (bf16) permute_kernel<__nv_bfloat16><<<nchunks, kThreads, 0, st>>>(a, nchunks);
         else permute_kernel<float><<<nchunks, kThreads, 0, st>>>(a, nchunks);
     }

@@ -1,0 +1,405 @@
+// router_sm100.cu -- router GEMM, fp32 scores, top-k selection, gates and the
+// per-block score sums for bf16 layers, on the tcgen05 tensor cores.
+//
+// "Mixture-of-Experts" (Vector Institute post), router section: one score per
+// expert h = x W_r, softmax over the experts, the k best, gates from the full
+// softmax (Eq. moe-output) or renormalised over the selected experts.
+// "Fine-tuning and serving MoE models", How an MoE layer actually works, and
+// the "Mixture of Experts" tutorial, Selective precision: the router runs in
+// fp32 even when the layer is bf16.  "Fine-Tuning Mixture of Experts (MoE)
+// Models: Router Optimization Techniques", How It Works 2: a per-expert bias
+// steers the selection only.
+//
+// fp32 accuracy on bf16 tensor cores: x is bf16 already; W_r (fp32) is split
+// exactly into three bf16 terms, W = hi + mid + lo (8 + 8 + 8 significand
+// bits), so x W = x hi + x mid + x lo with every product exact and the three
+// partial GEMMs accumulated into one fp32 TMEM accumulator.
+//
+// One CTA per 128 tokens (MMA M = 128, N = E rounded up to 16, K = d_model):
+//   warp 0      TMA producer: x tile 128 x 64 and the three W_r terms
+//               N x 64 per stage (128-byte swizzle), 2-4 stages
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue, one thread per token: the token's E logits come out
+//               of TMEM 32 columns at a time (three passes: max, sum, then
+//               scores, selection keys and a register-resident top-k list);
+//               per-expert sums of the normalised scores over the CTA's 128
+//               tokens by an in-warp transpose-reduce and a fixed-order sum of
+//               the four warps (deterministic).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int RM = 128;                       // tokens per CTA
+constexpr int RBK = 64;                       // K per stage
+constexpr int kThreads = 192;
+constexpr uint32_t A_BYTES = RM * RBK * 2;    // 16 KiB
+constexpr int kSmemCap = 227 * 1024;
+
+struct TcRouterParams {
+    const float *logit_bias;
+    const float *sel_bias;
+    int32_t *idx;
+    float *gate;
+    float *logits_out;
+    float *psum;
+    int32_t *status;
+    int T, d, E, k, score, renorm;
+    int n_pad;                 // MMA N
+    int stages;
+    uint32_t b_bytes;          // one W_r term per stage: n_pad x 64 bf16
+    uint32_t idesc;
+    uint32_t tmem_cols;
+    uint64_t timeout_ns;
+};
+
+struct RouterTail {
+    uint64_t full[4];
+    uint64_t empty[4];
+    uint64_t accf;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// W_r [d, E] fp32 -> three bf16 matrices [3][E][d] (K-major), w = hi + mid + lo.
+__global__ void __launch_bounds__(256) split_router_weights(const float *__restrict__ Wr, int d, int E,
+                                                            __nv_bfloat16 *__restrict__ out) {
+    __shared__ float tile[32][33];
+    const int j0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int r = ty; r < 32; r += 8) {
+        const int j = j0 + r, e = e0 + tx;
+        tile[r][tx] = (j < d && e < E) ? Wr[(size_t)j * E + e] : 0.f;
+    }
+    __syncthreads();
+    const size_t plane = (size_t)E * d;
+    for (int r = ty; r < 32; r += 8) {
+        const int e = e0 + r, j = j0 + tx;
+        if (e < E && j < d) {
+            const float w = tile[tx][r];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+            const float r1 = w - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(mid);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+            const size_t o = (size_t)e * d + j;
+            out[o] = hi;
+            out[plane + o] = mid;
+            out[2 * plane + o] = lo;
+        }
+    }
+}
+
+// (key desc, expert id asc): is (ka, ea) ahead of (kb, eb)?
+__device__ __forceinline__ bool ahead(float ka, int ea, float kb, int eb) {
+    return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const TcRouterParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    const uint32_t stage_bytes = A_BYTES + 3u * p.b_bytes;
+    RouterTail &s = *reinterpret_cast<RouterTail *>(smem + p.stages * stage_bytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.x * RM;
+    const int nk = (p.d + RBK - 1) / RBK;
+
+    if (tid == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < p.stages; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
+        mbar_init(smem_u32(&s.accf), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), p.tmem_cols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) {
+                    record_error(p.status, MOE_ERR_TIMEOUT, 11);
+                    s.abort_flag = 1;
+                    break;
+                }
+                const uint32_t fb = smem_u32(&s.full[stage]);
+                const uint32_t st = base + stage * stage_bytes;
+                mbar_arrive_expect_tx(fb, stage_bytes);
+                tma_load_2d(st, &tmX, fb, kb * RBK, t0);
+#pragma unroll
+                for (int j = 0; j < 3; ++j) tma_load_3d(st + A_BYTES + j * p.b_bytes, &tmW, fb, kb * RBK, 0, j);
+                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) {
+                    record_error(p.status, MOE_ERR_TIMEOUT, 12);
+                    s.abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = base + stage * stage_bytes;
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+#pragma unroll
+                    for (int k = 0; k < RBK / 16; ++k)
+                        mma_bf16(tmem, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
+                                 (kb | j | k) ? 1u : 0u);
+                mma_commit(smem_u32(&s.empty[stage]));
+                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+            }
+            if (ok) mma_commit(smem_u32(&s.accf));
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int t = t0 + row;
+        const bool tok_ok = t < p.T;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(smem_u32(&s.accf), 0, p.timeout_ns) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            if (lane == 0) { record_error(p.status, MOE_ERR_TIMEOUT, 13); s.abort_flag = 1; }
+        } else {
+            __syncwarp();
+            tc_fence_after();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            float *part = reinterpret_cast<float *>(smem);     // [4][E], reuses the drained stage buffers
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
+            const int E = p.E;
+            const int nchunk = (E + 31) / 32;
+            const bool softmax = p.score == MOE_SCORE_SOFTMAX;
+            float v[32];
+            // pass 1: max logit (softmax) / sum of sigmoids
+            float m = -INFINITY, ssum = 0.f;
+            for (int c = 0; c < nchunk; ++c) {
+                __syncwarp();
+                tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int e = c * 32 + j;
+                    if (e < E) {
+                        const float h = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
+                        if (softmax) m = fmaxf(m, h);
+                        else ssum += 1.f / (1.f + expf(-h));
+                    }
+                }
+            }
+            // pass 2: softmax normaliser
+            float z = 0.f;
+            if (softmax) {
+                for (int c = 0; c < nchunk; ++c) {
+                    __syncwarp();
+                    tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int e = c * 32 + j;
+                        if (e < E) z += expf(v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f) - m);
+                    }
+                }
+            }
+            // pass 3: scores, keys, top-k, per-block sums
+            float tk[KMAX], ts[KMAX];
+            int te[KMAX];
+#pragma unroll
+            for (int i = 0; i < KMAX; ++i) { tk[i] = -INFINITY; ts[i] = 0.f; te[i] = 0x7fffffff; }
+            float thr_k = -INFINITY;
+            int thr_e = 0x7fffffff;
+            const int k = p.k;
+            for (int c = 0; c < nchunk; ++c) {
+                __syncwarp();
+                tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int e = c * 32 + j;
+                    float pn = 0.f;
+                    if (e < E) {
+                        const float h = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
+                        float sc, key;
+                        if (softmax) {
+                            sc = expf(h - m) / z;
+                            pn = sc;
+                            key = h;
+                        } else {
+                            sc = 1.f / (1.f + expf(-h));
+                            pn = sc / ssum;
+                            key = sc;
+                        }
+                        if (p.sel_bias) key += __ldg(p.sel_bias + e);
+                        if (p.logits_out && tok_ok) p.logits_out[(size_t)t * E + e] = h;
+                        if (ahead(key, e, thr_k, thr_e)) {
+                            float ck = key, cs = sc;
+                            int ce = e;
+#pragma unroll
+                            for (int i = 0; i < KMAX; ++i) {
+                                if (i < k && ahead(ck, ce, tk[i], te[i])) {
+                                    const float a = tk[i], b = ts[i];
+                                    const int ei = te[i];
+                                    tk[i] = ck; ts[i] = cs; te[i] = ce;
+                                    ck = a; cs = b; ce = ei;
+                                }
+                            }
+#pragma unroll
+                            for (int i = 0; i < KMAX; ++i)
+                                if (i == k - 1) { thr_k = tk[i]; thr_e = te[i]; }
+                        }
+                    }
+                    v[j] = tok_ok ? pn : 0.f;
+                }
+                // transpose-reduce: lane L ends with the sum over the warp's 32
+                // tokens of the score of expert c*32 + L
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+                    for (int j = 0; j < o; ++j) {
+                        const bool upper = (lane & o) != 0;
+                        const float send = upper ? v[j] : v[j + o];
+                        const float keep = upper ? v[j + o] : v[j];
+                        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                }
+                if (c * 32 + lane < E) part[q * E + c * 32 + lane] = v[0];
+            }
+            if (tok_ok) {
+                float selsum = 0.f;
+#pragma unroll
+                for (int i = 0; i < KMAX; ++i) if (i < k) selsum += ts[i];
+#pragma unroll
+                for (int i = 0; i < KMAX; ++i) {
+                    if (i < k) {
+                        const float g = (softmax && !p.renorm) ? ts[i] : ts[i] / selsum;
+                        p.idx[(size_t)t * k + i] = te[i];
+                        p.gate[(size_t)t * k + i] = g;
+                    }
+                }
+            }
+        }
+        // the four epilogue warps meet here whether or not the wait succeeded
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok) {
+            const float *part = reinterpret_cast<const float *>(smem);
+            const int E = p.E;
+            for (int e = row; e < E; e += 128)
+                p.psum[(size_t)blockIdx.x * E + e] = ((part[e] + part[E + e]) + part[2 * E + e]) + part[3 * E + e];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, const cuuint64_t *strides,
+            const cuuint32_t *box) {
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KMAX>
+cudaError_t launch_tc(const CUtensorMap &mx, const CUtensorMap &mw, const TcRouterParams &p, size_t smem,
+                      cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemCap);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int grid = (p.T + RM - 1) / RM;
+    router_tc_kernel<KMAX><<<grid, kThreads, smem, st>>>(mx, mw, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int router_tc_blocks(int T) { return (T + RM - 1) / RM; }
+
+size_t router_split_bytes(int d, int E) { return (size_t)3 * E * d * 2; }
+
+cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status, cudaStream_t st) {
+    if (a.T == 0) return cudaSuccess;
+    dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
+    split_router_weights<<<sg, 256, 0, st>>>(a.Wr, a.d, a.E, static_cast<__nv_bfloat16 *>(wsplit));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    TcRouterParams p{};
+    p.logit_bias = a.logit_bias; p.sel_bias = a.sel_bias; p.idx = a.idx; p.gate = a.gate;
+    p.logits_out = a.logits_out; p.psum = a.psum; p.status = status;
+    p.T = a.T; p.d = a.d; p.E = a.E; p.k = a.k; p.score = a.score; p.renorm = a.renorm;
+    p.n_pad = (a.E + 15) / 16 * 16;
+    p.b_bytes = (uint32_t)p.n_pad * RBK * 2;
+    p.idesc = make_idesc_bf16(RM, (uint32_t)p.n_pad);
+    uint32_t cols = 32;
+    while ((int)cols < p.n_pad) cols <<= 1;
+    p.tmem_cols = cols;
+    p.timeout_ns = 2000000000ull;
+    const size_t stage_bytes = A_BYTES + 3 * (size_t)p.b_bytes;
+    const size_t fixed = 1024 + 256;
+    int stages = (int)((kSmemCap - fixed) / stage_bytes);
+    if (stages > 4) stages = 4;
+    if (stages < 2) return cudaErrorInvalidValue;
+    p.stages = stages;
+    // the epilogue reuses the stage buffers for its [4][E] partial sums
+    const size_t smem = fixed + stages * stage_bytes;
+
+    CUtensorMap mx, mw;
+    const cuuint64_t xd[2] = {(cuuint64_t)a.d, (cuuint64_t)a.T};
+    const cuuint64_t xs[1] = {(cuuint64_t)a.d * 2};
+    const cuuint32_t xb[2] = {RBK, RM};
+    if (!encode(&mx, 2, a.x, xd, xs, xb)) return cudaErrorInvalidValue;
+    const cuuint64_t wd[3] = {(cuuint64_t)a.d, (cuuint64_t)a.E, 3};
+    const cuuint64_t wst[2] = {(cuuint64_t)a.d * 2, (cuuint64_t)a.E * a.d * 2};
+    const cuuint32_t wb[3] = {RBK, (cuuint32_t)p.n_pad, 1};
+    if (!encode(&mw, 3, wsplit, wd, wst, wb)) return cudaErrorInvalidValue;
+
+    if (a.k <= 1) return launch_tc<1>(mx, mw, p, smem, st);
+    if (a.k <= 2) return launch_tc<2>(mx, mw, p, smem, st);
+    if (a.k <= 4) return launch_tc<4>(mx, mw, p, smem, st);
+    if (a.k <= 8) return launch_tc<8>(mx, mw, p, smem, st);
+    if (a.k <= 16) return launch_tc<16>(mx, mw, p, smem, st);
+    return launch_tc<32>(mx, mw, p, smem, st);
+}
+
+}  // namespace moe

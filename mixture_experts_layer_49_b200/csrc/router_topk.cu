@@ -8,6 +8,7 @@
 // Optimization Techniques", How It Works 2: a per-expert bias steers the
 // selection only; gates come from the unbiased scores.
 //
+// This FFMA version serves fp32 layers; bf16 layers use router_sm100.cu.
 // One CTA handles 32 tokens and all E (<= 256) experts.  The logits of a token
 // live in the registers of one warp (expert e on lane e % 32), so the softmax,
 // the k rounds of warp arg-max and the gates never leave registers.
@@ -36,13 +37,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename TX>
 __device__ __forceinline__ void load_x_vec(const TX *src, float *dst);
 
-template <>
-__device__ __forceinline__ void load_x_vec<__nv_bfloat16>(const __nv_bfloat16 *src, float *dst) {
-    uint4 v = *reinterpret_cast<const uint4 *>(src);
-    const __nv_bfloat16 *h = reinterpret_cast<const __nv_bfloat16 *>(&v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = __bfloat162float(h[i]);
-}
 template <>
 __device__ __forceinline__ void load_x_vec<float>(const float *src, float *dst) {
     float4 v = *reinterpret_cast<const float4 *>(src);
@@ -208,11 +202,14 @@ cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int router_blocks(int T) { return (T + kTok - 1) / kTok; }
+int router_blocks(int T, bool bf16) { return bf16 ? router_tc_blocks(T) : (T + kTok - 1) / kTok; }
 
+// bf16 layers take the tensor-core router (router_sm100.cu); fp32 layers this
+// FFMA kernel, which keeps every product in fp32.
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
-    return bf16 ? launch_router_t<__nv_bfloat16>(a, st) : launch_router_t<float>(a, st);
+    if (bf16) return launch_router_tc(a, a.wsplit, a.status, st);
+    return launch_router_t<float>(a, st);
 }
 
 }  // namespace moe
