@@ -12,8 +12,11 @@
 //
 // fp32 accuracy on bf16 tensor cores: x is bf16 already; W_r (fp32) is split
 // exactly into three bf16 terms, W = hi + mid + lo (8 + 8 + 8 significand
-// bits), so x W = x hi + x mid + x lo with every product exact and the three
-// partial GEMMs accumulated into one fp32 TMEM accumulator.
+// bits), so x W = x hi + x mid + x lo with every product exact.  The tensor
+// core's fp32 accumulator rounds each K=16 step toward zero, a bias that grows
+// with the number of steps, so K is split over up to 8 separate TMEM
+// accumulators whose partial sums the epilogue adds in fp32 (round to
+// nearest) before anything else reads the logits.
 //
 // One CTA per 128 tokens (MMA M = 128, N = E rounded up to 16, K = d_model):
 //   warp 0      TMA producer: x tile 128 x 64 and the three W_r terms
@@ -51,6 +54,8 @@ struct TcRouterParams {
     int32_t *status;
     int T, d, E, k, score, renorm;
     int n_pad;                 // MMA N
+    int nparts;                // K-split: separate accumulators
+    int pstride;               // TMEM columns between accumulators (>= n_pad, multiple of 32)
     int stages;
     uint32_t b_bytes;          // one W_r term per stage: n_pad x 64 bf16
     uint32_t idesc;
@@ -152,6 +157,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            int prev_part = -1;
             for (int kb = 0; kb < nk; ++kb) {
                 if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) {
                     record_error(p.status, MOE_ERR_TIMEOUT, 12);
@@ -161,12 +167,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
                 tc_fence_after();
                 const uint32_t st = base + stage * stage_bytes;
+                const int part = kb * p.nparts / nk;             // contiguous K ranges per accumulator
+                const uint32_t dtm = tmem + (uint32_t)(part * p.pstride);
+                const uint32_t fresh = part != prev_part;
+                prev_part = part;
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
 #pragma unroll
                     for (int k = 0; k < RBK / 16; ++k)
-                        mma_bf16(tmem, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
-                                 (kb | j | k) ? 1u : 0u);
+                        mma_bf16(dtm, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
+                                 (fresh && j == 0 && k == 0) ? 0u : 1u);
                 mma_commit(smem_u32(&s.empty[stage]));
                 if (++stage == p.stages) { stage = 0; phase ^= 1u; }
             }
@@ -192,20 +202,30 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const int nchunk = (E + 31) / 32;
             const bool softmax = p.score == MOE_SCORE_SOFTMAX;
             float v[32];
-            // pass 1: max logit (softmax) / sum of sigmoids
+            // pass 1: logits h = sum of the K-split accumulators (fixed order) +
+            // logit offset, written back over accumulator 0; max logit (softmax)
+            // or sum of sigmoids
             float m = -INFINITY, ssum = 0.f;
             for (int c = 0; c < nchunk; ++c) {
                 __syncwarp();
                 tmem_ld32(taddr + c * 32, v);
+                for (int r = 1; r < p.nparts; ++r) {
+                    float w[32];
+                    tmem_ld32(taddr + r * p.pstride + c * 32, w);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] += w[j];
+                }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int e = c * 32 + j;
                     if (e < E) {
                         const float h = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
+                        v[j] = h;
                         if (softmax) m = fmaxf(m, h);
                         else ssum += 1.f / (1.f + expf(-h));
                     }
                 }
+                tmem_st32(taddr + c * 32, v);
             }
             // pass 2: softmax normaliser
             float z = 0.f;
@@ -216,7 +236,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int e = c * 32 + j;
-                        if (e < E) z += expf(v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f) - m);
+                        if (e < E) z += expf(v[j] - m);
                     }
                 }
             }
@@ -236,7 +256,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const int e = c * 32 + j;
                     float pn = 0.f;
                     if (e < E) {
-                        const float h = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
+                        const float h = v[j];
                         float sc, key;
                         if (softmax) {
                             sc = expf(h - m) / z;
@@ -371,8 +391,14 @@ cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status,
     p.n_pad = (a.E + 15) / 16 * 16;
     p.b_bytes = (uint32_t)p.n_pad * RBK * 2;
     p.idesc = make_idesc_bf16(RM, (uint32_t)p.n_pad);
+    p.pstride = (p.n_pad + 31) / 32 * 32;
+    const int nk = (a.d + RBK - 1) / RBK;
+    int nparts = 512 / p.pstride;
+    if (nparts > 8) nparts = 8;
+    if (nparts > nk) nparts = nk;
+    p.nparts = nparts;
     uint32_t cols = 32;
-    while ((int)cols < p.n_pad) cols <<= 1;
+    while ((int)cols < p.nparts * p.pstride) cols <<= 1;
     p.tmem_cols = cols;
     p.timeout_ns = 2000000000ull;
     const size_t stage_bytes = A_BYTES + 3 * (size_t)p.b_bytes;
