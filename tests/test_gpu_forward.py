@@ -16,7 +16,7 @@ import oracle
 from mixture_experts_layer_49_b200 import native as nat
 from mixture_experts_layer_49_b200 import synthetic as syn
 
-from helpers import (TOL_BF16, TOL_F32, TOL_LOSS, check_routing, make_case, oracle_dims, rel_err,
+from helpers import (TOL_BF16, TOL_F32, TOL_LOGIT, TOL_LOSS, check_routing, make_case, oracle_dims, rel_err,
                      sample_tokens, to_f64, weights_host)
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +44,7 @@ def check_forward(wl, inp, host, n_sample=None, seed=0):
     swapped = check_routing(out.idx.cpu().numpy(), out.gate.cpu().numpy(), r)
     np.testing.assert_array_equal(out.counts.cpu().numpy(), dp["counts"])
     assert int(out.n_dropped.item()) == dp["n_dropped"]
-    assert rel_err(out.logits.cpu().numpy(), r["logits"]) < 1e-5
+    assert rel_err(out.logits.cpu().numpy(), r["logits"]) < TOL_LOGIT
     loss = float(out.loss.item())
     assert abs(loss - bal["loss"]) <= TOL_LOSS * abs(bal["loss"])
     np.testing.assert_allclose(out.f.cpu().numpy(), bal["f"], rtol=1e-6)
