@@ -184,7 +184,6 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int n
         __syncwarp();
     }
     __syncthreads();
-    if (a.x_perm == nullptr) return;              // the consumer gathers rows from x itself
     // copy the kept rows of x into x_perm, one warp per row, 16-byte vectors
     const int nvec = a.d * (int)sizeof(TX) / 16;
     const uint4 *xs = static_cast<const uint4 *>(a.x);

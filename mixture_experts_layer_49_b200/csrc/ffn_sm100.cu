@@ -56,7 +56,6 @@ constexpr uint32_t kIdesc = make_idesc_bf16(BM, BNB);   // M=128, N=256
 
 struct GemmParams {
     const int32_t *offsets;   // [E+1]
-    const int32_t *row_token; // gather mode: token of every routed row
     const float *bias;        // [E, N_routed] or null (GELU b1 / b2)
     const float *row_gate;    // [rows] (GM_DOWN) or null
     __nv_bfloat16 *out;       // row stride ldo
@@ -117,10 +116,7 @@ __device__ __forceinline__ void fail(SmemTail &s, const GemmParams &p, int where
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
-// GATHER: routed A rows come straight from x through the row -> token map
-// (TMA tile::gather4, four rows per instruction, issued by all 32 lanes of
-// the producer warp) instead of from a pre-permuted copy of x.
-template <int MODE, bool GATHER>
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
@@ -180,54 +176,34 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const uint32_t tmem_base = s.tmem_base;
 
     if (warp == 0) {
-        // ================= TMA producer (lane 0; all lanes for gathered A tiles)
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            if (__shfl_sync(0xffffffffu, aborted(s) ? 1 : 0, 0)) break;
-            int g, mt, nt;
-            decode(s, G, tile, g, mt, nt);
-            const bool sh = g >= p.E;
-            const bool gather = GATHER && !sh;
-            const int K = sh ? p.K_shared : p.K_routed;
-            const int nk = (K + BK - 1) / BK;
-            const int a_row = sh ? (int)p.shared_a_row + mt * BM : s.row0[g] + mt * BM;
-            const CUtensorMap *mA = sh ? &tmAs : &tmA;
-            const CUtensorMap *mB = sh ? &tmBs : &tmB;
-            const CUtensorMap *mB2 = sh ? &tmBs2 : &tmB2;
-            const int e = sh ? 0 : g;
-            int tok[4] = {0, 0, 0, 0};
-            if (gather) {           // rows 4*lane .. 4*lane+3 of the tile; rows past the group read token 0
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = mt * BM + lane * 4 + i;
-                    tok[i] = r < s.rows[g] ? __ldg(p.row_token + s.row0[g] + r) : 0;
-                }
-            }
-            for (int kb = 0; kb < nk; ++kb) {
-                int ok = 1;
-                const uint32_t fb = smem_u32(&s.full[stage]);
-                if (lane == 0) {
-                    ok = mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns) ? 1 : 0;
-                    if (ok) mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) { if (lane == 0) fail(s, p, 1); break; }
-                if (gather) {
-                    tma_gather4(smA + stage * A_BYTES + lane * 4 * 128, &tmA, fb, kb * BK, tok[0], tok[1], tok[2],
-                                tok[3]);
-                } else if (lane == 0) {
+        // ================= TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
+                int g, mt, nt;
+                decode(s, G, tile, g, mt, nt);
+                const bool sh = g >= p.E;
+                const int K = sh ? p.K_shared : p.K_routed;
+                const int nk = (K + BK - 1) / BK;
+                const int a_row = sh ? (int)p.shared_a_row + mt * BM : s.row0[g] + mt * BM;
+                const CUtensorMap *mA = sh ? &tmAs : &tmA;
+                const CUtensorMap *mB = sh ? &tmBs : &tmB;
+                const CUtensorMap *mB2 = sh ? &tmBs2 : &tmB2;
+                const int e = sh ? 0 : g;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail(s, p, 1); break; }
+                    const uint32_t fb = smem_u32(&s.full[stage]);
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     tma_load_2d(smA + stage * A_BYTES, mA, fb, kb * BK, a_row);
-                }
-                if (lane == 0) {
                     if (MODE == GM_SWIGLU) {
                         tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * 128, e);
                         tma_load_3d(smB + stage * B_BYTES + B_BYTES / 2, mB2, fb, kb * BK, nt * 128, e);
                     } else {
                         tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * BNB, e);
                     }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
         }
     } else if (warp == 1) {
@@ -374,17 +350,17 @@ bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE, bool GATHER>
+template <int MODE>
 cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
                         const CUtensorMap &Bs, const CUtensorMap &Bs2, const GemmParams &p, int grid, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, GATHER>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    tc_grouped_gemm<MODE, GATHER><<<grid, kThreads, kSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
+    tc_grouped_gemm<MODE><<<grid, kThreads, kSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
     return cudaGetLastError();
 }
 
@@ -399,16 +375,10 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     const int grid = a.num_sms > 0 ? a.num_sms : 148;
     const uint64_t timeout_ns = 2000000000ull;
 
-    // ---- GEMM 1: H = act(X W1^T [+ b1])   (A: x_perm, or x gathered through
-    // row_token; shared expert: x.  B: W1 (+Wu) / Wsg (+Wsu))
+    // ---- GEMM 1: H = act(X W1^T [+ b1])   (A: x_perm / x, B: W1 (+Wu) / Wsg (+Wsu))
     CUtensorMap A1, A1s, B1, B1u, B1s, B1su;
     const uint32_t box1 = swiglu ? 128 : 256;
-    const bool gather = a.row_token != nullptr;
-    if (gather) {
-        if (!make_map(&A1, 2, a.x, a.d, a.T, 1, a.d, 0, 1)) return cudaErrorInvalidValue;   // one-row box
-    } else {
-        if (!make_map(&A1, 2, a.x_perm, a.d, routed_rows, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
-    }
+    if (!make_map(&A1, 2, a.x_perm, a.d, routed_rows, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
     if (!make_map(&B1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
     if (swiglu) {
         if (!make_map(&B1u, 3, a.Wu, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
@@ -428,7 +398,6 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     }
     GemmParams p1{};
     p1.offsets = a.offsets;
-    p1.row_token = a.row_token;
     p1.bias = swiglu ? nullptr : a.b1;
     p1.row_gate = nullptr;
     p1.out = static_cast<__nv_bfloat16 *>(a.H);
@@ -441,13 +410,8 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p1.shared_a_row = 0;
     p1.shared_out_row = a.shared_base;
     p1.timeout_ns = timeout_ns;
-    cudaError_t err;
-    if (gather)
-        err = swiglu ? launch_gemm<GM_SWIGLU, true>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
-                     : launch_gemm<GM_GELU, true>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
-    else
-        err = swiglu ? launch_gemm<GM_SWIGLU, false>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
-                     : launch_gemm<GM_GELU, false>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
+    cudaError_t err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
+                             : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
     if (err != cudaSuccess) return err;
 
     // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
@@ -474,7 +438,7 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p2.shared_a_row = a.shared_base;
     p2.shared_out_row = a.shared_base;
     p2.timeout_ns = timeout_ns;
-    return launch_gemm<GM_DOWN, false>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st);
+    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st);
 }
 
 }  // namespace moe

@@ -40,7 +40,7 @@ struct DispatchArgs {
     int32_t *row_of;             // [T, k]
     int32_t *row_token;          // [T*k]
     float *row_gate;             // [T*k]
-    void *x_perm;                // [T*k, d], or null: rows are not copied
+    void *x_perm;                // [T*k, d]
     int32_t *n_dropped;          // device scalar or null
     int32_t *status;             // workspace status word
     int T, d, E, k, capacity;    // capacity < 0: unlimited
@@ -52,8 +52,7 @@ cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st);
 // offsets[g+1] of x_perm / H / y_perm); group E is the shared expert (rows
 // 0..T-1 of x, rows shared_base.. of H / y_perm).
 struct FfnArgs {
-    const void *x_perm;          // [T*k, d]; unused when row_token is set
-    const int32_t *row_token;    // [T*k] or null: bf16 GEMM 1 gathers x rows through it
+    const void *x_perm;          // [T*k, d]
     const void *x;               // [T, d] (shared expert) or null
     const int32_t *offsets;      // [E+1]
     const float *row_gate;       // [T*k]

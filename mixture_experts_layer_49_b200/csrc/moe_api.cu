@@ -130,7 +130,6 @@ moe::FfnArgs ffn_args(const moe_config *c, const void *x_perm, const int32_t *of
     a.x_perm = x_perm; a.x = x; a.offsets = offsets; a.row_gate = row_gate;
     a.W1 = W1; a.Wu = Wu; a.W2 = W2; a.b1 = b1; a.b2 = b2;
     a.Wsg = Wsg; a.Wsu = Wsu; a.Wsd = Wsd;
-    a.row_token = nullptr;
     a.H = at<char>(ws, L.H);
     a.y_perm = y_perm;
     a.status = status_word(ws);
@@ -308,8 +307,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     da.chunk_base = at<int32_t>(ws, L.chunk_base);
     da.counts = counts; da.kept = at<int32_t>(ws, L.kept); da.offsets = offsets;
     da.row_of = row_of; da.row_token = at<int32_t>(ws, L.row_token); da.row_gate = row_gate;
-    // bf16 layers: GEMM 1 gathers the rows of x itself (no permuted copy)
-    da.x_perm = bf16 ? nullptr : at<char>(ws, L.x_perm);
+    da.x_perm = at<char>(ws, L.x_perm);
     da.n_dropped = n_dropped;
     da.status = status_word(ws);
     da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
@@ -318,7 +316,6 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
 
     moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
                                y_perm, ws);
-    if (bf16) fa.row_token = da.row_token;
     e = bf16 ? moe::launch_ffn_bf16(fa, st) : moe::launch_ffn_f32(fa, st);
     if (e != cudaSuccess) return cuda_fail(e, "grouped_ffn");
 
