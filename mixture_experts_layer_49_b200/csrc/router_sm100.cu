@@ -240,7 +240,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     }
                 }
             }
-            // pass 3: scores, keys, top-k, per-block sums
+            // pass 3: scores and keys (unrolled, cheap), staged per chunk in
+            // shared memory [32][128] so the top-k insertion runs as one rolled
+            // loop (a fully unrolled insertion would overflow the instruction
+            // cache); per-block sums of the normalised scores
+            float *kbuf = part + 4 * 256;           // [32][128] keys of the current chunk
+            float *sbuf = kbuf + 32 * 128;          // [32][128] scores of the current chunk
             float tk[KMAX], ts[KMAX];
             int te[KMAX];
 #pragma unroll
@@ -254,10 +259,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int e = c * 32 + j;
-                    float pn = 0.f;
+                    float pn = 0.f, sc = 0.f, key = -INFINITY;
                     if (e < E) {
                         const float h = v[j];
-                        float sc, key;
                         if (softmax) {
                             sc = expf(h - m) / z;
                             pn = sc;
@@ -269,24 +273,33 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         }
                         if (p.sel_bias) key += __ldg(p.sel_bias + e);
                         if (p.logits_out && tok_ok) p.logits_out[(size_t)t * E + e] = h;
-                        if (ahead(key, e, thr_k, thr_e)) {
-                            float ck = key, cs = sc;
-                            int ce = e;
-#pragma unroll
-                            for (int i = 0; i < KMAX; ++i) {
-                                if (i < k && ahead(ck, ce, tk[i], te[i])) {
-                                    const float a = tk[i], b = ts[i];
-                                    const int ei = te[i];
-                                    tk[i] = ck; ts[i] = cs; te[i] = ce;
-                                    ck = a; cs = b; ce = ei;
-                                }
-                            }
-#pragma unroll
-                            for (int i = 0; i < KMAX; ++i)
-                                if (i == k - 1) { thr_k = tk[i]; thr_e = te[i]; }
-                        }
                     }
+                    kbuf[j * 128 + row] = key;
+                    sbuf[j * 128 + row] = sc;
                     v[j] = tok_ok ? pn : 0.f;
+                }
+                const int jn = E - c * 32 < 32 ? E - c * 32 : 32;
+#pragma unroll 1
+                for (int j = 0; j < jn; ++j) {
+                    const float key = kbuf[j * 128 + row];
+                    const int e = c * 32 + j;
+                    // a sorted top-KMAX list (KMAX >= k, so its first k entries are
+                    // the top-k); all indices compile-time, so it stays in registers
+                    if (ahead(key, e, thr_k, thr_e)) {
+                        float ck = key, cs = sbuf[j * 128 + row];
+                        int ce = e;
+#pragma unroll
+                        for (int i = 0; i < KMAX; ++i) {
+                            if (ahead(ck, ce, tk[i], te[i])) {
+                                const float a = tk[i], b = ts[i];
+                                const int ei = te[i];
+                                tk[i] = ck; ts[i] = cs; te[i] = ce;
+                                ck = a; cs = b; ce = ei;
+                            }
+                        }
+                        thr_k = tk[KMAX - 1];
+                        thr_e = te[KMAX - 1];
+                    }
                 }
                 // transpose-reduce: lane L ends with the sum over the warp's 32
                 // tokens of the score of expert c*32 + L
@@ -406,6 +419,8 @@ cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status,
     int stages = (int)((kSmemCap - fixed) / stage_bytes);
     if (stages > 4) stages = 4;
     if (stages < 2) return cudaErrorInvalidValue;
+    // the epilogue reuses the drained stages for part[4][256] + keys/scores [2][32][128]
+    if ((size_t)stages * stage_bytes < (4 * 256 + 2 * 32 * 128) * sizeof(float)) return cudaErrorInvalidValue;
     p.stages = stages;
     // the epilogue reuses the stage buffers for its [4][E] partial sums
     const size_t smem = fixed + stages * stage_bytes;
