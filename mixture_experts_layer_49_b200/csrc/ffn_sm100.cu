@@ -9,14 +9,15 @@
 // recommend (Router Optimization page, What Most Articles Miss 2; serving
 // tutorial, grouped GEMM remark).
 //
-// Kernel shape (one persistent CTA per SM, 192 threads, warp-specialised):
+// Kernel shape (one persistent CTA per SM, 320 threads, warp-specialised):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
 //               swizzle) per stage, 4 stages, mbarrier transaction counts
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (M=128, N=256, K=16, fp32 accumulators in TMEM), two
 //               256-column accumulators so the epilogue of tile i overlaps
 //               the mainloop of tile i+1
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, fused activation
+//   warps 2..9  epilogue (two warps per TMEM lane quadrant, each taking half
+//               of the columns): tcgen05.ld 32 lanes x 32 columns, fused activation
 //               (SwiGLU: gate and up halves of one N=256 accumulator; GELU:
 //               bias + exact-erf GELU) or fused bias + gate scale, bf16 stores
 // Tiles: groups are the routed experts (rows offsets[e]..offsets[e+1] of the
@@ -43,7 +44,7 @@ constexpr int BM = 128;                 // rows per tile (MMA M)
 constexpr int BK = 64;                  // K per stage: one 128-byte swizzle atom of bf16
 constexpr int BNB = 256;                // B rows per stage (MMA N)
 constexpr int STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                // 10 warps: producer, MMA, 8 epilogue
 constexpr uint32_t A_BYTES = BM * BK * 2;       // 16 KiB
 constexpr uint32_t B_BYTES = BNB * BK * 2;      // 32 KiB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -149,7 +150,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         s.tile_start[0] = 0;
         s.abort_flag = 0;
         for (int i = 0; i < STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 4); }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 8); }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -238,8 +239,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
         }
     } else {
-        // ================= epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        // ================= epilogue: warps 2..9.  TMEM lane quadrant = warp % 4;
+        // warps 2-5 take the first half of the tile's columns, warps 6-9 the second
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
         int ab = 0;
         uint32_t aphase = 0;
@@ -247,6 +250,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int g, mt, nt;
             decode(s, G, tile, g, mt, nt);
             const bool sh = g >= p.E;
+            const int grow = mt * BM + r_in_tile;
+            const bool valid = grow < s.rows[g];
+            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            // the row's gate is fetched before the accumulator wait, hiding its latency
+            float gscale = 1.f;
+            if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
             // lane 0 waits, the warp follows its verdict (keeps the warp converged
             // for the .sync.aligned TMEM loads)
             int ok = 1;
@@ -255,15 +264,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (!ok) { if (lane == 0) fail(s, p, 4); break; }
             __syncwarp();
             tc_fence_after();
-            const int grow = mt * BM + r_in_tile;
-            const bool valid = grow < s.rows[g];
-            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
             const int N = sh ? p.N_shared : p.N_routed;
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             if (MODE == GM_SWIGLU) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = half * 2; c < half * 2 + 2; ++c) {
                     float gv[32], uv[32];
                     tmem_ld32(taddr + c * 32, gv);
                     tmem_ld32(taddr + 128 + c * 32, uv);
@@ -280,10 +286,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             } else {
                 const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-                float gscale = 1.f;
-                if (MODE == GM_DOWN && !sh && valid) gscale = p.row_gate[orow];
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = half * 4; c < half * 4 + 4; ++c) {
                     float acc[32];
                     tmem_ld32(taddr + c * 32, acc);
                     const int col0 = nt * BNB + c * 32;
