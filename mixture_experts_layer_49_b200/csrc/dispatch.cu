@@ -27,7 +27,8 @@ namespace {
 
 constexpr int kChunk = 64;        // tokens per chunk
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kPermThreads = 512;            // permute: 16 warps share the row copies
+constexpr int kWarps = kPermThreads / 32;
 
 __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, int nchunks) {
     __shared__ int cnt[256];
@@ -90,14 +91,14 @@ __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nc
 }
 
 template <typename TX>
-__global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int nchunks) {
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, int nchunks) {
     __shared__ int base[256];
     __shared__ int offs[256];
     __shared__ int wcnt[kWarps][256];
     __shared__ int2 list[kChunk * 32];           // (row, token) of each pair, k <= 32
     const int c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, k = a.k;
-    for (int e = tid; e < E; e += kThreads) {
+    for (int e = tid; e < E; e += kPermThreads) {
         base[e] = a.chunk_base[(size_t)e * nchunks + c];
         offs[e] = a.kept[e];
 #pragma unroll
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int n
     }
     __syncthreads();
     // exclusive scan over warps, per expert
-    for (int e = tid; e < E; e += kThreads) {
+    for (int e = tid; e < E; e += kPermThreads) {
         int run = 0;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) { const int v = wcnt[w][e]; wcnt[w][e] = run; run += v; }
@@ -191,13 +192,15 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(DispatchArgs a, int n
     for (int q = warp; q < npairs; q += kWarps) {
         const int2 rt = list[q];
         if (rt.x < 0) continue;
-        const uint4 *src = xs + (size_t)rt.y * nvec;
-        uint4 *dst = xd + (size_t)rt.x * nvec;
+        const uint4 *__restrict__ src = xs + (size_t)rt.y * nvec;
+        uint4 *__restrict__ dst = xd + (size_t)rt.x * nvec;
         int v = lane;
-        for (; v + 96 < nvec; v += 128) {          // four 16-byte loads in flight per lane
-            const uint4 r0 = __ldg(src + v), r1 = __ldg(src + v + 32);
-            const uint4 r2 = __ldg(src + v + 64), r3 = __ldg(src + v + 96);
-            dst[v] = r0; dst[v + 32] = r1; dst[v + 64] = r2; dst[v + 96] = r3;
+        for (; v + 224 < nvec; v += 256) {         // eight 16-byte loads in flight per lane
+            uint4 r[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) r[i] = __ldg(src + v + 32 * i);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[v + 32 * i] = r[i];
         }
         for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
     }
@@ -219,8 +222,8 @@ cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
     if (nchunks == 0) {           // no tokens: every count is zero, offsets all zero
         empty_offsets_kernel<<<1, 256, 0, st>>>(a);
     } else {
-        if (bf16) permute_kernel<__nv_bfloat16><<<nchunks, kThreads, 0, st>>>(a, nchunks);
-        else permute_kernel<float><<<nchunks, kThreads, 0, st>>>(a, nchunks);
+        if (bf16) permute_kernel<__nv_bfloat16><<<nchunks, kPermThreads, 0, st>>>(a, nchunks);
+        else permute_kernel<float><<<nchunks, kPermThreads, 0, st>>>(a, nchunks);
     }
     return cudaGetLastError();
 }

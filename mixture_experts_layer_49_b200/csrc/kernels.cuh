@@ -20,15 +20,14 @@ struct RouterArgs {
     float *psum;                 // [router_blocks(T, bf16), E]
     int T, d, E, k, score, renorm;
     void *wsplit;                // bf16 layers: [3, E, d] scratch for the split W_r
+    float *logits_ws;            // bf16 layers: [T, E] scratch for the logits (if no logits_out)
     int32_t *status;             // workspace status word
 };
-// Rows of the per-block score sums: 128 tokens per block on the tensor-core
-// router (bf16 layers), 32 on the fp32 router.
-int router_blocks(int T, bool bf16);
+// Rows of the per-block score sums (32 tokens per block).
+int router_blocks(int T);
 size_t router_split_bytes(int d, int E);
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st);
-int router_tc_blocks(int T);
-cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status, cudaStream_t st);
+cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStream_t st);
 
 struct DispatchArgs {
     const void *x;               // [T, d]

@@ -24,7 +24,7 @@ moe_status cuda_fail(cudaError_t e, const char *where) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-    size_t router_w, psum, chunk_cnt, chunk_base, kept, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
+    size_t router_w, logits, psum, chunk_cnt, chunk_base, kept, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
 };
 
 int64_t perm_rows(const moe_config *c) {
@@ -38,10 +38,11 @@ Layout layout(const moe_config *c) {
     const size_t rows = (size_t)perm_rows(c);
     const size_t hF = (size_t)(c->d_ff > c->d_ff_shared ? c->d_ff : c->d_ff_shared);
     const bool bf16 = c->dtype == MOE_BF16;
-    const size_t nblk = (size_t)moe::router_blocks(c->T, bf16);
+    const size_t nblk = (size_t)moe::router_blocks(c->T);
     const size_t nch = (size_t)moe::dispatch_chunks(c->T);
     size_t o = sizeof(moe::WsHeader);
     L.router_w = o;   o = align256(o + (bf16 ? moe::router_split_bytes(c->d_model, c->E) : 0));
+    L.logits = o;     o = align256(o + (bf16 ? (size_t)c->T * c->E * 4 : 0));
     L.psum = o;       o = align256(o + nblk * c->E * 4);
     L.chunk_cnt = o;  o = align256(o + nch * c->E * 4);
     L.chunk_base = o; o = align256(o + nch * c->E * 4);
@@ -166,7 +167,7 @@ int32_t moe_capacity(const moe_config *cfg) {
 
 int32_t moe_router_blocks(const moe_config *cfg) {
     if (check_cfg(cfg) != MOE_OK) return 0;
-    return moe::router_blocks(cfg->T, cfg->dtype == MOE_BF16);
+    return moe::router_blocks(cfg->T);
 }
 
 int64_t moe_perm_rows(const moe_config *cfg) {
@@ -194,7 +195,7 @@ moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
     moe::RouterArgs a{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
-                      at<char>(ws, layout(cfg).router_w), status_word(ws)};
+                      at<char>(ws, layout(cfg).router_w), at<float>(ws, layout(cfg).logits), status_word(ws)};
     cudaError_t e = moe::launch_router(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router");
 }
@@ -264,8 +265,7 @@ moe_status moe_balance_stats(const moe_config *cfg, const int32_t *counts, const
     NEED(counts); NEED(f); NEED(P); NEED(loss);
     if (cfg->T > 0) NEED(psum);
     ALIGNED(counts, 4); ALIGNED(psum, 4); ALIGNED(f, 4); ALIGNED(P, 4); ALIGNED(loss, 8);
-    moe::BalanceArgs a{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k,
-                       moe::router_blocks(cfg->T, cfg->dtype == MOE_BF16)};
+    moe::BalanceArgs a{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
     cudaError_t e = moe::launch_balance(a, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "balance");
 }
@@ -298,7 +298,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
 
     moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                        cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
-                       at<char>(ws, L.router_w), status_word(ws)};
+                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws)};
     if ((e = moe::launch_router(ra, bf16, st)) != cudaSuccess) return cuda_fail(e, "router");
 
     moe::DispatchArgs da{};
@@ -323,7 +323,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
 
-    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T, bf16)};
+    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
     if ((e = moe::launch_balance(ba, st)) != cudaSuccess) return cuda_fail(e, "balance");
     return MOE_OK;
 }

@@ -22,12 +22,11 @@
 //   warp 0      TMA producer: x tile 128 x 64 and the three W_r terms
 //               N x 64 per stage (128-byte swizzle), 2-4 stages
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5  epilogue, one thread per token: the token's E logits come out
-//               of TMEM 32 columns at a time (three passes: max, sum, then
-//               scores, selection keys and a register-resident top-k list);
-//               per-expert sums of the normalised scores over the CTA's 128
-//               tokens by an in-warp transpose-reduce and a fixed-order sum of
-//               the four warps (deterministic).
+//   warps 2..5  epilogue, one thread per token: add the K-split accumulators
+//               and the logit offset, store the fp32 logits row
+// Scores, top-k, gates and the per-block score sums then run in the
+// warp-per-token selection kernel of router_topk.cu (a per-thread top-k over
+// E values was instruction-bound here).
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -46,13 +45,9 @@ constexpr int kSmemCap = 227 * 1024;
 
 struct TcRouterParams {
     const float *logit_bias;
-    const float *sel_bias;
-    int32_t *idx;
-    float *gate;
-    float *logits_out;
-    float *psum;
+    float *logits;             // [T, E] fp32 out
     int32_t *status;
-    int T, d, E, k, score, renorm;
+    int T, d, E;
     int n_pad;                 // MMA N
     int nparts;                // K-split: separate accumulators
     int pstride;               // TMEM columns between accumulators (>= n_pad, multiple of 32)
@@ -100,12 +95,6 @@ __global__ void __launch_bounds__(256) split_router_weights(const float *__restr
     }
 }
 
-// (key desc, expert id asc): is (ka, ea) ahead of (kb, eb)?
-__device__ __forceinline__ bool ahead(float ka, int ea, float kb, int eb) {
-    return ka > kb || (ka == kb && ea < eb);
-}
-
-template <int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const TcRouterParams p) {
@@ -195,147 +184,27 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         } else {
             __syncwarp();
             tc_fence_after();
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            float *part = reinterpret_cast<float *>(smem);     // [4][E], reuses the drained stage buffers
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
             const int E = p.E;
-            const int nchunk = (E + 31) / 32;
-            const bool softmax = p.score == MOE_SCORE_SOFTMAX;
-            float v[32];
-            // pass 1: logits h = sum of the K-split accumulators (fixed order) +
-            // logit offset, written back over accumulator 0; max logit (softmax)
-            // or sum of sigmoids
-            float m = -INFINITY, ssum = 0.f;
-            for (int c = 0; c < nchunk; ++c) {
+            float *dst = p.logits + (size_t)t * E;
+            for (int c = 0; c < (E + 31) / 32; ++c) {
+                float v[32];
                 __syncwarp();
                 tmem_ld32(taddr + c * 32, v);
-                for (int r = 1; r < p.nparts; ++r) {
+                for (int r = 1; r < p.nparts; ++r) {       // fixed order: parts 0, 1, 2, ...
                     float w[32];
                     tmem_ld32(taddr + r * p.pstride + c * 32, w);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] += w[j];
                 }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int e = c * 32 + j;
-                    if (e < E) {
-                        const float h = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
-                        v[j] = h;
-                        if (softmax) m = fmaxf(m, h);
-                        else ssum += 1.f / (1.f + expf(-h));
-                    }
-                }
-                tmem_st32(taddr + c * 32, v);
-            }
-            // pass 2: softmax normaliser
-            float z = 0.f;
-            if (softmax) {
-                for (int c = 0; c < nchunk; ++c) {
-                    __syncwarp();
-                    tmem_ld32(taddr + c * 32, v);
+                if (tok_ok) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int e = c * 32 + j;
-                        if (e < E) z += expf(v[j] - m);
+                        if (e < E) dst[e] = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
                     }
                 }
             }
-            // pass 3: scores and keys (unrolled, cheap), staged per chunk in
-            // shared memory [32][128] so the top-k insertion runs as one rolled
-            // loop (a fully unrolled insertion would overflow the instruction
-            // cache); per-block sums of the normalised scores
-            float *kbuf = part + 4 * 256;           // [32][128] keys of the current chunk
-            float *sbuf = kbuf + 32 * 128;          // [32][128] scores of the current chunk
-            float tk[KMAX], ts[KMAX];
-            int te[KMAX];
-#pragma unroll
-            for (int i = 0; i < KMAX; ++i) { tk[i] = -INFINITY; ts[i] = 0.f; te[i] = 0x7fffffff; }
-            float thr_k = -INFINITY;
-            int thr_e = 0x7fffffff;
-            const int k = p.k;
-            for (int c = 0; c < nchunk; ++c) {
-                __syncwarp();
-                tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int e = c * 32 + j;
-                    float pn = 0.f, sc = 0.f, key = -INFINITY;
-                    if (e < E) {
-                        const float h = v[j];
-                        if (softmax) {
-                            sc = expf(h - m) / z;
-                            pn = sc;
-                            key = h;
-                        } else {
-                            sc = 1.f / (1.f + expf(-h));
-                            pn = sc / ssum;
-                            key = sc;
-                        }
-                        if (p.sel_bias) key += __ldg(p.sel_bias + e);
-                        if (p.logits_out && tok_ok) p.logits_out[(size_t)t * E + e] = h;
-                    }
-                    kbuf[j * 128 + row] = key;
-                    sbuf[j * 128 + row] = sc;
-                    v[j] = tok_ok ? pn : 0.f;
-                }
-                const int jn = E - c * 32 < 32 ? E - c * 32 : 32;
-#pragma unroll 1
-                for (int j = 0; j < jn; ++j) {
-                    const float key = kbuf[j * 128 + row];
-                    const int e = c * 32 + j;
-                    // a sorted top-KMAX list (KMAX >= k, so its first k entries are
-                    // the top-k); all indices compile-time, so it stays in registers
-                    if (ahead(key, e, thr_k, thr_e)) {
-                        float ck = key, cs = sbuf[j * 128 + row];
-                        int ce = e;
-#pragma unroll
-                        for (int i = 0; i < KMAX; ++i) {
-                            if (ahead(ck, ce, tk[i], te[i])) {
-                                const float a = tk[i], b = ts[i];
-                                const int ei = te[i];
-                                tk[i] = ck; ts[i] = cs; te[i] = ce;
-                                ck = a; cs = b; ce = ei;
-                            }
-                        }
-                        thr_k = tk[KMAX - 1];
-                        thr_e = te[KMAX - 1];
-                    }
-                }
-                // transpose-reduce: lane L ends with the sum over the warp's 32
-                // tokens of the score of expert c*32 + L
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-#pragma unroll
-                    for (int j = 0; j < o; ++j) {
-                        const bool upper = (lane & o) != 0;
-                        const float send = upper ? v[j] : v[j + o];
-                        const float keep = upper ? v[j + o] : v[j];
-                        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                    }
-                }
-                if (c * 32 + lane < E) part[q * E + c * 32 + lane] = v[0];
-            }
-            if (tok_ok) {
-                float selsum = 0.f;
-#pragma unroll
-                for (int i = 0; i < KMAX; ++i) if (i < k) selsum += ts[i];
-#pragma unroll
-                for (int i = 0; i < KMAX; ++i) {
-                    if (i < k) {
-                        const float g = (softmax && !p.renorm) ? ts[i] : ts[i] / selsum;
-                        p.idx[(size_t)t * k + i] = te[i];
-                        p.gate[(size_t)t * k + i] = g;
-                    }
-                }
-            }
-        }
-        // the four epilogue warps meet here whether or not the wait succeeded
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (ok) {
-            const float *part = reinterpret_cast<const float *>(smem);
-            const int E = p.E;
-            for (int e = row; e < E; e += 128)
-                p.psum[(size_t)blockIdx.x * E + e] = ((part[e] + part[E + e]) + part[2 * E + e]) + part[3 * E + e];
         }
     }
     tc_fence_before();
@@ -369,28 +238,26 @@ bool encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KMAX>
 cudaError_t launch_tc(const CUtensorMap &mx, const CUtensorMap &mw, const TcRouterParams &p, size_t smem,
                       cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemCap);
+        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     const int grid = (p.T + RM - 1) / RM;
-    router_tc_kernel<KMAX><<<grid, kThreads, smem, st>>>(mx, mw, p);
+    router_tc_kernel<<<grid, kThreads, smem, st>>>(mx, mw, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int router_tc_blocks(int T) { return (T + RM - 1) / RM; }
-
 size_t router_split_bytes(int d, int E) { return (size_t)3 * E * d * 2; }
 
-cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status, cudaStream_t st) {
+// Logits h = x W_r (+ logit offset) into `logits` [T, E] fp32.
+cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStream_t st) {
+    void *wsplit = a.wsplit;
     if (a.T == 0) return cudaSuccess;
     dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
     split_router_weights<<<sg, 256, 0, st>>>(a.Wr, a.d, a.E, static_cast<__nv_bfloat16 *>(wsplit));
@@ -398,9 +265,8 @@ cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status,
     if (e != cudaSuccess) return e;
 
     TcRouterParams p{};
-    p.logit_bias = a.logit_bias; p.sel_bias = a.sel_bias; p.idx = a.idx; p.gate = a.gate;
-    p.logits_out = a.logits_out; p.psum = a.psum; p.status = status;
-    p.T = a.T; p.d = a.d; p.E = a.E; p.k = a.k; p.score = a.score; p.renorm = a.renorm;
+    p.logit_bias = a.logit_bias; p.logits = logits; p.status = a.status;
+    p.T = a.T; p.d = a.d; p.E = a.E;
     p.n_pad = (a.E + 15) / 16 * 16;
     p.b_bytes = (uint32_t)p.n_pad * RBK * 2;
     p.idesc = make_idesc_bf16(RM, (uint32_t)p.n_pad);
@@ -419,10 +285,7 @@ cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status,
     int stages = (int)((kSmemCap - fixed) / stage_bytes);
     if (stages > 4) stages = 4;
     if (stages < 2) return cudaErrorInvalidValue;
-    // the epilogue reuses the drained stages for part[4][256] + keys/scores [2][32][128]
-    if ((size_t)stages * stage_bytes < (4 * 256 + 2 * 32 * 128) * sizeof(float)) return cudaErrorInvalidValue;
     p.stages = stages;
-    // the epilogue reuses the stage buffers for its [4][E] partial sums
     const size_t smem = fixed + stages * stage_bytes;
 
     CUtensorMap mx, mw;
@@ -435,12 +298,7 @@ cudaError_t launch_router_tc(const RouterArgs &a, void *wsplit, int32_t *status,
     const cuuint32_t wb[3] = {RBK, (cuuint32_t)p.n_pad, 1};
     if (!encode(&mw, 3, wsplit, wd, wst, wb)) return cudaErrorInvalidValue;
 
-    if (a.k <= 1) return launch_tc<1>(mx, mw, p, smem, st);
-    if (a.k <= 2) return launch_tc<2>(mx, mw, p, smem, st);
-    if (a.k <= 4) return launch_tc<4>(mx, mw, p, smem, st);
-    if (a.k <= 8) return launch_tc<8>(mx, mw, p, smem, st);
-    if (a.k <= 16) return launch_tc<16>(mx, mw, p, smem, st);
-    return launch_tc<32>(mx, mw, p, smem, st);
+    return launch_tc(mx, mw, p, smem, st);
 }
 
 }  // namespace moe

@@ -43,61 +43,15 @@ __device__ __forceinline__ void load_x_vec<float>(const float *src, float *dst) 
     dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
 }
 
-template <typename TX, int EPT>
-__global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
-    constexpr int VEC = 16 / sizeof(TX);              // x elements per 16-byte load
-    constexpr int EW = EPT * 32;                      // expert slots per warp row
-    __shared__ float xs[kTok][kKc + 1];
-    __shared__ float wsm[kKc][EW];
-    __shared__ float part[kThreads / 32][EW];
-
+// Scores, top-k, gates and the block's score sums for the 32 tokens starting
+// at t0 (warp w holds tokens t0 + 4w .. t0 + 4w + 3; acc[i][j] is the logit of
+// token 4w + i for expert lane + 32 j).  add_bias: add logit_bias to acc first
+// (the tensor-core path has added it already).  part: shared [8][EPT*32].
+template <int EPT>
+__device__ __forceinline__ void select_tokens(const RouterArgs &a, float (&acc)[4][EPT], int t0, bool add_bias,
+                                              float (*part)[EPT * 32]) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * kTok;
-    const int d = a.d, E = a.E, k = a.k;
-
-    float acc[4][EPT];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
-
-    const TX *x = static_cast<const TX *>(a.x);
-    for (int k0 = 0; k0 < d; k0 += kKc) {
-        // x chunk [32 tokens][32]: 16-byte vector loads (d % 8 == 0)
-        for (int v = tid; v < kTok * (kKc / VEC); v += kThreads) {
-            const int tt = v / (kKc / VEC), kv = (v % (kKc / VEC)) * VEC;
-            float vals[VEC];
-            const int t = t0 + tt;
-            if (t < a.T && k0 + kv < d) {
-                load_x_vec<TX>(x + (size_t)t * d + k0 + kv, vals);
-            } else {
-#pragma unroll
-                for (int i = 0; i < VEC; ++i) vals[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) xs[tt][kv + i] = vals[i];
-        }
-        // W_r chunk [32][E] (row-major [d, E], coalesced along E)
-        for (int v = tid; v < kKc * EW; v += kThreads) {
-            const int kk = v / EW, e = v % EW;
-            wsm[kk][e] = (k0 + kk < d && e < E) ? a.Wr[(size_t)(k0 + kk) * E + e] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < kKc; ++kk) {
-            float xv[4], wv[EPT];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) xv[i] = xs[warp * 4 + i][kk];
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) wv[j] = wsm[kk][lane + 32 * j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < EPT; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-
+    const int E = a.E, k = a.k;
     float psum_acc[EPT];
 #pragma unroll
     for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
@@ -112,7 +66,7 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
         for (int j = 0; j < EPT; ++j) {
             const int e = lane + 32 * j;
             valid[j] = e < E;
-            h[j] = acc[i][j] + ((a.logit_bias && valid[j]) ? a.logit_bias[e] : 0.f);
+            h[j] = acc[i][j] + ((add_bias && a.logit_bias && valid[j]) ? a.logit_bias[e] : 0.f);
         }
         float norm;
         if (a.score == MOE_SCORE_SOFTMAX) {
@@ -140,7 +94,7 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
             if (a.sel_bias && valid[j]) key[j] += a.sel_bias[lane + 32 * j];
             psum_acc[j] += (a.score == MOE_SCORE_SOFTMAX) ? sc[j] : sc[j] / norm;
         }
-        if (a.logits_out) {
+        if (a.logits_out && add_bias) {
 #pragma unroll
             for (int j = 0; j < EPT; ++j)
                 if (valid[j]) a.logits_out[(size_t)t * E + lane + 32 * j] = h[j];
@@ -190,6 +144,84 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
     }
 }
 
+template <typename TX, int EPT>
+__global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
+    constexpr int VEC = 16 / sizeof(TX);              // x elements per 16-byte load
+    constexpr int EW = EPT * 32;                      // expert slots per warp row
+    __shared__ float xs[kTok][kKc + 1];
+    __shared__ float wsm[kKc][EW];
+    __shared__ float part[kThreads / 32][EW];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * kTok;
+    const int d = a.d, E = a.E;
+
+    float acc[4][EPT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
+
+    const TX *x = static_cast<const TX *>(a.x);
+    for (int k0 = 0; k0 < d; k0 += kKc) {
+        // x chunk [32 tokens][32]: 16-byte vector loads (d % 8 == 0)
+        for (int v = tid; v < kTok * (kKc / VEC); v += kThreads) {
+            const int tt = v / (kKc / VEC), kv = (v % (kKc / VEC)) * VEC;
+            float vals[VEC];
+            const int t = t0 + tt;
+            if (t < a.T && k0 + kv < d) {
+                load_x_vec<TX>(x + (size_t)t * d + k0 + kv, vals);
+            } else {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) vals[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) xs[tt][kv + i] = vals[i];
+        }
+        // W_r chunk [32][E] (row-major [d, E], coalesced along E)
+        for (int v = tid; v < kKc * EW; v += kThreads) {
+            const int kk = v / EW, e = v % EW;
+            wsm[kk][e] = (k0 + kk < d && e < E) ? a.Wr[(size_t)(k0 + kk) * E + e] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kKc; ++kk) {
+            float xv[4], wv[EPT];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[i] = xs[warp * 4 + i][kk];
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) wv[j] = wsm[kk][lane + 32 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < EPT; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+
+    select_tokens<EPT>(a, acc, t0, /*add_bias=*/true, part);
+}
+
+// Selection for bf16 layers: logits [T, E] (offset already added) from the
+// tensor-core router, same per-warp selection as the fp32 path.
+template <int EPT>
+__global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ logits) {
+    __shared__ float part[kThreads / 32][EPT * 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = blockIdx.x * kTok;
+    float acc[4][EPT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + warp * 4 + i;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const int e = lane + 32 * j;
+            acc[i][j] = (t < a.T && e < a.E) ? logits[(size_t)t * a.E + e] : 0.f;
+        }
+    }
+    select_tokens<EPT>(a, acc, t0, /*add_bias=*/false, part);
+}
+
 template <typename TX>
 cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
     const int blocks = (a.T + kTok - 1) / kTok;
@@ -202,14 +234,23 @@ cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int router_blocks(int T, bool bf16) { return bf16 ? router_tc_blocks(T) : (T + kTok - 1) / kTok; }
+int router_blocks(int T) { return (T + kTok - 1) / kTok; }
 
-// bf16 layers take the tensor-core router (router_sm100.cu); fp32 layers this
-// FFMA kernel, which keeps every product in fp32.
+// bf16 layers: logits on the tensor cores (router_sm100.cu), then the
+// warp-per-token selection; fp32 layers: this FFMA kernel end to end, which
+// keeps every product in fp32.
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
-    if (bf16) return launch_router_tc(a, a.wsplit, a.status, st);
-    return launch_router_t<float>(a, st);
+    if (!bf16) return launch_router_t<float>(a, st);
+    float *logits = a.logits_out ? a.logits_out : a.logits_ws;
+    cudaError_t e = launch_router_logits_tc(a, logits, st);
+    if (e != cudaSuccess) return e;
+    const int blocks = (a.T + kTok - 1) / kTok;
+    if (a.E <= 32) router_select_kernel<1><<<blocks, kThreads, 0, st>>>(a, logits);
+    else if (a.E <= 64) router_select_kernel<2><<<blocks, kThreads, 0, st>>>(a, logits);
+    else if (a.E <= 128) router_select_kernel<4><<<blocks, kThreads, 0, st>>>(a, logits);
+    else router_select_kernel<8><<<blocks, kThreads, 0, st>>>(a, logits);
+    return cudaGetLastError();
 }
 
 }  // namespace moe
