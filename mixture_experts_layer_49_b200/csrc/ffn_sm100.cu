@@ -9,7 +9,8 @@
 // recommend (Router Optimization page, What Most Articles Miss 2; serving
 // tutorial, grouped GEMM remark).
 //
-// Kernel shape (one persistent CTA per SM, 320 threads, warp-specialised):
+// Kernel shape (1-CTA version; the CTA-pair version further down shares the
+// roles; one persistent CTA per SM, 320 threads, warp-specialised):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
 //               swizzle) per stage, 4 stages, mbarrier transaction counts
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
@@ -68,6 +69,8 @@ struct GemmParams {
     int ldo;
     int64_t shared_a_row;     // first A row of the shared group
     int64_t shared_out_row;   // first output row of the shared group
+    int tail_mode;            // 1-CTA kernel: 0 all rows; 1 only a group's last rows
+                              // when rows % 256 is in 1..128 (the rest runs in pair tiles)
     uint64_t timeout_ns;
 };
 
@@ -80,8 +83,9 @@ struct SmemTail {
     int abort_flag;
     int tile_start[kMaxGroups + 1];
     int mtiles[kMaxGroups];
-    int rows[kMaxGroups];
-    int row0[kMaxGroups];
+    int rows[kMaxGroups];     // rows this launch computes for the group
+    int row0[kMaxGroups];     // routed groups: first packed row (offsets[g] + start)
+    int start[kMaxGroups];    // first row of the group this launch computes
 };
 
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemTail);
@@ -138,11 +142,18 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // ---- tile table from the device-side offsets
     for (int g = tid; g < G; g += kThreads) {
         const bool sh = g >= p.E;
-        const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        int start = 0;
+        if (p.tail_mode) {
+            const int rem = rows % (2 * BM);
+            start = rows - rem;
+            rows = (rem > 0 && rem <= BM) ? rem : 0;
+        }
         const int n = sh ? p.N_shared : p.N_routed;
         const int mt = (rows + BM - 1) / BM;
         s.rows[g] = rows;
-        s.row0[g] = sh ? 0 : p.offsets[g];
+        s.start[g] = start;
+        s.row0[g] = sh ? 0 : p.offsets[g] + start;
         s.mtiles[g] = mt > 0 ? mt : 1;
         s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
     }
@@ -187,7 +198,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
                 const int nk = (K + BK - 1) / BK;
-                const int a_row = sh ? (int)p.shared_a_row + mt * BM : s.row0[g] + mt * BM;
+                const int a_row = sh ? (int)p.shared_a_row + s.start[g] + mt * BM : s.row0[g] + mt * BM;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = sh ? &tmBs : &tmB;
                 const CUtensorMap *mB2 = sh ? &tmBs2 : &tmB2;
@@ -252,7 +263,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const bool sh = g >= p.E;
             const int grow = mt * BM + r_in_tile;
             const bool valid = grow < s.rows[g];
-            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            const int64_t orow = sh ? p.shared_out_row + s.start[g] + grow : (int64_t)s.row0[g] + grow;
             // the row's gate is fetched before the accumulator wait, hiding its latency
             float gscale = 1.f;
             if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
@@ -323,6 +334,260 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
+
+// ============================================================================
+// CTA-pair version: one cluster of two CTAs computes a 256-row x 256-column
+// accumulator with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16).  Each
+// CTA loads its own 128 A rows and half of the B rows (SwiGLU: rank 0 the gate
+// rows, rank 1 the up rows), so a CTA moves 32 KiB per 64-deep K step instead
+// of 48 KiB, and six stages fit in shared memory.  Rank 0 issues the MMAs;
+// the full barriers live in rank 0 and collect both CTAs' TMA bytes; rank 0's
+// commits arrive on both CTAs' empty and accumulator-full barriers; both
+// CTAs' epilogue warps arrive on rank 0's accumulator-empty barriers.
+// Pair tiles cover a group's 256-row blocks and a last block of more than 128
+// rows; a last block of 1..128 rows runs in the 1-CTA kernel (tail mode), so
+// row padding never exceeds that of 128-row tiles.
+constexpr int P_STAGES = 6;
+constexpr uint32_t P_A_BYTES = BM * BK * 2;         // 16 KiB: this CTA's 128 A rows
+constexpr uint32_t P_B_BYTES = 128 * BK * 2;        // 16 KiB: this CTA's half of B
+constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int PM = 2 * BM;                          // rows per pair tile
+constexpr uint32_t kIdescPair = make_idesc_bf16(PM, BNB);
+
+struct PairTail {
+    uint64_t full[P_STAGES];     // rank 0's are used
+    uint64_t empty[P_STAGES];
+    uint64_t accf[2];
+    uint64_t acce[2];            // rank 0's are used: 8 warps x 2 CTAs
+    uint32_t tmem_base;
+    int abort_flag;
+    int tile_start[kMaxGroups + 1];
+    int mtiles[kMaxGroups];
+    int rows[kMaxGroups];
+    int row0[kMaxGroups];
+};
+
+constexpr size_t kPairSmemBytes = 1024 + P_STAGES * P_STAGE_BYTES + sizeof(PairTail);
+
+__device__ __forceinline__ void decode_pair(const PairTail &s, int G, int tile, int &g, int &mt, int &nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - s.tile_start[g];
+    mt = local % s.mtiles[g];
+    nt = local / s.mtiles[g];
+}
+
+__device__ __forceinline__ bool aborted_pair(const PairTail &s) {
+    return *reinterpret_cast<const volatile int *>(&s.abort_flag) != 0;
+}
+__device__ __forceinline__ void fail_pair(PairTail &s, const GemmParams &p, int where) {
+    record_error(p.status, MOE_ERR_TIMEOUT, where);
+    *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                     const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
+                     const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    PairTail &s = *reinterpret_cast<PairTail *>(smem + P_STAGES * P_STAGE_BYTES);
+    const uint32_t smA = base;                           // P_STAGES x 16 KiB
+    const uint32_t smB = base + P_STAGES * P_A_BYTES;    // P_STAGES x 16 KiB
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = (int)cluster_id_x(), npairs = (int)ncluster_x();
+    constexpr int BNO = (MODE == GM_SWIGLU) ? 128 : 256;
+    const int G = p.E + (p.has_shared ? 1 : 0);
+
+    for (int g = tid; g < G; g += kThreads) {
+        const bool sh = g >= p.E;
+        const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        const int n = sh ? p.N_shared : p.N_routed;
+        const int mt = rows / PM + ((rows % PM) > BM ? 1 : 0);
+        s.rows[g] = rows;
+        s.row0[g] = sh ? 0 : p.offsets[g];
+        s.mtiles[g] = mt > 0 ? mt : 1;
+        s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
+    }
+    if (tid == 0) {
+        s.tile_start[0] = 0;
+        s.abort_flag = 0;
+        for (int i = 0; i < P_STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 16); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            int v = g < G ? s.tile_start[g + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (g < G) s.tile_start[g + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(&s.tmem_base), TMEM_COLS);   // warp 1 of both CTAs
+    tc_fence_before();
+    cluster_sync();                                  // barriers of both CTAs initialised
+    tc_fence_after();
+    const int total = s.tile_start[G];
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == 0) {
+        // ================= TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+                int g, mt, nt;
+                decode_pair(s, G, tile, g, mt, nt);
+                const bool sh = g >= p.E;
+                const int K = sh ? p.K_shared : p.K_routed;
+                const int nk = (K + BK - 1) / BK;
+                const int a_row = (sh ? (int)p.shared_a_row : s.row0[g]) + mt * PM + (int)rank * BM;
+                const CUtensorMap *mA = sh ? &tmAs : &tmA;
+                const CUtensorMap *mB = (MODE == GM_SWIGLU && rank == 1) ? (sh ? &tmBs2 : &tmB2) : (sh ? &tmBs : &tmB);
+                const int b_row = (MODE == GM_SWIGLU) ? nt * 128 : nt * BNB + (int)rank * 128;
+                const int e = sh ? 0 : g;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 21); break; }
+                    const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * P_STAGE_BYTES);
+                    tma_load_2d_pair(smA + stage * P_A_BYTES, mA, fb, kb * BK, a_row);
+                    tma_load_3d_pair(smB + stage * P_B_BYTES, mB, fb, kb * BK, b_row, e);
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer (rank 0 only)
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int ab = 0;
+            uint32_t aphase = 0;
+            for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+                int g, mt, nt;
+                decode_pair(s, G, tile, g, mt, nt);
+                const int K = g >= p.E ? p.K_shared : p.K_routed;
+                const int nk = (K + BK - 1) / BK;
+                if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 22); break; }
+                tc_fence_after();
+                const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) { fail_pair(s, p, 23); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smA + stage * P_A_BYTES, b0 = smB + stage * P_B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | k) ? 1u : 0u);
+                    mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit_pair(smem_u32(&s.accf[ab]), (uint16_t)0x3);
+                if (++ab == 2) { ab = 0; aphase ^= 1u; }
+            }
+        }
+    } else {
+        // ================= epilogue (both CTAs), warps 2..9 as in the 1-CTA kernel
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int r_in_tile = q * 32 + lane;
+        int ab = 0;
+        uint32_t aphase = 0;
+        for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+            int g, mt, nt;
+            decode_pair(s, G, tile, g, mt, nt);
+            const bool sh = g >= p.E;
+            const int grow = mt * PM + (int)rank * BM + r_in_tile;
+            const bool valid = grow < s.rows[g];
+            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            float gscale = 1.f;
+            if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(smem_u32(&s.accf[ab]), aphase, p.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { if (lane == 0) fail_pair(s, p, 24); break; }
+            __syncwarp();
+            tc_fence_after();
+            const int N = sh ? p.N_shared : p.N_routed;
+            const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
+            __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
+            if (MODE == GM_SWIGLU) {
+#pragma unroll 1
+                for (int c = half * 2; c < half * 2 + 2; ++c) {
+                    float gv[32], uv[32];
+                    tmem_ld32(taddr + c * 32, gv);
+                    tmem_ld32(taddr + 128 + c * 32, uv);
+                    const int col0 = nt * 128 + c * 32;
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) h[i] = silu(gv[v * 8 + i]) * uv[v * 8 + i];
+                            if (col0 + v * 8 < N) store8(orow_ptr + col0 + v * 8, h);
+                        }
+                    }
+                }
+            } else {
+                const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+#pragma unroll 1
+                for (int c = half * 4; c < half * 4 + 4; ++c) {
+                    float acc[32];
+                    tmem_ld32(taddr + c * 32, acc);
+                    const int col0 = nt * BNB + c * 32;
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int cb = col0 + v * 8;
+                            if (cb >= N) continue;
+                            float h[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float t = acc[v * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
+                                h[i] = (MODE == GM_GELU) ? gelu_erf(t) : gscale * t;
+                            }
+                            store8(orow_ptr + cb, h);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
+            if (++ab == 2) { ab = 0; aphase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                  // no CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -368,8 +633,40 @@ cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUten
     return cudaGetLastError();
 }
 
+template <int MODE>
+cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B,
+                             const CUtensorMap &B2, const CUtensorMap &Bs, const CUtensorMap &Bs2,
+                             const GemmParams &p, int num_sms, cudaStream_t st) {
+    static int grid = 0;
+    if (grid == 0) {
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kPairSmemBytes);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kPairSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_grouped_gemm_pair<MODE>, &cfg);
+        if (e != cudaSuccess || nclusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        grid = 2 * nclusters;
+    }
+    tc_grouped_gemm_pair<MODE><<<grid, kThreads, kPairSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
+// Each GEMM runs as two launches on the stream: the CTA-pair kernel over the
+// 256-row blocks of every group (and a last block of > 128 rows), then the
+// 1-CTA kernel over the remaining last blocks of 1..128 rows.
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
     const bool swiglu = a.act == MOE_ACT_SWIGLU;
@@ -414,8 +711,26 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p1.shared_a_row = 0;
     p1.shared_out_row = a.shared_base;
     p1.timeout_ns = timeout_ns;
-    cudaError_t err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
-                             : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
+    // pair kernel: B boxes of 128 rows (each CTA loads half of the tile's B rows)
+    CUtensorMap P1, P1u, P1s, P1su;
+    if (swiglu) {
+        P1 = B1; P1u = B1u; P1s = B1s; P1su = B1su;
+    } else {
+        if (!make_map(&P1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, 128)) return cudaErrorInvalidValue;
+        P1u = P1;
+        if (has_sh) {
+            if (!make_map(&P1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, 128)) return cudaErrorInvalidValue;
+        } else {
+            P1s = P1;
+        }
+        P1su = P1s;
+    }
+    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st)
+                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st);
+    if (err != cudaSuccess) return err;
+    p1.tail_mode = 1;
+    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
+                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
     if (err != cudaSuccess) return err;
 
     // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
@@ -442,6 +757,16 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p2.shared_a_row = a.shared_base;
     p2.shared_out_row = a.shared_base;
     p2.timeout_ns = timeout_ns;
+    CUtensorMap P2, P2s;
+    if (!make_map(&P2, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, 128)) return cudaErrorInvalidValue;
+    if (has_sh) {
+        if (!make_map(&P2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, 128)) return cudaErrorInvalidValue;
+    } else {
+        P2s = P2;
+    }
+    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, p2, grid, st);
+    if (err != cudaSuccess) return err;
+    p2.tail_mode = 1;
     return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st);
 }
 
