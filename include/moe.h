@@ -203,6 +203,25 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        double *loss, float *logits_out, int32_t *n_dropped,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Auxiliary-loss-free bias update, to run after a training step on the
+ * counts that step's routing produced ("Fine-Tuning Mixture of Experts (MoE)
+ * Models: Router Optimization Techniques", How It Works 2, and its router
+ * module): with L_target = T * top_k / E,
+ *   sel_bias[e] <- sel_bias[e] - gamma * sign(counts[e] - L_target)
+ * computed in double and stored as fp32 (sign(0) = 0).  counts [E] int32,
+ * sel_bias [E] fp32 in/out (the selection bias moe_router_topk takes).     */
+MOE_API moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float *sel_bias,
+                                   float gamma, moe_stream_t stream);
+
+/* Routing health: out[0] = -sum_e P_e log P_e, the Shannon entropy of the
+ * mean routing distribution (Router Optimization page, Best Practices 6);
+ * out[1] = max_e counts / min_e counts (+inf when an expert got nothing) and
+ * out[2] = max_e counts / (T * top_k) ("Fine-tuning and serving MoE models",
+ * Utilization is a first-class metric).  counts [E] int32, P [E] fp32 (from
+ * moe_balance_stats), out [3] fp64, all device pointers.                    */
+MOE_API moe_status moe_routing_health(const moe_config *cfg, const int32_t *counts, const float *P,
+                                      double *out, moe_stream_t stream);
+
 /* moe_permute for callers that cannot allocate device memory.  The paper has
  * no counterpart: this entry point exists for integration only.
  * Same computation, arguments and outputs as moe_permute, but no workspace:

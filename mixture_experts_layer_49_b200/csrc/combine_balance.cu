@@ -129,7 +129,63 @@ __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
     if (threadIdx.x == 0) *a.loss = (double)a.E * red[0];
 }
 
+// Auxiliary-loss-free bias update ("Fine-Tuning Mixture of Experts (MoE)
+// Models: Router Optimization Techniques", How It Works 2, and its router
+// module): b_e <- b_e - gamma * sign(count_e - T k / E), in double.
+__global__ void bias_update_kernel(const int32_t *counts, float *bias, double gamma, int T, int k, int E) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const double err = (double)counts[e] - (double)T * (double)k / (double)E;
+    const double sgn = err > 0.0 ? 1.0 : (err < 0.0 ? -1.0 : 0.0);
+    bias[e] = (float)((double)bias[e] - gamma * sgn);
+}
+
+// Routing health: entropy -sum P log P of the mean routing distribution
+// (Router Optimization page, Best Practices 6), max/min count ratio and the
+// largest load share ("Fine-tuning and serving MoE models", Utilization is a
+// first-class metric).  One CTA; fixed-order tree sums in double.
+__global__ void __launch_bounds__(256) routing_health_kernel(const int32_t *counts, const float *P, double *out,
+                                                             int T, int k, int E) {
+    __shared__ double hs[256];
+    __shared__ int mx[256], mn[256];
+    const int e = threadIdx.x;
+    double h = 0.0;
+    int cmax = -1, cmin = 0x7fffffff;
+    if (e < E) {
+        const double p = (double)P[e];
+        if (p > 0.0) h = -p * log(p);
+        cmax = cmin = counts[e];
+    }
+    hs[e] = h; mx[e] = cmax; mn[e] = cmin;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (e < o) {
+            hs[e] += hs[e + o];
+            mx[e] = max(mx[e], mx[e + o]);
+            mn[e] = min(mn[e], mn[e + o]);
+        }
+        __syncthreads();
+    }
+    if (e == 0) {
+        out[0] = hs[0];
+        out[1] = mn[0] > 0 ? (double)mx[0] / (double)mn[0] : (double)INFINITY;
+        out[2] = (double)mx[0] / ((double)T * (double)k);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_bias_update(const int32_t *counts, float *bias, double gamma, int T, int k, int E,
+                               cudaStream_t st) {
+    bias_update_kernel<<<(E + 255) / 256, 256, 0, st>>>(counts, bias, gamma, T, k, E);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_routing_health(const int32_t *counts, const float *P, double *out, int T, int k, int E,
+                                  cudaStream_t st) {
+    routing_health_kernel<<<1, 256, 0, st>>>(counts, P, out, T, k, E);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;

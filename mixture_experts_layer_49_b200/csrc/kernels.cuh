@@ -23,8 +23,9 @@ struct RouterArgs {
     float *logits_ws;            // bf16 layers: [T, E] scratch for the logits (if no logits_out)
     int32_t *status;             // workspace status word
 };
-// Rows of the per-block score sums (32 tokens per block).
-int router_blocks(int T);
+// Rows of the per-block score sums: 128 tokens per block for bf16 layers,
+// 32 for fp32 layers.
+int router_blocks(int T, bool bf16);
 size_t router_split_bytes(int d, int E);
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStream_t st);
@@ -88,6 +89,11 @@ struct BalanceArgs {
     int T, E, k, nblk;
 };
 cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st);
+
+cudaError_t launch_bias_update(const int32_t *counts, float *bias, double gamma, int T, int k, int E,
+                               cudaStream_t st);
+cudaError_t launch_routing_health(const int32_t *counts, const float *P, double *out, int T, int k, int E,
+                                  cudaStream_t st);
 
 // Host-side helpers shared by the entry points (moe_api.cu).
 moe_status validate_config(const moe_config *cfg);        // sets the error detail

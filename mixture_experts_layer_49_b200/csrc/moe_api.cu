@@ -38,7 +38,7 @@ Layout layout(const moe_config *c) {
     const size_t rows = (size_t)perm_rows(c);
     const size_t hF = (size_t)(c->d_ff > c->d_ff_shared ? c->d_ff : c->d_ff_shared);
     const bool bf16 = c->dtype == MOE_BF16;
-    const size_t nblk = (size_t)moe::router_blocks(c->T);
+    const size_t nblk = (size_t)moe::router_blocks(c->T, bf16);
     const size_t nch = (size_t)moe::dispatch_chunks(c->T);
     size_t o = sizeof(moe::WsHeader);
     L.router_w = o;   o = align256(o + (bf16 ? moe::router_split_bytes(c->d_model, c->E) : 0));
@@ -167,7 +167,7 @@ int32_t moe_capacity(const moe_config *cfg) {
 
 int32_t moe_router_blocks(const moe_config *cfg) {
     if (check_cfg(cfg) != MOE_OK) return 0;
-    return moe::router_blocks(cfg->T);
+    return moe::router_blocks(cfg->T, cfg->dtype == MOE_BF16);
 }
 
 int64_t moe_perm_rows(const moe_config *cfg) {
@@ -265,7 +265,8 @@ moe_status moe_balance_stats(const moe_config *cfg, const int32_t *counts, const
     NEED(counts); NEED(f); NEED(P); NEED(loss);
     if (cfg->T > 0) NEED(psum);
     ALIGNED(counts, 4); ALIGNED(psum, 4); ALIGNED(f, 4); ALIGNED(P, 4); ALIGNED(loss, 8);
-    moe::BalanceArgs a{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
+    moe::BalanceArgs a{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k,
+                       moe::router_blocks(cfg->T, cfg->dtype == MOE_BF16)};
     cudaError_t e = moe::launch_balance(a, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "balance");
 }
@@ -323,9 +324,32 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
 
-    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T)};
+    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T, bf16)};
     if ((e = moe::launch_balance(ba, st)) != cudaSuccess) return cuda_fail(e, "balance");
     return MOE_OK;
+}
+
+moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float *sel_bias, float gamma,
+                           moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(counts); NEED(sel_bias);
+    ALIGNED(counts, 4); ALIGNED(sel_bias, 4);
+    if (!isfinite(gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma not finite%s");
+    cudaError_t e = moe::launch_bias_update(counts, sel_bias, (double)gamma, cfg->T, cfg->top_k, cfg->E,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "bias_update");
+}
+
+moe_status moe_routing_health(const moe_config *cfg, const int32_t *counts, const float *P, double *out,
+                              moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(counts); NEED(P); NEED(out);
+    ALIGNED(counts, 4); ALIGNED(P, 4); ALIGNED(out, 8);
+    cudaError_t e = moe::launch_routing_health(counts, P, out, cfg->T, cfg->top_k, cfg->E,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "routing_health");
 }
 
 moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out) {

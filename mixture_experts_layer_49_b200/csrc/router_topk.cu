@@ -43,19 +43,15 @@ __device__ __forceinline__ void load_x_vec<float>(const float *src, float *dst) 
     dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
 }
 
-// Scores, top-k, gates and the block's score sums for the 32 tokens starting
-// at t0 (warp w holds tokens t0 + 4w .. t0 + 4w + 3; acc[i][j] is the logit of
-// token 4w + i for expert lane + 32 j).  add_bias: add logit_bias to acc first
-// (the tensor-core path has added it already).  part: shared [8][EPT*32].
+// Scores, top-k and gates for the 32 tokens starting at t0 (warp w holds
+// tokens t0 + 4w .. t0 + 4w + 3; acc[i][j] is the logit of token 4w + i for
+// expert lane + 32 j), adding each token's normalised scores into psum_acc.
+// add_bias: add logit_bias to acc first (the tensor-core path has added it).
 template <int EPT>
 __device__ __forceinline__ void select_tokens(const RouterArgs &a, float (&acc)[4][EPT], int t0, bool add_bias,
-                                              float (*part)[EPT * 32]) {
+                                              float (&psum_acc)[EPT]) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, k = a.k;
-    float psum_acc[EPT];
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
-
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int t = t0 + warp * 4 + i;
@@ -132,15 +128,20 @@ __device__ __forceinline__ void select_tokens(const RouterArgs &a, float (&acc)[
             a.gate[(size_t)t * k + lane] = g;
         }
     }
-    // per-CTA partial sums of the normalised scores, fixed order
+}
+
+// The CTA's row of the per-block score sums: warp partials added in warp order.
+template <int EPT>
+__device__ __forceinline__ void write_psum(const RouterArgs &a, float (*part)[EPT * 32], const float (&psum_acc)[EPT]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #pragma unroll
     for (int j = 0; j < EPT; ++j) part[warp][lane + 32 * j] = psum_acc[j];
     __syncthreads();
-    for (int e = tid; e < E; e += kThreads) {
+    for (int e = tid; e < a.E; e += kThreads) {
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) s += part[w][e];
-        a.psum[(size_t)blockIdx.x * E + e] = s;
+        a.psum[(size_t)blockIdx.x * a.E + e] = s;
     }
 }
 
@@ -199,27 +200,41 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
         __syncthreads();
     }
 
-    select_tokens<EPT>(a, acc, t0, /*add_bias=*/true, part);
+    float psum_acc[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
+    select_tokens<EPT>(a, acc, t0, /*add_bias=*/true, psum_acc);
+    write_psum<EPT>(a, part, psum_acc);
 }
 
 // Selection for bf16 layers: logits [T, E] (offset already added) from the
-// tensor-core router, same per-warp selection as the fp32 path.
+// tensor-core router, same per-warp selection as the fp32 path; one CTA takes
+// 128 tokens (four groups of 32), so the score sums have T/128 rows.
+constexpr int kSelTok = 128;
+
 template <int EPT>
 __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ logits) {
     __shared__ float part[kThreads / 32][EPT * 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t0 = blockIdx.x * kTok;
-    float acc[4][EPT];
+    float psum_acc[EPT];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + warp * 4 + i;
+    for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
+    for (int grp = 0; grp < kSelTok / kTok; ++grp) {
+        const int t0 = blockIdx.x * kSelTok + grp * kTok;
+        if (t0 >= a.T) break;
+        float acc[4][EPT];
 #pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            const int e = lane + 32 * j;
-            acc[i][j] = (t < a.T && e < a.E) ? logits[(size_t)t * a.E + e] : 0.f;
+        for (int i = 0; i < 4; ++i) {
+            const int t = t0 + warp * 4 + i;
+#pragma unroll
+            for (int j = 0; j < EPT; ++j) {
+                const int e = lane + 32 * j;
+                acc[i][j] = (t < a.T && e < a.E) ? logits[(size_t)t * a.E + e] : 0.f;
+            }
         }
+        select_tokens<EPT>(a, acc, t0, /*add_bias=*/false, psum_acc);
     }
-    select_tokens<EPT>(a, acc, t0, /*add_bias=*/false, part);
+    write_psum<EPT>(a, part, psum_acc);
 }
 
 template <typename TX>
@@ -234,7 +249,7 @@ cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int router_blocks(int T) { return (T + kTok - 1) / kTok; }
+int router_blocks(int T, bool bf16) { return bf16 ? (T + kSelTok - 1) / kSelTok : (T + kTok - 1) / kTok; }
 
 // bf16 layers: logits on the tensor cores (router_sm100.cu), then the
 // warp-per-token selection; fp32 layers: this FFMA kernel end to end, which
@@ -245,7 +260,7 @@ cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
     float *logits = a.logits_out ? a.logits_out : a.logits_ws;
     cudaError_t e = launch_router_logits_tc(a, logits, st);
     if (e != cudaSuccess) return e;
-    const int blocks = (a.T + kTok - 1) / kTok;
+    const int blocks = (a.T + kSelTok - 1) / kSelTok;
     if (a.E <= 32) router_select_kernel<1><<<blocks, kThreads, 0, st>>>(a, logits);
     else if (a.E <= 64) router_select_kernel<2><<<blocks, kThreads, 0, st>>>(a, logits);
     else if (a.E <= 128) router_select_kernel<4><<<blocks, kThreads, 0, st>>>(a, logits);

@@ -27,7 +27,8 @@ MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_rows",
            "moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
-           "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc")
+           "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
+           "moe_bias_update", "moe_routing_health")
 
 
 class MoEError(RuntimeError):
@@ -80,6 +81,10 @@ def lib():
         L.moe_balance_stats.argtypes = [P(MoeConfig)] + [c_vp] * 6
         L.moe_forward.argtypes = [P(MoeConfig)] + [c_vp] * 22 + [ctypes.c_size_t, c_vp]
         L.moe_get_device_status.argtypes = [c_vp, c_vp, P(c_i32)]
+        L.moe_bias_update.restype = ctypes.c_int
+        L.moe_bias_update.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_float, c_vp]
+        L.moe_routing_health.restype = ctypes.c_int
+        L.moe_routing_health.argtypes = [P(MoeConfig), c_vp, c_vp, c_vp, c_vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_permute_noalloc.argtypes = [P(MoeConfig)] + [c_vp] * 11 + [c_vp]
         _lib = L
@@ -211,6 +216,16 @@ def moe_forward(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh
                              _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g), _p(Wsh_u), _p(Wsh_d), _p(y),
                              _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss), _p(logits_out),
                              _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_bias_update(cfg, counts, sel_bias, gamma, stream=None):
+    _check(lib().moe_bias_update(ctypes.byref(cfg), _p(counts), _p(sel_bias), float(gamma), _stream(stream)),
+           "moe_bias_update")
+
+
+def moe_routing_health(cfg, counts, P, out, stream=None):
+    _check(lib().moe_routing_health(ctypes.byref(cfg), _p(counts), _p(P), _p(out), _stream(stream)),
+           "moe_routing_health")
 
 
 def moe_get_device_status(ws, stream=None) -> int:

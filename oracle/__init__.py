@@ -46,7 +46,8 @@ def _load():
         lib.oracle_capacity.restype = ctypes.c_int32
         lib.oracle_capacity.argtypes = [ctypes.c_double, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         for name in ("oracle_route", "oracle_dispatch", "oracle_balance",
-                     "oracle_expert_apply", "oracle_layer_tokens"):
+                     "oracle_expert_apply", "oracle_layer_tokens", "oracle_bias_update",
+                     "oracle_routing_health"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -206,6 +207,25 @@ def forward(dims, x, Wr, weights, logit_bias=None, sel_bias=None, tokens=None):
     out["y"] = y
     out["tokens"] = tok
     return out
+
+
+def bias_update(dims, counts, bias, gamma):
+    """b_e - gamma * sign(count_e - T k / E), returned as a new float32 array."""
+    lib = _load()
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    b = np.array(bias, dtype=np.float32, copy=True)
+    lib.oracle_bias_update(ctypes.byref(dims), _ptr(counts), ctypes.c_double(gamma), _ptr(b))
+    return b
+
+
+def routing_health(dims, counts, P):
+    """dict(entropy = -sum P log P, ratio = max/min count, max_share)."""
+    lib = _load()
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    P = np.ascontiguousarray(P, dtype=np.float64)
+    out = np.empty(3, np.float64)
+    lib.oracle_routing_health(ctypes.byref(dims), _ptr(counts), _ptr(P), _ptr(out))
+    return dict(entropy=float(out[0]), ratio=float(out[1]), max_share=float(out[2]))
 
 
 def bf16_bits_to_f64(a):

@@ -406,3 +406,41 @@ int oracle_layer_tokens(const oracle_dims *dm, int64_t ntok, const int32_t *toke
     parallel_for(ntok, dm->nthreads, layer_range, &c);
     return 0;
 }
+
+/* ---- auxiliary-loss-free bias update -------------------------------------
+ * [RO] How It Works 2 and the dynamic-bias router module, step 5: after a
+ * step, with L_e the assignments expert e received and L_target = T k / E,
+ *   b_e <- b_e - gamma * sign(L_e - L_target)
+ * (overloaded experts lose gamma, underloaded ones gain it, exactly loaded
+ * ones keep their bias).  Arithmetic in double, result stored as float.     */
+int oracle_bias_update(const oracle_dims *dm, const int32_t *counts, double gamma, float *bias)
+{
+    const double target = (double)dm->T * (double)dm->k / (double)dm->E;
+    for (int e = 0; e < dm->E; ++e) {
+        const double err = (double)counts[e] - target;
+        const double sgn = err > 0.0 ? 1.0 : (err < 0.0 ? -1.0 : 0.0);
+        bias[e] = (float)((double)bias[e] - gamma * sgn);
+    }
+    return 0;
+}
+
+/* ---- routing health ------------------------------------------------------
+ * [RO] Best Practices 6: Shannon entropy H = -sum_e P_e log P_e of the layer's
+ * mean routing distribution P (terms with P_e = 0 add 0); [IS] "Utilization
+ * is a first-class metric": the max/min ratio of the per-expert counts
+ * (HUGE_VAL when some expert received nothing), and the largest share
+ * max_e counts_e / (T k).  out = {H, ratio, max share}.                     */
+int oracle_routing_health(const oracle_dims *dm, const int32_t *counts, const double *P, double *out)
+{
+    double H = 0.0;
+    int32_t mx = counts[0], mn = counts[0];
+    for (int e = 0; e < dm->E; ++e) {
+        if (P[e] > 0.0) H -= P[e] * log(P[e]);
+        if (counts[e] > mx) mx = counts[e];
+        if (counts[e] < mn) mn = counts[e];
+    }
+    out[0] = H;
+    out[1] = mn > 0 ? (double)mx / (double)mn : HUGE_VAL;
+    out[2] = (double)mx / ((double)dm->T * (double)dm->k);
+    return 0;
+}

@@ -398,3 +398,59 @@ def test_expert_apply_matches_layer_sum():
     np.testing.assert_allclose(y, out["y"], rtol=1e-12, atol=1e-14)
     with pytest.raises(ValueError):
         oracle.expert_apply(dims, x, w, [0], [E + 1])
+
+
+# --------------------------------------------------------------------------
+# auxiliary-loss-free bias update and routing health
+# --------------------------------------------------------------------------
+def test_bias_update_follows_the_sign_rule():
+    fx = facts()["bias_rule"]
+    gamma = fx["gamma"]
+    T, k, E = 12, 2, 4                      # target load T k / E = 6
+    dims = oracle.make_dims(T, 8, E, 8, k, x_dtype="f32")
+    counts = np.array([9, 6, 3, 6], np.int32)
+    b0 = np.array([0.5, -0.25, 0.0, 1.0], np.float32)
+    b1 = oracle.bias_update(dims, counts, b0, gamma)
+    # overloaded expert 0 loses gamma, underloaded expert 2 gains it, exactly
+    # loaded experts 1 and 3 keep their bias
+    np.testing.assert_array_equal(b1, np.array([0.5 - gamma, -0.25, 0.0 + gamma, 1.0], np.float32))
+    np.testing.assert_array_equal(b0, [0.5, -0.25, 0.0, 1.0])      # input untouched
+
+
+def test_bias_update_balances_a_skewed_router():
+    # repeated updates on a fixed, skewed router move load off the hot expert
+    rng = np.random.default_rng(21)
+    T, d, E, k = 256, 16, 8, 2
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    Wr = (rng.standard_normal((d, E)) * 0.3).astype(np.float32)
+    lb = np.array([2.0, 1.0] + [0.0] * (E - 2), np.float32)
+    dims = oracle.make_dims(T, d, E, 8, k, x_dtype="f32", score="sigmoid")
+    b = np.zeros(E, np.float32)
+    first = None
+    for _ in range(400):
+        r = oracle.route(dims, x, Wr, lb, b, want_pnorm=False)
+        counts = oracle.dispatch(dims, r["idx"])["counts"]
+        if first is None:
+            first = counts.max() / (T * k / E)
+        b = oracle.bias_update(dims, counts, b, 0.01)
+    last = counts.max() / (T * k / E)
+    assert first > 2.0 and last < first / 1.5
+
+
+def test_routing_health_closed_forms():
+    E = facts()["entropy_max_128"]["num_experts"]
+    T, k = 256, 2
+    dims = oracle.make_dims(T, 8, E, 8, k, x_dtype="f32")
+    uniform = oracle.routing_health(dims, np.full(E, T * k // E, np.int32), np.full(E, 1.0 / E))
+    assert abs(uniform["entropy"] - np.log(E)) < 1e-12
+    assert round(uniform["entropy"], facts()["entropy_max_128"]["printed_digits"]) == facts()["entropy_max_128"]["value"]
+    assert uniform["ratio"] == 1.0 and abs(uniform["max_share"] - 1.0 / E) < 1e-15
+    onehot_P = np.zeros(E); onehot_P[3] = 1.0
+    counts = np.zeros(E, np.int32); counts[3] = T * k
+    collapsed = oracle.routing_health(dims, counts, onehot_P)
+    assert collapsed["entropy"] == 0.0 and collapsed["ratio"] == float("inf") and collapsed["max_share"] == 1.0
+    # a 2:1 split of the load between two halves of the experts
+    c = np.array([2] * (E // 2) + [1] * (E // 2), np.int32) * 4
+    h = oracle.routing_health(dims, c, c / c.sum())
+    assert h["ratio"] == 2.0
+    assert abs(h["entropy"] - stats.entropy(c / c.sum())) < 1e-12   # scipy's Shannon entropy
