@@ -90,36 +90,45 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     }
 }
 
-// 1024 threads: quarter g (= threadIdx.x / 256) of expert e (= threadIdx.x %
-// 256) adds the block rows b = g, g+4, ... in order; the four quarter sums
-// are then added in quarter order, and the loss terms f_e P_e in a fixed
-// tree.  Everything in double; the result does not depend on scheduling.
+// 1024 threads: with EP = E rounded up to a power of two, thread (g, e)
+// (g = threadIdx.x / EP) adds the block rows b = g, g + 1024/EP, ... in
+// order; the 1024/EP partial sums of an expert are then added in g order and
+// the loss terms f_e P_e in a fixed tree.  Everything in double; the result
+// does not depend on scheduling.
 __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
-    __shared__ double quarter[4][256];
+    __shared__ double partial[1024];
     __shared__ double red[256];
-    const int e = threadIdx.x & 255, g = threadIdx.x >> 8;
+    int EP = 1;
+    while (EP < a.E) EP <<= 1;
+    const int groups = 1024 / EP;
+    const int e = threadIdx.x % EP, g = threadIdx.x / EP;
     double s = 0.0;
     if (e < a.E) {
         int b = g;
-        for (; b + 12 < a.nblk; b += 16) {       // four independent loads in flight
-            const float v0 = a.psum[(size_t)b * a.E + e], v1 = a.psum[(size_t)(b + 4) * a.E + e];
-            const float v2 = a.psum[(size_t)(b + 8) * a.E + e], v3 = a.psum[(size_t)(b + 12) * a.E + e];
+        for (; b + 3 * groups < a.nblk; b += 4 * groups) {     // four independent loads in flight
+            const float v0 = a.psum[(size_t)b * a.E + e];
+            const float v1 = a.psum[(size_t)(b + groups) * a.E + e];
+            const float v2 = a.psum[(size_t)(b + 2 * groups) * a.E + e];
+            const float v3 = a.psum[(size_t)(b + 3 * groups) * a.E + e];
             s += (double)v0; s += (double)v1; s += (double)v2; s += (double)v3;
         }
-        for (; b < a.nblk; b += 4) s += (double)a.psum[(size_t)b * a.E + e];
+        for (; b < a.nblk; b += groups) s += (double)a.psum[(size_t)b * a.E + e];
     }
-    quarter[g][e] = s;
+    partial[threadIdx.x] = s;
     __syncthreads();
-    if (g == 0) {
+    if (threadIdx.x < 256) {
         double contrib = 0.0;
-        if (e < a.E) {
-            const double P = (((quarter[0][e] + quarter[1][e]) + quarter[2][e]) + quarter[3][e]) / (double)a.T;
-            const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
-            a.f[e] = (float)f;
-            a.P[e] = (float)P;
+        const int ee = threadIdx.x;
+        if (ee < a.E) {
+            double tot = 0.0;
+            for (int gg = 0; gg < groups; ++gg) tot += partial[gg * EP + ee];
+            const double P = tot / (double)a.T;
+            const double f = (double)a.counts[ee] / ((double)a.T * (double)a.k);
+            a.f[ee] = (float)f;
+            a.P[ee] = (float)P;
             contrib = f * P;
         }
-        red[e] = contrib;
+        red[ee] = contrib;
     }
     __syncthreads();
     for (int o = 128; o > 0; o >>= 1) {

@@ -23,7 +23,7 @@ struct RouterArgs {
     float *logits_ws;            // bf16 layers: [T, E] scratch for the logits (if no logits_out)
     int32_t *status;             // workspace status word
 };
-// Rows of the per-block score sums: 128 tokens per block for bf16 layers,
+// Rows of the per-block score sums: 64 tokens per block for bf16 layers,
 // 32 for fp32 layers.
 int router_blocks(int T, bool bf16);
 size_t router_split_bytes(int d, int E);

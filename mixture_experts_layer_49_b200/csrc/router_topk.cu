@@ -34,6 +34,12 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Order-preserving map of a finite fp32 key to an unsigned integer.
+__device__ __forceinline__ unsigned ordered_key(float f) {
+    const unsigned u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 template <typename TX>
 __device__ __forceinline__ void load_x_vec(const TX *src, float *dst);
 
@@ -95,37 +101,42 @@ __device__ __forceinline__ void select_tokens(const RouterArgs &a, float (&acc)[
             for (int j = 0; j < EPT; ++j)
                 if (valid[j]) a.logits_out[(size_t)t * E + lane + 32 * j] = h[j];
         }
-        // k rounds of warp arg-max on (key desc, expert id asc)
+        // k rounds of warp arg-max on (key desc, expert id asc): each lane
+        // offers its best untaken expert; redux.sync picks the largest key
+        // (as an order-preserving integer), then the lowest expert id among
+        // the lanes holding it.  The owner lane records the slot.
         unsigned taken = 0;
-        int my_e = -1;
-        float my_sc = 0.f;
+        int slot[EPT];
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) slot[j] = -1;
         for (int r = 0; r < k; ++r) {
-            float bk = -INFINITY, bs = 0.f;
-            int be = 0x7fffffff;
+            float bk = 0.f;
+            int bj = -1;
 #pragma unroll
-            for (int j = 0; j < EPT; ++j) {
-                const int e = lane + 32 * j;
-                if (valid[j] && !(taken & (1u << j)) && (key[j] > bk || (key[j] == bk && e < be))) {
-                    bk = key[j]; be = e; bs = sc[j];
-                }
-            }
+            for (int j = 0; j < EPT; ++j)
+                if (valid[j] && !(taken & (1u << j)) && (bj < 0 || key[j] > bk)) { bk = key[j]; bj = j; }
+            const unsigned offer = (bj >= 0 && bk == bk) ? ordered_key(bk) : 0u;
+            const unsigned kmax = __reduce_max_sync(0xffffffffu, offer);
+            const unsigned cand = (bj >= 0 && offer == kmax) ? (unsigned)(lane + 32 * bj) : 0xffffffffu;
+            const unsigned be = __reduce_min_sync(0xffffffffu, cand);
+            if (be < (unsigned)E && (int)(be & 31u) == lane) {
+                taken |= 1u << (be >> 5);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-                if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; bs = os; }
+                for (int j = 0; j < EPT; ++j)
+                    if ((unsigned)j == (be >> 5)) slot[j] = r;
             }
-            if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == r) { my_e = be; my_sc = bs; }
         }
-        const float selsum = warp_sum(lane < k ? my_sc : 0.f);
-        if (lane < k) {
-            float g;
-            if (a.score == MOE_SCORE_SOFTMAX && !a.renorm) g = my_sc;
-            else g = my_sc / selsum;
-            a.idx[(size_t)t * k + lane] = my_e;
-            a.gate[(size_t)t * k + lane] = g;
+        float mine = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) if (slot[j] >= 0) mine += sc[j];
+        const float selsum = warp_sum(mine);
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            if (slot[j] >= 0) {
+                const float g = (a.score == MOE_SCORE_SOFTMAX && !a.renorm) ? sc[j] : sc[j] / selsum;
+                a.idx[(size_t)t * k + slot[j]] = lane + 32 * j;
+                a.gate[(size_t)t * k + slot[j]] = g;
+            }
         }
     }
 }
@@ -209,8 +220,8 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
 
 // Selection for bf16 layers: logits [T, E] (offset already added) from the
 // tensor-core router, same per-warp selection as the fp32 path; one CTA takes
-// 128 tokens (four groups of 32), so the score sums have T/128 rows.
-constexpr int kSelTok = 128;
+// 64 tokens (two groups of 32), so the score sums have T/64 rows.
+constexpr int kSelTok = 64;
 
 template <int EPT>
 __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ logits) {
