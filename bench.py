@@ -351,6 +351,15 @@ def run_ours(args, wl, dev, world, rank):
     return result
 
 
+def launches_per_forward(wl):
+    """Kernels one moe_forward call launches (T > 0).  bf16: W_r split, logits
+    GEMM, selection, histogram, scan (+ balance statistics), permute, two
+    launches per expert GEMM (CTA-pair kernel, then the 1-CTA kernel for last
+    blocks of 1..128 rows), combine.  fp32: router, histogram, scan, permute,
+    two SIMT GEMMs, combine."""
+    return 11 if wl.dtype == "bf16" else 7
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -402,7 +411,7 @@ def main():
         "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
         "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": launches_per_forward(wl) * args.steps,
         "clocks": r["clocks"],
         "routing": {"kept_rows": r["kept_rows"], "dropped": r["n_dropped"], "loss": r["loss"],
                     "max_count": int(r["counts"].max()), "min_count": int(r["counts"].min()),

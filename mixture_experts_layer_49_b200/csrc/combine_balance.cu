@@ -10,8 +10,10 @@
 //
 // Balance: f_e = counts_e / (T k), P_e = mean over tokens of the normalised
 // score, L = E sum f_e P_e (Vector Institute post, Eq. balance; Router
-// Optimization page, How It Works 1).  The per-block partial sums written by
-// the router are added in block order in double precision.
+// Optimization page, How It Works 1), in the reduction order of balance.cuh.
+// The forward pass computes them in the dispatch scan instead; this kernel
+// serves the standalone entry point.
+#include "balance.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -90,52 +92,25 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     }
 }
 
-// 1024 threads: with EP = E rounded up to a power of two, thread (g, e)
-// (g = threadIdx.x / EP) adds the block rows b = g, g + 1024/EP, ... in
-// order; the 1024/EP partial sums of an expert are then added in g order and
-// the loss terms f_e P_e in a fixed tree.  Everything in double; the result
-// does not depend on scheduling.
+// 32 warps; warp w takes experts w, w + 32, ... (P_e by psum_column), then
+// the loss terms meet in loss_tree.  Everything in double; the result does
+// not depend on scheduling and equals the forward pass's (dispatch scan).
 __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
-    __shared__ double partial[1024];
     __shared__ double red[256];
-    int EP = 1;
-    while (EP < a.E) EP <<= 1;
-    const int groups = 1024 / EP;
-    const int e = threadIdx.x % EP, g = threadIdx.x / EP;
-    double s = 0.0;
-    if (e < a.E) {
-        int b = g;
-        for (; b + 3 * groups < a.nblk; b += 4 * groups) {     // four independent loads in flight
-            const float v0 = a.psum[(size_t)b * a.E + e];
-            const float v1 = a.psum[(size_t)(b + groups) * a.E + e];
-            const float v2 = a.psum[(size_t)(b + 2 * groups) * a.E + e];
-            const float v3 = a.psum[(size_t)(b + 3 * groups) * a.E + e];
-            s += (double)v0; s += (double)v1; s += (double)v2; s += (double)v3;
-        }
-        for (; b < a.nblk; b += groups) s += (double)a.psum[(size_t)b * a.E + e];
-    }
-    partial[threadIdx.x] = s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x < 256) red[threadIdx.x] = 0.0;
     __syncthreads();
-    if (threadIdx.x < 256) {
-        double contrib = 0.0;
-        const int ee = threadIdx.x;
-        if (ee < a.E) {
-            double tot = 0.0;
-            for (int gg = 0; gg < groups; ++gg) tot += partial[gg * EP + ee];
-            const double P = tot / (double)a.T;
-            const double f = (double)a.counts[ee] / ((double)a.T * (double)a.k);
-            a.f[ee] = (float)f;
-            a.P[ee] = (float)P;
-            contrib = f * P;
+    for (int e = warp; e < a.E; e += 32) {
+        const double P = psum_column(a.psum, a.nblk, a.E, e) / (double)a.T;
+        const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
+        if (lane == 0) {
+            a.f[e] = (float)f;
+            a.P[e] = (float)P;
+            red[e] = f * P;
         }
-        red[ee] = contrib;
     }
-    __syncthreads();
-    for (int o = 128; o > 0; o >>= 1) {
-        if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) *a.loss = (double)a.E * red[0];
+    const double s = loss_tree(red);
+    if (threadIdx.x == 0) *a.loss = (double)a.E * s;
 }
 
 // Auxiliary-loss-free bias update ("Fine-Tuning Mixture of Experts (MoE)

@@ -18,6 +18,7 @@
 //                assignments to the same expert comes from __match_any_sync
 //                over flattened (t, s) order, so rows are stable by token id;
 //                then the kept rows of x are copied with 16-byte vectors.
+#include "balance.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -51,42 +52,69 @@ __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, in
 // One warp per expert: exclusive scan of the expert's per-chunk counts (each
 // lane first sums 8 consecutive chunks, then a warp scan of the lane totals),
 // the expert's total count and its kept count.  Experts are independent, so
-// the grid covers them 32 per CTA.
+// the grid covers them 32 per CTA.  With balance outputs, the same warp
+// computes f_e and P_e (balance.cuh order) and the last CTA to finish adds
+// the loss terms.
 __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
+    __shared__ double red[256];
+    __shared__ int last;
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
-    if (e >= a.E) return;
-    const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
-    int32_t *dst = a.chunk_base + (size_t)e * nchunks;
-    int running = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 256) {
-        int v[8];
+    if (e < a.E) {
+        const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
+        int32_t *dst = a.chunk_base + (size_t)e * nchunks;
+        int running = 0;
+        for (int c0 = 0; c0 < nchunks; c0 += 256) {
+            int v[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int c = c0 + lane * 8 + i;
-            v[i] = c < nchunks ? src[c] : 0;
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + lane * 8 + i;
+                v[i] = c < nchunks ? src[c] : 0;
+            }
+            int tot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tot += v[i];
+            int incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            int run = running + incl - tot;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + lane * 8 + i;
+                if (c < nchunks) dst[c] = run;
+                run += v[i];
+            }
+            running += __shfl_sync(0xffffffffu, incl, 31);
         }
-        int tot = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) tot += v[i];
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += n;
+        if (lane == 0) {
+            a.counts[e] = running;
+            a.kept[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
         }
-        int run = running + incl - tot;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int c = c0 + lane * 8 + i;
-            if (c < nchunks) dst[c] = run;
-            run += v[i];
+        if (a.loss) {
+            const double P = psum_column(a.psum, a.nblk, a.E, e) / (double)a.T;
+            const double f = (double)running / ((double)a.T * (double)a.k);
+            if (lane == 0) {
+                a.f[e] = (float)f;
+                a.P[e] = (float)P;
+                a.contrib[e] = f * P;
+            }
         }
-        running += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-        a.counts[e] = running;
-        a.kept[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
+    if (a.loss == nullptr) return;                   // uniform over the grid
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(a.ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;                               // uniform over the block
+    __threadfence();
+    if (threadIdx.x < 256) red[threadIdx.x] = (int)threadIdx.x < a.E ? __ldcg(a.contrib + threadIdx.x) : 0.0;
+    const double s = loss_tree(red);
+    if (threadIdx.x == 0) {
+        *a.loss = (double)a.E * s;
+        *a.ticket = 0;
     }
 }
 

@@ -20,15 +20,21 @@ struct RouterArgs {
     float *psum;                 // [router_blocks(T, bf16), E]
     int T, d, E, k, score, renorm;
     void *wsplit;                // bf16 layers: [3, E, d] scratch for the split W_r
-    float *logits_ws;            // bf16 layers: [T, E] scratch for the logits (if no logits_out)
+    float *logits_ws;            // bf16 layers: [router_logit_splits_max(T), T, E] scratch for
+                                 // the (partial) logits
     int32_t *status;             // workspace status word
+    int num_sms;
 };
 // Rows of the per-block score sums: 64 tokens per block for bf16 layers,
 // 32 for fp32 layers.
 int router_blocks(int T, bool bf16);
 size_t router_split_bytes(int d, int E);
+// K-split count of the tensor-core logits GEMM: the bound the workspace is
+// sized for, and the count used on a GPU with num_sms SMs.
+int router_logit_splits_max(int T);
+int router_logit_splits(int T, int d, int num_sms);
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st);
-cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStream_t st);
+cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits, cudaStream_t st);
 
 struct DispatchArgs {
     const void *x;               // [T, d]
@@ -44,6 +50,14 @@ struct DispatchArgs {
     int32_t *n_dropped;          // device scalar or null
     int32_t *status;             // workspace status word
     int T, d, E, k, capacity;    // capacity < 0: unlimited
+    // Optional (loss != null): the balance statistics, computed in the scan
+    // kernel from the router's per-block score sums.
+    const float *psum;           // [nblk, E]
+    float *f, *P;                // [E]
+    double *loss;                // device scalar
+    double *contrib;             // [E] scratch: f_e P_e
+    int32_t *ticket;             // zero-initialised counter, reset by the last CTA
+    int nblk;
 };
 int dispatch_chunks(int T);
 cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st);

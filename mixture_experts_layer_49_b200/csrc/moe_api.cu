@@ -24,7 +24,7 @@ moe_status cuda_fail(cudaError_t e, const char *where) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-    size_t router_w, logits, psum, chunk_cnt, chunk_base, kept, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
+    size_t router_w, logits, psum, chunk_cnt, chunk_base, kept, contrib, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
 };
 
 int64_t perm_rows(const moe_config *c) {
@@ -42,11 +42,12 @@ Layout layout(const moe_config *c) {
     const size_t nch = (size_t)moe::dispatch_chunks(c->T);
     size_t o = sizeof(moe::WsHeader);
     L.router_w = o;   o = align256(o + (bf16 ? moe::router_split_bytes(c->d_model, c->E) : 0));
-    L.logits = o;     o = align256(o + (bf16 ? (size_t)c->T * c->E * 4 : 0));
+    L.logits = o;     o = align256(o + (bf16 ? (size_t)moe::router_logit_splits_max(c->T) * c->T * c->E * 4 : 0));
     L.psum = o;       o = align256(o + nblk * c->E * 4);
     L.chunk_cnt = o;  o = align256(o + nch * c->E * 4);
     L.chunk_base = o; o = align256(o + nch * c->E * 4);
     L.kept = o;       o = align256(o + (size_t)c->E * 4);
+    L.contrib = o;    o = align256(o + (size_t)c->E * 8);
     L.offsets = o;    o = align256(o + (size_t)(c->E + 1) * 4);
     L.row_of = o;     o = align256(o + Tk * 4);
     L.row_token = o;  o = align256(o + Tk * 4);
@@ -195,7 +196,8 @@ moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
     moe::RouterArgs a{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
-                      at<char>(ws, layout(cfg).router_w), at<float>(ws, layout(cfg).logits), status_word(ws)};
+                      at<char>(ws, layout(cfg).router_w), at<float>(ws, layout(cfg).logits), status_word(ws),
+                      num_sms()};
     cudaError_t e = moe::launch_router(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router");
 }
@@ -299,7 +301,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
 
     moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                        cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
-                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws)};
+                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
     if ((e = moe::launch_router(ra, bf16, st)) != cudaSuccess) return cuda_fail(e, "router");
 
     moe::DispatchArgs da{};
@@ -313,6 +315,11 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     da.status = status_word(ws);
     da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
     da.capacity = moe_capacity(cfg);
+    // the balance statistics ride on the dispatch scan
+    da.psum = psum; da.f = f; da.P = P; da.loss = loss;
+    da.contrib = at<double>(ws, L.contrib);
+    da.ticket = &reinterpret_cast<moe::WsHeader *>(ws)->balance_ticket;
+    da.nblk = moe::router_blocks(cfg->T, bf16);
     if ((e = moe::launch_dispatch(da, bf16, st)) != cudaSuccess) return cuda_fail(e, "permute");
 
     moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
@@ -323,9 +330,6 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
-
-    moe::BalanceArgs ba{counts, psum, f, P, loss, cfg->T, cfg->E, cfg->top_k, moe::router_blocks(cfg->T, bf16)};
-    if ((e = moe::launch_balance(ba, st)) != cudaSuccess) return cuda_fail(e, "balance");
     return MOE_OK;
 }
 

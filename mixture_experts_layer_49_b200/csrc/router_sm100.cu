@@ -18,12 +18,19 @@
 // accumulators whose partial sums the epilogue adds in fp32 (round to
 // nearest) before anything else reads the logits.
 //
-// One CTA per 128 tokens (MMA M = 128, N = E rounded up to 16, K = d_model):
-//   warp 0      TMA producer: x tile 128 x 64 and the three W_r terms
-//               N x 64 per stage (128-byte swizzle), 2-4 stages
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+// One CTA pair (tcgen05.mma.cta_group::2) per 256 tokens and K range:
+//   MMA M = 256 (128 tokens per CTA), N = E rounded up to 16 (each CTA loads
+//   half of the rows of the three W_r terms), K = d_model or a slice of it.
+//   When the tokens alone give fewer pairs than the GPU holds, K is split
+//   over up to four pairs per token block; each writes its partial logits and
+//   the selection kernel adds them in split order.
+//   warp 0      TMA producer (both CTAs): x tile 128 x 64 and the CTA's half
+//               of the three W_r terms per stage (128-byte swizzle)
+//   warp 1      TMEM allocator (both CTAs) + single-thread MMA issuer (rank 0)
 //   warps 2..5  epilogue, one thread per token: add the K-split accumulators
-//               and the logit offset, store the fp32 logits row
+//               (and the logit offset in split 0), stage the row in shared
+//               memory, then each warp stores its 32 rows as one contiguous
+//               block with 16-byte vector stores
 // Scores, top-k, gates and the per-block score sums then run in the
 // warp-per-token selection kernel of router_topk.cu (a per-thread top-k over
 // E values was instruction-bound here).
@@ -42,25 +49,30 @@ constexpr int RBK = 64;                       // K per stage
 constexpr int kThreads = 192;
 constexpr uint32_t A_BYTES = RM * RBK * 2;    // 16 KiB
 constexpr int kSmemCap = 227 * 1024;
+constexpr int kMaxStages = 8;
+constexpr int kMaxSplits = 4;
 
 struct TcRouterParams {
     const float *logit_bias;
-    float *logits;             // [T, E] fp32 out
+    float *out;                // [splits][T][E] fp32 (one split: the logits)
     int32_t *status;
     int T, d, E;
     int n_pad;                 // MMA N
-    int nparts;                // K-split: separate accumulators
+    int nparts;                // K-split inside the CTA: separate accumulators
     int pstride;               // TMEM columns between accumulators (>= n_pad, multiple of 32)
     int stages;
-    uint32_t b_bytes;          // one W_r term per stage: n_pad x 64 bf16
+    int splits;                // K-split across CTA pairs
+    int kb_per_split;
+    int ld;                    // staging row stride in floats
+    uint32_t b_bytes;          // one W_r term, this CTA's half: n_pad/2 x 64 bf16
     uint32_t idesc;
     uint32_t tmem_cols;
     uint64_t timeout_ns;
 };
 
 struct RouterTail {
-    uint64_t full[4];
-    uint64_t empty[4];
+    uint64_t full[kMaxStages];     // rank 0's collect both CTAs' bytes
+    uint64_t empty[kMaxStages];
     uint64_t accf;
     uint32_t tmem_base;
     int abort_flag;
@@ -95,7 +107,7 @@ __global__ void __launch_bounds__(256) split_router_weights(const float *__restr
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const TcRouterParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -106,8 +118,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     RouterTail &s = *reinterpret_cast<RouterTail *>(smem + p.stages * stage_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.x * RM;
+    const uint32_t rank = cluster_ctarank();
+    const int cl = (int)cluster_id_x();
+    const int split = cl % p.splits;
+    const int t0 = (cl / p.splits) * (2 * RM) + (int)rank * RM;
     const int nk = (p.d + RBK - 1) / RBK;
+    const int kb0 = split * p.kb_per_split;
+    const int kb1 = min(nk, kb0 + p.kb_per_split);
 
     if (tid == 0) {
         s.abort_flag = 0;
@@ -116,9 +133,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), p.tmem_cols);
+    if (warp == 1) tmem_alloc_pair(smem_u32(&s.tmem_base), p.tmem_cols);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = s.tmem_base;
 
@@ -126,28 +143,31 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int kb = 0; kb < nk; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) {
                     record_error(p.status, MOE_ERR_TIMEOUT, 11);
                     s.abort_flag = 1;
                     break;
                 }
-                const uint32_t fb = smem_u32(&s.full[stage]);
+                const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
                 const uint32_t st = base + stage * stage_bytes;
-                mbar_arrive_expect_tx(fb, stage_bytes);
-                tma_load_2d(st, &tmX, fb, kb * RBK, t0);
+                if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * stage_bytes);
+                tma_load_2d_pair(st, &tmX, fb, kb * RBK, t0);
 #pragma unroll
-                for (int j = 0; j < 3; ++j) tma_load_3d(st + A_BYTES + j * p.b_bytes, &tmW, fb, kb * RBK, 0, j);
+                for (int j = 0; j < 3; ++j)
+                    tma_load_3d_pair(st + A_BYTES + j * p.b_bytes, &tmW, fb, kb * RBK, (int)rank * (p.n_pad / 2), j);
                 if (++stage == p.stages) { stage = 0; phase ^= 1u; }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             int prev_part = -1;
-            for (int kb = 0; kb < nk; ++kb) {
+            const int nkl = kb1 - kb0;
+            const int np = min(p.nparts, nkl);
+            for (int i = 0; i < nkl; ++i) {
                 if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) {
                     record_error(p.status, MOE_ERR_TIMEOUT, 12);
                     s.abort_flag = 1;
@@ -156,7 +176,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
                 tc_fence_after();
                 const uint32_t st = base + stage * stage_bytes;
-                const int part = kb * p.nparts / nk;             // contiguous K ranges per accumulator
+                const int part = i * np / nkl;                   // contiguous K ranges per accumulator
                 const uint32_t dtm = tmem + (uint32_t)(part * p.pstride);
                 const uint32_t fresh = part != prev_part;
                 prev_part = part;
@@ -164,18 +184,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 for (int j = 0; j < 3; ++j)
 #pragma unroll
                     for (int k = 0; k < RBK / 16; ++k)
-                        mma_bf16(dtm, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
-                                 (fresh && j == 0 && k == 0) ? 0u : 1u);
-                mma_commit(smem_u32(&s.empty[stage]));
+                        mma_bf16_pair(dtm, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
+                                      (fresh && j == 0 && k == 0) ? 0u : 1u);
+                mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
                 if (++stage == p.stages) { stage = 0; phase ^= 1u; }
             }
-            if (ok) mma_commit(smem_u32(&s.accf));
+            if (ok) mma_commit_pair(smem_u32(&s.accf), (uint16_t)0x3);
         }
     } else {
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int t = t0 + row;
-        const bool tok_ok = t < p.T;
+        const int row0 = t0 + q * 32;                     // the warp's first token
         int ok = 1;
         if (lane == 0) ok = mbar_wait(smem_u32(&s.accf), 0, p.timeout_ns) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -184,35 +202,66 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         } else {
             __syncwarp();
             tc_fence_after();
+            // every MMA has completed, so the stage buffers are free: the warp
+            // stages its 32 rows there (row stride ld floats)
+            const int E = p.E, ld = p.ld;
+            float *stg = reinterpret_cast<float *>(smem) + (size_t)q * 32 * ld;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-            const int E = p.E;
-            float *dst = p.logits + (size_t)t * E;
+            // 16-byte vectors need E % 4 == 0 and a 16-byte aligned output
+            const bool vec = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
+            const bool add_bias = split == 0 && p.logit_bias != nullptr;
+            const int np = min(p.nparts, kb1 - kb0);      // accumulators this split wrote
             for (int c = 0; c < (E + 31) / 32; ++c) {
                 float v[32];
                 __syncwarp();
                 tmem_ld32(taddr + c * 32, v);
-                for (int r = 1; r < p.nparts; ++r) {       // fixed order: parts 0, 1, 2, ...
+                for (int r = 1; r < np; ++r) {             // fixed order: parts 0, 1, 2, ...
                     float w[32];
                     tmem_ld32(taddr + r * p.pstride + c * 32, w);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] += w[j];
                 }
-                if (tok_ok) {
+                if (add_bias) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int e = c * 32 + j;
-                        if (e < E) dst[e] = v[j] + (p.logit_bias ? __ldg(p.logit_bias + e) : 0.f);
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        if (c * 32 + j < E) v[j] += __ldg(p.logit_bias + c * 32 + j);
+                }
+                float *dst = stg + (size_t)lane * ld + c * 32;
+                if (vec) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        if (c * 32 + j < E) *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c * 32 + j < E) dst[j] = v[j];
+                }
+            }
+            __syncwarp();
+            // the warp's rows are contiguous in the output: copy them as one block
+            const int nrows = max(0, min(32, p.T - row0));
+            float *out = p.out + ((size_t)split * p.T + row0) * E;
+            const int n = nrows * E;
+            if (vec) {
+                for (int f = lane * 4; f < n; f += 128) {
+                    const int r = f / E, col = f - r * E;
+                    *reinterpret_cast<float4 *>(out + f) = *reinterpret_cast<const float4 *>(stg + (size_t)r * ld + col);
+                }
+            } else {
+                for (int f = lane; f < n; f += 32) {
+                    const int r = f / E, col = f - r * E;
+                    out[f] = stg[(size_t)r * ld + col];
                 }
             }
         }
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                                  // no CTA leaves while its peer may still signal it
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, p.tmem_cols);
+        tmem_dealloc_pair(tmem, p.tmem_cols);
     }
 }
 
@@ -238,25 +287,35 @@ bool encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_tc(const CUtensorMap &mx, const CUtensorMap &mw, const TcRouterParams &p, size_t smem,
-                      cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    const int grid = (p.T + RM - 1) / RM;
-    router_tc_kernel<<<grid, kThreads, smem, st>>>(mx, mw, p);
-    return cudaGetLastError();
-}
+// Pairs of 256 tokens; the K-split count multiplies them up to the number of
+// pairs the GPU holds at once, at most kMaxSplits and at most one split per
+// two 64-deep K steps.
+int pair_blocks(int T) { return (T + 2 * RM - 1) / (2 * RM); }
 
 }  // namespace
 
+int router_logit_splits_max(int T) {
+    const int pairs = pair_blocks(T);
+    if (pairs <= 0) return 1;
+    const int s = 128 / pairs;
+    return s < 1 ? 1 : (s > kMaxSplits ? kMaxSplits : s);
+}
+
+int router_logit_splits(int T, int d, int num_sms) {
+    const int pairs = pair_blocks(T);
+    if (pairs <= 0) return 1;
+    int s = (num_sms / 2) / pairs;
+    const int nk = (d + RBK - 1) / RBK;
+    if (s > nk / 2) s = nk / 2;
+    const int cap = router_logit_splits_max(T);
+    if (s > cap) s = cap;
+    return s < 1 ? 1 : s;
+}
+
 size_t router_split_bytes(int d, int E) { return (size_t)3 * E * d * 2; }
 
-// Logits h = x W_r (+ logit offset) into `logits` [T, E] fp32.
-cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStream_t st) {
+// Logits h = x W_r (+ logit offset) into `out`: [splits][T][E] partial sums.
+cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits, cudaStream_t st) {
     void *wsplit = a.wsplit;
     if (a.T == 0) return cudaSuccess;
     dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
@@ -265,28 +324,37 @@ cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStre
     if (e != cudaSuccess) return e;
 
     TcRouterParams p{};
-    p.logit_bias = a.logit_bias; p.logits = logits; p.status = a.status;
+    p.logit_bias = a.logit_bias; p.out = out; p.status = a.status;
     p.T = a.T; p.d = a.d; p.E = a.E;
     p.n_pad = (a.E + 15) / 16 * 16;
-    p.b_bytes = (uint32_t)p.n_pad * RBK * 2;
-    p.idesc = make_idesc_bf16(RM, (uint32_t)p.n_pad);
+    p.b_bytes = (uint32_t)(p.n_pad / 2) * RBK * 2;
+    p.idesc = make_idesc_bf16(2 * RM, (uint32_t)p.n_pad);
     p.pstride = (p.n_pad + 31) / 32 * 32;
     const int nk = (a.d + RBK - 1) / RBK;
+    p.splits = splits;
+    p.kb_per_split = (nk + splits - 1) / splits;
+    const int nkl = p.kb_per_split;
     int nparts = 512 / p.pstride;
     if (nparts > 8) nparts = 8;
-    if (nparts > nk) nparts = nk;
+    if (nparts > nkl) nparts = nkl;
     p.nparts = nparts;
     uint32_t cols = 32;
     while ((int)cols < p.nparts * p.pstride) cols <<= 1;
     p.tmem_cols = cols;
     p.timeout_ns = 2000000000ull;
+    p.ld = (a.E & 3) == 0 ? a.E + 4 : a.E + 1;
     const size_t stage_bytes = A_BYTES + 3 * (size_t)p.b_bytes;
-    const size_t fixed = 1024 + 256;
+    const size_t fixed = 1024 + sizeof(RouterTail);
     int stages = (int)((kSmemCap - fixed) / stage_bytes);
-    if (stages > 4) stages = 4;
+    if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return cudaErrorInvalidValue;
+    // the epilogue stages 128 rows of ld floats in the stage buffers
+    const size_t staging = (size_t)RM * p.ld * 4;
+    if (staging > (size_t)stages * stage_bytes) return cudaErrorInvalidValue;
     p.stages = stages;
     const size_t smem = fixed + stages * stage_bytes;
+    // every split must own at least one K step
+    if ((size_t)(splits - 1) * p.kb_per_split >= (size_t)nk) return cudaErrorInvalidValue;
 
     CUtensorMap mx, mw;
     const cuuint64_t xd[2] = {(cuuint64_t)a.d, (cuuint64_t)a.T};
@@ -295,10 +363,18 @@ cudaError_t launch_router_logits_tc(const RouterArgs &a, float *logits, cudaStre
     if (!encode(&mx, 2, a.x, xd, xs, xb)) return cudaErrorInvalidValue;
     const cuuint64_t wd[3] = {(cuuint64_t)a.d, (cuuint64_t)a.E, 3};
     const cuuint64_t wst[2] = {(cuuint64_t)a.d * 2, (cuuint64_t)a.E * a.d * 2};
-    const cuuint32_t wb[3] = {RBK, (cuuint32_t)p.n_pad, 1};
+    const cuuint32_t wb[3] = {RBK, (cuuint32_t)(p.n_pad / 2), 1};
     if (!encode(&mw, 3, wsplit, wd, wst, wb)) return cudaErrorInvalidValue;
 
-    return launch_tc(mx, mw, p, smem, st);
+    static bool attr = false;
+    if (!attr) {
+        e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int grid = 2 * pair_blocks(a.T) * splits;
+    router_tc_kernel<<<grid, kThreads, smem, st>>>(mx, mw, p);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

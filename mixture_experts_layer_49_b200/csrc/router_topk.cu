@@ -49,96 +49,138 @@ __device__ __forceinline__ void load_x_vec<float>(const float *src, float *dst) 
     dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
 }
 
-// Scores, top-k and gates for the 32 tokens starting at t0 (warp w holds
-// tokens t0 + 4w .. t0 + 4w + 3; acc[i][j] is the logit of token 4w + i for
-// expert lane + 32 j), adding each token's normalised scores into psum_acc.
-// add_bias: add logit_bias to acc first (the tensor-core path has added it).
+// Compare-exchange for the lane-local sort: order by key descending, then
+// expert id ascending (the tie rule of the selection).
+__device__ __forceinline__ void cex(unsigned &ka, int &ia, float &ga, unsigned &kb, int &ib, float &gb) {
+    const bool sw = ka < kb || (ka == kb && ia > ib);
+    const unsigned tk = sw ? kb : ka; kb = sw ? ka : kb; ka = tk;
+    const int ti = sw ? ib : ia; ib = sw ? ia : ib; ia = ti;
+    const float tg = sw ? gb : ga; gb = sw ? ga : gb; ga = tg;
+}
+
+// Sorting networks for 2, 4 and 8 candidates per lane (Batcher's odd-even
+// merge sort for 8).
+template <int EPT>
+__device__ __forceinline__ void lane_sort(unsigned (&k)[EPT], int (&id)[EPT], float (&g)[EPT]) {
+#define CEX(i, j) cex(k[i], id[i], g[i], k[j], id[j], g[j])
+    if constexpr (EPT == 2) {
+        CEX(0, 1);
+    } else if constexpr (EPT == 4) {
+        CEX(0, 1); CEX(2, 3); CEX(0, 2); CEX(1, 3); CEX(1, 2);
+    } else if constexpr (EPT == 8) {
+        CEX(0, 1); CEX(2, 3); CEX(4, 5); CEX(6, 7);
+        CEX(0, 2); CEX(1, 3); CEX(4, 6); CEX(5, 7);
+        CEX(1, 2); CEX(5, 6);
+        CEX(0, 4); CEX(1, 5); CEX(2, 6); CEX(3, 7);
+        CEX(2, 4); CEX(3, 5);
+        CEX(1, 2); CEX(3, 4); CEX(5, 6);
+    }
+#undef CEX
+}
+
+// Scores, top-k and gates of token t, whose logits h[j] (expert lane + 32 j,
+// logit offset included) sit in the registers of one warp; sb[j] is the
+// selection bias of the same expert (0 without one).  The token's
+// normalised scores are added into psum_acc.
+//
+// Selection: each lane sorts its EPT candidates by (key desc, id asc); then
+// k rounds, each taking the largest head key over the warp (redux.sync on an
+// order-preserving integer image of the fp32 key) and, among the lanes that
+// hold it, the lowest expert id.  The winner lane pops its head.  Lane r
+// keeps the winner of round r, so slot r of idx and gate is written by lane r.
+template <int EPT>
+__device__ __forceinline__ void select_token(const RouterArgs &a, const float (&h)[EPT], const float (&sb)[EPT],
+                                             int t, float (&psum_acc)[EPT]) {
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    const bool softmax = a.score == MOE_SCORE_SOFTMAX;
+    float gs[EPT], kf[EPT];                  // gate source; selection key
+    if (softmax) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) if (lane + 32 * j < E) m = fmaxf(m, h[j]);
+        m = warp_max(m);
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) { gs[j] = (lane + 32 * j < E) ? expf(h[j] - m) : 0.f; z += gs[j]; }
+        const float inv = 1.f / warp_sum(z);
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) { gs[j] *= inv; psum_acc[j] += gs[j]; kf[j] = h[j] + sb[j]; }
+    } else {
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            gs[j] = (lane + 32 * j < E) ? 1.f / (1.f + expf(-h[j])) : 0.f;
+            z += gs[j];
+        }
+        const float inv = 1.f / warp_sum(z);
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) { psum_acc[j] += gs[j] * inv; kf[j] = gs[j] + sb[j]; }
+    }
+    unsigned key[EPT];
+    int id[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        id[j] = lane + 32 * j;
+        // absent experts rank below every real key; a NaN key ranks just above them
+        key[j] = id[j] < E ? (kf[j] == kf[j] ? ordered_key(kf[j]) : 1u) : 0u;
+    }
+    lane_sort<EPT>(key, id, gs);
+    unsigned my_id = 0;
+    float my_g = 0.f;
+    for (int r = 0; r < k; ++r) {
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, key[0]);
+        const unsigned be = __reduce_min_sync(0xffffffffu, key[0] == kmax ? (unsigned)id[0] : 0xffffffffu);
+        const int wl = (int)(be & 31u);
+        const float gw = __shfl_sync(0xffffffffu, gs[0], wl);
+        if (lane == r) { my_id = be; my_g = gw; }
+        if (lane == wl) {
+#pragma unroll
+            for (int j = 0; j + 1 < EPT; ++j) { key[j] = key[j + 1]; id[j] = id[j + 1]; gs[j] = gs[j + 1]; }
+            key[EPT - 1] = 0u;
+            id[EPT - 1] = 0x7fffffff;
+        }
+    }
+    const float selsum = warp_sum(lane < k ? my_g : 0.f);
+    if (lane < k) {
+        a.idx[(size_t)t * k + lane] = (int)my_id;
+        a.gate[(size_t)t * k + lane] = (softmax && !a.renorm) ? my_g : my_g / selsum;
+    }
+}
+
+// The 32 tokens starting at t0 (warp w holds tokens t0 + 4w .. t0 + 4w + 3;
+// acc[i][j] is the logit of token 4w + i for expert lane + 32 j).
+// add_bias: add logit_bias to acc first (the tensor-core path has);
+// write_logits: store the logits to logits_out.
 template <int EPT>
 __device__ __forceinline__ void select_tokens(const RouterArgs &a, float (&acc)[4][EPT], int t0, bool add_bias,
-                                              float (&psum_acc)[EPT]) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int E = a.E, k = a.k;
+                                              bool write_logits, const float (&sb)[EPT], float (&psum_acc)[EPT]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = a.E;
+    float lb[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) lb[j] = (add_bias && a.logit_bias && lane + 32 * j < E) ? a.logit_bias[lane + 32 * j] : 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int t = t0 + warp * 4 + i;
         if (t >= a.T) break;                         // uniform across the warp
-        float h[EPT], sc[EPT], key[EPT];
-        bool valid[EPT];
+        float h[EPT];
 #pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            const int e = lane + 32 * j;
-            valid[j] = e < E;
-            h[j] = acc[i][j] + ((add_bias && a.logit_bias && valid[j]) ? a.logit_bias[e] : 0.f);
-        }
-        float norm;
-        if (a.score == MOE_SCORE_SOFTMAX) {
-            float m = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) if (valid[j]) m = fmaxf(m, h[j]);
-            m = warp_max(m);
-            float z = 0.f;
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) { sc[j] = valid[j] ? expf(h[j] - m) : 0.f; z += sc[j]; }
-            norm = warp_sum(z);
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) { sc[j] = sc[j] / norm; key[j] = h[j]; }
-            norm = 1.f;                              // sc already normalised
-        } else {
-            float z = 0.f;
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) { sc[j] = valid[j] ? 1.f / (1.f + expf(-h[j])) : 0.f; z += sc[j]; }
-            norm = warp_sum(z);
-#pragma unroll
-            for (int j = 0; j < EPT; ++j) key[j] = sc[j];
-        }
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            if (a.sel_bias && valid[j]) key[j] += a.sel_bias[lane + 32 * j];
-            psum_acc[j] += (a.score == MOE_SCORE_SOFTMAX) ? sc[j] : sc[j] / norm;
-        }
-        if (a.logits_out && add_bias) {
+        for (int j = 0; j < EPT; ++j) h[j] = acc[i][j] + lb[j];
+        if (write_logits) {
 #pragma unroll
             for (int j = 0; j < EPT; ++j)
-                if (valid[j]) a.logits_out[(size_t)t * E + lane + 32 * j] = h[j];
+                if (lane + 32 * j < E) a.logits_out[(size_t)t * E + lane + 32 * j] = h[j];
         }
-        // k rounds of warp arg-max on (key desc, expert id asc): each lane
-        // offers its best untaken expert; redux.sync picks the largest key
-        // (as an order-preserving integer), then the lowest expert id among
-        // the lanes holding it.  The owner lane records the slot.
-        unsigned taken = 0;
-        int slot[EPT];
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) slot[j] = -1;
-        for (int r = 0; r < k; ++r) {
-            float bk = 0.f;
-            int bj = -1;
-#pragma unroll
-            for (int j = 0; j < EPT; ++j)
-                if (valid[j] && !(taken & (1u << j)) && (bj < 0 || key[j] > bk)) { bk = key[j]; bj = j; }
-            const unsigned offer = (bj >= 0 && bk == bk) ? ordered_key(bk) : 0u;
-            const unsigned kmax = __reduce_max_sync(0xffffffffu, offer);
-            const unsigned cand = (bj >= 0 && offer == kmax) ? (unsigned)(lane + 32 * bj) : 0xffffffffu;
-            const unsigned be = __reduce_min_sync(0xffffffffu, cand);
-            if (be < (unsigned)E && (int)(be & 31u) == lane) {
-                taken |= 1u << (be >> 5);
-#pragma unroll
-                for (int j = 0; j < EPT; ++j)
-                    if ((unsigned)j == (be >> 5)) slot[j] = r;
-            }
-        }
-        float mine = 0.f;
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) if (slot[j] >= 0) mine += sc[j];
-        const float selsum = warp_sum(mine);
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            if (slot[j] >= 0) {
-                const float g = (a.score == MOE_SCORE_SOFTMAX && !a.renorm) ? sc[j] : sc[j] / selsum;
-                a.idx[(size_t)t * k + slot[j]] = lane + 32 * j;
-                a.gate[(size_t)t * k + slot[j]] = g;
-            }
-        }
+        select_token<EPT>(a, h, sb, t, psum_acc);
     }
+}
+
+template <int EPT>
+__device__ __forceinline__ void load_sel_bias(const RouterArgs &a, float (&sb)[EPT]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) sb[j] = (a.sel_bias && lane + 32 * j < a.E) ? a.sel_bias[lane + 32 * j] : 0.f;
 }
 
 // The CTA's row of the per-block score sums: warp partials added in warp order.
@@ -211,25 +253,30 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
         __syncthreads();
     }
 
-    float psum_acc[EPT];
+    float psum_acc[EPT], sb[EPT];
 #pragma unroll
     for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
-    select_tokens<EPT>(a, acc, t0, /*add_bias=*/true, psum_acc);
+    load_sel_bias<EPT>(a, sb);
+    select_tokens<EPT>(a, acc, t0, /*add_bias=*/true, a.logits_out != nullptr, sb, psum_acc);
     write_psum<EPT>(a, part, psum_acc);
 }
 
-// Selection for bf16 layers: logits [T, E] (offset already added) from the
-// tensor-core router, same per-warp selection as the fp32 path; one CTA takes
-// 64 tokens (two groups of 32), so the score sums have T/64 rows.
+// Selection for bf16 layers: `parts` holds `splits` partial logits [T, E]
+// (offset already added to split 0) from the tensor-core router, added in
+// split order; then the same per-warp selection as the fp32 path.  One CTA
+// takes 64 tokens (two groups of 32), so the score sums have T/64 rows.
 constexpr int kSelTok = 64;
 
 template <int EPT>
-__global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ logits) {
+__global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ parts,
+                                                                 int splits) {
     __shared__ float part[kThreads / 32][EPT * 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float psum_acc[EPT];
+    float psum_acc[EPT], sb[EPT];
 #pragma unroll
     for (int j = 0; j < EPT; ++j) psum_acc[j] = 0.f;
+    load_sel_bias<EPT>(a, sb);
+    const size_t plane = (size_t)a.T * a.E;
     for (int grp = 0; grp < kSelTok / kTok; ++grp) {
         const int t0 = blockIdx.x * kSelTok + grp * kTok;
         if (t0 >= a.T) break;
@@ -240,10 +287,21 @@ __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, c
 #pragma unroll
             for (int j = 0; j < EPT; ++j) {
                 const int e = lane + 32 * j;
-                acc[i][j] = (t < a.T && e < a.E) ? logits[(size_t)t * a.E + e] : 0.f;
+                acc[i][j] = (t < a.T && e < a.E) ? parts[(size_t)t * a.E + e] : 0.f;
             }
         }
-        select_tokens<EPT>(a, acc, t0, /*add_bias=*/false, psum_acc);
+        for (int sp = 1; sp < splits; ++sp) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = t0 + warp * 4 + i;
+#pragma unroll
+                for (int j = 0; j < EPT; ++j) {
+                    const int e = lane + 32 * j;
+                    if (t < a.T && e < a.E) acc[i][j] += parts[sp * plane + (size_t)t * a.E + e];
+                }
+            }
+        }
+        select_tokens<EPT>(a, acc, t0, /*add_bias=*/false, splits > 1 && a.logits_out != nullptr, sb, psum_acc);
     }
     write_psum<EPT>(a, part, psum_acc);
 }
@@ -268,14 +326,17 @@ int router_blocks(int T, bool bf16) { return bf16 ? (T + kSelTok - 1) / kSelTok 
 cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
     if (!bf16) return launch_router_t<float>(a, st);
-    float *logits = a.logits_out ? a.logits_out : a.logits_ws;
-    cudaError_t e = launch_router_logits_tc(a, logits, st);
+    // one split writes the logits straight to logits_out when asked for them;
+    // several write partials to the workspace and the selection adds them
+    const int splits = router_logit_splits(a.T, a.d, a.num_sms);
+    float *parts = (splits == 1 && a.logits_out) ? a.logits_out : a.logits_ws;
+    cudaError_t e = launch_router_logits_tc(a, parts, splits, st);
     if (e != cudaSuccess) return e;
     const int blocks = (a.T + kSelTok - 1) / kSelTok;
-    if (a.E <= 32) router_select_kernel<1><<<blocks, kThreads, 0, st>>>(a, logits);
-    else if (a.E <= 64) router_select_kernel<2><<<blocks, kThreads, 0, st>>>(a, logits);
-    else if (a.E <= 128) router_select_kernel<4><<<blocks, kThreads, 0, st>>>(a, logits);
-    else router_select_kernel<8><<<blocks, kThreads, 0, st>>>(a, logits);
+    if (a.E <= 32) router_select_kernel<1><<<blocks, kThreads, 0, st>>>(a, parts, splits);
+    else if (a.E <= 64) router_select_kernel<2><<<blocks, kThreads, 0, st>>>(a, parts, splits);
+    else if (a.E <= 128) router_select_kernel<4><<<blocks, kThreads, 0, st>>>(a, parts, splits);
+    else router_select_kernel<8><<<blocks, kThreads, 0, st>>>(a, parts, splits);
     return cudaGetLastError();
 }
 
