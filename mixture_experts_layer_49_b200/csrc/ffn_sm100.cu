@@ -101,6 +101,53 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
     *reinterpret_cast<uint4 *>(dst) = pk;
 }
 
+// Epilogue of one accumulator row (this thread's TMEM lane) for one tile:
+// the warp's half of the columns (SwiGLU: gate chunks half*2, half*2+1 and
+// the up chunks 128 columns on; otherwise chunks half*4 .. half*4+3) arrive
+// with one TMEM wait, then the fused activation or bias + gate scale and
+// 16-byte bf16 stores of the valid row's columns below N.
+template <int MODE>
+__device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
+                                             __nv_bfloat16 *orow_ptr, const float *bias, float gscale) {
+    float v[128];
+    if (MODE == GM_SWIGLU) {
+        const int c0 = half * 2;
+        tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + 128 + c0 * 32, taddr + 128 + (c0 + 1) * 32, v);
+        if (!valid) return;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int col0 = nt * 128 + (c0 + cc) * 32;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float h[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h[i] = silu(v[cc * 32 + u * 8 + i]) * v[64 + cc * 32 + u * 8 + i];
+                if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, h);
+            }
+        }
+    } else {
+        const int c0 = half * 4;
+        tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + (c0 + 2) * 32, taddr + (c0 + 3) * 32, v);
+        if (!valid) return;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const int col0 = nt * BNB + (c0 + cc) * 32;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int cb = col0 + u * 8;
+                if (cb >= N) continue;
+                float h[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float z = v[cc * 32 + u * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
+                    h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
+                }
+                store8(orow_ptr + cb, h);
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void decode(const SmemTail &s, int G, int tile, int &g, int &mt, int &nt) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {
@@ -278,46 +325,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int N = sh ? p.N_shared : p.N_routed;
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
-            if (MODE == GM_SWIGLU) {
-#pragma unroll 1
-                for (int c = half * 2; c < half * 2 + 2; ++c) {
-                    float gv[32], uv[32];
-                    tmem_ld32(taddr + c * 32, gv);
-                    tmem_ld32(taddr + 128 + c * 32, uv);
-                    const int col0 = nt * 128 + c * 32;
-                    if (valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            float h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) h[i] = silu(gv[v * 8 + i]) * uv[v * 8 + i];
-                            if (col0 + v * 8 < N) store8(orow_ptr + col0 + v * 8, h);
-                        }
-                    }
-                }
-            } else {
-                const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-#pragma unroll 1
-                for (int c = half * 4; c < half * 4 + 4; ++c) {
-                    float acc[32];
-                    tmem_ld32(taddr + c * 32, acc);
-                    const int col0 = nt * BNB + c * 32;
-                    if (valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int cb = col0 + v * 8;
-                            if (cb >= N) continue;
-                            float h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                float t = acc[v * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
-                                h[i] = (MODE == GM_GELU) ? gelu_erf(t) : gscale * t;
-                            }
-                            store8(orow_ptr + cb, h);
-                        }
-                    }
-                }
-            }
+            const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
@@ -531,46 +540,8 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const int N = sh ? p.N_shared : p.N_routed;
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
-            if (MODE == GM_SWIGLU) {
-#pragma unroll 1
-                for (int c = half * 2; c < half * 2 + 2; ++c) {
-                    float gv[32], uv[32];
-                    tmem_ld32(taddr + c * 32, gv);
-                    tmem_ld32(taddr + 128 + c * 32, uv);
-                    const int col0 = nt * 128 + c * 32;
-                    if (valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            float h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) h[i] = silu(gv[v * 8 + i]) * uv[v * 8 + i];
-                            if (col0 + v * 8 < N) store8(orow_ptr + col0 + v * 8, h);
-                        }
-                    }
-                }
-            } else {
-                const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-#pragma unroll 1
-                for (int c = half * 4; c < half * 4 + 4; ++c) {
-                    float acc[32];
-                    tmem_ld32(taddr + c * 32, acc);
-                    const int col0 = nt * BNB + c * 32;
-                    if (valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int cb = col0 + v * 8;
-                            if (cb >= N) continue;
-                            float h[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                float t = acc[v * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
-                                h[i] = (MODE == GM_GELU) ? gelu_erf(t) : gscale * t;
-                            }
-                            store8(orow_ptr + cb, h);
-                        }
-                    }
-                }
-            }
+            const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
