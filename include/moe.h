@@ -148,7 +148,8 @@ MOE_API moe_status moe_router_topk(const moe_config *cfg, const void *x, const f
  *   row_of     [T, top_k] int32 out: row of each assignment, -1 when dropped
  *   row_token  [T*top_k] int32 out: token of each row (first offsets[E] valid)
  *   row_gate   [T*top_k] fp32 out: gate of each row
- *   x_perm     [T*top_k, d_model] cfg->dtype out: x rows in row order
+ *   x_perm     [T*top_k, d_model] cfg->dtype out: x rows in row order, or NULL
+ *              to write the row tables only
  *   n_dropped  device int32 out (may be NULL): assignments dropped by capacity
  * An expert id outside [0, E) is recorded as MOE_ERR_DEVICE_BOUNDS and the
  * assignment is treated as dropped.                                          */

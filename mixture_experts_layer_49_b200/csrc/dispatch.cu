@@ -17,7 +17,8 @@
 //                publishes them); the rank of (t, s) among the chunk's
 //                assignments to the same expert comes from __match_any_sync
 //                over flattened (t, s) order, so rows are stable by token id;
-//                then the kept rows of x are copied with 16-byte vectors.
+//                then, unless x_perm is null, the kept rows of x are copied
+//                with 16-byte vectors.
 #include "balance.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
         }
         __syncwarp();
     }
+    if (a.x_perm == nullptr) return;             // row tables only
     __syncthreads();
     // copy the kept rows of x into x_perm, one warp per row, 16-byte vectors
     const int nvec = a.d * (int)sizeof(TX) / 16;

@@ -209,7 +209,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *idx,
     moe_status s = check_cfg(cfg);
     if (s != MOE_OK) return s;
     NEED(counts); NEED(kept); NEED(offsets);
-    if (cfg->T > 0) { NEED(x); NEED(idx); NEED(gate); NEED(row_of); NEED(row_token); NEED(row_gate); NEED(x_perm); }
+    if (cfg->T > 0) { NEED(x); NEED(idx); NEED(gate); NEED(row_of); NEED(row_token); NEED(row_gate); }
     ALIGNED(x, 16); ALIGNED(x_perm, 16); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(kept, 4);
     ALIGNED(offsets, 4); ALIGNED(row_of, 4); ALIGNED(row_token, 4); ALIGNED(row_gate, 4); ALIGNED(n_dropped, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;

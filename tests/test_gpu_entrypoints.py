@@ -119,6 +119,15 @@ def test_entry_points(wl, cuda_device):
             if ro[t, s] >= 0:
                 exp_gate[ro[t, s]] = g[t, s]
     np.testing.assert_array_equal(st.row_gate[:nrows].cpu().numpy(), exp_gate)
+    # without x_perm the same row tables come out and nothing else is written
+    rt2 = torch.full_like(st.row_token, -7)
+    ro2 = torch.full_like(st.row_of, -7)
+    rg2 = torch.zeros_like(st.row_gate)
+    nat.moe_permute(st.cfg, inp["x"], st.idx, st.gate, st.counts, st.kept, st.offsets, ro2, rt2, rg2, None,
+                    st.n_dropped, st.ws)
+    assert st.status() == nat.MOE_OK
+    assert torch.equal(ro2, st.row_of) and torch.equal(rt2[:nrows], st.row_token[:nrows])
+    assert torch.equal(rg2[:nrows], st.row_gate[:nrows])
 
     # ---- grouped FFN: each packed row against the oracle expert on its token
     st.ffn()
