@@ -61,6 +61,7 @@ constexpr int kCombThreads = 256;
 // One warp per token (grid-stride); lanes stride over 16-byte column vectors.
 template <typename TY>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
+    pdl_wait_then_release();
     using V = Vec16<TY>;
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (kCombThreads / 32);
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 // the loss terms meet in loss_tree.  Everything in double; the result does
 // not depend on scheduling and equals the forward pass's (dispatch scan).
 __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
+    pdl_wait_then_release();
     __shared__ double red[256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x < 256) red[threadIdx.x] = 0.0;
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
 // Models: Router Optimization Techniques", How It Works 2, and its router
 // module): b_e <- b_e - gamma * sign(count_e - T k / E), in double.
 __global__ void bias_update_kernel(const int32_t *counts, float *bias, double gamma, int T, int k, int E) {
+    pdl_wait_then_release();
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     const double err = (double)counts[e] - (double)T * (double)k / (double)E;
@@ -130,6 +133,7 @@ __global__ void bias_update_kernel(const int32_t *counts, float *bias, double ga
 // first-class metric).  One CTA; fixed-order tree sums in double.
 __global__ void __launch_bounds__(256) routing_health_kernel(const int32_t *counts, const float *P, double *out,
                                                              int T, int k, int E) {
+    pdl_wait_then_release();
     __shared__ double hs[256];
     __shared__ int mx[256], mn[256];
     const int e = threadIdx.x;
@@ -177,9 +181,8 @@ cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st) {
     int blocks = (a.T + warps_per_block - 1) / warps_per_block;
     const int cap = a.num_sms * 8;
     if (blocks > cap) blocks = cap;
-    if (bf16) combine_kernel<__nv_bfloat16><<<blocks, kCombThreads, 0, st>>>(a);
-    else combine_kernel<float><<<blocks, kCombThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    if (bf16) return launch_kernel(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(kCombThreads), 0, st, a.pdl, a);
+    return launch_kernel(combine_kernel<float>, dim3(blocks), dim3(kCombThreads), 0, st, a.pdl, a);
 }
 
 cudaError_t launch_balance(const BalanceArgs &a, cudaStream_t st) {

@@ -33,6 +33,7 @@ constexpr int kPermThreads = 512;            // permute: 16 warps share the row 
 constexpr int kWarps = kPermThreads / 32;
 
 __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, int nchunks) {
+    pdl_wait_then_release();
     __shared__ int cnt[256];
     const int c = blockIdx.x;
     for (int e = threadIdx.x; e < a.E; e += kThreads) cnt[e] = 0;
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, in
 // computes f_e and P_e (balance.cuh order) and the last CTA to finish adds
 // the loss terms.
 __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
+    pdl_wait_then_release();
     __shared__ double red[256];
     __shared__ int last;
     const int lane = threadIdx.x & 31;
@@ -121,6 +123,7 @@ __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nc
 
 template <typename TX>
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, int nchunks) {
+    pdl_wait_then_release();
     __shared__ int base[256];
     __shared__ int offs[256];
     __shared__ int wcnt[kWarps][256];
@@ -237,6 +240,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
 }
 
 __global__ void empty_offsets_kernel(DispatchArgs a) {
+    pdl_wait_then_release();
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.offsets[e] = 0;
     if (threadIdx.x == 0 && a.n_dropped) *a.n_dropped = 0;
 }
@@ -247,15 +251,15 @@ int dispatch_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 
 cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
     const int nchunks = dispatch_chunks(a.T);
-    if (nchunks > 0) chunk_hist_kernel<<<nchunks, kThreads, 0, st>>>(a, nchunks);
-    chunk_scan_kernel<<<(a.E + 31) / 32, 1024, 0, st>>>(a, nchunks);
-    if (nchunks == 0) {           // no tokens: every count is zero, offsets all zero
-        empty_offsets_kernel<<<1, 256, 0, st>>>(a);
-    } else {
-        if (bf16) permute_kernel<__nv_bfloat16><<<nchunks, kPermThreads, 0, st>>>(a, nchunks);
-        else permute_kernel<float><<<nchunks, kPermThreads, 0, st>>>(a, nchunks);
-    }
-    return cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if (nchunks > 0) e = launch_kernel(chunk_hist_kernel, dim3(nchunks), dim3(kThreads), 0, st, a.pdl, a, nchunks);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(chunk_scan_kernel, dim3((a.E + 31) / 32), dim3(1024), 0, st, nchunks > 0 || a.pdl, a, nchunks);
+    if (e != cudaSuccess) return e;
+    if (nchunks == 0)             // no tokens: every count is zero, offsets all zero
+        return launch_kernel(empty_offsets_kernel, dim3(1), dim3(256), 0, st, true, a);
+    if (bf16) return launch_kernel(permute_kernel<__nv_bfloat16>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
+    return launch_kernel(permute_kernel<float>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
 }
 
 }  // namespace moe

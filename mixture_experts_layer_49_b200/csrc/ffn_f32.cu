@@ -32,6 +32,7 @@ __device__ __forceinline__ float silu(float v) { return v / (1.f + expf(-v)); }
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads) simt_grouped_gemm(FfnArgs a) {
+    pdl_wait_then_release();
     __shared__ GroupTable tab;
     __shared__ float As[BK][BM + 4];
     __shared__ float Bs[BK][BN + 4];
@@ -159,11 +160,12 @@ cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st) {
     if (a.S > 0) mtiles += (a.T + BM - 1) / BM + 1;
     const int n1 = (a.F > a.S ? a.F : a.S);
     dim3 g1((unsigned)mtiles, (unsigned)((n1 + BN - 1) / BN));
-    if (a.act == MOE_ACT_SWIGLU) simt_grouped_gemm<MODE_SWIGLU><<<g1, kThreads, 0, st>>>(a);
-    else simt_grouped_gemm<MODE_GELU><<<g1, kThreads, 0, st>>>(a);
+    cudaError_t e = a.act == MOE_ACT_SWIGLU
+                        ? launch_kernel(simt_grouped_gemm<MODE_SWIGLU>, g1, dim3(kThreads), 0, st, a.pdl, a)
+                        : launch_kernel(simt_grouped_gemm<MODE_GELU>, g1, dim3(kThreads), 0, st, a.pdl, a);
+    if (e != cudaSuccess) return e;
     dim3 g2((unsigned)mtiles, (unsigned)((a.d + BN - 1) / BN));
-    simt_grouped_gemm<MODE_DOWN><<<g2, kThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(simt_grouped_gemm<MODE_DOWN>, g2, dim3(kThreads), 0, st, true, a);
 }
 
 }  // namespace moe

@@ -174,6 +174,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                 const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
                 const GemmParams p) {
+    pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -404,6 +405,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
                      const GemmParams p) {
+    pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -592,7 +594,8 @@ bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64
 
 template <int MODE>
 cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
-                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const GemmParams &p, int grid, cudaStream_t st) {
+                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const GemmParams &p, int grid, cudaStream_t st,
+                        bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -600,14 +603,13 @@ cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUten
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    tc_grouped_gemm<MODE><<<grid, kThreads, kSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
-    return cudaGetLastError();
+    return launch_kernel(tc_grouped_gemm<MODE>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs, Bs2, p);
 }
 
 template <int MODE>
 cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B,
                              const CUtensorMap &B2, const CUtensorMap &Bs, const CUtensorMap &Bs2,
-                             const GemmParams &p, int num_sms, cudaStream_t st) {
+                             const GemmParams &p, int num_sms, cudaStream_t st, bool pdl) {
     static int grid = 0;
     if (grid == 0) {
         cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -629,8 +631,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const 
         if (e != cudaSuccess || nclusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
         grid = 2 * nclusters;
     }
-    tc_grouped_gemm_pair<MODE><<<grid, kThreads, kPairSmemBytes, st>>>(A, As, B, B2, Bs, Bs2, p);
-    return cudaGetLastError();
+    return launch_kernel(tc_grouped_gemm_pair<MODE>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A, As, B, B2,
+                         Bs, Bs2, p);
 }
 
 }  // namespace
@@ -696,12 +698,12 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
         }
         P1su = P1s;
     }
-    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st)
-                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st);
+    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st, a.pdl)
+                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st, a.pdl);
     if (err != cudaSuccess) return err;
     p1.tail_mode = 1;
-    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st)
-                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st);
+    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st, true)
+                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st, true);
     if (err != cudaSuccess) return err;
 
     // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
@@ -735,10 +737,10 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     } else {
         P2s = P2;
     }
-    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, p2, grid, st);
+    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, p2, grid, st, true);
     if (err != cudaSuccess) return err;
     p2.tail_mode = 1;
-    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st);
+    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st, true);
 }
 
 }  // namespace moe

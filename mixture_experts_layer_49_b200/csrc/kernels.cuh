@@ -9,6 +9,26 @@
 
 namespace moe {
 
+// Launch `kernel` on `st`; pdl: with programmatic stream serialization, so the
+// launch overlaps the previous kernel of the stream (the kernel itself waits
+// for that kernel's completion before touching memory).  The first kernel of
+// an entry point launches without it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 bool pdl, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 struct RouterArgs {
     const void *x;               // [T, d] bf16 or fp32
     const float *Wr;             // [d, E]
@@ -24,6 +44,7 @@ struct RouterArgs {
                                  // the (partial) logits
     int32_t *status;             // workspace status word
     int num_sms;
+    bool pdl;                    // the first launch overlaps the stream's previous kernel
 };
 // Rows of the per-block score sums: 64 tokens per block for bf16 layers,
 // 32 for fp32 layers.
@@ -58,6 +79,7 @@ struct DispatchArgs {
     double *contrib;             // [E] scratch: f_e P_e
     int32_t *ticket;             // zero-initialised counter, reset by the last CTA
     int nblk;
+    bool pdl;                    // the first launch overlaps the stream's previous kernel
 };
 int dispatch_chunks(int T);
 cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st);
@@ -80,6 +102,7 @@ struct FfnArgs {
     int hF;                      // row stride of H in elements
     int64_t shared_base;         // = T*k
     int num_sms;
+    bool pdl;                    // the first launch overlaps the stream's previous kernel
 };
 cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st);
@@ -92,6 +115,7 @@ struct CombineArgs {
     int T, d, k, has_shared;
     int64_t rows_routed;         // T*k: valid routed row indices are below it
     int num_sms;
+    bool pdl;                    // the launch overlaps the stream's previous kernel
 };
 cudaError_t launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
 

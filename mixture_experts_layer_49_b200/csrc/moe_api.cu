@@ -320,15 +320,17 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     da.contrib = at<double>(ws, L.contrib);
     da.ticket = &reinterpret_cast<moe::WsHeader *>(ws)->balance_ticket;
     da.nblk = moe::router_blocks(cfg->T, bf16);
+    da.pdl = true;                                 // every launch after the first overlaps its predecessor
     if ((e = moe::launch_dispatch(da, bf16, st)) != cudaSuccess) return cuda_fail(e, "permute");
 
     moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
                                y_perm, ws);
+    fa.pdl = true;
     e = bf16 ? moe::launch_ffn_bf16(fa, st) : moe::launch_ffn_f32(fa, st);
     if (e != cudaSuccess) return cuda_fail(e, "grouped_ffn");
 
     moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
-                        cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms()};
+                        cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
 }

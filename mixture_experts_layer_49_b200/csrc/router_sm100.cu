@@ -81,6 +81,7 @@ struct RouterTail {
 // W_r [d, E] fp32 -> three bf16 matrices [3][E][d] (K-major), w = hi + mid + lo.
 __global__ void __launch_bounds__(256) split_router_weights(const float *__restrict__ Wr, int d, int E,
                                                             __nv_bfloat16 *__restrict__ out) {
+    pdl_wait_then_release();
     __shared__ float tile[32][33];
     const int j0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(256) split_router_weights(const float *__restr
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const TcRouterParams p) {
+    pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -319,8 +321,8 @@ cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits,
     void *wsplit = a.wsplit;
     if (a.T == 0) return cudaSuccess;
     dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
-    split_router_weights<<<sg, 256, 0, st>>>(a.Wr, a.d, a.E, static_cast<__nv_bfloat16 *>(wsplit));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(split_router_weights, sg, dim3(256), 0, st, a.pdl, a.Wr, a.d, a.E,
+                                  static_cast<__nv_bfloat16 *>(wsplit));
     if (e != cudaSuccess) return e;
 
     TcRouterParams p{};
@@ -373,8 +375,7 @@ cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits,
         attr = true;
     }
     const int grid = 2 * pair_blocks(a.T) * splits;
-    router_tc_kernel<<<grid, kThreads, smem, st>>>(mx, mw, p);
-    return cudaGetLastError();
+    return launch_kernel(router_tc_kernel, dim3(grid), dim3(kThreads), smem, st, true, mx, mw, p);
 }
 
 }  // namespace moe

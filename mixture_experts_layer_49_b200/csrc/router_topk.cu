@@ -200,6 +200,7 @@ __device__ __forceinline__ void write_psum(const RouterArgs &a, float (*part)[EP
 
 template <typename TX, int EPT>
 __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
+    pdl_wait_then_release();
     constexpr int VEC = 16 / sizeof(TX);              // x elements per 16-byte load
     constexpr int EW = EPT * 32;                      // expert slots per warp row
     __shared__ float xs[kTok][kKc + 1];
@@ -270,6 +271,7 @@ constexpr int kSelTok = 64;
 template <int EPT>
 __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ parts,
                                                                  int splits) {
+    pdl_wait_then_release();
     __shared__ float part[kThreads / 32][EPT * 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float psum_acc[EPT], sb[EPT];
@@ -308,12 +310,11 @@ __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, c
 
 template <typename TX>
 cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
-    const int blocks = (a.T + kTok - 1) / kTok;
-    if (a.E <= 32) router_topk_kernel<TX, 1><<<blocks, kThreads, 0, st>>>(a);
-    else if (a.E <= 64) router_topk_kernel<TX, 2><<<blocks, kThreads, 0, st>>>(a);
-    else if (a.E <= 128) router_topk_kernel<TX, 4><<<blocks, kThreads, 0, st>>>(a);
-    else router_topk_kernel<TX, 8><<<blocks, kThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    const dim3 blocks((a.T + kTok - 1) / kTok), threads(kThreads);
+    if (a.E <= 32) return launch_kernel(router_topk_kernel<TX, 1>, blocks, threads, 0, st, a.pdl, a);
+    if (a.E <= 64) return launch_kernel(router_topk_kernel<TX, 2>, blocks, threads, 0, st, a.pdl, a);
+    if (a.E <= 128) return launch_kernel(router_topk_kernel<TX, 4>, blocks, threads, 0, st, a.pdl, a);
+    return launch_kernel(router_topk_kernel<TX, 8>, blocks, threads, 0, st, a.pdl, a);
 }
 
 }  // namespace
@@ -332,12 +333,12 @@ cudaError_t launch_router(const RouterArgs &a, bool bf16, cudaStream_t st) {
     float *parts = (splits == 1 && a.logits_out) ? a.logits_out : a.logits_ws;
     cudaError_t e = launch_router_logits_tc(a, parts, splits, st);
     if (e != cudaSuccess) return e;
-    const int blocks = (a.T + kSelTok - 1) / kSelTok;
-    if (a.E <= 32) router_select_kernel<1><<<blocks, kThreads, 0, st>>>(a, parts, splits);
-    else if (a.E <= 64) router_select_kernel<2><<<blocks, kThreads, 0, st>>>(a, parts, splits);
-    else if (a.E <= 128) router_select_kernel<4><<<blocks, kThreads, 0, st>>>(a, parts, splits);
-    else router_select_kernel<8><<<blocks, kThreads, 0, st>>>(a, parts, splits);
-    return cudaGetLastError();
+    const dim3 blocks((a.T + kSelTok - 1) / kSelTok), threads(kThreads);
+    const float *cparts = parts;
+    if (a.E <= 32) return launch_kernel(router_select_kernel<1>, blocks, threads, 0, st, true, a, cparts, splits);
+    if (a.E <= 64) return launch_kernel(router_select_kernel<2>, blocks, threads, 0, st, true, a, cparts, splits);
+    if (a.E <= 128) return launch_kernel(router_select_kernel<4>, blocks, threads, 0, st, true, a, cparts, splits);
+    return launch_kernel(router_select_kernel<8>, blocks, threads, 0, st, true, a, cparts, splits);
 }
 
 }  // namespace moe
