@@ -88,7 +88,12 @@ struct SmemTail {
     int start[kMaxGroups];    // first row of the group this launch computes
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemTail);
+// Epilogue staging: one 2 KiB buffer per epilogue warp (32 rows x 32 bf16),
+// 1024-byte aligned after the tail.
+constexpr uint32_t STG_BYTES = 32 * 32 * 2;
+constexpr size_t kStgOff = (STAGES * STAGE_BYTES + sizeof(SmemTail) + 1023) / 1024 * 1024;
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStgOff + 8 * STG_BYTES;
+static_assert(kSmemBytes <= 227 * 1024, "1-CTA kernel shared memory");
 
 __device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.f + erff(v * 0.70710678118654752f)); }
 __device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
@@ -101,48 +106,84 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
     *reinterpret_cast<uint4 *>(dst) = pk;
 }
 
+// Store one 32-column chunk of the warp's 32 rows (h: this lane's row) with a
+// TMA tensor store: the chunk goes to the warp's 2 KiB staging buffer in the
+// 64-byte swizzled layout (16-byte piece c of row r at piece c ^ ((r / 2) % 4),
+// conflict-free), then one store writes the 32 x 32 block in whole 64-byte row
+// segments.  The previous store from the buffer must have read it first.
+__device__ __forceinline__ void stage_store32(uint32_t stg, const CUtensorMap *tmO, int col0, int row0, const float *h) {
+    const int lane = threadIdx.x & 31;
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(h[2 * i], h[2 * i + 1]);
+        pk[i] = *reinterpret_cast<const uint32_t *>(&b);
+    }
+    if (lane == 0) tma_store_wait_read();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t a = stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
+                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3]) : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmO, stg, col0, row0);
+        tma_store_commit();
+    }
+}
+
 // Epilogue of one accumulator row (this thread's TMEM lane) for one tile:
 // the warp's half of the columns (SwiGLU: gate chunks half*2, half*2+1 and
 // the up chunks 128 columns on; otherwise chunks half*4 .. half*4+3) arrive
-// with one TMEM wait, then the fused activation or bias + gate scale and
-// 16-byte bf16 stores of the valid row's columns below N.
+// with one TMEM wait, then the fused activation or bias + gate scale.  When
+// all 32 rows of the warp are valid, each 32-column chunk leaves through the
+// staging buffer and a TMA store (row0: the warp's first output row);
+// otherwise each valid row stores its columns below N with 16-byte stores.
 template <int MODE>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
-                                             __nv_bfloat16 *orow_ptr, const float *bias, float gscale) {
+                                             __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
+                                             const CUtensorMap *tmO, uint32_t stg, int row0) {
     float v[128];
+    const bool staged = __all_sync(0xffffffffu, valid);
     if (MODE == GM_SWIGLU) {
         const int c0 = half * 2;
         tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + 128 + c0 * 32, taddr + 128 + (c0 + 1) * 32, v);
-        if (!valid) return;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = nt * 128 + (c0 + cc) * 32;
+            float *h = v + cc * 32;                  // in place of the gate values
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float h[8];
+            for (int i = 0; i < 32; ++i) h[i] = silu(h[i]) * v[64 + cc * 32 + i];
+            if (staged) {
+                if (col0 < N) stage_store32(stg, tmO, col0, row0, h);
+            } else if (valid) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) h[i] = silu(v[cc * 32 + u * 8 + i]) * v[64 + cc * 32 + u * 8 + i];
-                if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, h);
+                for (int u = 0; u < 4; ++u)
+                    if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, h + u * 8);
             }
         }
     } else {
         const int c0 = half * 4;
         tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + (c0 + 2) * 32, taddr + (c0 + 3) * 32, v);
-        if (!valid) return;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             const int col0 = nt * BNB + (c0 + cc) * 32;
+            if (col0 >= N) continue;                  // uniform over the warp
+            float *h = v + cc * 32;                  // in place
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int cb = col0 + u * 8;
-                if (cb >= N) continue;
-                float h[8];
+            for (int i = 0; i < 32; ++i) {
+                const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
+                h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
+            }
+            if (staged) {
+                stage_store32(stg, tmO, col0, row0, h);
+            } else if (valid) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float z = v[cc * 32 + u * 8 + i] + (bias ? __ldg(bias + cb + i) : 0.f);
-                    h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
-                }
-                store8(orow_ptr + cb, h);
+                for (int u = 0; u < 4; ++u)
+                    if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, h + u * 8);
             }
         }
     }
@@ -173,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                 const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
-                const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
     pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -303,6 +344,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
+        const uint32_t stg = base + (uint32_t)kStgOff + (uint32_t)(warp - 2) * STG_BYTES;
         int ab = 0;
         uint32_t aphase = 0;
         for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
@@ -327,12 +369,13 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale);
+            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
             if (++ab == 2) { ab = 0; aphase ^= 1u; }
         }
+        if (lane == 0) tma_store_wait_all();            // the staged stores have landed
     }
 
     tc_fence_before();
@@ -377,7 +420,9 @@ struct PairTail {
     int row0[kMaxGroups];
 };
 
-constexpr size_t kPairSmemBytes = 1024 + P_STAGES * P_STAGE_BYTES + sizeof(PairTail);
+constexpr size_t kPairStgOff = (P_STAGES * P_STAGE_BYTES + sizeof(PairTail) + 1023) / 1024 * 1024;
+constexpr size_t kPairSmemBytes = 1024 + kPairStgOff + 8 * STG_BYTES;
+static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
 __device__ __forceinline__ void decode_pair(const PairTail &s, int G, int tile, int &g, int &mt, int &nt) {
     int lo = 0, hi = G - 1;
@@ -404,7 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
-                     const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
     pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -522,6 +567,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
+        const uint32_t stg = base + (uint32_t)kPairStgOff + (uint32_t)(warp - 2) * STG_BYTES;
         int ab = 0;
         uint32_t aphase = 0;
         for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
@@ -543,12 +589,13 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale);
+            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
             if (++ab == 2) { ab = 0; aphase ^= 1u; }
         }
+        if (lane == 0) tma_store_wait_all();            // the staged stores have landed
     }
 
     tc_fence_before();
@@ -592,10 +639,25 @@ bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64
     return r == CUDA_SUCCESS;
 }
 
+// Output map for the staged epilogue stores: bf16 [rows][cols] with row
+// stride ld elements, box 32 x 32, 64-byte swizzle.
+bool make_store_map(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows, uint64_t ld) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int MODE>
 cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
-                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const GemmParams &p, int grid, cudaStream_t st,
-                        bool pdl) {
+                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const CUtensorMap &O, const GemmParams &p,
+                        int grid, cudaStream_t st, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -603,13 +665,14 @@ cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUten
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_kernel(tc_grouped_gemm<MODE>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs, Bs2, p);
+    return launch_kernel(tc_grouped_gemm<MODE>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs, Bs2, O,
+                         p);
 }
 
 template <int MODE>
 cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B,
                              const CUtensorMap &B2, const CUtensorMap &Bs, const CUtensorMap &Bs2,
-                             const GemmParams &p, int num_sms, cudaStream_t st, bool pdl) {
+                             const CUtensorMap &O, const GemmParams &p, int num_sms, cudaStream_t st, bool pdl) {
     static int grid = 0;
     if (grid == 0) {
         cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -632,7 +695,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const 
         grid = 2 * nclusters;
     }
     return launch_kernel(tc_grouped_gemm_pair<MODE>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A, As, B, B2,
-                         Bs, Bs2, p);
+                         Bs, Bs2, O, p);
 }
 
 }  // namespace
@@ -698,12 +761,15 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
         }
         P1su = P1s;
     }
-    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st, a.pdl)
-                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, p1, grid, st, a.pdl);
+    // the first GEMM's output: H [all rows, hF], stored in 32 x 32 blocks
+    CUtensorMap O1;
+    if (!make_store_map(&O1, a.H, a.hF, all_rows, a.hF)) return cudaErrorInvalidValue;
+    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl)
+                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl);
     if (err != cudaSuccess) return err;
     p1.tail_mode = 1;
-    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st, true)
-                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, p1, grid, st, true);
+    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true)
+                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true);
     if (err != cudaSuccess) return err;
 
     // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
@@ -737,10 +803,12 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     } else {
         P2s = P2;
     }
-    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, p2, grid, st, true);
+    CUtensorMap O2;                               // y_perm [all rows, d_model]
+    if (!make_store_map(&O2, a.y_perm, a.d, all_rows, a.d)) return cudaErrorInvalidValue;
+    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, O2, p2, grid, st, true);
     if (err != cudaSuccess) return err;
     p2.tail_mode = 1;
-    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, p2, grid, st, true);
+    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, O2, p2, grid, st, true);
 }
 
 }  // namespace moe
