@@ -329,15 +329,21 @@ def run_ours(args, wl, dev, world, rank):
     kept_np = np.minimum(counts, cap) if cap >= 0 else counts
     flops, alg_bytes, kept_rows = algorithmic_counts(wl, counts, kept_np)
     peaks, peak_src = load_peaks()
-    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    # The step runs back to back for the whole timed region (power-capped
+    # clocks, sw_power_cap active): the sustained bf16 figure is the tensor
+    # peak; the burst figure is reported beside it.
+    t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_tensor_burst = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
     layer_roof_ms = max(t_tensor, t_hbm) * 1e3
+    layer_roof_burst_ms = max(t_tensor_burst, t_hbm) * 1e3
     ffn_ms = stage_avg["grouped_ffn"]
     ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(wl.name)
     result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts,
                   flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
-                  layer_roof_ms=layer_roof_ms, ffn_tflops=ffn_tflops, traffic=traffic,
+                  layer_roof_ms=layer_roof_ms, layer_roof_burst_ms=layer_roof_burst_ms, ffn_tflops=ffn_tflops,
+                  traffic=traffic,
                   loss=float(out.loss.item()), n_dropped=int(out.n_dropped.item()),
                   bound="tensor" if t_tensor >= t_hbm else "hbm",
                   h2d=x_host.numel() * x_host.element_size(),
@@ -395,7 +401,7 @@ def main():
     e2e_tokens_per_s = world * wl.T / (r["e2e_ms"] * 1e-3)
     peaks = r["peaks"]
     tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
-    peak_tensor = peaks["bf16_tflops"]
+    peak_tensor = peaks["bf16_tflops_sustained"]
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
@@ -404,10 +410,16 @@ def main():
         "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
         "layer_roofline": {"bound": r["bound"], "time_ms": r["layer_roof_ms"],
                            "frac": r["layer_roof_ms"] / r["ms"], "flops": r["flops"],
-                           "alg_bytes": r["alg_bytes"], "peak_note": "burst bf16 and copy bandwidth, " + tag},
+                           "alg_bytes": r["alg_bytes"],
+                           "frac_burst": r["layer_roof_burst_ms"] / r["ms"],
+                           "peak_note": "sustained bf16 (timed inside the back-to-back step loop) and copy "
+                                        "bandwidth, " + tag + "; frac_burst against the burst bf16 figure"},
         "roofline": {"kernel": "grouped_ffn (tcgen05 gemm1 + gemm2)", "bound": "tensor",
                      "achieved": r["ffn_tflops"], "peak": peak_tensor, "unit": "TFLOP/s",
-                     "frac": r["ffn_tflops"] / peak_tensor, "traffic": r["traffic"], "peak_note": "burst, " + tag},
+                     "frac": r["ffn_tflops"] / peak_tensor, "traffic": r["traffic"],
+                     "frac_burst": r["ffn_tflops"] / peaks["bf16_tflops"],
+                     "peak_note": "sustained, " + tag + " (the kernel runs inside the back-to-back step loop); "
+                                  "frac_burst against the burst figure"},
         "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
         "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

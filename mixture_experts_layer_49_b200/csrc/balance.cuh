@@ -18,15 +18,17 @@ namespace moe {
 __device__ __forceinline__ double psum_column(const float *psum, int nblk, int E, int e) {
     const int lane = threadIdx.x & 31;
     double s = 0.0;
-    int b = lane;
-    for (; b + 96 < nblk; b += 128) {           // four independent loads in flight
-        const float v0 = psum[(size_t)b * E + e];
-        const float v1 = psum[(size_t)(b + 32) * E + e];
-        const float v2 = psum[(size_t)(b + 64) * E + e];
-        const float v3 = psum[(size_t)(b + 96) * E + e];
-        s += (double)v0; s += (double)v1; s += (double)v2; s += (double)v3;
+    for (int b0 = 0; b0 < nblk; b0 += 32 * 16) {   // sixteen independent loads in flight
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int b = b0 + lane + 32 * j;
+            v[j] = b < nblk ? psum[(size_t)b * E + e] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (b0 + lane + 32 * j < nblk) s += (double)v[j];
     }
-    for (; b < nblk; b += 32) s += (double)psum[(size_t)b * E + e];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     return s;
@@ -42,6 +44,25 @@ __device__ __forceinline__ double loss_tree(double *red) {
     }
     __syncthreads();
     return red[0];
+}
+
+// The same tree run by one warp over contrib[0..E) (zero past E): lane l
+// holds entries l + 32 j; the halving steps 128, 64, 32 are register adds in
+// the same operand order, 16 .. 1 are shuffles.  Every lane returns lane 0's
+// value, which equals loss_tree's bit for bit.
+__device__ __forceinline__ double loss_tree_warp(const double *contrib, int E) {
+    const int lane = threadIdx.x & 31;
+    double v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = lane + 32 * j < E ? contrib[lane + 32 * j] : 0.0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] += v[j + 4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) v[j] += v[j + 2];
+    v[0] += v[1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[0] += __shfl_down_sync(0xffffffffu, v[0], o);
+    return __shfl_sync(0xffffffffu, v[0], 0);
 }
 
 }  // namespace moe

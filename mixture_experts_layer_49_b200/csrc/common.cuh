@@ -15,10 +15,9 @@ namespace moe {
 
 // Workspace header: first 256 bytes of every workspace.
 struct WsHeader {
-    int32_t status;          // first recorded device error (moe_status), 0 = none
-    int32_t detail;          // free-form detail of that error (an index, a stage)
-    int32_t balance_ticket;  // CTAs of the dispatch scan done with their balance terms
-    int32_t pad[61];
+    int32_t status;      // first recorded device error (moe_status), 0 = none
+    int32_t detail;      // free-form detail of that error (an index, a stage)
+    int32_t pad[62];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

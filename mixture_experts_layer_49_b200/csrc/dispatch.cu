@@ -55,69 +55,55 @@ __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, in
 // lane first sums 8 consecutive chunks, then a warp scan of the lane totals),
 // the expert's total count and its kept count.  Experts are independent, so
 // the grid covers them 32 per CTA.  With balance outputs, the same warp
-// computes f_e and P_e (balance.cuh order) and the last CTA to finish adds
-// the loss terms.
+// computes f_e, P_e and the loss term f_e P_e (balance.cuh order; its score
+// sums are loaded before the scan so the two latencies overlap); the permute
+// kernel adds the terms.
 __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
     pdl_wait_then_release();
-    __shared__ double red[256];
-    __shared__ int last;
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
-    if (e < a.E) {
-        const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
-        int32_t *dst = a.chunk_base + (size_t)e * nchunks;
-        int running = 0;
-        for (int c0 = 0; c0 < nchunks; c0 += 256) {
-            int v[8];
+    if (e >= a.E) return;
+    double psum_e = 0.0;
+    const bool bal = a.loss != nullptr;
+    if (bal) psum_e = psum_column(a.psum, a.nblk, a.E, e);
+    const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
+    int32_t *dst = a.chunk_base + (size_t)e * nchunks;
+    int running = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 256) {
+        int v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = c0 + lane * 8 + i;
-                v[i] = c < nchunks ? src[c] : 0;
-            }
-            int tot = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) tot += v[i];
-            int incl = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            int run = running + incl - tot;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = c0 + lane * 8 + i;
-                if (c < nchunks) dst[c] = run;
-                run += v[i];
-            }
-            running += __shfl_sync(0xffffffffu, incl, 31);
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + lane * 8 + i;
+            v[i] = c < nchunks ? src[c] : 0;
         }
-        if (lane == 0) {
-            a.counts[e] = running;
-            a.kept[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
+        int tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tot += v[i];
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
         }
-        if (a.loss) {
-            const double P = psum_column(a.psum, a.nblk, a.E, e) / (double)a.T;
-            const double f = (double)running / ((double)a.T * (double)a.k);
-            if (lane == 0) {
-                a.f[e] = (float)f;
-                a.P[e] = (float)P;
-                a.contrib[e] = f * P;
-            }
+        int run = running + incl - tot;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + lane * 8 + i;
+            if (c < nchunks) dst[c] = run;
+            run += v[i];
         }
+        running += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (a.loss == nullptr) return;                   // uniform over the grid
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(a.ticket, 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!last) return;                               // uniform over the block
-    __threadfence();
-    if (threadIdx.x < 256) red[threadIdx.x] = (int)threadIdx.x < a.E ? __ldcg(a.contrib + threadIdx.x) : 0.0;
-    const double s = loss_tree(red);
-    if (threadIdx.x == 0) {
-        *a.loss = (double)a.E * s;
-        *a.ticket = 0;
+    if (lane == 0) {
+        a.counts[e] = running;
+        a.kept[e] = (a.capacity >= 0 && running > a.capacity) ? a.capacity : running;
+        if (bal) {
+            const double P = psum_e / (double)a.T;
+            const double f = (double)running / ((double)a.T * (double)a.k);
+            a.f[e] = (float)f;
+            a.P[e] = (float)P;
+            a.contrib[e] = f * P;
+        }
     }
 }
 
@@ -161,6 +147,9 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
             a.offsets[E] = running;
             if (a.n_dropped) *a.n_dropped = dropped;
         }
+    } else if (warp == 1 && c == 0 && a.loss) {       // the balance loss from the scan's terms
+        const double sum = loss_tree_warp(a.contrib, E);
+        if (lane == 0) *a.loss = (double)E * sum;
     }
     __syncthreads();
     const int t0 = c * kChunk;
@@ -243,6 +232,10 @@ __global__ void empty_offsets_kernel(DispatchArgs a) {
     pdl_wait_then_release();
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.offsets[e] = 0;
     if (threadIdx.x == 0 && a.n_dropped) *a.n_dropped = 0;
+    if (a.loss && threadIdx.x < 32) {
+        const double sum = loss_tree_warp(a.contrib, a.E);
+        if (threadIdx.x == 0) *a.loss = (double)a.E * sum;
+    }
 }
 
 }  // namespace

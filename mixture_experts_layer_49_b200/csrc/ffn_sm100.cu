@@ -215,7 +215,6 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                 const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
                 const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-    pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -228,6 +227,21 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     constexpr int BNO = (MODE == GM_SWIGLU) ? 128 : 256;   // output columns per tile
     const int G = p.E + (p.has_shared ? 1 : 0);
 
+    // ---- independent of the previous kernel: barriers, TMEM, descriptors
+    if (tid == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 8); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), TMEM_COLS);   // whole warp; address lands in smem
+    if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+    }
+    pdl_wait_then_release();
+    if (tid == 0) s.tile_start[0] = 0;
     // ---- tile table from the device-side offsets
     for (int g = tid; g < G; g += kThreads) {
         const bool sh = g >= p.E;
@@ -246,14 +260,6 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         s.mtiles[g] = mt > 0 ? mt : 1;
         s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
     }
-    if (tid == 0) {
-        s.tile_start[0] = 0;
-        s.abort_flag = 0;
-        for (int i = 0; i < STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 8); }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
     __syncthreads();
     if (warp == 0) {            // inclusive scan of the per-group tile counts
         int carry = 0;
@@ -269,7 +275,6 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             carry += __shfl_sync(0xffffffffu, v, 31);
         }
     }
-    if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), TMEM_COLS);   // whole warp; address lands in smem
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -450,7 +455,6 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
                      const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
-    pdl_wait_then_release();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -465,6 +469,22 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
     constexpr int BNO = (MODE == GM_SWIGLU) ? 128 : 256;
     const int G = p.E + (p.has_shared ? 1 : 0);
 
+    // ---- independent of the previous kernel: barriers, TMEM, descriptors
+    if (tid == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < P_STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 16); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(&s.tmem_base), TMEM_COLS);   // warp 1 of both CTAs
+    if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB2) : "memory");
+    }
+    pdl_wait_then_release();
+    if (tid == 0) s.tile_start[0] = 0;
     for (int g = tid; g < G; g += kThreads) {
         const bool sh = g >= p.E;
         const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
@@ -474,14 +494,6 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
         s.row0[g] = sh ? 0 : p.offsets[g];
         s.mtiles[g] = mt > 0 ? mt : 1;
         s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
-    }
-    if (tid == 0) {
-        s.tile_start[0] = 0;
-        s.abort_flag = 0;
-        for (int i = 0; i < P_STAGES; ++i) { mbar_init(smem_u32(&s.full[i]), 1); mbar_init(smem_u32(&s.empty[i]), 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 16); }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
     if (warp == 0) {
@@ -498,7 +510,6 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             carry += __shfl_sync(0xffffffffu, v, 31);
         }
     }
-    if (warp == 1) tmem_alloc_pair(smem_u32(&s.tmem_base), TMEM_COLS);   // warp 1 of both CTAs
     tc_fence_before();
     cluster_sync();                                  // barriers of both CTAs initialised
     tc_fence_after();

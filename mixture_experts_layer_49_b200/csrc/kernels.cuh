@@ -71,13 +71,13 @@ struct DispatchArgs {
     int32_t *n_dropped;          // device scalar or null
     int32_t *status;             // workspace status word
     int T, d, E, k, capacity;    // capacity < 0: unlimited
-    // Optional (loss != null): the balance statistics, computed in the scan
-    // kernel from the router's per-block score sums.
+    // Optional (loss != null): the balance statistics, f and P computed in the
+    // scan kernel from the router's per-block score sums, the loss added by
+    // the permute kernel (or the empty-input kernel).
     const float *psum;           // [nblk, E]
     float *f, *P;                // [E]
     double *loss;                // device scalar
     double *contrib;             // [E] scratch: f_e P_e
-    int32_t *ticket;             // zero-initialised counter, reset by the last CTA
     int nblk;
     bool pdl;                    // the first launch overlaps the stream's previous kernel
 };

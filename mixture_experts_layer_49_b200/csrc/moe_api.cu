@@ -318,7 +318,6 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     // the balance statistics ride on the dispatch scan
     da.psum = psum; da.f = f; da.P = P; da.loss = loss;
     da.contrib = at<double>(ws, L.contrib);
-    da.ticket = &reinterpret_cast<moe::WsHeader *>(ws)->balance_ticket;
     da.nblk = moe::router_blocks(cfg->T, bf16);
     da.pdl = true;                                 // every launch after the first overlaps its predecessor
     if ((e = moe::launch_dispatch(da, bf16, st)) != cudaSuccess) return cuda_fail(e, "permute");

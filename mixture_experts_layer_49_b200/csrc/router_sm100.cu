@@ -127,6 +127,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int nk = (p.d + RBK - 1) / RBK;
     const int kb0 = split * p.kb_per_split;
     const int kb1 = min(nk, kb0 + p.kb_per_split);
+    // K steps kb0 .. kb1-1 in np contiguous parts (one accumulator each).
+    // Pairs start at different parts (rotation by cluster index), so pairs
+    // running together read different W_r tiles instead of all hitting the
+    // same L2 lines; each part is still summed in ascending K order, so the
+    // result does not depend on the rotation.
+    const int nkl = kb1 - kb0;
+    const int np = min(p.nparts, nkl);
+    const int rot = cl % np;
+    auto part_begin = [&](int part) { return (part * nkl + np - 1) / np; };
 
     if (tid == 0) {
         s.abort_flag = 0;
@@ -145,20 +154,26 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) {
-                    record_error(p.status, MOE_ERR_TIMEOUT, 11);
-                    s.abort_flag = 1;
-                    break;
-                }
-                const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
-                const uint32_t st = base + stage * stage_bytes;
-                if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * stage_bytes);
-                tma_load_2d_pair(st, &tmX, fb, kb * RBK, t0);
+            bool ok = true;
+            for (int pp = 0; pp < np && ok; ++pp) {
+                const int part = (pp + rot) % np;
+                for (int i = part_begin(part); i < part_begin(part + 1); ++i) {
+                    const int kb = kb0 + i;
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) {
+                        record_error(p.status, MOE_ERR_TIMEOUT, 11);
+                        s.abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
+                    const uint32_t st = base + stage * stage_bytes;
+                    if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * stage_bytes);
+                    tma_load_2d_pair(st, &tmX, fb, kb * RBK, t0);
 #pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    tma_load_3d_pair(st + A_BYTES + j * p.b_bytes, &tmW, fb, kb * RBK, (int)rank * (p.n_pad / 2), j);
-                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+                    for (int j = 0; j < 3; ++j)
+                        tma_load_3d_pair(st + A_BYTES + j * p.b_bytes, &tmW, fb, kb * RBK, (int)rank * (p.n_pad / 2), j);
+                    if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+                }
             }
         }
     } else if (warp == 1) {
@@ -166,30 +181,28 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            int prev_part = -1;
-            const int nkl = kb1 - kb0;
-            const int np = min(p.nparts, nkl);
-            for (int i = 0; i < nkl; ++i) {
-                if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) {
-                    record_error(p.status, MOE_ERR_TIMEOUT, 12);
-                    s.abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t st = base + stage * stage_bytes;
-                const int part = i * np / nkl;                   // contiguous K ranges per accumulator
+            for (int pp = 0; pp < np && ok; ++pp) {
+                const int part = (pp + rot) % np;
                 const uint32_t dtm = tmem + (uint32_t)(part * p.pstride);
-                const uint32_t fresh = part != prev_part;
-                prev_part = part;
+                for (int i = part_begin(part); i < part_begin(part + 1); ++i) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) {
+                        record_error(p.status, MOE_ERR_TIMEOUT, 12);
+                        s.abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = base + stage * stage_bytes;
+                    const uint32_t fresh = i == part_begin(part);   // the part's first K step starts its sum
 #pragma unroll
-                for (int j = 0; j < 3; ++j)
+                    for (int j = 0; j < 3; ++j)
 #pragma unroll
-                    for (int k = 0; k < RBK / 16; ++k)
-                        mma_bf16_pair(dtm, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32), p.idesc,
-                                      (fresh && j == 0 && k == 0) ? 0u : 1u);
-                mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
-                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+                        for (int k = 0; k < RBK / 16; ++k)
+                            mma_bf16_pair(dtm, sdesc(st + k * 32), sdesc(st + A_BYTES + j * p.b_bytes + k * 32),
+                                          p.idesc, (fresh && j == 0 && k == 0) ? 0u : 1u);
+                    mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
+                    if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+                }
             }
             if (ok) mma_commit_pair(smem_u32(&s.accf), (uint16_t)0x3);
         }
@@ -212,7 +225,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             // 16-byte vectors need E % 4 == 0 and a 16-byte aligned output
             const bool vec = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
             const bool add_bias = split == 0 && p.logit_bias != nullptr;
-            const int np = min(p.nparts, kb1 - kb0);      // accumulators this split wrote
             for (int c = 0; c < (E + 31) / 32; ++c) {
                 float v[32];
                 __syncwarp();

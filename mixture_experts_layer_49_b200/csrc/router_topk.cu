@@ -265,8 +265,9 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(RouterArgs a) {
 // Selection for bf16 layers: `parts` holds `splits` partial logits [T, E]
 // (offset already added to split 0) from the tensor-core router, added in
 // split order; then the same per-warp selection as the fp32 path.  One CTA
-// takes 64 tokens (two groups of 32), so the score sums have T/64 rows.
-constexpr int kSelTok = 64;
+// takes 32 tokens (many small CTAs keep the SMs evenly loaded), so the score
+// sums have T/32 rows, as for fp32 layers.
+constexpr int kSelTok = 32;
 
 template <int EPT>
 __global__ void __launch_bounds__(kThreads) router_select_kernel(RouterArgs a, const float *__restrict__ parts,
@@ -320,6 +321,7 @@ cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
 }  // namespace
 
 int router_blocks(int T, bool bf16) { return bf16 ? (T + kSelTok - 1) / kSelTok : (T + kTok - 1) / kTok; }
+static_assert(kSelTok % kTok == 0, "selection blocks hold whole 32-token groups");
 
 // bf16 layers: logits on the tensor cores (router_sm100.cu), then the
 // warp-per-token selection; fp32 layers: this FFMA kernel end to end, which

@@ -46,9 +46,9 @@ def cfg(**kw):
 def test_sizes_and_capacity():
     c = cfg()
     assert nat.workspace_size(c) > 0
-    assert nat.router_blocks(c) == 1                     # bf16: 64 tokens per router block
-    assert nat.router_blocks(cfg(T=300)) == 5
-    assert nat.router_blocks(cfg(dtype="f32")) == 2      # fp32: 32 tokens per router block
+    assert nat.router_blocks(c) == 2                     # 32 tokens per router block
+    assert nat.router_blocks(cfg(T=300)) == 10
+    assert nat.router_blocks(cfg(dtype="f32")) == 2
     assert nat.perm_rows(c) == 128
     assert nat.perm_rows(cfg(d_ff_shared=64)) == 128 + 64
     assert nat.capacity(c) == -1

@@ -168,6 +168,11 @@ def test_entry_points(wl, cuda_device):
     # ---- balance statistics
     st.balance()
     bal = oracle.balance(dims, dp["counts"], r["pnorm"])
+    # the forward pass computes them inside the dispatch kernels in the same
+    # reduction order: identical bits
+    out = nat.Outputs(st.cfg, cuda_device)
+    nat.forward(st.cfg, inp, out, st.ws)
+    assert torch.equal(out.f, st.f) and torch.equal(out.P, st.P) and torch.equal(out.loss, st.loss)
     assert abs(float(st.loss.item()) - bal["loss"]) <= TOL_LOSS * bal["loss"]
     np.testing.assert_allclose(st.f.cpu().numpy(), bal["f"], rtol=1e-6)
     np.testing.assert_allclose(st.P.cpu().numpy(), bal["P"], rtol=1e-4, atol=1e-7)
