@@ -40,6 +40,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ----------------------------------------------------------------------- util
+def max_over_ranks(values, world, device):
+    """Per-rank timings reduced to the slowest rank's (all_reduce MAX); with
+    one rank, the values themselves."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(world, T, ms):
+    """Whole-job throughput: every rank runs a replica on its own T tokens, so
+    the job moves world * T tokens per step of the slowest rank."""
+    return world * T / (ms * 1e-3)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -343,10 +358,7 @@ def run_ours(args, wl, dev, world, rank):
     y_host, loss_host = y_host[0], loss_host[0]
 
     # ---- max over ranks
-    tm = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
-    ms, e2e_ms = float(tm[0]), float(tm[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
     counts = out.counts.cpu().numpy()
     cap = nat.capacity(cfg)
@@ -421,8 +433,8 @@ def main():
             torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    tokens_per_s = world * wl.T / (r["ms"] * 1e-3)
-    e2e_tokens_per_s = world * wl.T / (r["e2e_ms"] * 1e-3)
+    tokens_per_s = job_tokens_per_s(world, wl.T, r["ms"])
+    e2e_tokens_per_s = job_tokens_per_s(world, wl.T, r["e2e_ms"])
     peaks = r["peaks"]
     tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
     peak_tensor = peaks["bf16_tflops_sustained"]

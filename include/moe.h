@@ -250,6 +250,16 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, con
  * (a moe_status) and clear it.  Returns MOE_ERR_CUDA if the read fails.   */
 MOE_API moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out);
 
+/* Self-check of the bounded waits that every tensor-core kernel of the
+ * library uses on its pipeline barriers (failure detection without a GPU
+ * fault): one CTA initialises a shared-memory barrier that nothing ever
+ * arrives on and waits on it with the library's bounded wait; after limit_ns
+ * nanoseconds (1 us .. 10 s) the wait gives up, MOE_ERR_TIMEOUT is recorded in
+ * the status word of `ws` (an initialised workspace of at least 256 bytes)
+ * and the kernel returns normally, leaving the context usable.  Read the
+ * outcome with moe_get_device_status.  The paper has no counterpart.        */
+MOE_API moe_status moe_check_wait_timeout(void *ws, uint64_t limit_ns, moe_stream_t stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(moe_status s);
 

@@ -9,6 +9,16 @@
 
 namespace {
 
+// One CTA waits on a barrier nothing arrives on; the bounded wait gives up
+// after limit_ns and the timeout lands in the status word.
+__global__ void wait_timeout_kernel(int32_t *status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    moe::mbar_init(moe::smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!moe::mbar_wait(moe::smem_u32(&bar), 0, limit_ns)) moe::record_error(status, MOE_ERR_TIMEOUT, 77);
+}
+
 thread_local char g_detail[256] = "";
 
 moe_status fail(moe_status s, const char *fmt, const char *what = "") {
@@ -355,6 +365,16 @@ moe_status moe_routing_health(const moe_config *cfg, const int32_t *counts, cons
     cudaError_t e = moe::launch_routing_health(counts, P, out, cfg->T, cfg->top_k, cfg->E,
                                                reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "routing_health");
+}
+
+moe_status moe_check_wait_timeout(void *ws, uint64_t limit_ns, moe_stream_t stream) {
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL%s");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    if (limit_ns < 1000ull || limit_ns > 10000000000ull)
+        return fail(MOE_ERR_INVALID_ARG, "limit_ns outside 1 us .. 10 s%s");
+    wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status_word(ws), limit_ns);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "check_wait_timeout");
 }
 
 moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_out) {

@@ -28,7 +28,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
-           "moe_bias_update", "moe_routing_health")
+           "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout")
 
 
 class MoEError(RuntimeError):
@@ -85,6 +85,8 @@ def lib():
         L.moe_bias_update.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_float, c_vp]
         L.moe_routing_health.restype = ctypes.c_int
         L.moe_routing_health.argtypes = [P(MoeConfig), c_vp, c_vp, c_vp, c_vp]
+        L.moe_check_wait_timeout.restype = ctypes.c_int
+        L.moe_check_wait_timeout.argtypes = [c_vp, ctypes.c_uint64, c_vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_permute_noalloc.argtypes = [P(MoeConfig)] + [c_vp] * 11 + [c_vp]
         _lib = L
@@ -233,6 +235,12 @@ def moe_get_device_status(ws, stream=None) -> int:
     _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(out)),
            "moe_get_device_status")
     return int(out.value)
+
+
+def moe_check_wait_timeout(ws, limit_ns, stream=None):
+    """Launch the bounded-wait self-check (records MOE_ERR_TIMEOUT in ws)."""
+    _check(lib().moe_check_wait_timeout(_p(ws), ctypes.c_uint64(int(limit_ns)), _stream(stream)),
+           "moe_check_wait_timeout")
 
 
 def layer_dtype(cfg):

@@ -114,6 +114,14 @@ def test_workspace_checks():
     assert nat.lib().moe_get_device_status(None, None, ctypes.byref(out)) == nat.MOE_ERR_WORKSPACE
 
 
+def test_wait_timeout_check_arguments():
+    L = nat.lib()
+    assert L.moe_check_wait_timeout(None, 1000000, None) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_check_wait_timeout(ctypes.c_void_p(4096 + 16), 1000000, None) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_check_wait_timeout(ctypes.c_void_p(4096), 10, None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_check_wait_timeout(ctypes.c_void_p(4096), 20 * 10**9, None) == nat.MOE_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for s in range(7):
         assert nat.status_string(s) != "unknown status"
