@@ -12,26 +12,36 @@
 
 namespace moe {
 
-// Column e of psum summed in double by one warp: lane l adds rows l, l + 32,
-// l + 64, ... in order, then the 32 lane sums meet in a butterfly (addition
-// is commutative, so every lane ends with the same value).
-__device__ __forceinline__ double psum_column(const float *psum, int nblk, int E, int e) {
-    const int lane = threadIdx.x & 31;
+// P sums of the 32 experts e0 .. e0+31 in double, by a block of 32 warps.
+// The order, for expert e: residue class w of rows (w, w + 32, w + 64, ...)
+// summed in ascending row order, then the 32 class sums meet in a butterfly
+// over w (addition is commutative, so every lane of the butterfly ends with
+// the same value).  Warp w reads rows of class w, its lane l takes expert
+// e0 + l, so every load is one 128-byte row segment; the class sums cross
+// over through shared memory and warp w then returns expert e0 + w's sum.
+// Every thread of the block must call it; red is a [32][33] shared array.
+__device__ __forceinline__ double psum_block32(const float *psum, int nblk, int E, int e0, double (*red)[33]) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int e = e0 + lane;
     double s = 0.0;
-    for (int b0 = 0; b0 < nblk; b0 += 32 * 16) {   // sixteen independent loads in flight
+    for (int b0 = w; b0 < nblk; b0 += 32 * 16) {     // sixteen independent loads in flight
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const int b = b0 + lane + 32 * j;
-            v[j] = b < nblk ? psum[(size_t)b * E + e] : 0.f;
+            const int b = b0 + 32 * j;
+            v[j] = (b < nblk && e < E) ? psum[(size_t)b * E + e] : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            if (b0 + lane + 32 * j < nblk) s += (double)v[j];
+            if (b0 + 32 * j < nblk) s += (double)v[j];
     }
+    red[w][lane] = s;
+    __syncthreads();
+    double t = red[lane][w];                         // lane = residue class, warp w = expert e0 + w
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    return s;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    __syncthreads();                                 // red may be reused
+    return t;
 }
 
 // The loss from the per-expert terms f_e P_e in red[0..255] (zero past E):

@@ -93,19 +93,22 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     }
 }
 
-// 32 warps; warp w takes experts w, w + 32, ... (P_e by psum_column), then
-// the loss terms meet in loss_tree.  Everything in double; the result does
-// not depend on scheduling and equals the forward pass's (dispatch scan).
+// 32 warps; for each block of 32 experts, the P sums in the balance.cuh order
+// (psum_block32: warp w ends with expert e0 + w), then the loss terms meet in
+// loss_tree.  Everything in double; the result does not depend on scheduling
+// and equals the forward pass's (dispatch scan and permute).
 __global__ void __launch_bounds__(1024) balance_kernel(BalanceArgs a) {
     pdl_wait_then_release();
     __shared__ double red[256];
+    __shared__ double cls[32][33];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x < 256) red[threadIdx.x] = 0.0;
-    __syncthreads();
-    for (int e = warp; e < a.E; e += 32) {
-        const double P = psum_column(a.psum, a.nblk, a.E, e) / (double)a.T;
-        const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
-        if (lane == 0) {
+    for (int e0 = 0; e0 < a.E; e0 += 32) {
+        const double sum = psum_block32(a.psum, a.nblk, a.E, e0, cls);
+        const int e = e0 + warp;
+        if (e < a.E && lane == 0) {
+            const double P = sum / (double)a.T;
+            const double f = (double)a.counts[e] / ((double)a.T * (double)a.k);
             a.f[e] = (float)f;
             a.P[e] = (float)P;
             red[e] = f * P;

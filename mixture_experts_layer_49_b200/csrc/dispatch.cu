@@ -55,17 +55,18 @@ __global__ void __launch_bounds__(kThreads) chunk_hist_kernel(DispatchArgs a, in
 // lane first sums 8 consecutive chunks, then a warp scan of the lane totals),
 // the expert's total count and its kept count.  Experts are independent, so
 // the grid covers them 32 per CTA.  With balance outputs, the same warp
-// computes f_e, P_e and the loss term f_e P_e (balance.cuh order; its score
-// sums are loaded before the scan so the two latencies overlap); the permute
-// kernel adds the terms.
+// computes f_e, P_e and the loss term f_e P_e (balance.cuh order, the score
+// sums read as whole rows of the CTA's 32 experts); the permute kernel adds
+// the terms.
 __global__ void __launch_bounds__(1024) chunk_scan_kernel(DispatchArgs a, int nchunks) {
     pdl_wait_then_release();
+    __shared__ double red[32][33];
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * 32 + (threadIdx.x >> 5);
-    if (e >= a.E) return;
     double psum_e = 0.0;
-    const bool bal = a.loss != nullptr;
-    if (bal) psum_e = psum_column(a.psum, a.nblk, a.E, e);
+    const bool bal = a.loss != nullptr;                    // uniform over the grid
+    if (bal) psum_e = psum_block32(a.psum, a.nblk, a.E, blockIdx.x * 32, red);
+    if (e >= a.E) return;
     const int32_t *src = a.chunk_cnt + (size_t)e * nchunks;
     int32_t *dst = a.chunk_base + (size_t)e * nchunks;
     int running = 0;
