@@ -26,16 +26,6 @@ __device__ __forceinline__ void record_error(int32_t *status, int32_t code, int3
     if (atomicCAS(status, 0, code) == 0) status[1] = detail;
 }
 
-__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
-
-template <typename T> __device__ __forceinline__ float to_f32(T v);
-template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
-
-template <typename T> __device__ __forceinline__ T from_f32(float v);
-template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
-
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -45,8 +35,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
 // Programmatic dependent launch.  Every kernel of the library starts with
 // this: wait until the grids it depends on have completed and their writes

@@ -9,18 +9,25 @@
 // recommend (Router Optimization page, What Most Articles Miss 2; serving
 // tutorial, grouped GEMM remark).
 //
-// Kernel shape (1-CTA version; the CTA-pair version further down shares the
-// roles; one persistent CTA per SM, 320 threads, warp-specialised):
-//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
-//               swizzle) per stage, 4 stages, mbarrier transaction counts
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//               (M=128, N=256, K=16, fp32 accumulators in TMEM), two
-//               256-column accumulators so the epilogue of tile i overlaps
-//               the mainloop of tile i+1
+// Two persistent kernels per GEMM, launched back to back on the stream:
+//   tc_grouped_gemm_pair  one cluster of two CTAs per pair of SMs
+//               (tcgen05.mma.cta_group::2, M = 256, N = 256): every group's
+//               256-row blocks and a last block of more than 128 rows
+//   tc_grouped_gemm       one CTA per SM (M = 128, N = 256): a last block of
+//               1..128 rows, which mostly streams the weights of small experts
+// Roles (both kernels, 320 threads, warp-specialised):
+//   warp 0      TMA producer: A (activations) and B (weights) tiles, 64 deep
+//               in K, 128-byte swizzle, mbarrier transaction counts
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer, fp32
+//               accumulators in TMEM, two 256-column accumulators so the
+//               epilogue of tile i overlaps the mainloop of tile i+1
 //   warps 2..9  epilogue (two warps per TMEM lane quadrant, each taking half
-//               of the columns): tcgen05.ld 32 lanes x 32 columns, fused activation
-//               (SwiGLU: gate and up halves of one N=256 accumulator; GELU:
-//               bias + exact-erf GELU) or fused bias + gate scale, bf16 stores
+//               of the columns): four tcgen05.ld of 32 columns under one
+//               wait, fused activation (SwiGLU: gate and up halves of one
+//               N=256 accumulator; GELU: bias + exact-erf GELU) or fused bias
+//               + gate scale; a warp whose 32 rows are all valid stores
+//               through a 2 KiB swizzled staging buffer and TMA tensor
+//               stores, others store directly
 // Tiles: groups are the routed experts (rows offsets[e]..offsets[e+1] of the
 // packed activations) plus an optional shared expert over all T tokens.  The
 // tile list is built on the device from `offsets` (no host round trip); a
