@@ -78,17 +78,23 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
             }
         }
         const int64_t shared_row = a.rows_routed + t;
-        for (int v = lane; v < nvec; v += 32) {
+        // every lane runs the column loop (the row indices come by shuffle
+        // from lanes 0..k-1); lanes past the row's last vector only idle
+        for (int v0 = 0; v0 < nvec; v0 += 32) {
+            const int v = v0 + lane;
+            const bool in_row = v < nvec;
             float acc[V::N];
 #pragma unroll
             for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
 #pragma unroll 4
             for (int s = 0; s < a.k; ++s) {
                 const int r = __shfl_sync(0xffffffffu, my_row, s);
-                if (r >= 0) V::add(__ldg(yp + (size_t)r * nvec + v), acc);
+                if (in_row && r >= 0) V::add(__ldg(yp + (size_t)r * nvec + v), acc);
             }
-            if (a.has_shared) V::add(__ldg(yp + (size_t)shared_row * nvec + v), acc);
-            y[(size_t)t * nvec + v] = V::pack(acc);
+            if (in_row) {
+                if (a.has_shared) V::add(__ldg(yp + (size_t)shared_row * nvec + v), acc);
+                y[(size_t)t * nvec + v] = V::pack(acc);
+            }
         }
     }
 }

@@ -77,6 +77,10 @@ SMALL = [
     W("soft_mixture_k_eq_E", T=130, d_model=128, E=4, d_ff=128, top_k=4, renorm=0, act="gelu"),
     W("tight_capacity", T=400, d_model=128, E=8, d_ff=128, top_k=2, capacity_factor=0.3,
       logit_skew="normal"),
+    # selection edge cases: every lane keeps a slot (k = 32); eight candidates
+    # per lane with softmax scores (E = 256)
+    W("k32", T=160, d_model=128, E=64, d_ff=128, top_k=32),
+    W("e256_softmax", T=300, d_model=256, E=256, d_ff=64, top_k=4, logit_skew="normal"),
 ]
 
 
