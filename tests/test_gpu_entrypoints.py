@@ -173,6 +173,10 @@ def test_entry_points(wl, cuda_device):
     out = nat.Outputs(st.cfg, cuda_device)
     nat.forward(st.cfg, inp, out, st.ws)
     assert torch.equal(out.f, st.f) and torch.equal(out.P, st.P) and torch.equal(out.loss, st.loss)
+    # in bf16 the forward's first expert GEMM gathers its rows from x by token
+    # instead of reading x_perm: the same operands in the same order, so the
+    # same bits as the entry-point chain
+    assert torch.equal(out.idx, st.idx) and torch.equal(out.y, st.y)
     assert abs(float(st.loss.item()) - bal["loss"]) <= TOL_LOSS * bal["loss"]
     np.testing.assert_allclose(st.f.cpu().numpy(), bal["f"], rtol=1e-6)
     np.testing.assert_allclose(st.P.cpu().numpy(), bal["P"], rtol=1e-4, atol=1e-7)
