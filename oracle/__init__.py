@@ -11,12 +11,20 @@ formulation used to pin the first.
 Inputs: x and expert weights are fp32 arrays or bf16 arrays given as their raw
 uint16 bit patterns; router weights and biases are fp32.
 
+FP8 experts (``e4m3_value``, ``e4m3_round``, ``quantize_rows``,
+``expert_apply_fp8``, ``layer_tokens_fp8``): e4m3 codes with per-channel
+weight scales and per-row activation scales, defined in ``moe_oracle.c``.
+
 Parity pins (tests/test_oracle_pins.py): brute-force top-k on tiny inputs,
 library softmax / sigmoid for the gates, sums of counts, closed-form balance
 loss (exactly 1 under uniform routing, E under collapse), the dense-FFN
 special case (E = 1, k = 1) against a direct matrix product with library
 GELU / SiLU, the full soft mixture (k = E, no renormalisation), and agreement
-with the loop-over-experts formulation.
+with the loop-over-experts formulation.  FP8: every e4m3 code's value and the
+rounding of fp32 values against the library's float8_e4m3fn type and a brute-
+force nearest-code search, the row quantizer's closed facts (largest code 448,
+error within half a step, zero rows), and the FP8 experts against an
+independent loop-over-experts formulation.
 """
 import ctypes
 import os
@@ -47,8 +55,12 @@ def _load():
         lib.oracle_capacity.argtypes = [ctypes.c_double, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         for name in ("oracle_route", "oracle_dispatch", "oracle_balance",
                      "oracle_expert_apply", "oracle_layer_tokens", "oracle_bias_update",
-                     "oracle_routing_health"):
+                     "oracle_routing_health", "oracle_quantize_rows", "oracle_expert_apply_fp8"):
             getattr(lib, name).restype = ctypes.c_int
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_round.restype = ctypes.c_uint8
+        lib.oracle_e4m3_round.argtypes = [ctypes.c_float]
         _lib = lib
     return _lib
 
@@ -234,3 +246,84 @@ def bf16_bits_to_f64(a):
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return a.astype(np.float64)
+
+
+# ---------------------------------------------------------------- FP8 experts
+def e4m3_value(codes):
+    """float64 value of each e4m3 code (NaN for the NaN codes)."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_value(int(v)) for v in c.ravel()], np.float64).reshape(c.shape)
+
+
+def e4m3_round(q):
+    """e4m3 code nearest to each fp32 value (ties to even, saturating at 448)."""
+    lib = _load()
+    q = np.asarray(q, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_round(float(v)) for v in q.ravel()], np.uint8).reshape(q.shape)
+
+
+def quantize_rows(v):
+    """(codes uint8 [rows, cols], scale float32 [rows]) of a float32 matrix."""
+    lib = _load()
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, cols = v.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scale = np.empty(rows, np.float32)
+    lib.oracle_quantize_rows(_ptr(v), ctypes.c_int64(rows), ctypes.c_int32(cols), ctypes.c_int64(cols),
+                             _ptr(codes), _ptr(scale))
+    return codes, scale
+
+
+def _fp8_weights(w):
+    def u8(a):
+        return None if a is None else np.ascontiguousarray(a, dtype=np.uint8)
+    return (u8(w.get("W1")), _f32(w.get("W1_scale")), _f32(w.get("b1")),
+            u8(w.get("Wu")), _f32(w.get("Wu_scale")),
+            u8(w.get("W2")), _f32(w.get("W2_scale")), _f32(w.get("b2")),
+            u8(w.get("Wsg")), _f32(w.get("Wsg_scale")), u8(w.get("Wsu")), _f32(w.get("Wsu_scale")),
+            u8(w.get("Wsd")), _f32(w.get("Wsd_scale")))
+
+
+def expert_apply_fp8(dims, x8, xs, weights, token, expert, scale=None):
+    """out[r] = scale[r] * E8_{expert[r]}(x8[token[r]]) with FP8 experts.
+
+    x8: e4m3 codes [T, d] with row scales xs [T]; weights: W1, Wu, W2 (and
+    Wsg, Wsu, Wsd) as e4m3 codes with per-output-channel scales under the
+    same names + "_scale", biases b1, b2 fp32."""
+    lib = _load()
+    x8 = np.ascontiguousarray(x8, dtype=np.uint8)
+    xs = _f32(xs)
+    token = np.ascontiguousarray(token, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.float64)
+    out = np.empty((len(token), dims.d), np.float64)
+    ws = _fp8_weights(weights)
+    rc = lib.oracle_expert_apply_fp8(ctypes.byref(dims), ctypes.c_int64(len(token)), _ptr(token), _ptr(expert),
+                                     _ptr(sc), _ptr(x8), _ptr(xs), *[_ptr(a) for a in ws], _ptr(out))
+    if rc:
+        raise ValueError("oracle_expert_apply_fp8: bad expert id")
+    return out
+
+
+def layer_tokens_fp8(dims, x8, xs, weights, idx, gate, row_of, tokens):
+    """y[n] for the listed tokens with FP8 experts: the gate-weighted sum of
+    the kept experts (+ the shared expert, weight 1), summed in float64."""
+    idx = np.asarray(idx, np.int32)
+    gate = np.asarray(gate, np.float64)
+    tokens = np.asarray(tokens, np.int32)
+    k = dims.k
+    tok, ex, g, owner = [], [], [], []
+    for n, t in enumerate(tokens):
+        for s in range(k):
+            if row_of is not None and row_of[t, s] < 0:
+                continue
+            tok.append(t); ex.append(idx[t, s]); g.append(gate[t, s]); owner.append(n)
+        if dims.d_ff_shared > 0:
+            tok.append(t); ex.append(dims.E); g.append(1.0); owner.append(n)
+    y = np.zeros((len(tokens), dims.d), np.float64)
+    if tok:
+        rows = expert_apply_fp8(dims, x8, xs, weights, np.array(tok), np.array(ex), np.array(g))
+        for r, n in enumerate(owner):
+            y[n] += rows[r]
+    return y

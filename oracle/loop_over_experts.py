@@ -106,3 +106,117 @@ def layer(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1,
     P = probs.mean(0)
     return dict(y=y, idx=idx, gate=gate, counts=counts, kept=kept, perm_rows=perm_rows,
                 f=f, P=P, loss=float(E * np.sum(f * P)), logits=logits, probs=probs)
+
+
+# ---------------------------------------------------------------- FP8 experts
+# The same layer with FP8 (e4m3) experts, written from the format's bit
+# fields and a nearest-value search over the whole code table (no shared
+# code with the C oracle's closed-form rounding).
+
+def _e4m3_table():
+    """Value of every e4m3 code 0..255 from its sign / exponent / mantissa."""
+    c = np.arange(256)
+    s, e, m = c >> 7, (c >> 3) & 15, c & 7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = np.where(s == 1, -mag, mag)
+    val[(e == 15) & (m == 7)] = np.nan
+    return val
+
+
+E4M3 = _e4m3_table()
+
+
+def e4m3_nearest(q):
+    """Code of the e4m3 value nearest to each float32 q, by searching the
+    table of the 127 finite magnitudes; ties go to the even code; the sign
+    bit follows q's sign (so a negative q that rounds to zero gives -0)."""
+    q = np.asarray(q, np.float32)
+    a = np.abs(q.astype(np.float64)).ravel()
+    mags = E4M3[:127]                                 # codes 0x00 .. 0x7E, increasing
+    dist = np.abs(a[:, None] - mags[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    # among equally near codes prefer the even one (at most two candidates)
+    even = cand & (np.arange(127)[None, :] % 2 == 0)
+    pick = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1))
+    code = pick.astype(np.uint8) | np.where(np.signbit(q.ravel()), 0x80, 0).astype(np.uint8)
+    return code.reshape(q.shape)
+
+
+def bf16_round(h):
+    """Nearest bf16 (ties to even) of float64 values, returned as float64:
+    keep the top 7 fraction bits of the float64 pattern."""
+    h = np.asarray(h, np.float64)
+    bits = h.view(np.uint64)
+    drop = np.uint64(52 - 7)
+    lsb = (bits >> drop) & np.uint64(1)
+    rounded = (bits + (np.uint64(1) << (drop - np.uint64(1))) - np.uint64(1) + lsb) >> drop << drop
+    out = rounded.view(np.float64)
+    return np.where(h == 0, h, out)
+
+
+def quantize_rows_np(v):
+    """Per-row e4m3 quantization in float32 arithmetic: inv = 448 / amax,
+    code = nearest(v * inv), scale = amax / 448."""
+    v = np.asarray(v, np.float32)
+    amax = np.abs(v).max(axis=1)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, np.float32(448.0) / amax, np.float32(0.0)).astype(np.float32)
+    codes = e4m3_nearest((v * inv[:, None]).astype(np.float32))
+    scale = (amax / np.float32(448.0)).astype(np.float32)
+    return codes, scale
+
+
+def dequant_rows(codes, scale):
+    return E4M3[np.asarray(codes, np.uint8)] * np.asarray(scale, np.float64)[..., None]
+
+
+def expert_fn_fp8(act, xd, Wa, Wb, Wo, b_a=None, b_o=None):
+    """One FP8 expert on dequantized rows xd; Wa/Wb/Wo dequantized weights.
+    H is rounded to bf16 and quantized per row before the second product."""
+    a = xd @ Wa.T
+    if act == "gelu":
+        if b_a is not None:
+            a = a + b_a
+        h = a * stats.norm.cdf(a)
+    else:
+        h = a * special.expit(a) * (xd @ Wb.T)
+    hc, hs = quantize_rows_np(bf16_round(h).astype(np.float32))
+    o = dequant_rows(hc, hs) @ Wo.T
+    if b_o is not None:
+        o = o + b_o
+    return o
+
+
+def layer_fp8(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1,
+              logit_bias=None, sel_bias=None):
+    """The layer with FP8 experts.  weights: e4m3 codes W1, Wu, W2 (Wsg, Wsu,
+    Wsd) with per-output-channel scales "<name>_scale", biases b1, b2.
+    Returns dict(y, idx, gate, x8, xs)."""
+    idx, gate, _, _ = route(x, Wr, k, score=score, renorm=renorm, logit_bias=logit_bias, sel_bias=sel_bias)
+    x8, xs = quantize_rows_np(_f64(x).astype(np.float32))
+    xd = dequant_rows(x8, xs)
+    T, d = xd.shape
+    E = np.asarray(Wr).shape[1]
+
+    def wdeq(name):
+        if weights.get(name) is None:
+            return None
+        return E4M3[np.asarray(weights[name], np.uint8)] * np.asarray(weights[name + "_scale"], np.float64)[..., None]
+
+    W1, Wu, W2 = wdeq("W1"), wdeq("Wu"), wdeq("W2")
+    b1 = np.asarray(weights["b1"], np.float64) if weights.get("b1") is not None else None
+    b2 = np.asarray(weights["b2"], np.float64) if weights.get("b2") is not None else None
+    y = np.zeros((T, d), np.float64)
+    for e in range(E):
+        tok, slot = np.nonzero(idx == e)
+        if capacity >= 0:
+            tok, slot = tok[:capacity], slot[:capacity]
+        if len(tok) == 0:
+            continue
+        o = expert_fn_fp8(act, xd[tok], W1[e], None if Wu is None else Wu[e], W2[e],
+                          None if b1 is None else b1[e], None if b2 is None else b2[e])
+        np.add.at(y, tok, o * gate[tok, slot][:, None])
+    if weights.get("Wsg") is not None:
+        y += expert_fn_fp8(act, xd, wdeq("Wsg"), wdeq("Wsu"), wdeq("Wsd"))
+    return dict(y=y, idx=idx, gate=gate, x8=x8, xs=xs)

@@ -444,3 +444,196 @@ int oracle_routing_health(const oracle_dims *dm, const int32_t *counts, const do
     out[2] = (double)mx / ((double)dm->T * (double)dm->k);
     return 0;
 }
+
+/* ---- FP8 (e4m3) experts ----------------------------------------------------
+ * [IS] "Serving: throughput does not scale the way you expect", its list of
+ * consequences for capacity planning: quantize the experts to FP8 (or INT4),
+ * since memory binds.  The pages give no recipe; the reading written out
+ * here is W8A8 e4m3:
+ *   e4m3 (OCP 8-bit floating point, E4M3): sign bit, 4 exponent bits with
+ *   bias 7, 3 mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6;
+ *   no infinities; S.1111.111 is NaN; the largest finite magnitude is 448.
+ *   Expert weights: one e4m3 code per element and one fp32 scale per output
+ *   channel (row of the nn.Linear [out, in] matrix): W[n][j] = code * scale[n].
+ *   Activations (x, and the hidden activation H of each expert): one scale per
+ *   row, from fp32 arithmetic on the row's values v:
+ *     amax  = max_j |v_j|
+ *     inv   = 448 / amax          (fp32 quotient; 0 when amax = 0)
+ *     code  = e4m3 nearest to v_j * inv (fp32 product), ties to the even
+ *             mantissa, magnitudes above 448 saturated to 448, sign kept
+ *     scale = amax / 448          (fp32 quotient)
+ *   H is held in bf16 (nearest, ties to even, from its exact value) before its
+ *   row is quantized.  Everything else is the expert of the bf16 layer, in
+ *   double, on the exactly dequantized values.                              */
+
+/* Value of an e4m3 code (NaN for the two NaN codes).                        */
+double oracle_e4m3_value(uint8_t c)
+{
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Nearest integer to a non-negative x, ties to even.                        */
+static double round_half_even(double x)
+{
+    const double fl = floor(x), diff = x - fl;
+    if (diff > 0.5) return fl + 1.0;
+    if (diff < 0.5) return fl;
+    return fmod(fl, 2.0) == 0.0 ? fl : fl + 1.0;
+}
+
+/* e4m3 code nearest to q (see above).  Within a binade the e4m3 values are
+ * the multiples of step = 2^(e-3) (2^-9 below 2^-6), so the magnitude is
+ * rounded to a multiple of its binade's step; the division is exact.        */
+uint8_t oracle_e4m3_round(float q)
+{
+    const double a = fabs((double)q);
+    const uint8_t sign = signbit(q) ? 0x80 : 0x00;
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        const double n = round_half_even(a / ldexp(1.0, -9));      /* 0 .. 8 */
+        return sign | (uint8_t)(n >= 8.0 ? 0x08 : (int)n);
+    }
+    int x;
+    (void)frexp(a, &x);                      /* a = f * 2^x, f in [0.5, 1)  */
+    int e = x - 1;                           /* 2^e <= a < 2^(e+1), -6..8   */
+    double n = round_half_even(a / ldexp(1.0, e - 3));              /* 8 .. 16 */
+    if (n >= 16.0) { e += 1; n = 8.0; }
+    if (e > 8 || (e == 8 && n > 14.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)n - 8));
+}
+
+/* Per-row quantization of rows x cols fp32 values (row stride ld).          */
+int oracle_quantize_rows(const float *v, int64_t rows, int32_t cols, int64_t ld, uint8_t *codes,
+                         float *scale)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = v + r * ld;
+        float amax = 0.0f;
+        for (int j = 0; j < cols; ++j) {
+            const float a = fabsf(row[j]);
+            if (a > amax) amax = a;
+        }
+        const float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+        for (int j = 0; j < cols; ++j) {
+            const float p = row[j] * inv;
+            codes[r * (int64_t)cols + j] = oracle_e4m3_round(p);
+        }
+        scale[r] = amax / 448.0f;
+    }
+    return 0;
+}
+
+/* Nearest bf16 to h (ties to even), returned as a float (exact).            */
+static float round_bf16(double h)
+{
+    if (h == 0.0 || !isfinite(h)) return (float)h;
+    const double a = fabs(h);
+    int x;
+    (void)frexp(a, &x);                      /* 2^(x-1) <= a < 2^x          */
+    int e = x - 1;
+    if (e < -126) e = -126;                  /* bf16 subnormals: fixed step */
+    const double step = ldexp(1.0, e - 7);   /* 8 significant bits          */
+    const double r = round_half_even(a / step) * step;
+    return (float)(h < 0 ? -r : r);
+}
+
+typedef struct {
+    const oracle_dims *dm;
+    const uint8_t *x8; const float *xs;                     /* [T, d], [T]       */
+    const uint8_t *W1; const float *s1; const float *b1;    /* [E, d_ff, d] ...  */
+    const uint8_t *Wu; const float *su;
+    const uint8_t *W2; const float *s2; const float *b2;    /* [E, d, d_ff], [E, d] */
+    const uint8_t *Wsg; const float *ssg;
+    const uint8_t *Wsu; const float *ssu;
+    const uint8_t *Wsd; const float *ssd;
+} fp8_experts;
+
+static double wq(const uint8_t *W, const float *s, size_t row, size_t cols, size_t j)
+{
+    return oracle_e4m3_value(W[row * cols + j]) * (double)s[row];
+}
+
+/* One FP8 expert on token t (e == E: the shared expert).  hbuf: d_ff doubles,
+ * hf: d_ff floats, hc: d_ff bytes of scratch.                               */
+static void expert_apply_fp8_one(const fp8_experts *w, int64_t t, int e, double *hbuf, float *hf,
+                                 uint8_t *hc, double *out)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const uint8_t *Wa = shared ? w->Wsg : w->W1, *Wb = shared ? w->Wsu : w->Wu, *Wo = shared ? w->Wsd : w->W2;
+    const float *sa = shared ? w->ssg : w->s1, *sb = shared ? w->ssu : w->su, *so = shared ? w->ssd : w->s2;
+    const size_t eb = shared ? 0 : (size_t)e;
+    const double xscale = (double)w->xs[t];
+    for (int j = 0; j < dff; ++j) {
+        double a = 0.0;
+        for (int i = 0; i < d; ++i)
+            a += wq(Wa, sa, eb * dff + j, d, i) * (oracle_e4m3_value(w->x8[(size_t)t * d + i]) * xscale);
+        if (dm->act == 0) {
+            if (!shared && w->b1) a += (double)w->b1[eb * dff + j];
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else {
+            double u = 0.0;
+            for (int i = 0; i < d; ++i)
+                u += wq(Wb, sb, eb * dff + j, d, i) * (oracle_e4m3_value(w->x8[(size_t)t * d + i]) * xscale);
+            hbuf[j] = a / (1.0 + exp(-a)) * u;
+        }
+        hf[j] = round_bf16(hbuf[j]);
+    }
+    float hs;
+    oracle_quantize_rows(hf, 1, dff, dff, hc, &hs);
+    for (int i = 0; i < d; ++i) {
+        double o = 0.0;
+        for (int j = 0; j < dff; ++j)
+            o += wq(Wo, so, eb * d + i, dff, j) * (oracle_e4m3_value(hc[j]) * (double)hs);
+        if (dm->act == 0 && !shared && w->b2) o += (double)w->b2[eb * d + i];
+        out[i] = o;
+    }
+}
+
+typedef struct {
+    fp8_experts w;
+    const int32_t *token; const int32_t *expert; const double *scale; double *out;
+} apply8_ctx;
+
+static void apply8_range(void *vctx, int64_t lo, int64_t hi)
+{
+    apply8_ctx *c = (apply8_ctx *)vctx;
+    const oracle_dims *dm = c->w.dm;
+    const int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    const size_t hn = (size_t)(hmax > 0 ? hmax : 1);
+    double *hbuf = (double *)malloc(sizeof(double) * hn);
+    float *hf = (float *)malloc(sizeof(float) * hn);
+    uint8_t *hc = (uint8_t *)malloc(hn);
+    for (int64_t r = lo; r < hi; ++r) {
+        double *o = c->out + (size_t)r * dm->d;
+        expert_apply_fp8_one(&c->w, c->token[r], c->expert[r], hbuf, hf, hc, o);
+        const double sc = c->scale ? c->scale[r] : 1.0;
+        for (int i = 0; i < dm->d; ++i) o[i] *= sc;
+    }
+    free(hbuf); free(hf); free(hc);
+}
+
+/* out[r,:] = scale[r] * E8_{expert[r]}(x8[token[r],:]) for FP8 experts;
+ * expert == E selects the shared expert.                                    */
+int oracle_expert_apply_fp8(const oracle_dims *dm, int64_t nrows, const int32_t *token,
+                            const int32_t *expert, const double *scale, const uint8_t *x8, const float *xs,
+                            const uint8_t *W1, const float *s1, const float *b1,
+                            const uint8_t *Wu, const float *su,
+                            const uint8_t *W2, const float *s2, const float *b2,
+                            const uint8_t *Wsg, const float *ssg, const uint8_t *Wsu, const float *ssu,
+                            const uint8_t *Wsd, const float *ssd, double *out)
+{
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (expert[r] < 0 || expert[r] > dm->E) return 1;
+        if (expert[r] == dm->E && dm->d_ff_shared <= 0) return 1;
+    }
+    apply8_ctx c = { { dm, x8, xs, W1, s1, b1, Wu, su, W2, s2, b2, Wsg, ssg, Wsu, ssu, Wsd, ssd },
+                     token, expert, scale, out };
+    parallel_for(nrows, dm->nthreads, apply8_range, &c);
+    return 0;
+}
