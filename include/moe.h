@@ -204,6 +204,63 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        double *loss, float *logits_out, int32_t *n_dropped,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- FP8 (e4m3) experts -----------------------------------------------
+ * Quantized experts for serving ("Fine-tuning and serving MoE models",
+ * Serving: throughput does not scale the way you expect, consequences for
+ * capacity planning: quantize the experts to FP8 since memory binds).  The
+ * expert GEMMs run on the tensor cores with e4m3 x e4m3 products and fp32
+ * accumulation (W8A8):
+ *   e4m3: OCP 8-bit float E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa
+ *     bits, no infinities, largest finite 448), one byte per element.
+ *   weights: e4m3 codes in the nn.Linear [out, in] layout stacked over
+ *     experts, one fp32 scale per output channel: W[e][n][j] = code * scale[e][n].
+ *   activations: x and each expert's hidden activation H are quantized per
+ *     row on the device (moe_quantize_rows_e4m3: scale = max|v| / 448, code =
+ *     e4m3(v * 448 / max|v|), round to nearest even, saturating); H is formed
+ *     in bf16 first, as in the bf16 layer.
+ *   Everything else (router, dispatch, gates, combine, statistics) is the
+ *   bf16 layer's.  Only bf16 layers (cfg->dtype == MOE_BF16) with d_model,
+ *   d_ff and d_ff_shared multiples of 16 (else MOE_ERR_UNSUPPORTED).
+ * All pointers in the struct are device pointers; the struct itself is a
+ * host object read during the call.                                        */
+typedef struct {
+    const uint8_t *W1;    const float *W1_scale;     /* [E, d_ff, d_model], [E, d_ff]   */
+    const uint8_t *Wu;    const float *Wu_scale;     /* SwiGLU W_up (same shapes), else NULL */
+    const uint8_t *W2;    const float *W2_scale;     /* [E, d_model, d_ff], [E, d_model] */
+    const uint8_t *Wsh_g; const float *Wsh_g_scale;  /* shared expert [d_ff_shared, d_model],
+                                                        [d_ff_shared], or NULL          */
+    const uint8_t *Wsh_u; const float *Wsh_u_scale;  /* SwiGLU shared W_up, or NULL      */
+    const uint8_t *Wsh_d; const float *Wsh_d_scale;  /* [d_model, d_ff_shared], [d_model] */
+} moe_fp8_experts;
+
+/* Per-row e4m3 quantization of a bf16 matrix: for each of `rows` rows of
+ * `cols` values (row stride ld_in elements), amax = max |v| (fp32),
+ * codes[r, j] = e4m3(v_j * (448 / amax)) (0 for a zero row; correctly rounded
+ * fp32 quotient and product, nearest-even conversion, saturating at 448),
+ * scale[r] = amax / 448.  codes: row stride ld_out bytes.  cols, ld_in and
+ * ld_out multiples of 8; `in` 16-byte aligned, `codes` 8-byte aligned.     */
+MOE_API moe_status moe_quantize_rows_e4m3(const void *in, int64_t rows, int32_t cols, int64_t ld_in,
+                                          uint8_t *codes, int64_t ld_out, float *scale, moe_stream_t stream);
+
+/* moe_grouped_ffn with FP8 experts.  x8_perm [T*top_k, d_model] e4m3 codes of
+ * the packed rows with their row scales x8_perm_scale [T*top_k]; x8 / x8_scale
+ * the codes and scales of x [T, d_model] (the shared expert's input, NULL
+ * without one); b1, b2 fp32 as in moe_grouped_ffn.  Output y_perm as in
+ * moe_grouped_ffn (bf16).  H, its codes and scales live in ws.             */
+MOE_API moe_status moe_grouped_ffn_fp8(const moe_config *cfg, const uint8_t *x8_perm, const float *x8_perm_scale,
+                                       const int32_t *offsets, const float *row_gate, const moe_fp8_experts *w,
+                                       const float *b1, const float *b2, const uint8_t *x8, const float *x8_scale,
+                                       void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with FP8 experts: router on the bf16 x, then x quantized per
+ * row, the permute of its codes, the e4m3 grouped FFN, combine, statistics.
+ * Arguments and outputs as in moe_forward, the expert weights in *w.       */
+MOE_API moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr,
+                                   const float *logit_bias, const float *sel_bias, const moe_fp8_experts *w,
+                                   const float *b1, const float *b2, void *y, int32_t *idx, float *gate,
+                                   int32_t *counts, float *f, float *P, double *loss, float *logits_out,
+                                   int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Auxiliary-loss-free bias update, to run after a training step on the
  * counts that step's routing produced ("Fine-Tuning Mixture of Experts (MoE)
  * Models: Router Optimization Techniques", How It Works 2, and its router

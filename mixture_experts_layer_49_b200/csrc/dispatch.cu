@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
                 row = offs[e] + rank;
                 a.row_token[row] = t;
                 a.row_gate[row] = a.gate[(size_t)t0 * k + p];
+                if (a.row_scale) a.row_scale[row] = a.x_scale[t];
             }
             a.row_of[(size_t)t0 * k + p] = row;
             list[p] = make_int2(row, t);
@@ -243,7 +244,7 @@ __global__ void empty_offsets_kernel(DispatchArgs a) {
 
 int dispatch_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 
-cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
+cudaError_t launch_dispatch(const DispatchArgs &a, int x_bytes, cudaStream_t st) {
     const int nchunks = dispatch_chunks(a.T);
     cudaError_t e = cudaSuccess;
     if (nchunks > 0) e = launch_kernel(chunk_hist_kernel, dim3(nchunks), dim3(kThreads), 0, st, a.pdl, a, nchunks);
@@ -252,7 +253,8 @@ cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (nchunks == 0)             // no tokens: every count is zero, offsets all zero
         return launch_kernel(empty_offsets_kernel, dim3(1), dim3(256), 0, st, true, a);
-    if (bf16) return launch_kernel(permute_kernel<__nv_bfloat16>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
+    if (x_bytes == 1) return launch_kernel(permute_kernel<uint8_t>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
+    if (x_bytes == 2) return launch_kernel(permute_kernel<__nv_bfloat16>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
     return launch_kernel(permute_kernel<float>, dim3(nchunks), dim3(kPermThreads), 0, st, true, a, nchunks);
 }
 

@@ -62,6 +62,9 @@ constexpr int kMaxGroups = 257;
 enum { GM_SWIGLU = 0, GM_GELU = 1, GM_DOWN = 2 };
 
 constexpr uint32_t kIdesc = make_idesc_bf16(BM, BNB);   // M=128, N=256
+constexpr uint32_t kIdescF8 = make_idesc_e4m3(BM, BNB);
+// K elements per stage: one 128-byte swizzle row of bf16 or of e4m3
+template <bool F8> constexpr int bk_elems() { return F8 ? 128 : 64; }
 
 struct GemmParams {
     const int32_t *offsets;   // [E+1]
@@ -79,6 +82,14 @@ struct GemmParams {
     int tail_mode;            // 1-CTA kernel: 0 all rows; 1 only a group's last rows
                               // when rows % 256 is in 1..128 (the rest runs in pair tiles)
     uint64_t timeout_ns;
+    // e4m3 operands: the accumulator is scaled by its A row's scale and its
+    // output column's scale before the epilogue's arithmetic
+    const float *row_scale;         // routed groups: scale of packed A row r
+    const float *shared_row_scale;  // shared group: scale of A row shared_a_row + i
+    const float *col_scale;         // [E, N_routed] (SwiGLU: the gate projection)
+    const float *col_scale2;        // [E, N_routed] SwiGLU up projection
+    const float *sh_col_scale;      // [N_shared]
+    const float *sh_col_scale2;     // [N_shared]
 };
 
 struct SmemTail {
@@ -149,10 +160,11 @@ __device__ __forceinline__ void stage_store32(uint32_t stg, const CUtensorMap *t
 // all 32 rows of the warp are valid, each 32-column chunk leaves through the
 // staging buffer and a TMA store (row0: the warp's first output row);
 // otherwise each valid row stores its columns below N with 16-byte stores.
-template <int MODE>
+template <int MODE, bool F8>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
                                              __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
-                                             const CUtensorMap *tmO, uint32_t stg, int row0) {
+                                             const CUtensorMap *tmO, uint32_t stg, int row0, float rscale,
+                                             const float *cs, const float *cs2) {
     float v[128];
     const bool staged = __all_sync(0xffffffffu, valid);
     if (MODE == GM_SWIGLU) {
@@ -162,6 +174,14 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = nt * 128 + (c0 + cc) * 32;
             float *h = v + cc * 32;                  // in place of the gate values
+            if (F8) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool in = col0 + i < N;
+                    h[i] *= rscale * (in ? __ldg(cs + col0 + i) : 0.f);
+                    v[64 + cc * 32 + i] *= rscale * (in ? __ldg(cs2 + col0 + i) : 0.f);
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) h[i] = silu(h[i]) * v[64 + cc * 32 + i];
             if (staged) {
@@ -182,7 +202,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
             float *h = v + cc * 32;                  // in place
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
+                const float acc = F8 ? h[i] * (rscale * (col0 + i < N ? __ldg(cs + col0 + i) : 0.f)) : h[i];
+                const float z = acc + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
                 h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
             }
             if (staged) {
@@ -216,7 +237,7 @@ __device__ __forceinline__ void fail(SmemTail &s, const GemmParams &p, int where
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
@@ -298,7 +319,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 decode(s, G, tile, g, mt, nt);
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
-                const int nk = (K + BK - 1) / BK;
+                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 const int a_row = sh ? (int)p.shared_a_row + s.start[g] + mt * BM : s.row0[g] + mt * BM;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = sh ? &tmBs : &tmB;
@@ -308,12 +329,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail(s, p, 1); break; }
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(smA + stage * A_BYTES, mA, fb, kb * BK, a_row);
+                    tma_load_2d(smA + stage * A_BYTES, mA, fb, kb * bk_elems<F8>(), a_row);
                     if (MODE == GM_SWIGLU) {
-                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * 128, e);
-                        tma_load_3d(smB + stage * B_BYTES + B_BYTES / 2, mB2, fb, kb * BK, nt * 128, e);
+                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * bk_elems<F8>(), nt * 128, e);
+                        tma_load_3d(smB + stage * B_BYTES + B_BYTES / 2, mB2, fb, kb * bk_elems<F8>(), nt * 128, e);
                     } else {
-                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * BK, nt * BNB, e);
+                        tma_load_3d(smB + stage * B_BYTES, mB, fb, kb * bk_elems<F8>(), nt * BNB, e);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -330,7 +351,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 int g, mt, nt;
                 decode(s, G, tile, g, mt, nt);
                 const int K = g >= p.E ? p.K_shared : p.K_routed;
-                const int nk = (K + BK - 1) / BK;
+                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail(s, p, 2); break; }
                 tc_fence_after();
                 const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
@@ -341,7 +362,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     const uint32_t a0 = smA + stage * A_BYTES, b0 = smB + stage * B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdesc, (kb | k) ? 1u : 0u);
+                        if (F8)
+                            mma_e4m3(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescF8, (kb | k) ? 1u : 0u);
+                        else
+                            mma_bf16(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdesc, (kb | k) ? 1u : 0u);
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -381,7 +405,16 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane));
+            float rscale = 0.f;
+            const float *cs = nullptr, *cs2 = nullptr;
+            if (F8) {
+                const int64_t arow = sh ? p.shared_a_row + s.start[g] + grow : orow;
+                if (valid) rscale = __ldg((sh ? p.shared_row_scale : p.row_scale) + arow);
+                cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
+                cs2 = sh ? p.sh_col_scale2 : (p.col_scale2 ? p.col_scale2 + (size_t)g * p.N_routed : nullptr);
+            }
+            epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
+                                   rscale, cs, cs2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
@@ -418,6 +451,7 @@ constexpr uint32_t P_B_BYTES = 128 * BK * 2;        // 16 KiB: this CTA's half o
 constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int PM = 2 * BM;                          // rows per pair tile
 constexpr uint32_t kIdescPair = make_idesc_bf16(PM, BNB);
+constexpr uint32_t kIdescPairF8 = make_idesc_e4m3(PM, BNB);
 
 struct PairTail {
     uint64_t full[P_STAGES];     // rank 0's are used
@@ -456,7 +490,7 @@ __device__ __forceinline__ void fail_pair(PairTail &s, const GemmParams &p, int 
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
@@ -533,7 +567,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 decode_pair(s, G, tile, g, mt, nt);
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
-                const int nk = (K + BK - 1) / BK;
+                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 const int a_row = (sh ? (int)p.shared_a_row : s.row0[g]) + mt * PM + (int)rank * BM;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = (MODE == GM_SWIGLU && rank == 1) ? (sh ? &tmBs2 : &tmB2) : (sh ? &tmBs : &tmB);
@@ -543,8 +577,8 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 21); break; }
                     const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * P_STAGE_BYTES);
-                    tma_load_2d_pair(smA + stage * P_A_BYTES, mA, fb, kb * BK, a_row);
-                    tma_load_3d_pair(smB + stage * P_B_BYTES, mB, fb, kb * BK, b_row, e);
+                    tma_load_2d_pair(smA + stage * P_A_BYTES, mA, fb, kb * bk_elems<F8>(), a_row);
+                    tma_load_3d_pair(smB + stage * P_B_BYTES, mB, fb, kb * bk_elems<F8>(), b_row, e);
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -560,7 +594,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 int g, mt, nt;
                 decode_pair(s, G, tile, g, mt, nt);
                 const int K = g >= p.E ? p.K_shared : p.K_routed;
-                const int nk = (K + BK - 1) / BK;
+                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 22); break; }
                 tc_fence_after();
                 const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
@@ -571,7 +605,10 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     const uint32_t a0 = smA + stage * P_A_BYTES, b0 = smB + stage * P_B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | k) ? 1u : 0u);
+                        if (F8)
+                            mma_e4m3_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPairF8, (kb | k) ? 1u : 0u);
+                        else
+                            mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | k) ? 1u : 0u);
                     mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -607,7 +644,16 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            epilogue_row<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane));
+            float rscale = 0.f;
+            const float *cs = nullptr, *cs2 = nullptr;
+            if (F8) {
+                const int64_t arow = sh ? p.shared_a_row + grow : orow;
+                if (valid) rscale = __ldg((sh ? p.shared_row_scale : p.row_scale) + arow);
+                cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
+                cs2 = sh ? p.sh_col_scale2 : (p.col_scale2 ? p.col_scale2 + (size_t)g * p.N_routed : nullptr);
+            }
+            epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
+                                   rscale, cs, cs2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
@@ -639,19 +685,21 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// bf16 tensor [outer][mid][inner] (inner contiguous), box {64, box_mid(, 1)}.
-// rank 2 maps (A operands) ignore `outer`; rank 3 maps (expert-stacked B
-// operands) are indexed by expert in the third coordinate.
+// Tensor [outer][mid][inner] (inner contiguous) of bf16 (esize 2) or e4m3
+// codes (esize 1), box {one 128-byte row of elements, box_mid(, 1)}.  rank 2
+// maps (A operands) ignore `outer`; rank 3 maps (expert-stacked B operands)
+// are indexed by expert in the third coordinate.
 bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
-              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid) {
+              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, int esize = 2) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     if (outer_stride_elems == 0) outer_stride_elems = mid * mid_stride_elems;
     cuuint64_t dims[3] = {inner, mid, outer};
-    cuuint64_t strides[2] = {mid_stride_elems * 2, outer_stride_elems * 2};
-    cuuint32_t box[3] = {(cuuint32_t)BK, box_mid, 1};
+    cuuint64_t strides[2] = {mid_stride_elems * esize, outer_stride_elems * esize};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / esize), box_mid, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+    const CUtensorMapDataType dt = esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = enc(m, dt, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -672,28 +720,28 @@ bool make_store_map(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
                         const CUtensorMap &Bs, const CUtensorMap &Bs2, const CUtensorMap &O, const GemmParams &p,
                         int grid, cudaStream_t st, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_kernel(tc_grouped_gemm<MODE>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs, Bs2, O,
-                         p);
+    return launch_kernel(tc_grouped_gemm<MODE, F8>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs,
+                         Bs2, O, p);
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B,
                              const CUtensorMap &B2, const CUtensorMap &Bs, const CUtensorMap &Bs2,
                              const CUtensorMap &O, const GemmParams &p, int num_sms, cudaStream_t st, bool pdl) {
     static int grid = 0;
     if (grid == 0) {
-        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kPairSmemBytes);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
@@ -708,11 +756,11 @@ cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_grouped_gemm_pair<MODE>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_grouped_gemm_pair<MODE, F8>, &cfg);
         if (e != cudaSuccess || nclusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
         grid = 2 * nclusters;
     }
-    return launch_kernel(tc_grouped_gemm_pair<MODE>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A, As, B, B2,
+    return launch_kernel(tc_grouped_gemm_pair<MODE, F8>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A, As, B, B2,
                          Bs, Bs2, O, p);
 }
 
@@ -720,9 +768,15 @@ cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const 
 
 // Each GEMM runs as two launches on the stream: the CTA-pair kernel over the
 // 256-row blocks of every group (and a last block of > 128 rows), then the
-// 1-CTA kernel over the remaining last blocks of 1..128 rows.
-cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
-    if (a.T == 0) return cudaSuccess;
+// 1-CTA kernel over the remaining last blocks of 1..128 rows.  With e4m3
+// experts the first GEMM reads e4m3 x rows and weights and still writes H in
+// bf16; H is then quantized per row (kept routed rows, then the shared rows)
+// and the second GEMM reads the e4m3 H.
+namespace {
+
+template <bool F8>
+cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
+    constexpr int es = F8 ? 1 : 2;                 // bytes per A / B element
     const bool swiglu = a.act == MOE_ACT_SWIGLU;
     const bool has_sh = a.S > 0;
     const uint64_t routed_rows = (uint64_t)a.T * a.k;
@@ -733,18 +787,18 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     // ---- GEMM 1: H = act(X W1^T [+ b1])   (A: x_perm / x, B: W1 (+Wu) / Wsg (+Wsu))
     CUtensorMap A1, A1s, B1, B1u, B1s, B1su;
     const uint32_t box1 = swiglu ? 128 : 256;
-    if (!make_map(&A1, 2, a.x_perm, a.d, routed_rows, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&B1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
+    if (!make_map(&A1, 2, a.x_perm, a.d, routed_rows, 1, a.d, 0, BM, es)) return cudaErrorInvalidValue;
+    if (!make_map(&B1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1, es)) return cudaErrorInvalidValue;
     if (swiglu) {
-        if (!make_map(&B1u, 3, a.Wu, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1)) return cudaErrorInvalidValue;
+        if (!make_map(&B1u, 3, a.Wu, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, box1, es)) return cudaErrorInvalidValue;
     } else {
         B1u = B1;
     }
     if (has_sh) {
-        if (!make_map(&A1s, 2, a.x, a.d, a.T, 1, a.d, 0, BM)) return cudaErrorInvalidValue;
-        if (!make_map(&B1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, box1)) return cudaErrorInvalidValue;
+        if (!make_map(&A1s, 2, a.x, a.d, a.T, 1, a.d, 0, BM, es)) return cudaErrorInvalidValue;
+        if (!make_map(&B1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, box1, es)) return cudaErrorInvalidValue;
         if (swiglu) {
-            if (!make_map(&B1su, 3, a.Wsu, a.d, a.S, 1, a.d, 0, box1)) return cudaErrorInvalidValue;
+            if (!make_map(&B1su, 3, a.Wsu, a.d, a.S, 1, a.d, 0, box1, es)) return cudaErrorInvalidValue;
         } else {
             B1su = B1s;
         }
@@ -765,15 +819,23 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p1.shared_a_row = 0;
     p1.shared_out_row = a.shared_base;
     p1.timeout_ns = timeout_ns;
+    if (F8) {
+        p1.row_scale = a.xperm_scale;
+        p1.shared_row_scale = a.x_scale;
+        p1.col_scale = a.W1s;
+        p1.col_scale2 = swiglu ? a.Wus : nullptr;
+        p1.sh_col_scale = a.Wsgs;
+        p1.sh_col_scale2 = swiglu ? a.Wsus : nullptr;
+    }
     // pair kernel: B boxes of 128 rows (each CTA loads half of the tile's B rows)
     CUtensorMap P1, P1u, P1s, P1su;
     if (swiglu) {
         P1 = B1; P1u = B1u; P1s = B1s; P1su = B1su;
     } else {
-        if (!make_map(&P1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, 128)) return cudaErrorInvalidValue;
+        if (!make_map(&P1, 3, a.W1, a.d, a.F, a.E, a.d, (uint64_t)a.F * a.d, 128, es)) return cudaErrorInvalidValue;
         P1u = P1;
         if (has_sh) {
-            if (!make_map(&P1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, 128)) return cudaErrorInvalidValue;
+            if (!make_map(&P1s, 3, a.Wsg, a.d, a.S, 1, a.d, 0, 128, es)) return cudaErrorInvalidValue;
         } else {
             P1s = P1;
         }
@@ -782,21 +844,46 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     // the first GEMM's output: H [all rows, hF], stored in 32 x 32 blocks
     CUtensorMap O1;
     if (!make_store_map(&O1, a.H, a.hF, all_rows, a.hF)) return cudaErrorInvalidValue;
-    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl)
-                             : launch_gemm_pair<GM_GELU>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl);
+    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl)
+                             : launch_gemm_pair<GM_GELU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl);
     if (err != cudaSuccess) return err;
     p1.tail_mode = 1;
-    err = swiglu ? launch_gemm<GM_SWIGLU>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true)
-                 : launch_gemm<GM_GELU>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true);
+    err = swiglu ? launch_gemm<GM_SWIGLU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true)
+                 : launch_gemm<GM_GELU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true);
     if (err != cudaSuccess) return err;
 
-    // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H, B: W2 / Wsd)
+    // ---- e4m3: quantize H per row (kept routed rows, then the shared rows)
+    if (F8) {
+        QuantArgs q{};
+        q.in = static_cast<const __nv_bfloat16 *>(a.H);
+        q.ld_in = a.hF;
+        q.out = a.H8;
+        q.ld_out = a.hF;
+        q.scale = a.h_scale;
+        q.rows = (int64_t)routed_rows;
+        q.row0 = 0;
+        q.cols = a.F;
+        q.rows_limit = a.offsets + a.E;
+        q.num_sms = a.num_sms;
+        q.pdl = true;
+        if ((err = launch_quant_rows(q, st)) != cudaSuccess) return err;
+        if (has_sh) {
+            q.rows = a.T;
+            q.row0 = a.shared_base;
+            q.cols = a.S;
+            q.rows_limit = nullptr;
+            if ((err = launch_quant_rows(q, st)) != cudaSuccess) return err;
+        }
+    }
+
+    // ---- GEMM 2: Y = gate * (H W2^T [+ b2])   (A: H / H8, B: W2 / Wsd)
+    const void *Ain = F8 ? static_cast<const void *>(a.H8) : a.H;
     CUtensorMap A2, A2s, B2m, B2s;
-    if (!make_map(&A2, 2, a.H, a.F, all_rows, 1, a.hF, 0, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&B2m, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, BNB)) return cudaErrorInvalidValue;
+    if (!make_map(&A2, 2, Ain, a.F, all_rows, 1, a.hF, 0, BM, es)) return cudaErrorInvalidValue;
+    if (!make_map(&B2m, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, BNB, es)) return cudaErrorInvalidValue;
     if (has_sh) {
-        if (!make_map(&A2s, 2, a.H, a.S, all_rows, 1, a.hF, 0, BM)) return cudaErrorInvalidValue;
-        if (!make_map(&B2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, BNB)) return cudaErrorInvalidValue;
+        if (!make_map(&A2s, 2, Ain, a.S, all_rows, 1, a.hF, 0, BM, es)) return cudaErrorInvalidValue;
+        if (!make_map(&B2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, BNB, es)) return cudaErrorInvalidValue;
     } else {
         A2s = A2; B2s = B2m;
     }
@@ -814,19 +901,32 @@ cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     p2.shared_a_row = a.shared_base;
     p2.shared_out_row = a.shared_base;
     p2.timeout_ns = timeout_ns;
+    if (F8) {
+        p2.row_scale = a.h_scale;
+        p2.shared_row_scale = a.h_scale;
+        p2.col_scale = a.W2s;
+        p2.sh_col_scale = a.Wsds;
+    }
     CUtensorMap P2, P2s;
-    if (!make_map(&P2, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&P2, 3, a.W2, a.F, a.d, a.E, a.F, (uint64_t)a.d * a.F, 128, es)) return cudaErrorInvalidValue;
     if (has_sh) {
-        if (!make_map(&P2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, 128)) return cudaErrorInvalidValue;
+        if (!make_map(&P2s, 3, a.Wsd, a.S, a.d, 1, a.S, 0, 128, es)) return cudaErrorInvalidValue;
     } else {
         P2s = P2;
     }
     CUtensorMap O2;                               // y_perm [all rows, d_model]
     if (!make_store_map(&O2, a.y_perm, a.d, all_rows, a.d)) return cudaErrorInvalidValue;
-    err = launch_gemm_pair<GM_DOWN>(A2, A2s, P2, P2, P2s, P2s, O2, p2, grid, st, true);
+    err = launch_gemm_pair<GM_DOWN, F8>(A2, A2s, P2, P2, P2s, P2s, O2, p2, grid, st, true);
     if (err != cudaSuccess) return err;
     p2.tail_mode = 1;
-    return launch_gemm<GM_DOWN>(A2, A2s, B2m, B2m, B2s, B2s, O2, p2, grid, st, true);
+    return launch_gemm<GM_DOWN, F8>(A2, A2s, B2m, B2m, B2s, B2s, O2, p2, grid, st, true);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
+    if (a.T == 0) return cudaSuccess;
+    return a.f8 ? run_ffn<true>(a, st) : run_ffn<false>(a, st);
 }
 
 }  // namespace moe

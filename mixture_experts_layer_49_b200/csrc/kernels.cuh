@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -68,6 +69,8 @@ struct DispatchArgs {
     int32_t *row_token;          // [T*k]
     float *row_gate;             // [T*k]
     void *x_perm;                // [T*k, d]
+    const float *x_scale;        // [T] per-row scales of e4m3 x, or null
+    float *row_scale;            // [T*k]: x_scale of each packed row's token, or null
     int32_t *n_dropped;          // device scalar or null
     int32_t *status;             // workspace status word
     int T, d, E, k, capacity;    // capacity < 0: unlimited
@@ -82,7 +85,8 @@ struct DispatchArgs {
     bool pdl;                    // the first launch overlaps the stream's previous kernel
 };
 int dispatch_chunks(int T);
-cudaError_t launch_dispatch(const DispatchArgs &a, bool bf16, cudaStream_t st);
+// x_bytes: bytes per element of x and x_perm (4 fp32, 2 bf16, 1 e4m3 codes)
+cudaError_t launch_dispatch(const DispatchArgs &a, int x_bytes, cudaStream_t st);
 
 // Grouped expert FFN.  Group g < E is routed expert g (rows offsets[g] ..
 // offsets[g+1] of x_perm / H / y_perm); group E is the shared expert (rows
@@ -103,9 +107,36 @@ struct FfnArgs {
     int64_t shared_base;         // = T*k
     int num_sms;
     bool pdl;                    // the first launch overlaps the stream's previous kernel
+    // e4m3 experts (bf16 layers): x_perm and x hold e4m3 codes with per-row
+    // scales, the weights e4m3 codes with per-output-channel scales; the
+    // first GEMM's bf16 H is quantized per row into H8 for the second GEMM
+    bool f8;
+    const float *xperm_scale;    // [T*k] scale of each packed row
+    const float *x_scale;        // [T] (shared expert rows)
+    const float *W1s, *Wus, *W2s;      // [E, F], [E, F], [E, d]
+    const float *Wsgs, *Wsus, *Wsds;   // [S], [S], [d]
+    uint8_t *H8;                 // [T*k (+T), hF] codes
+    float *h_scale;              // [T*k (+T)]
 };
 cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st);
+
+// Per-row e4m3 quantization of bf16 rows (row0 + r for r < rows, or fewer
+// when rows_limit points at a smaller device count): in [.., ld_in] bf16,
+// out [.., ld_out] e4m3 codes, scale [..] fp32.  cols % 8 == 0.
+struct QuantArgs {
+    const __nv_bfloat16 *in;
+    int64_t ld_in;
+    uint8_t *out;
+    int64_t ld_out;
+    float *scale;
+    int64_t rows, row0;
+    int cols;
+    const int32_t *rows_limit;   // device count of rows to quantize, or null
+    int num_sms;
+    bool pdl;                    // the launch overlaps the stream's previous kernel
+};
+cudaError_t launch_quant_rows(const QuantArgs &a, cudaStream_t st);
 
 struct CombineArgs {
     const void *y_perm;

@@ -34,7 +34,11 @@ moe_status cuda_fail(cudaError_t e, const char *where) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-    size_t router_w, logits, psum, chunk_cnt, chunk_base, kept, contrib, offsets, row_of, row_token, row_gate, x_perm, H, y_perm, total;
+    size_t router_w, logits, psum, chunk_cnt, chunk_base, kept, contrib, offsets, row_of, row_token, row_gate, x_perm, H, y_perm;
+    // e4m3 experts (bf16 layers): codes and row scales of x, the packed rows'
+    // scales (the codes themselves go to x_perm), codes and scales of H
+    size_t x8, x8_scale, xperm_scale, H8, h_scale;
+    size_t total;
 };
 
 int64_t perm_rows(const moe_config *c) {
@@ -65,6 +69,12 @@ Layout layout(const moe_config *c) {
     L.x_perm = o;     o = align256(o + Tk * c->d_model * esz);
     L.H = o;          o = align256(o + rows * hF * esz);
     L.y_perm = o;     o = align256(o + rows * c->d_model * esz);
+    const size_t f8 = bf16 ? 1 : 0;
+    L.x8 = o;         o = align256(o + f8 * (size_t)c->T * c->d_model);
+    L.x8_scale = o;   o = align256(o + f8 * (size_t)c->T * 4);
+    L.xperm_scale = o; o = align256(o + f8 * Tk * 4);
+    L.H8 = o;         o = align256(o + f8 * rows * hF);
+    L.h_scale = o;    o = align256(o + f8 * rows * 4);
     L.total = o;
     return L;
 }
@@ -103,6 +113,30 @@ moe_status check_ws(const moe_config *c, void *ws, size_t ws_bytes) {
 #define ALIGNED(p, a) \
     do { if ((p) && (reinterpret_cast<uintptr_t>(p) % (a))) \
         return fail(MOE_ERR_INVALID_ARG, "misaligned pointer: %s", #p); } while (0)
+
+// e4m3 experts: bf16 layers only; every e4m3 row (x, weights, H) must be a
+// multiple of 16 bytes for the tensor maps.
+moe_status check_fp8_cfg(const moe_config *c) {
+    if (c->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "FP8 experts need a bf16 layer%s");
+    if (c->d_model % 16 || c->d_ff % 16 || c->d_ff_shared % 16)
+        return fail(MOE_ERR_UNSUPPORTED, "FP8 experts need d_model, d_ff, d_ff_shared multiples of 16%s");
+    return MOE_OK;
+}
+
+moe_status check_fp8_weights(const moe_config *c, const moe_fp8_experts *w) {
+    NEED(w);
+    NEED(w->W1); NEED(w->W1_scale); NEED(w->W2); NEED(w->W2_scale);
+    ALIGNED(w->W1, 16); ALIGNED(w->Wu, 16); ALIGNED(w->W2, 16);
+    ALIGNED(w->Wsh_g, 16); ALIGNED(w->Wsh_u, 16); ALIGNED(w->Wsh_d, 16);
+    ALIGNED(w->W1_scale, 4); ALIGNED(w->Wu_scale, 4); ALIGNED(w->W2_scale, 4);
+    ALIGNED(w->Wsh_g_scale, 4); ALIGNED(w->Wsh_u_scale, 4); ALIGNED(w->Wsh_d_scale, 4);
+    if (c->act == MOE_ACT_SWIGLU) { NEED(w->Wu); NEED(w->Wu_scale); }
+    if (c->d_ff_shared > 0) {
+        NEED(w->Wsh_g); NEED(w->Wsh_g_scale); NEED(w->Wsh_d); NEED(w->Wsh_d_scale);
+        if (c->act == MOE_ACT_SWIGLU) { NEED(w->Wsh_u); NEED(w->Wsh_u_scale); }
+    }
+    return MOE_OK;
+}
 
 int num_sms() {
     static int cache[64] = {0};
@@ -151,6 +185,19 @@ moe::FfnArgs ffn_args(const moe_config *c, const void *x_perm, const int32_t *of
     a.shared_base = (int64_t)c->T * c->top_k;
     a.num_sms = num_sms();
     return a;
+}
+
+// The e4m3 fields of the FFN arguments (x_perm / x hold codes).
+void set_fp8(moe::FfnArgs &a, const moe_config *c, const moe_fp8_experts *w, const float *xperm_scale,
+             const float *x_scale, void *ws) {
+    const Layout L = layout(c);
+    a.f8 = true;
+    a.xperm_scale = xperm_scale;
+    a.x_scale = x_scale;
+    a.W1s = w->W1_scale; a.Wus = w->Wu_scale; a.W2s = w->W2_scale;
+    a.Wsgs = w->Wsh_g_scale; a.Wsus = w->Wsh_u_scale; a.Wsds = w->Wsh_d_scale;
+    a.H8 = at<uint8_t>(ws, L.H8);
+    a.h_scale = at<float>(ws, L.h_scale);
 }
 
 }  // namespace
@@ -234,7 +281,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *idx,
     a.status = status_word(ws);
     a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.k = cfg->top_k;
     a.capacity = moe_capacity(cfg);
-    cudaError_t e = moe::launch_dispatch(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = moe::launch_dispatch(a, cfg->dtype == MOE_BF16 ? 2 : 4, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "permute");
 }
 
@@ -330,7 +377,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     da.contrib = at<double>(ws, L.contrib);
     da.nblk = moe::router_blocks(cfg->T, bf16);
     da.pdl = true;                                 // every launch after the first overlaps its predecessor
-    if ((e = moe::launch_dispatch(da, bf16, st)) != cudaSuccess) return cuda_fail(e, "permute");
+    if ((e = moe::launch_dispatch(da, bf16 ? 2 : 4, st)) != cudaSuccess) return cuda_fail(e, "permute");
 
     moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
                                y_perm, ws);
@@ -390,6 +437,127 @@ moe_status moe_get_device_status(void *ws, moe_stream_t stream, int32_t *status_
     if (e != cudaSuccess) return cuda_fail(e, "moe_get_device_status clear");
     *status_out = h[0];
     if (h[0] != 0) snprintf(g_detail, sizeof g_detail, "device status %d, detail %d", h[0], h[1]);
+    return MOE_OK;
+}
+
+moe_status moe_quantize_rows_e4m3(const void *in, int64_t rows, int32_t cols, int64_t ld_in, uint8_t *codes,
+                                  int64_t ld_out, float *scale, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return fail(MOE_ERR_INVALID_ARG, "negative rows or cols%s");
+    if (rows == 0 || cols == 0) return MOE_OK;
+    NEED(in); NEED(codes); NEED(scale);
+    if (cols % 8) return fail(MOE_ERR_UNSUPPORTED, "cols must be a multiple of 8%s");
+    if (ld_in < cols || ld_in % 8) return fail(MOE_ERR_INVALID_ARG, "ld_in < cols or not a multiple of 8%s");
+    if (ld_out < cols || ld_out % 8) return fail(MOE_ERR_INVALID_ARG, "ld_out < cols or not a multiple of 8%s");
+    ALIGNED(in, 16); ALIGNED(codes, 8); ALIGNED(scale, 4);
+    moe::QuantArgs q{};
+    q.in = static_cast<const __nv_bfloat16 *>(in);
+    q.ld_in = ld_in;
+    q.out = codes;
+    q.ld_out = ld_out;
+    q.scale = scale;
+    q.rows = rows;
+    q.cols = cols;
+    q.num_sms = num_sms();
+    cudaError_t e = moe::launch_quant_rows(q, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "quantize_rows");
+}
+
+moe_status moe_grouped_ffn_fp8(const moe_config *cfg, const uint8_t *x8_perm, const float *x8_perm_scale,
+                               const int32_t *offsets, const float *row_gate, const moe_fp8_experts *w,
+                               const float *b1, const float *b2, const uint8_t *x8, const float *x8_scale,
+                               void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    if ((s = check_fp8_cfg(cfg)) != MOE_OK) return s;
+    if (cfg->T > 0) {
+        NEED(x8_perm); NEED(x8_perm_scale); NEED(offsets); NEED(row_gate); NEED(y_perm);
+        if ((s = check_fp8_weights(cfg, w)) != MOE_OK) return s;
+        if (cfg->d_ff_shared > 0) { NEED(x8); NEED(x8_scale); }
+    }
+    ALIGNED(x8_perm, 16); ALIGNED(x8, 16); ALIGNED(y_perm, 16); ALIGNED(x8_perm_scale, 4); ALIGNED(x8_scale, 4);
+    ALIGNED(offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4); ALIGNED(b2, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    if (cfg->T == 0) return MOE_OK;
+    moe::FfnArgs a = ffn_args(cfg, x8_perm, offsets, row_gate, w->W1, b1, w->Wu, w->W2, b2, x8, w->Wsh_g, w->Wsh_u,
+                              w->Wsh_d, y_perm, ws);
+    set_fp8(a, cfg, w, x8_perm_scale, x8_scale, ws);
+    cudaError_t e = moe::launch_ffn_bf16(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "grouped_ffn_fp8");
+}
+
+moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                           const float *sel_bias, const moe_fp8_experts *w, const float *b1, const float *b2,
+                           void *y, int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                           float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    if ((s = check_fp8_cfg(cfg)) != MOE_OK) return s;
+    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    if (cfg->T > 0) {
+        NEED(x); NEED(Wr); NEED(y); NEED(idx); NEED(gate);
+        if ((s = check_fp8_weights(cfg, w)) != MOE_OK) return s;
+    }
+    ALIGNED(x, 16); ALIGNED(y, 16); ALIGNED(Wr, 4); ALIGNED(logit_bias, 4); ALIGNED(sel_bias, 4);
+    ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
+    ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    const Layout L = layout(cfg);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *psum = at<float>(ws, L.psum);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *row_of = at<int32_t>(ws, L.row_of);
+    float *row_gate = at<float>(ws, L.row_gate);
+    void *y_perm = at<char>(ws, L.y_perm);
+    uint8_t *x8 = at<uint8_t>(ws, L.x8);
+    float *x8_scale = at<float>(ws, L.x8_scale);
+    float *xperm_scale = at<float>(ws, L.xperm_scale);
+    cudaError_t e;
+
+    moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
+                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
+                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
+    if ((e = moe::launch_router(ra, true, st)) != cudaSuccess) return cuda_fail(e, "router");
+
+    moe::QuantArgs q{};                           // x -> e4m3 codes + row scales
+    q.in = static_cast<const __nv_bfloat16 *>(x);
+    q.ld_in = cfg->d_model;
+    q.out = x8;
+    q.ld_out = cfg->d_model;
+    q.scale = x8_scale;
+    q.rows = cfg->T;
+    q.cols = cfg->d_model;
+    q.num_sms = num_sms();
+    q.pdl = true;
+    if ((e = moe::launch_quant_rows(q, st)) != cudaSuccess) return cuda_fail(e, "quantize_x");
+
+    moe::DispatchArgs da{};
+    da.x = x8; da.idx = idx; da.gate = gate;
+    da.chunk_cnt = at<int32_t>(ws, L.chunk_cnt);
+    da.chunk_base = at<int32_t>(ws, L.chunk_base);
+    da.counts = counts; da.kept = at<int32_t>(ws, L.kept); da.offsets = offsets;
+    da.row_of = row_of; da.row_token = at<int32_t>(ws, L.row_token); da.row_gate = row_gate;
+    da.x_perm = at<char>(ws, L.x_perm);
+    da.x_scale = x8_scale;
+    da.row_scale = xperm_scale;
+    da.n_dropped = n_dropped;
+    da.status = status_word(ws);
+    da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
+    da.capacity = moe_capacity(cfg);
+    da.psum = psum; da.f = f; da.P = P; da.loss = loss;
+    da.contrib = at<double>(ws, L.contrib);
+    da.nblk = moe::router_blocks(cfg->T, true);
+    da.pdl = true;
+    if ((e = moe::launch_dispatch(da, 1, st)) != cudaSuccess) return cuda_fail(e, "permute");
+
+    moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, w->W1, b1, w->Wu, w->W2, b2, x8, w->Wsh_g,
+                               w->Wsh_u, w->Wsh_d, y_perm, ws);
+    set_fp8(fa, cfg, w, xperm_scale, x8_scale, ws);
+    fa.pdl = true;
+    if ((e = moe::launch_ffn_bf16(fa, st)) != cudaSuccess) return cuda_fail(e, "grouped_ffn_fp8");
+
+    moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
+                        cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
+    if ((e = moe::launch_combine(ca, true, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
 }
 

@@ -106,7 +106,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, 
     a.status = reinterpret_cast<int32_t *>(b);
     a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.k = cfg->top_k;
     a.capacity = moe_capacity(cfg);
-    e = moe::launch_dispatch(a, cfg->dtype == MOE_BF16, st);
+    e = moe::launch_dispatch(a, cfg->dtype == MOE_BF16 ? 2 : 4, st);
     if (e != cudaSuccess) return reject(MOE_ERR_CUDA, cudaGetErrorString(e));
     return MOE_OK;
 }

@@ -28,7 +28,16 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_workspace_init", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
-           "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout")
+           "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
+           "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8")
+
+
+class MoeFp8Experts(ctypes.Structure):
+    """moe_fp8_experts: e4m3 expert weights (device pointers) and their
+    per-output-channel fp32 scales."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
+        "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")]
 
 
 class MoEError(RuntimeError):
@@ -89,6 +98,15 @@ def lib():
         L.moe_check_wait_timeout.argtypes = [c_vp, ctypes.c_uint64, c_vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_permute_noalloc.argtypes = [P(MoeConfig)] + [c_vp] * 11 + [c_vp]
+        L.moe_quantize_rows_e4m3.restype = ctypes.c_int
+        L.moe_quantize_rows_e4m3.argtypes = [c_vp, ctypes.c_int64, c_i32, ctypes.c_int64, c_vp, ctypes.c_int64,
+                                             c_vp, c_vp]
+        L.moe_grouped_ffn_fp8.restype = ctypes.c_int
+        L.moe_grouped_ffn_fp8.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeFp8Experts)] + [c_vp] * 6 + [
+            ctypes.c_size_t, c_vp]
+        L.moe_forward_fp8.restype = ctypes.c_int
+        L.moe_forward_fp8.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeFp8Experts)] + [c_vp] * 12 + [
+            ctypes.c_size_t, c_vp]
         _lib = L
     return _lib
 
@@ -270,3 +288,54 @@ def forward(cfg, inp, out: Outputs, ws, stream=None):
                 inp.get("Wsg"), inp.get("Wsu"), inp.get("Wsd"),
                 out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss, out.logits,
                 out.n_dropped, ws, stream)
+
+
+# ---------------------------------------------------------------- FP8 experts
+FP8_WEIGHTS = ("W1", "Wu", "W2", "Wsg", "Wsu", "Wsd")
+_FP8_FIELD = {"W1": "W1", "Wu": "Wu", "W2": "W2", "Wsg": "Wsh_g", "Wsu": "Wsh_u", "Wsd": "Wsh_d"}
+
+
+def fp8_experts(w) -> MoeFp8Experts:
+    """moe_fp8_experts from a dict of device tensors: e4m3 codes (uint8)
+    under W1, Wu, W2, Wsg, Wsu, Wsd and fp32 scales under "<name>_scale"."""
+    s = MoeFp8Experts()
+    for name in FP8_WEIGHTS:
+        field = _FP8_FIELD[name]
+        setattr(s, field, _p(w.get(name)))
+        setattr(s, field + "_scale", _p(w.get(name + "_scale")))
+    return s
+
+
+def moe_quantize_rows_e4m3(x, codes, scale, rows=None, cols=None, ld_in=None, ld_out=None, stream=None):
+    """Per-row e4m3 quantization of a bf16 [rows, cols] tensor into codes
+    (uint8, same shape unless ld_out is given) and scale [rows] fp32."""
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld_in = x.shape[1] if ld_in is None else ld_in
+    ld_out = codes.shape[1] if ld_out is None else ld_out
+    _check(lib().moe_quantize_rows_e4m3(_p(x), rows, cols, ld_in, _p(codes), ld_out, _p(scale), _stream(stream)),
+           "moe_quantize_rows_e4m3")
+
+
+def moe_grouped_ffn_fp8(cfg, x8_perm, x8_perm_scale, offsets, row_gate, w, b1, b2, x8, x8_scale, y_perm, ws,
+                        stream=None):
+    ex = fp8_experts(w)
+    _check(lib().moe_grouped_ffn_fp8(ctypes.byref(cfg), _p(x8_perm), _p(x8_perm_scale), _p(offsets), _p(row_gate),
+                                     ctypes.byref(ex), _p(b1), _p(b2), _p(x8), _p(x8_scale), _p(y_perm), _p(ws),
+                                     ws.numel(), _stream(stream)), "moe_grouped_ffn_fp8")
+
+
+def moe_forward_fp8(cfg, x, Wr, logit_bias, sel_bias, w, b1, b2, y, idx, gate, counts, f, P, loss, logits_out,
+                    n_dropped, ws, stream=None):
+    ex = fp8_experts(w)
+    _check(lib().moe_forward_fp8(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias), ctypes.byref(ex),
+                                 _p(b1), _p(b2), _p(y), _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss),
+                                 _p(logits_out), _p(n_dropped), _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward_fp8")
+
+
+def forward_fp8(cfg, inp, w8, out: Outputs, ws, stream=None):
+    """moe_forward_fp8 on a dict of device inputs and a dict of FP8 experts."""
+    moe_forward_fp8(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"), w8,
+                    inp.get("b1"), inp.get("b2"), out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss,
+                    out.logits, out.n_dropped, ws, stream)

@@ -170,3 +170,47 @@ def to_numpy_raw(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view("uint16")
     return t.numpy()
+
+
+def _fp8_stack(wl, name, E, rows, cols, device, seed):
+    """E x rows x cols e4m3 codes of N(0, 1) draws (through torch's
+    float8_e4m3fn cast) and E x rows scales U(0.5, 1.5) / sqrt(cols)."""
+    codes = torch.empty((E, rows, cols), dtype=torch.uint8, device=device)
+    scale = torch.empty((E, rows), dtype=torch.float32, device=device)
+    for e in range(E):
+        g = _gen(device, seed, wl, name + "_e4m3", e)
+        codes[e].copy_(torch.randn((rows, cols), generator=g, device=device).to(torch.float8_e4m3fn)
+                       .view(torch.uint8))
+        scale[e].copy_((torch.rand((rows,), generator=g, device=device) + 0.5) * cols ** -0.5)
+    return codes, scale
+
+
+def generate_fp8_experts(wl: Workload, device="cpu", seed: int = 0) -> dict:
+    """FP8 expert weights for a bf16 workload: e4m3 codes (uint8, nn.Linear
+    [out, in] layout) with one fp32 scale per output channel, spread like the
+    bf16 weights (N(0, 1/fan_in)).  Keys W1, Wu, W2, Wsg, Wsu, Wsd and
+    "<key>_scale" (absent ones None), and for GELU experts the fp32 biases
+    b1, b2 (the same draws as generate()'s)."""
+    dev = torch.device(device)
+    d, E, F = wl.d_model, wl.E, wl.d_ff
+    w = {k: None for k in ("W1", "Wu", "W2", "Wsg", "Wsu", "Wsd")}
+    w.update({k + "_scale": None for k in list(w)})
+    w["W1"], w["W1_scale"] = _fp8_stack(wl, "W1", E, F, d, dev, seed)
+    w["W2"], w["W2_scale"] = _fp8_stack(wl, "W2", E, d, F, dev, seed)
+    if wl.act == "swiglu":
+        w["Wu"], w["Wu_scale"] = _fp8_stack(wl, "Wu", E, F, d, dev, seed)
+    if wl.act == "gelu":            # the GELU experts' fp32 biases, as generate() draws them
+        g = _gen(dev, seed, wl, "b1")
+        w["b1"] = (torch.rand((E, F), generator=g, device=dev) * 0.02 - 0.01)
+        g = _gen(dev, seed, wl, "b2")
+        w["b2"] = (torch.rand((E, d), generator=g, device=dev) * 0.02 - 0.01)
+    if wl.d_ff_shared:
+        S = wl.d_ff_shared
+        c, s = _fp8_stack(wl, "Wsg", 1, S, d, dev, seed)
+        w["Wsg"], w["Wsg_scale"] = c[0], s[0]
+        c, s = _fp8_stack(wl, "Wsd", 1, d, S, dev, seed)
+        w["Wsd"], w["Wsd_scale"] = c[0], s[0]
+        if wl.act == "swiglu":
+            c, s = _fp8_stack(wl, "Wsu", 1, S, d, dev, seed)
+            w["Wsu"], w["Wsu_scale"] = c[0], s[0]
+    return w

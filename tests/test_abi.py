@@ -133,3 +133,41 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError):
         nat.moe_combine(c, torch.zeros(4), torch.zeros(4, dtype=torch.int32), torch.zeros(4),
                         torch.zeros(256, dtype=torch.uint8))
+
+
+def fp8_raw(c, w=None, **null):
+    if w is None:
+        w = nat.MoeFp8Experts(W1=4096, W1_scale=4096, Wu=4096, Wu_scale=4096, W2=4096, W2_scale=4096)
+    args = dict(x=fake(), Wr=fake(), lb=None, sb=None)
+    rest = dict(b1=None, b2=None, y=fake(), idx=fake(), gate=fake(), counts=fake(), f=fake(), P=fake(),
+                loss=fake(), logits=None, nd=None)
+    for k in null:
+        (args if k in args else rest)[k] = None
+    return nat.lib().moe_forward_fp8(ctypes.byref(c), *args.values(), ctypes.byref(w), *rest.values(), fake(16),
+                                     nat.workspace_size(c), None)
+
+
+def test_fp8_entry_points_check_arguments():
+    # FP8 experts need a bf16 layer and widths that are multiples of 16
+    assert fp8_raw(cfg(dtype="f32")) == nat.MOE_ERR_UNSUPPORTED
+    assert fp8_raw(cfg(d_model=136)) == nat.MOE_ERR_UNSUPPORTED
+    assert fp8_raw(cfg(d_ff=264)) == nat.MOE_ERR_UNSUPPORTED
+    assert fp8_raw(cfg(d_ff_shared=24)) == nat.MOE_ERR_UNSUPPORTED
+    # missing weights, scales or outputs
+    assert fp8_raw(cfg(), w=nat.MoeFp8Experts(W1=4096, W2=4096, W2_scale=4096, Wu=4096, Wu_scale=4096)) \
+        == nat.MOE_ERR_INVALID_ARG
+    assert "W1_scale" in nat.last_error_detail()
+    assert fp8_raw(cfg(), w=nat.MoeFp8Experts(W1=4096, W1_scale=4096, W2=4096, W2_scale=4096)) \
+        == nat.MOE_ERR_INVALID_ARG                        # SwiGLU without W_up
+    assert fp8_raw(cfg(d_ff_shared=64)) == nat.MOE_ERR_INVALID_ARG      # no shared expert weights
+    assert fp8_raw(cfg(), y=None) == nat.MOE_ERR_INVALID_ARG
+    # misaligned codes
+    assert fp8_raw(cfg(), w=nat.MoeFp8Experts(W1=4096 + 8, W1_scale=4096, Wu=4096, Wu_scale=4096, W2=4096,
+                                              W2_scale=4096)) == nat.MOE_ERR_INVALID_ARG
+    # the row quantizer
+    L = nat.lib()
+    assert L.moe_quantize_rows_e4m3(fake(), 4, 12, 12, fake(), 12, fake(), None) == nat.MOE_ERR_UNSUPPORTED
+    assert L.moe_quantize_rows_e4m3(fake(), 4, 16, 8, fake(), 16, fake(), None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(fake(), 4, 16, 16, fake(), 12, fake(), None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(None, 4, 16, 16, fake(), 16, fake(), None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(None, 0, 16, 16, None, 16, None, None) == nat.MOE_OK
