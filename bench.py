@@ -141,17 +141,21 @@ def recorded_traffic(workload):
     return None
 
 
-def algorithmic_counts(wl, counts, kept):
+def algorithmic_counts(wl, counts, kept, fp8=False):
     """Expert FLOPs on kept rows (+ shared expert), and the layer's algorithmic
-    bytes: x, y, W_r and the weights of every expert with a kept row."""
+    bytes: x, y, W_r and the weights of every expert with a kept row (e4m3
+    experts: one byte per weight plus a 4-byte scale per output channel)."""
     esz = 2 if wl.dtype == "bf16" else 4
+    wsz = 1 if fp8 else esz
     mats = 3 if wl.act == "swiglu" else 2
     kept_rows = int(kept.sum())
     flops = wl.expert_flops(kept_rows)
     touched = int((kept > 0).sum())
-    w_bytes = touched * mats * wl.d_model * wl.d_ff * esz
+    w_bytes = touched * mats * wl.d_model * wl.d_ff * wsz
+    if fp8:                                        # per-channel scales
+        w_bytes += touched * 4 * ((mats - 1) * wl.d_ff + wl.d_model)
     if wl.d_ff_shared:
-        w_bytes += 3 * wl.d_model * wl.d_ff_shared * esz
+        w_bytes += 3 * wl.d_model * wl.d_ff_shared * wsz
     b = 2 * wl.T * wl.d_model * esz + wl.d_model * wl.E * 4 + w_bytes
     return flops, b, kept_rows
 
@@ -235,11 +239,22 @@ def workload_config(wl):
 def run_ours(args, wl, dev, world, rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    inp = syn.generate(wl, dev, seed=0)
+    fp8 = args.experts == "fp8"
+    inp = syn.generate(wl, dev, seed=0, weights=not fp8)
+    w8 = None
+    if fp8:                                         # e4m3 experts (bf16 layer around them)
+        w8 = syn.generate_fp8_experts(wl, dev, seed=0)
+        inp["b1"], inp["b2"] = w8.get("b1"), w8.get("b2")
     cfg = nat.config_from_workload(wl)
     out = nat.Outputs(cfg, dev)
     ws = nat.alloc_workspace(cfg, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def layer(inp_, out_):
+        if fp8:
+            nat.forward_fp8(cfg, inp_, w8, out_, ws, stream)
+        else:
+            nat.forward(cfg, inp_, out_, ws, stream)
 
     def barrier():
         if world > 1:
@@ -247,7 +262,7 @@ def run_ours(args, wl, dev, world, rank):
 
     for _ in range(args.warmup):
         flush.zero_()
-        nat.forward(cfg, inp, out, ws, stream)
+        layer(inp, out)
     torch.cuda.synchronize(dev)
     st = nat.moe_get_device_status(ws, stream)
     if st != nat.MOE_OK:
@@ -262,7 +277,7 @@ def run_ours(args, wl, dev, world, rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        nat.forward(cfg, inp, out, ws, stream)
+        layer(inp, out)
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -282,8 +297,22 @@ def run_ours(args, wl, dev, world, rank):
     row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
     row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
     row_gate = torch.empty(T * k, dtype=torch.float32, device=dev)
-    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)
+    x_perm = torch.empty((T * k, d), dtype=torch.uint8 if fp8 else dt, device=dev)
     y_perm = torch.empty((nat.perm_rows(cfg), d), dtype=dt, device=dev)
+    if fp8:
+        # e4m3 x and its packed rows, built once from this step's routing (the
+        # forward quantizes x and copies its rows on the device; here the
+        # staged pass times the quantizer, the row tables and the FFN)
+        x8 = torch.empty((T, d), dtype=torch.uint8, device=dev)
+        xs = torch.empty(T, dtype=torch.float32, device=dev)
+        xps = torch.zeros(T * k, dtype=torch.float32, device=dev)
+        nat.moe_quantize_rows_e4m3(inp["x"], x8, xs, stream=stream)
+        nat.moe_permute(cfg, inp["x"], out.idx, out.gate, out.counts, kept, offsets, row_of, row_token, row_gate,
+                        None, out.n_dropped, ws, stream)
+        torch.cuda.synchronize(dev)
+        nrows = int(offsets[-1].item())
+        x_perm[:nrows] = x8[row_token[:nrows].long()]
+        xps[:nrows] = xs[row_token[:nrows].long()]
     stages = ["router", "permute", "grouped_ffn", "combine", "balance"]
     stage_ms = {s: [] for s in stages}
     all_evs = []
@@ -294,11 +323,20 @@ def run_ours(args, wl, dev, world, rank):
         nat.moe_router_topk(cfg, inp["x"], inp["Wr"], inp["logit_bias"], inp["sel_bias"], out.idx, out.gate,
                             None, psum, ws, stream)
         evs[1].record(stream)
-        nat.moe_permute(cfg, inp["x"], out.idx, out.gate, out.counts, kept, offsets, row_of, row_token, row_gate,
-                        x_perm, out.n_dropped, ws, stream)
+        if fp8:
+            nat.moe_quantize_rows_e4m3(inp["x"], x8, xs, stream=stream)
+            nat.moe_permute(cfg, inp["x"], out.idx, out.gate, out.counts, kept, offsets, row_of, row_token,
+                            row_gate, None, out.n_dropped, ws, stream)
+        else:
+            nat.moe_permute(cfg, inp["x"], out.idx, out.gate, out.counts, kept, offsets, row_of, row_token,
+                            row_gate, x_perm, out.n_dropped, ws, stream)
         evs[2].record(stream)
-        nat.moe_grouped_ffn(cfg, x_perm, offsets, row_gate, inp["W1"], inp["b1"], inp["Wu"], inp["W2"], inp["b2"],
-                            inp["x"], inp["Wsg"], inp["Wsu"], inp["Wsd"], y_perm, ws, stream)
+        if fp8:
+            nat.moe_grouped_ffn_fp8(cfg, x_perm, xps, offsets, row_gate, w8, inp["b1"], inp["b2"], x8, xs, y_perm,
+                                    ws, stream)
+        else:
+            nat.moe_grouped_ffn(cfg, x_perm, offsets, row_gate, inp["W1"], inp["b1"], inp["Wu"], inp["W2"],
+                                inp["b2"], inp["x"], inp["Wsg"], inp["Wsu"], inp["Wsd"], y_perm, ws, stream)
         evs[3].record(stream)
         nat.moe_combine(cfg, y_perm, row_of, out.y, ws, stream)
         evs[4].record(stream)
@@ -345,7 +383,7 @@ def run_ours(args, wl, dev, world, rank):
             stream.wait_event(ev_out[i - nbuf])      # outs[b] is free once its results are out
         inp_i = dict(inp)
         inp_i["x"] = x_dev[b]
-        nat.forward(cfg, inp_i, outs[b], ws, stream)
+        layer(inp_i, outs[b])
         ev_comp[i].record(stream)
         s_out.wait_event(ev_comp[i])
         with torch.cuda.stream(s_out):
@@ -363,8 +401,11 @@ def run_ours(args, wl, dev, world, rank):
     counts = out.counts.cpu().numpy()
     cap = nat.capacity(cfg)
     kept_np = np.minimum(counts, cap) if cap >= 0 else counts
-    flops, alg_bytes, kept_rows = algorithmic_counts(wl, counts, kept_np)
+    flops, alg_bytes, kept_rows = algorithmic_counts(wl, counts, kept_np, fp8)
     peaks, peak_src = load_peaks()
+    if fp8:       # e4m3 contractions: the measured bf16 peaks x the nominal fp8 : bf16 ratio (2)
+        peaks = dict(peaks, bf16_tflops=2 * peaks["bf16_tflops"],
+                     bf16_tflops_sustained=2 * peaks["bf16_tflops_sustained"])
     # The step runs back to back for the whole timed region (power-capped
     # clocks, sw_power_cap active): the sustained bf16 figure is the tensor
     # peak; the burst figure is reported beside it.
@@ -375,7 +416,7 @@ def run_ours(args, wl, dev, world, rank):
     layer_roof_burst_ms = max(t_tensor_burst, t_hbm) * 1e3
     ffn_ms = stage_avg["grouped_ffn"]
     ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
-    traffic = recorded_traffic(wl.name)
+    traffic = None if fp8 else recorded_traffic(wl.name)
     result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts,
                   flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
                   layer_roof_ms=layer_roof_ms, layer_roof_burst_ms=layer_roof_burst_ms, ffn_tflops=ffn_tflops,
@@ -384,7 +425,7 @@ def run_ours(args, wl, dev, world, rank):
                   bound="tensor" if t_tensor >= t_hbm else "hbm",
                   h2d=x_host.numel() * x_host.element_size(),
                   d2h=y_host.numel() * y_host.element_size() + 8, host_inp=None)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and not fp8:
         host = host_inputs(inp)
         n, dt_cpu, cores = oracle_sample(wl, host, args.cpu_seconds)
         result["cpu"] = {"value": n / dt_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -393,12 +434,15 @@ def run_ours(args, wl, dev, world, rank):
     return result
 
 
-def launches_per_forward(wl):
+def launches_per_forward(wl, fp8=False):
     """Kernels one moe_forward call launches (T > 0).  bf16: W_r split, logits
     GEMM, selection, histogram, scan (+ balance statistics), permute, two
     launches per expert GEMM (CTA-pair kernel, then the 1-CTA kernel for last
     blocks of 1..128 rows), combine.  fp32: router, histogram, scan, permute,
-    two SIMT GEMMs, combine."""
+    two SIMT GEMMs, combine.  moe_forward_fp8 adds the quantization of x and
+    of H (the routed rows, and the shared rows when there is a shared expert)."""
+    if fp8:
+        return 13 + (1 if wl.d_ff_shared else 0)
     return 11 if wl.dtype == "bf16" else 7
 
 
@@ -411,11 +455,15 @@ def main():
     ap.add_argument("--workload", default="qwen3_moe", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: e4m3 experts through moe_forward_fp8 (bf16 layers only; no CPU baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()
     wl = syn.WORKLOADS[args.workload]
+    if args.experts == "fp8" and wl.dtype != "bf16":
+        ap.error("--experts fp8 needs a bf16 workload")
     if args.impl == "reference":
         if rank == 0:
             dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
@@ -438,30 +486,36 @@ def main():
     peaks = r["peaks"]
     tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
     peak_tensor = peaks["bf16_tflops_sustained"]
+    fp8 = args.experts == "fp8"
+    peak_kind = ("fp8 (2 x the measured bf16 figure, the nominal fp8 : bf16 ratio)" if fp8 else "bf16")
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": dict(workload_config(wl), parallelism="replicas x%d" % world),
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3 experts (fp32 accumulation), bf16 layer" if fp8 else ("bf16" if wl.dtype == "bf16"
+                                                                                   else "f32"),
+        "data": "synthetic",
+        "config": dict(workload_config(wl), parallelism="replicas x%d" % world, experts=args.experts),
         "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
         "layer_roofline": {"bound": r["bound"], "time_ms": r["layer_roof_ms"],
                            "frac": r["layer_roof_ms"] / r["ms"], "flops": r["flops"],
                            "alg_bytes": r["alg_bytes"],
                            "frac_burst": r["layer_roof_burst_ms"] / r["ms"],
-                           "peak_note": "sustained bf16 (timed inside the back-to-back step loop) and copy "
-                                        "bandwidth, " + tag + "; frac_burst against the burst bf16 figure"},
-        "roofline": {"kernel": "grouped_ffn (tcgen05 gemm1 + gemm2)", "bound": "tensor",
+                           "peak_note": "sustained " + peak_kind + " (timed inside the back-to-back step loop) "
+                                        "and copy bandwidth, " + tag + "; frac_burst against the burst figure"},
+        "roofline": {"kernel": ("grouped_ffn_fp8 (tcgen05 e4m3 gemm1 + H quantization + gemm2)" if fp8
+                                else "grouped_ffn (tcgen05 gemm1 + gemm2)"), "bound": "tensor",
                      "achieved": r["ffn_tflops"], "peak": peak_tensor, "unit": "TFLOP/s",
                      "frac": r["ffn_tflops"] / peak_tensor, "traffic": r["traffic"],
                      "frac_burst": r["ffn_tflops"] / peaks["bf16_tflops"],
-                     "peak_note": "sustained, " + tag + " (the kernel runs inside the back-to-back step loop); "
-                                  "frac_burst against the burst figure"},
+                     "peak_note": "sustained " + peak_kind + ", " + tag + " (the kernel runs inside the "
+                                  "back-to-back step loop); frac_burst against the burst figure"},
         "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
         "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],
                 "copies": "every step's x in and y + loss out, on their own streams, overlapping the "
                           "neighbouring steps' layers (double-buffered device buffers)"},
-        "gpu_launches": launches_per_forward(wl) * args.steps,
+        "gpu_launches": launches_per_forward(wl, fp8) * args.steps,
         "clocks": r["clocks"],
         "routing": {"kept_rows": r["kept_rows"], "dropped": r["n_dropped"], "loss": r["loss"],
                     "max_count": int(r["counts"].max()), "min_count": int(r["counts"].min()),

@@ -221,8 +221,9 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
  *   Everything else (router, dispatch, gates, combine, statistics) is the
  *   bf16 layer's.  Only bf16 layers (cfg->dtype == MOE_BF16) with d_model,
  *   d_ff and d_ff_shared multiples of 16 (else MOE_ERR_UNSUPPORTED).
- * All pointers in the struct are device pointers; the struct itself is a
- * host object read during the call.                                        */
+ * All pointers in the struct are device pointers (codes 16-byte aligned,
+ * scales 4-byte aligned); the struct itself is a host object read during
+ * the call.                                                                 */
 typedef struct {
     const uint8_t *W1;    const float *W1_scale;     /* [E, d_ff, d_model], [E, d_ff]   */
     const uint8_t *Wu;    const float *Wu_scale;     /* SwiGLU W_up (same shapes), else NULL */

@@ -153,6 +153,14 @@ __device__ __forceinline__ void stage_store32(uint32_t stg, const CUtensorMap *t
     }
 }
 
+// The scale of column col0 + lane (0 past N): one coalesced load per warp
+// and 32-column chunk; the epilogue hands each column's scale to every row
+// (lane) with a shuffle.
+__device__ __forceinline__ float col_scale_lane(const float *cs, int col0, int N) {
+    const int c = col0 + (int)(threadIdx.x & 31);
+    return c < N ? __ldg(cs + c) : 0.f;
+}
+
 // Epilogue of one accumulator row (this thread's TMEM lane) for one tile:
 // the warp's half of the columns (SwiGLU: gate chunks half*2, half*2+1 and
 // the up chunks 128 columns on; otherwise chunks half*4 .. half*4+3) arrive
@@ -174,12 +182,12 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = nt * 128 + (c0 + cc) * 32;
             float *h = v + cc * 32;                  // in place of the gate values
-            if (F8) {
+            if (F8) {                                // gate and up column scales
+                const float sg = col_scale_lane(cs, col0, N), su = col_scale_lane(cs2, col0, N);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool in = col0 + i < N;
-                    h[i] *= rscale * (in ? __ldg(cs + col0 + i) : 0.f);
-                    v[64 + cc * 32 + i] *= rscale * (in ? __ldg(cs2 + col0 + i) : 0.f);
+                    h[i] *= rscale * __shfl_sync(0xffffffffu, sg, i);
+                    v[64 + cc * 32 + i] *= rscale * __shfl_sync(0xffffffffu, su, i);
                 }
             }
 #pragma unroll
@@ -200,10 +208,14 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
             const int col0 = nt * BNB + (c0 + cc) * 32;
             if (col0 >= N) continue;                  // uniform over the warp
             float *h = v + cc * 32;                  // in place
+            if (F8) {
+                const float sc = col_scale_lane(cs, col0, N);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] *= rscale * __shfl_sync(0xffffffffu, sc, i);
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float acc = F8 ? h[i] * (rscale * (col0 + i < N ? __ldg(cs + col0 + i) : 0.f)) : h[i];
-                const float z = acc + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
+                const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
                 h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
             }
             if (staged) {
