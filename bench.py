@@ -127,17 +127,18 @@ def source_hash(path):
         return hashlib.sha256(f.read()).hexdigest()[:12]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the grouped-FFN kernels from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
+def recorded_traffic(workload, kernel="grouped_ffn"):
+    """DRAM bytes per launch of the grouped-FFN kernels (kernel: grouped_ffn or
+    grouped_ffn_fp8) from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
     if not os.path.exists(path):
         return None
     src = source_hash(os.path.join(ROOT, "mixture_experts_layer_49_b200", "csrc", "ffn_sm100.cu"))
     for line in open(path):
-        m = re.match(r"\|\s*grouped_ffn\s*\|\s*(\w+)\s*\|\s*([0-9a-f]+)\s*\|\s*([0-9.eE+]+)\s*\|", line)
-        if m and m.group(1) == workload and m.group(2) == src:
-            return float(m.group(3))
+        m = re.match(r"\|\s*(\w+)\s*\|\s*(\w+)\s*\|\s*([0-9a-f]+)\s*\|\s*([0-9.eE+]+)\s*\|", line)
+        if m and m.group(1) == kernel and m.group(2) == workload and m.group(3) == src:
+            return float(m.group(4))
     return None
 
 
@@ -416,7 +417,7 @@ def run_ours(args, wl, dev, world, rank):
     layer_roof_burst_ms = max(t_tensor_burst, t_hbm) * 1e3
     ffn_ms = stage_avg["grouped_ffn"]
     ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
-    traffic = None if fp8 else recorded_traffic(wl.name)
+    traffic = recorded_traffic(wl.name, "grouped_ffn_fp8" if fp8 else "grouped_ffn")
     result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts,
                   flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
                   layer_roof_ms=layer_roof_ms, layer_roof_burst_ms=layer_roof_burst_ms, ffn_tflops=ffn_tflops,

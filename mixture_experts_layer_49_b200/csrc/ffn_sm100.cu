@@ -161,6 +161,29 @@ __device__ __forceinline__ float col_scale_lane(const float *cs, int col0, int N
     return c < N ? __ldg(cs + c) : 0.f;
 }
 
+// e4m3 tiles: this thread's row scale and the column scales its warp's
+// chunks need (SwiGLU: gate scales of chunks half*2, half*2+1, then the up
+// scales; otherwise chunks half*4 .. half*4+3), loaded before the accumulator
+// wait so their latency overlaps it.
+template <int MODE>
+__device__ __forceinline__ void preload_scales(const GemmParams &p, bool sh, int g, int nt, int half, int N,
+                                               bool valid, int64_t arow, float &rscale, float *csv) {
+    rscale = valid ? __ldg((sh ? p.shared_row_scale : p.row_scale) + arow) : 0.f;
+    const float *cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
+    if (MODE == GM_SWIGLU) {
+        const float *cs2 = sh ? p.sh_col_scale2 : p.col_scale2 + (size_t)g * p.N_routed;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int col0 = nt * 128 + (half * 2 + cc) * 32;
+            csv[cc] = col_scale_lane(cs, col0, N);
+            csv[2 + cc] = col_scale_lane(cs2, col0, N);
+        }
+    } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) csv[cc] = col_scale_lane(cs, nt * BNB + (half * 4 + cc) * 32, N);
+    }
+}
+
 // Epilogue of one accumulator row (this thread's TMEM lane) for one tile:
 // the warp's half of the columns (SwiGLU: gate chunks half*2, half*2+1 and
 // the up chunks 128 columns on; otherwise chunks half*4 .. half*4+3) arrive
@@ -172,7 +195,7 @@ template <int MODE, bool F8>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
                                              __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
                                              const CUtensorMap *tmO, uint32_t stg, int row0, float rscale,
-                                             const float *cs, const float *cs2) {
+                                             const float *csv) {
     float v[128];
     const bool staged = __all_sync(0xffffffffu, valid);
     if (MODE == GM_SWIGLU) {
@@ -183,11 +206,10 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
             const int col0 = nt * 128 + (c0 + cc) * 32;
             float *h = v + cc * 32;                  // in place of the gate values
             if (F8) {                                // gate and up column scales
-                const float sg = col_scale_lane(cs, col0, N), su = col_scale_lane(cs2, col0, N);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    h[i] *= rscale * __shfl_sync(0xffffffffu, sg, i);
-                    v[64 + cc * 32 + i] *= rscale * __shfl_sync(0xffffffffu, su, i);
+                    h[i] *= rscale * __shfl_sync(0xffffffffu, csv[cc], i);
+                    v[64 + cc * 32 + i] *= rscale * __shfl_sync(0xffffffffu, csv[2 + cc], i);
                 }
             }
 #pragma unroll
@@ -209,9 +231,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
             if (col0 >= N) continue;                  // uniform over the warp
             float *h = v + cc * 32;                  // in place
             if (F8) {
-                const float sc = col_scale_lane(cs, col0, N);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) h[i] *= rscale * __shfl_sync(0xffffffffu, sc, i);
+                for (int i = 0; i < 32; ++i) h[i] *= rscale * __shfl_sync(0xffffffffu, csv[cc], i);
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -402,9 +423,15 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int grow = mt * BM + r_in_tile;
             const bool valid = grow < s.rows[g];
             const int64_t orow = sh ? p.shared_out_row + s.start[g] + grow : (int64_t)s.row0[g] + grow;
-            // the row's gate is fetched before the accumulator wait, hiding its latency
+            // the row's gate (and, for e4m3 tiles, the scales) are fetched
+            // before the accumulator wait, hiding their latency
             float gscale = 1.f;
             if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
+            const int N = sh ? p.N_shared : p.N_routed;
+            float rscale = 0.f, csv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (F8)
+                preload_scales<MODE>(p, sh, g, nt, half, N, valid, sh ? p.shared_a_row + s.start[g] + grow : orow,
+                                     rscale, csv);
             // lane 0 waits, the warp follows its verdict (keeps the warp converged
             // for the .sync.aligned TMEM loads)
             int ok = 1;
@@ -413,20 +440,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (!ok) { if (lane == 0) fail(s, p, 4); break; }
             __syncwarp();
             tc_fence_after();
-            const int N = sh ? p.N_shared : p.N_routed;
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            float rscale = 0.f;
-            const float *cs = nullptr, *cs2 = nullptr;
-            if (F8) {
-                const int64_t arow = sh ? p.shared_a_row + s.start[g] + grow : orow;
-                if (valid) rscale = __ldg((sh ? p.shared_row_scale : p.row_scale) + arow);
-                cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
-                cs2 = sh ? p.sh_col_scale2 : (p.col_scale2 ? p.col_scale2 + (size_t)g * p.N_routed : nullptr);
-            }
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, cs, cs2);
+                                   rscale, csv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
@@ -646,26 +664,20 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
             float gscale = 1.f;
             if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
+            const int N = sh ? p.N_shared : p.N_routed;
+            float rscale = 0.f, csv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (F8) preload_scales<MODE>(p, sh, g, nt, half, N, valid, sh ? p.shared_a_row + grow : orow, rscale, csv);
             int ok = 1;
             if (lane == 0) ok = mbar_wait(smem_u32(&s.accf[ab]), aphase, p.timeout_ns) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) { if (lane == 0) fail_pair(s, p, 24); break; }
             __syncwarp();
             tc_fence_after();
-            const int N = sh ? p.N_shared : p.N_routed;
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
-            float rscale = 0.f;
-            const float *cs = nullptr, *cs2 = nullptr;
-            if (F8) {
-                const int64_t arow = sh ? p.shared_a_row + grow : orow;
-                if (valid) rscale = __ldg((sh ? p.shared_row_scale : p.row_scale) + arow);
-                cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
-                cs2 = sh ? p.sh_col_scale2 : (p.col_scale2 ? p.col_scale2 + (size_t)g * p.N_routed : nullptr);
-            }
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, cs, cs2);
+                                   rscale, csv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
