@@ -123,8 +123,16 @@ class ClockSampler:
 
 
 def source_hash(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:12]
+    """sha256 (first 12 hex digits) of a source file with its comments, trailing
+    blanks and blank lines removed: a comment edit keeps the hash, any change to
+    the code changes it."""
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    lines = [ln.rstrip() for ln in text.splitlines()]
+    code = "\n".join(ln for ln in lines if ln)
+    return hashlib.sha256(code.encode()).hexdigest()[:12]
 
 
 def recorded_traffic(workload, kernel="grouped_ffn"):

@@ -35,6 +35,13 @@
 // are computed but never stored.  Within a group the m index runs fastest so
 // CTAs working at the same time share one weight tile through L2.
 //
+// e4m3 experts (the F8 instantiations): the same kernels with e4m3 A and B
+// tiles (128 elements per 128-byte swizzled row, kind::f8f6f4 MMAs of 32
+// elements of K); the epilogue multiplies each fp32 accumulator by its row's
+// activation scale and its column's weight scale before the activation or
+// gate (the scales are loaded before the accumulator wait; a column's scale
+// reaches the warp's rows by shuffle).
+//
 // Every mbarrier wait is bounded (a global-timer limit); a wait that runs out
 // records MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds,
 // freeing its TMEM.  No TMA multicast is used.
