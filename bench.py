@@ -170,9 +170,10 @@ def algorithmic_counts(wl, counts, kept, fp8=False):
 
 
 # ------------------------------------------------------------- CPU oracle leg
-def oracle_sample(wl, inp_host, target_s, max_tokens=None):
+def oracle_sample(wl, inp_host, target_s, max_tokens=None, threads=None):
     """Time the oracle (router + selection + expert FFNs in fp64) on the first
-    n tokens of the workload; n is grown until the run takes ~target_s."""
+    n tokens of the workload; n is grown until the run takes ~target_s.
+    threads: worker threads (default: every host core)."""
     import oracle
     cap = oracle.capacity(float(np.float32(wl.capacity_factor)), wl.top_k, wl.T, wl.E)
     weights = {k: inp_host[k] for k in ("W1", "Wu", "W2", "b1", "b2", "Wsg", "Wsu", "Wsd")
@@ -181,7 +182,7 @@ def oracle_sample(wl, inp_host, target_s, max_tokens=None):
     while True:
         dims = oracle.make_dims(n, wl.d_model, wl.E, wl.d_ff, wl.top_k, x_dtype=wl.dtype, act=wl.act,
                                 score=wl.score, renorm=wl.renorm, capacity=cap,
-                                d_ff_shared=wl.d_ff_shared)
+                                d_ff_shared=wl.d_ff_shared, nthreads=threads)
         x = inp_host["x"][:n]
         t0 = time.perf_counter()
         r = oracle.route(dims, x, inp_host["Wr"], inp_host["logit_bias"], inp_host["sel_bias"])
@@ -293,6 +294,8 @@ def run_ours(args, wl, dev, world, rank):
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = sum(step_ms) / args.steps
+    srt = sorted(step_ms)
+    step_pct = {q: srt[min(len(srt) - 1, int(round(q / 100 * (len(srt) - 1))))] for q in (10, 50, 90)}
     st = nat.moe_get_device_status(ws, stream)
     if st != nat.MOE_OK:
         raise RuntimeError("device status after timing: " + nat.status_string(st))
@@ -426,7 +429,7 @@ def run_ours(args, wl, dev, world, rank):
     ffn_ms = stage_avg["grouped_ffn"]
     ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(wl.name, "grouped_ffn_fp8" if fp8 else "grouped_ffn")
-    result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts,
+    result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts, step_pct=step_pct,
                   flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
                   layer_roof_ms=layer_roof_ms, layer_roof_burst_ms=layer_roof_burst_ms, ffn_tflops=ffn_tflops,
                   traffic=traffic,
@@ -437,9 +440,12 @@ def run_ours(args, wl, dev, world, rank):
     if rank == 0 and not args.no_cpu_baseline and not fp8:
         host = host_inputs(inp)
         n, dt_cpu, cores = oracle_sample(wl, host, args.cpu_seconds)
+        n1, dt1, _ = oracle_sample(wl, host, max(1.0, args.cpu_seconds / 5), threads=1)
         result["cpu"] = {"value": n / dt_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": "first %d tokens of %s: router, top-k, dispatch, balance and expert FFNs in "
-                                   "fp64 (%.1f s on the host cores)" % (n, wl.name, dt_cpu)}
+                                   "fp64 (%.1f s on the host cores)" % (n, wl.name, dt_cpu),
+                         "value_1core": n1 / dt1,
+                         "sample_1core": "first %d tokens, one thread (%.1f s)" % (n1, dt1)}
     return result
 
 
@@ -520,6 +526,7 @@ def main():
                      "peak_note": "sustained " + peak_kind + ", " + tag + " (the kernel runs inside the "
                                   "back-to-back step loop); frac_burst against the burst figure"},
         "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
+        "step_ms_percentiles": {"p10": r["step_pct"][10], "p50": r["step_pct"][50], "p90": r["step_pct"][90]},
         "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],
                 "copies": "every step's x in and y + loss out, on their own streams, overlapping the "
