@@ -469,6 +469,7 @@ moe_status moe_grouped_ffn_fp8(const moe_config *cfg, const uint8_t *x8_perm, co
     moe_status s = check_cfg(cfg);
     if (s != MOE_OK) return s;
     if ((s = check_fp8_cfg(cfg)) != MOE_OK) return s;
+    NEED(w);
     if (cfg->T > 0) {
         NEED(x8_perm); NEED(x8_perm_scale); NEED(offsets); NEED(row_gate); NEED(y_perm);
         if ((s = check_fp8_weights(cfg, w)) != MOE_OK) return s;
@@ -492,7 +493,7 @@ moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr
     moe_status s = check_cfg(cfg);
     if (s != MOE_OK) return s;
     if ((s = check_fp8_cfg(cfg)) != MOE_OK) return s;
-    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    NEED(counts); NEED(f); NEED(P); NEED(loss); NEED(w);
     if (cfg->T > 0) {
         NEED(x); NEED(Wr); NEED(y); NEED(idx); NEED(gate);
         if ((s = check_fp8_weights(cfg, w)) != MOE_OK) return s;

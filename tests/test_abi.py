@@ -161,6 +161,11 @@ def test_fp8_entry_points_check_arguments():
         == nat.MOE_ERR_INVALID_ARG                        # SwiGLU without W_up
     assert fp8_raw(cfg(d_ff_shared=64)) == nat.MOE_ERR_INVALID_ARG      # no shared expert weights
     assert fp8_raw(cfg(), y=None) == nat.MOE_ERR_INVALID_ARG
+    # the weights struct is required even for an empty batch
+    c0 = cfg(T=0)
+    assert nat.lib().moe_forward_fp8(ctypes.byref(c0), None, None, None, None, None, None, None, None, None,
+                                     None, fake(), fake(), fake(), fake(), None, None, fake(16),
+                                     nat.workspace_size(c0), None) == nat.MOE_ERR_INVALID_ARG
     # misaligned codes
     assert fp8_raw(cfg(), w=nat.MoeFp8Experts(W1=4096 + 8, W1_scale=4096, Wu=4096, Wu_scale=4096, W2=4096,
                                               W2_scale=4096)) == nat.MOE_ERR_INVALID_ARG
