@@ -388,9 +388,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int ab = 0;
             uint32_t aphase = 0;
             for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
-                int g, mt, nt;
-                decode(s, G, tile, g, mt, nt);
-                const int K = g >= p.E ? p.K_shared : p.K_routed;
+                // the shared group, when there is one, is the last: its tiles start
+                // at tile_start[E] (= total without one), so K needs no search
+                const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
                 const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail(s, p, 2); break; }
                 tc_fence_after();
@@ -628,9 +628,9 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             int ab = 0;
             uint32_t aphase = 0;
             for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
-                int g, mt, nt;
-                decode_pair(s, G, tile, g, mt, nt);
-                const int K = g >= p.E ? p.K_shared : p.K_routed;
+                // the shared group, when there is one, is the last: its tiles start
+                // at tile_start[E] (= total without one), so K needs no search
+                const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
                 const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 22); break; }
                 tc_fence_after();
