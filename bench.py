@@ -246,10 +246,15 @@ def workload_config(wl):
 
 
 # ------------------------------------------------------------------ GPU leg
-def run_ours(args, wl, dev, world, rank):
+def run_ours(args, wl, dev, world, rank, fp8=None, steps=None, warmup=None, full=True):
+    """Time K whole-layer steps of `wl` (and, with full, the end-to-end leg
+    and the CPU baseline).  Sub-records pass full=False: the device-resident
+    steps and the staged per-stage pass only."""
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    fp8 = args.experts == "fp8"
+    fp8 = (args.experts == "fp8") if fp8 is None else fp8
+    steps = steps if steps is None else steps
+    warmup = warmup if warmup is None else warmup
     inp = syn.generate(wl, dev, seed=0, weights=not fp8)
     w8 = None
     if fp8:                                         # e4m3 experts (bf16 layer around them)
@@ -270,7 +275,7 @@ def run_ours(args, wl, dev, world, rank):
         if world > 1:
             torch.distributed.barrier(device_ids=[dev.index])
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         layer(inp, out)
     torch.cuda.synchronize(dev)
@@ -281,10 +286,10 @@ def run_ours(args, wl, dev, world, rank):
     # ---- main timed region: K whole-layer steps through moe_forward
     sampler = ClockSampler(dev.index)
     sampler.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     torch.cuda.synchronize(dev)
     barrier()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         layer(inp, out)
@@ -293,7 +298,7 @@ def run_ours(args, wl, dev, world, rank):
     barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = sum(step_ms) / args.steps
+    ms = sum(step_ms) / steps
     srt = sorted(step_ms)
     step_pct = {q: srt[min(len(srt) - 1, int(round(q / 100 * (len(srt) - 1))))] for q in (10, 50, 90)}
     st = nat.moe_get_device_status(ws, stream)
@@ -328,7 +333,7 @@ def run_ours(args, wl, dev, world, rank):
     stages = ["router", "permute", "grouped_ffn", "combine", "balance"]
     stage_ms = {s: [] for s in stages}
     all_evs = []
-    for it in range(args.warmup + args.steps):
+    for it in range(warmup + steps):
         flush.zero_()
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
         evs[0].record(stream)
@@ -354,7 +359,7 @@ def run_ours(args, wl, dev, world, rank):
         evs[4].record(stream)
         nat.moe_balance_stats(cfg, out.counts, psum, out.f, out.P, out.loss, stream)
         evs[5].record(stream)
-        if it >= args.warmup:
+        if it >= warmup:
             all_evs.append(evs)
     torch.cuda.synchronize(dev)       # once: the host runs ahead, so no launch gaps land in a stage
     for evs in all_evs:
@@ -362,6 +367,17 @@ def run_ours(args, wl, dev, world, rank):
             stage_ms[name].append(evs[j].elapsed_time(evs[j + 1]))
     stage_avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
 
+    if not full:
+        e2e_ms = float("nan")
+        x_host = y_host = None
+    else:
+        e2e_ms, x_host, y_host = time_e2e(cfg, inp, out, layer, stream, dev, warmup, steps)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
+    return finish(args, wl, cfg, inp, out, dev, rank, fp8, full, ms, e2e_ms, x_host, y_host, clocks, stage_avg,
+                  step_pct)
+
+
+def time_e2e(cfg, inp, out, layer, stream, dev, warmup, steps):
     # ---- end to end through moe_forward: every step copies its own x in
     # (pinned host -> device) and its y and loss out, all inside the timed
     # region.  Copies run on their own streams with double-buffered device
@@ -375,7 +391,7 @@ def run_ours(args, wl, dev, world, rank):
     x_dev = [torch.empty_like(inp["x"]) for _ in range(nbuf)]
     outs = [nat.Outputs(cfg, dev) for _ in range(nbuf)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    n_e2e = args.warmup + args.steps
+    n_e2e = warmup + steps
     ev_in = [torch.cuda.Event() for _ in range(n_e2e)]
     ev_comp = [torch.cuda.Event() for _ in range(n_e2e)]
     ev_out = [torch.cuda.Event() for _ in range(n_e2e)]
@@ -385,7 +401,7 @@ def run_ours(args, wl, dev, world, rank):
         b = i % nbuf
         if i >= nbuf:
             s_in.wait_event(ev_comp[i - nbuf])       # x_dev[b] is free once its layer ran
-        if i == args.warmup:
+        if i == warmup:
             t_start.record(s_in)
         with torch.cuda.stream(s_in):
             x_dev[b].copy_(x_host, non_blocking=True)
@@ -404,12 +420,20 @@ def run_ours(args, wl, dev, world, rank):
         ev_out[i].record(s_out)
     t_end.record(s_out)
     torch.cuda.synchronize(dev)
-    e2e_ms = t_start.elapsed_time(t_end) / args.steps
-    y_host, loss_host = y_host[0], loss_host[0]
+    e2e_ms = t_start.elapsed_time(t_end) / steps
+    return e2e_ms, x_host, y_host[0]
 
-    # ---- max over ranks
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
+def tensor_peak(peaks, clocks):
+    """The tensor peak a run is held to: the burst figure, unless the clocks
+    sampled during that run's timed region show sw_power_cap active, in which
+    case the sustained (power-capped) figure.  Returns (TFLOP/s, which)."""
+    if "sw_power_cap" in (clocks.get("reasons") or []):
+        return peaks["bf16_tflops_sustained"], "sustained (sw_power_cap active during the timed region)"
+    return peaks["bf16_tflops"], "burst (no power cap during the timed region)"
+
+
+def finish(args, wl, cfg, inp, out, dev, rank, fp8, full, ms, e2e_ms, x_host, y_host, clocks, stage_avg, step_pct):
     counts = out.counts.cpu().numpy()
     cap = nat.capacity(cfg)
     kept_np = np.minimum(counts, cap) if cap >= 0 else counts
@@ -418,26 +442,26 @@ def run_ours(args, wl, dev, world, rank):
     if fp8:       # e4m3 contractions: the measured bf16 peaks x the nominal fp8 : bf16 ratio (2)
         peaks = dict(peaks, bf16_tflops=2 * peaks["bf16_tflops"],
                      bf16_tflops_sustained=2 * peaks["bf16_tflops_sustained"])
-    # The step runs back to back for the whole timed region (power-capped
-    # clocks, sw_power_cap active): the sustained bf16 figure is the tensor
-    # peak; the burst figure is reported beside it.
-    t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    peak_t, peak_which = tensor_peak(peaks, clocks)
+    t_tensor = flops / (peak_t * 1e12)
     t_tensor_burst = flops / (peaks["bf16_tflops"] * 1e12)
+    t_tensor_sust = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
-    layer_roof_ms = max(t_tensor, t_hbm) * 1e3
-    layer_roof_burst_ms = max(t_tensor_burst, t_hbm) * 1e3
     ffn_ms = stage_avg["grouped_ffn"]
     ffn_tflops = flops / (ffn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(wl.name, "grouped_ffn_fp8" if fp8 else "grouped_ffn")
     result = dict(rank=rank, ms=ms, e2e_ms=e2e_ms, clocks=clocks, stage_avg=stage_avg, counts=counts, step_pct=step_pct,
                   flops=flops, alg_bytes=alg_bytes, kept_rows=kept_rows, peaks=peaks, peak_src=peak_src,
-                  layer_roof_ms=layer_roof_ms, layer_roof_burst_ms=layer_roof_burst_ms, ffn_tflops=ffn_tflops,
+                  peak_t=peak_t, peak_which=peak_which,
+                  layer_roof_ms=max(t_tensor, t_hbm) * 1e3, layer_roof_burst_ms=max(t_tensor_burst, t_hbm) * 1e3,
+                  layer_roof_sust_ms=max(t_tensor_sust, t_hbm) * 1e3, ffn_tflops=ffn_tflops,
                   traffic=traffic,
                   loss=float(out.loss.item()), n_dropped=int(out.n_dropped.item()),
-                  bound="tensor" if t_tensor >= t_hbm else "hbm",
-                  h2d=x_host.numel() * x_host.element_size(),
-                  d2h=y_host.numel() * y_host.element_size() + 8, host_inp=None)
-    if rank == 0 and not args.no_cpu_baseline and not fp8:
+                  bound="tensor" if t_tensor >= t_hbm else "hbm")
+    if full:
+        result["h2d"] = x_host.numel() * x_host.element_size()
+        result["d2h"] = y_host.numel() * y_host.element_size() + 8
+    if full and rank == 0 and not args.no_cpu_baseline and not fp8:
         host = host_inputs(inp)
         n, dt_cpu, cores = oracle_sample(wl, host, args.cpu_seconds)
         n1, dt1, _ = oracle_sample(wl, host, max(1.0, args.cpu_seconds / 5), threads=1)
@@ -472,6 +496,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: e4m3 experts through moe_forward_fp8 (bf16 layers only; no CPU baseline)")
+    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8",
+                    help="further workloads (name or name:fp8) timed after the headline one and reported "
+                         "under sub_records; '' for none")
+    ap.add_argument("--sub-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -489,8 +517,12 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=dev)
+    subs = {}
     try:
         r = run_ours(args, wl, dev, world, rank)
+        for spec in [t for t in args.sub.split(",") if t] if args.experts == "bf16" else []:
+            torch.cuda.empty_cache()
+            subs[spec] = sub_record(args, spec, dev, world, rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
@@ -498,11 +530,7 @@ def main():
         return
     tokens_per_s = job_tokens_per_s(world, wl.T, r["ms"])
     e2e_tokens_per_s = job_tokens_per_s(world, wl.T, r["e2e_ms"])
-    peaks = r["peaks"]
-    tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
-    peak_tensor = peaks["bf16_tflops_sustained"]
     fp8 = args.experts == "fp8"
-    peak_kind = ("fp8 (2 x the measured bf16 figure, the nominal fp8 : bf16 ratio)" if fp8 else "bf16")
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
@@ -511,21 +539,9 @@ def main():
                                                                                    else "f32"),
         "data": "synthetic",
         "config": dict(workload_config(wl), parallelism="replicas x%d" % world, experts=args.experts),
-        "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
-        "layer_roofline": {"bound": r["bound"], "time_ms": r["layer_roof_ms"],
-                           "frac": r["layer_roof_ms"] / r["ms"], "flops": r["flops"],
-                           "alg_bytes": r["alg_bytes"],
-                           "frac_burst": r["layer_roof_burst_ms"] / r["ms"],
-                           "peak_note": "sustained " + peak_kind + " (timed inside the back-to-back step loop) "
-                                        "and copy bandwidth, " + tag + "; frac_burst against the burst figure"},
-        "roofline": {"kernel": ("grouped_ffn_fp8 (tcgen05 e4m3 gemm1 + H quantization + gemm2)" if fp8
-                                else "grouped_ffn (tcgen05 gemm1 + gemm2)"), "bound": "tensor",
-                     "achieved": r["ffn_tflops"], "peak": peak_tensor, "unit": "TFLOP/s",
-                     "frac": r["ffn_tflops"] / peak_tensor, "traffic": r["traffic"],
-                     "frac_burst": r["ffn_tflops"] / peaks["bf16_tflops"],
-                     "peak_note": "sustained " + peak_kind + ", " + tag + " (the kernel runs inside the "
-                                  "back-to-back step loop); frac_burst against the burst figure"},
-        "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
+    }
+    line.update(roofline_fields(r, fp8))
+    line.update({
         "step_ms_percentiles": {"p10": r["step_pct"][10], "p50": r["step_pct"][50], "p90": r["step_pct"][90]},
         "e2e": {"value": e2e_tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],
@@ -533,13 +549,57 @@ def main():
                           "neighbouring steps' layers (double-buffered device buffers)"},
         "gpu_launches": launches_per_forward(wl, fp8) * args.steps,
         "clocks": r["clocks"],
+    })
+    if "cpu" in r:
+        line["cpu_baseline"] = r["cpu"]
+    if subs:
+        line["sub_records"] = subs
+    print(json.dumps(line), flush=True)
+
+
+def roofline_fields(r, fp8):
+    """tflops, layer_roofline, roofline (grouped FFN), stages and routing of
+    one measured workload, fractions against the tensor peak its own clock
+    record calls for (tensor_peak), burst and sustained fractions beside."""
+    peaks = r["peaks"]
+    tag = "of measured" if r["peak_src"] == "measured" else "of fallback"
+    kind = "fp8 (2 x the measured bf16 figure, the nominal fp8 : bf16 ratio)" if fp8 else "bf16"
+    return {
+        "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
+        "layer_roofline": {"bound": r["bound"], "time_ms": r["layer_roof_ms"],
+                           "frac": r["layer_roof_ms"] / r["ms"], "flops": r["flops"],
+                           "alg_bytes": r["alg_bytes"],
+                           "frac_burst": r["layer_roof_burst_ms"] / r["ms"],
+                           "frac_sustained": r["layer_roof_sust_ms"] / r["ms"],
+                           "peak_note": "%s %s peak and copy bandwidth, %s" % (r["peak_which"], kind, tag)},
+        "roofline": {"kernel": ("grouped_ffn_fp8 (tcgen05 e4m3 gemm1 + H quantization + gemm2)" if fp8
+                                else "grouped_ffn (tcgen05 gemm1 + gemm2)"), "bound": "tensor",
+                     "achieved": r["ffn_tflops"], "peak": r["peak_t"], "unit": "TFLOP/s",
+                     "frac": r["ffn_tflops"] / r["peak_t"], "traffic": r["traffic"],
+                     "frac_burst": r["ffn_tflops"] / peaks["bf16_tflops"],
+                     "frac_sustained": r["ffn_tflops"] / peaks["bf16_tflops_sustained"],
+                     "peak_note": "%s %s peak, %s" % (r["peak_which"], kind, tag)},
+        "stages_ms": {k: round(v, 4) for k, v in r["stage_avg"].items()},
         "routing": {"kept_rows": r["kept_rows"], "dropped": r["n_dropped"], "loss": r["loss"],
                     "max_count": int(r["counts"].max()), "min_count": int(r["counts"].min()),
                     "active_experts": int((r["counts"] > 0).sum())},
     }
-    if "cpu" in r:
-        line["cpu_baseline"] = r["cpu"]
-    print(json.dumps(line), flush=True)
+
+
+def sub_record(args, spec, dev, world, rank):
+    """One further workload timed like the headline one (device-resident steps
+    with the L2 flushed between them, the staged per-stage pass), reported
+    with its own roofline fractions.  spec: "workload" or "workload:fp8"."""
+    name, _, experts = spec.partition(":")
+    wl = syn.WORKLOADS[name]
+    fp8 = experts == "fp8"
+    r = run_ours(args, wl, dev, world, rank, fp8=fp8, steps=args.sub_steps, warmup=3, full=False)
+    rec = {"workload": name, "experts": "fp8" if fp8 else "bf16", "steps": args.sub_steps, "warmup": 3,
+           "ms_per_step": r["ms"], "tokens_per_s": job_tokens_per_s(world, wl.T, r["ms"]),
+           "step_ms_percentiles": {"p10": r["step_pct"][10], "p50": r["step_pct"][50], "p90": r["step_pct"][90]},
+           "gpu_launches": launches_per_forward(wl, fp8) * args.sub_steps, "clocks": r["clocks"]}
+    rec.update(roofline_fields(r, fp8))
+    return rec
 
 
 if __name__ == "__main__":

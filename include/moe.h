@@ -204,6 +204,28 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        double *loss, float *logits_out, int32_t *n_dropped,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Where moe_forward / moe_forward_fp8 leave their intermediate results inside
+ * a workspace: the dispatch tables (rows in (expert, token) order, see
+ * moe_permute), the packed input rows, the hidden activation and the gated
+ * expert outputs.  They are valid after the forward pass on the workspace's
+ * stream has completed and until the next call that uses the workspace.  A
+ * host-only call: it computes addresses (device pointers into ws) and launches
+ * nothing.  Returns MOE_ERR_INVALID_ARG on a bad config or NULL out,
+ * MOE_ERR_WORKSPACE when ws is NULL, misaligned or smaller than
+ * moe_workspace_size(cfg).                                                  */
+typedef struct {
+    int32_t *kept;        /* [E]            min(counts, capacity)                     */
+    int32_t *offsets;     /* [E+1]          exclusive prefix sum of kept              */
+    int32_t *row_of;      /* [T, top_k]     row of each assignment, -1 when dropped   */
+    int32_t *row_token;   /* [T*top_k]      token of each row (first offsets[E] valid) */
+    float *row_gate;      /* [T*top_k]      gate of each row                          */
+    void *x_perm;         /* [T*top_k, d_model] packed x rows (e4m3 codes with FP8 experts) */
+    void *H;              /* [moe_perm_rows(cfg), hF] hidden activation, hF = h_stride */
+    void *y_perm;         /* [moe_perm_rows(cfg), d_model] gate-scaled expert outputs */
+    int64_t h_stride;     /* row stride of H in elements: max(d_ff, d_ff_shared)      */
+} moe_ws_view;
+MOE_API moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws_bytes, moe_ws_view *out);
+
 /* ---- FP8 (e4m3) experts -----------------------------------------------
  * Quantized experts for serving ("Fine-tuning and serving MoE models",
  * Serving: throughput does not scale the way you expect, consequences for
@@ -283,7 +305,8 @@ MOE_API moe_status moe_routing_health(const moe_config *cfg, const int32_t *coun
 
 /* moe_permute for callers that cannot allocate device memory.  The paper has
  * no counterpart: this entry point exists for integration only.
- * Same computation, arguments and outputs as moe_permute, but no workspace:
+ * Same computation, arguments and outputs as moe_permute (x_perm may be NULL
+ * for the row tables alone), but no workspace:
  * its scratch (per-chunk expert counts and their prefix sums) lives in a
  * static device array inside libmoe (2 MiB + 256 bytes on every GPU that
  * loads the library, held until the process exits).  It serves callers that
@@ -293,7 +316,9 @@ MOE_API moe_status moe_routing_health(const moe_config *cfg, const int32_t *coun
  *   - Limit: E * ceil(T / 64) <= 262144 (E = 256 allows T <= 65536); beyond it
  *     the call returns MOE_ERR_UNSUPPORTED and launches nothing.
  *   - The first call on a device looks up the array's address with that
- *     device current; make that first call before any stream capture.
+ *     device current and keeps it; make that first call before any stream
+ *     capture.  The address is that of the device's current context: after
+ *     cudaDeviceReset, reload the library before calling again.
  *   - All calls share the array: calls that overlap on the GPU race.
  *   - A bad expert id is dropped (row -1) as in moe_permute but, with no
  *     workspace status word, not reported.

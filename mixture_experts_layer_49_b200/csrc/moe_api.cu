@@ -391,6 +391,24 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     return MOE_OK;
 }
 
+moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws_bytes, moe_ws_view *out) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(out);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    const Layout L = layout(cfg);
+    out->kept = at<int32_t>(ws, L.kept);
+    out->offsets = at<int32_t>(ws, L.offsets);
+    out->row_of = at<int32_t>(ws, L.row_of);
+    out->row_token = at<int32_t>(ws, L.row_token);
+    out->row_gate = at<float>(ws, L.row_gate);
+    out->x_perm = at<char>(ws, L.x_perm);
+    out->H = at<char>(ws, L.H);
+    out->y_perm = at<char>(ws, L.y_perm);
+    out->h_stride = cfg->d_ff > cfg->d_ff_shared ? cfg->d_ff : cfg->d_ff_shared;
+    return MOE_OK;
+}
+
 moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float *sel_bias, float gamma,
                            moe_stream_t stream) {
     moe_status s = check_cfg(cfg);

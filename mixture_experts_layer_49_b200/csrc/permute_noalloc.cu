@@ -18,7 +18,10 @@
 //     problems are rejected with MOE_ERR_UNSUPPORTED before any launch.
 //   - The first call on a device looks up the array's device address
 //     (cudaGetSymbolAddress) with that device current and caches it; make that
-//     first call before any stream capture.
+//     first call before any stream capture.  The cached address belongs to the
+//     device's current context: after cudaDeviceReset on that device the
+//     library must be reloaded (the module, and so the array, may then sit at
+//     another address).
 //   - All calls share the one array: calls that overlap on the GPU (two
 //     streams, or two host threads) race on it.  Each call rewrites every
 //     count it reads, and clears the status header it owns first.
@@ -77,7 +80,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, 
     moe_status s = moe::validate_config(cfg);
     if (s != MOE_OK) return s;
     if (!counts || !kept || !offsets) return reject(MOE_ERR_INVALID_ARG, "NULL counts, kept or offsets");
-    if (cfg->T > 0 && (!x || !idx || !gate || !row_of || !row_token || !row_gate || !x_perm))
+    // x_perm may be NULL (row tables only), as in moe_permute
+    if (cfg->T > 0 && (!x || !idx || !gate || !row_of || !row_token || !row_gate))
         return reject(MOE_ERR_INVALID_ARG, "NULL input or output array");
     auto mis = [](const void *p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) != 0; };
     if (mis(x, 16) || mis(x_perm, 16) || mis(idx, 4) || mis(gate, 4) || mis(counts, 4) || mis(kept, 4) ||

@@ -29,7 +29,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
-           "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8")
+           "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -38,6 +38,14 @@ class MoeFp8Experts(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
         "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")]
+
+
+class MoeWsView(ctypes.Structure):
+    """moe_ws_view: device addresses of the forward pass's intermediate
+    results inside a workspace."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "kept", "offsets", "row_of", "row_token", "row_gate", "x_perm", "H", "y_perm")] + [
+        ("h_stride", ctypes.c_int64)]
 
 
 class MoEError(RuntimeError):
@@ -94,6 +102,8 @@ def lib():
         L.moe_bias_update.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_float, c_vp]
         L.moe_routing_health.restype = ctypes.c_int
         L.moe_routing_health.argtypes = [P(MoeConfig), c_vp, c_vp, c_vp, c_vp]
+        L.moe_workspace_view.restype = ctypes.c_int
+        L.moe_workspace_view.argtypes = [P(MoeConfig), c_vp, ctypes.c_size_t, P(MoeWsView)]
         L.moe_check_wait_timeout.restype = ctypes.c_int
         L.moe_check_wait_timeout.argtypes = [c_vp, ctypes.c_uint64, c_vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
@@ -236,6 +246,38 @@ def moe_forward(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh
                              _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g), _p(Wsh_u), _p(Wsh_d), _p(y),
                              _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss), _p(logits_out),
                              _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_workspace_view(cfg, ws) -> MoeWsView:
+    v = MoeWsView()
+    _check(lib().moe_workspace_view(ctypes.byref(cfg), _p(ws), ws.numel() * ws.element_size(), ctypes.byref(v)),
+           "moe_workspace_view")
+    return v
+
+
+def workspace_tables(cfg, ws) -> dict:
+    """The forward pass's dispatch tables and intermediate rows as tensors
+    that alias the workspace (slices of `ws` at the addresses
+    moe_workspace_view reports)."""
+    v = moe_workspace_view(cfg, ws)
+    base = ws.data_ptr()
+    T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.top_k
+    rows = perm_rows(cfg)
+    dt = layer_dtype(cfg)
+
+    def region(addr, n, dtype, shape):
+        off = addr - base
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype).view(shape)
+
+    return dict(kept=region(v.kept, E, torch.int32, (E,)),
+                offsets=region(v.offsets, E + 1, torch.int32, (E + 1,)),
+                row_of=region(v.row_of, T * k, torch.int32, (T, k)),
+                row_token=region(v.row_token, T * k, torch.int32, (T * k,)),
+                row_gate=region(v.row_gate, T * k, torch.float32, (T * k,)),
+                x_perm=region(v.x_perm, T * k * d, dt, (T * k, d)),
+                H=region(v.H, rows * v.h_stride, dt, (rows, v.h_stride)),
+                y_perm=region(v.y_perm, rows * d, dt, (rows, d)))
 
 
 def moe_bias_update(cfg, counts, sel_bias, gamma, stream=None):

@@ -176,3 +176,33 @@ def test_fp8_entry_points_check_arguments():
     assert L.moe_quantize_rows_e4m3(fake(), 4, 16, 16, fake(), 12, fake(), None) == nat.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_rows_e4m3(None, 4, 16, 16, fake(), 16, fake(), None) == nat.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_rows_e4m3(None, 0, 16, 16, None, 16, None, None) == nat.MOE_OK
+
+
+def test_workspace_view_addresses():
+    # a host-only call: addresses inside the workspace, in increasing order,
+    # aligned for their element type, every region inside ws_bytes
+    for c in (cfg(T=300), cfg(T=300, d_ff_shared=64), cfg(T=64, dtype="f32"), cfg(T=0)):
+        base, n = 1 << 20, nat.workspace_size(c)
+        v = nat.MoeWsView()
+        assert nat.lib().moe_workspace_view(ctypes.byref(c), ctypes.c_void_p(base), n, ctypes.byref(v)) == nat.MOE_OK
+        T, d, E, k = c.T, c.d_model, c.E, c.top_k
+        esz = 2 if c.dtype == nat.MOE_BF16 else 4
+        rows = nat.perm_rows(c)
+        regions = [(v.kept, 4 * E), (v.offsets, 4 * (E + 1)), (v.row_of, 4 * T * k), (v.row_token, 4 * T * k),
+                   (v.row_gate, 4 * T * k), (v.x_perm, esz * T * k * d), (v.H, esz * rows * v.h_stride),
+                   (v.y_perm, esz * rows * d)]
+        assert v.h_stride == max(c.d_ff, c.d_ff_shared)
+        end = base + 256                               # after the status header
+        for addr, nbytes in regions:
+            assert addr % 256 == 0 and addr >= end
+            end = addr + nbytes
+        assert end <= base + n
+    c = cfg()
+    v = nat.MoeWsView()
+    L = nat.lib()
+    assert L.moe_workspace_view(ctypes.byref(c), ctypes.c_void_p(4096), nat.workspace_size(c) - 1,
+                                ctypes.byref(v)) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_view(ctypes.byref(c), ctypes.c_void_p(4096 + 8), nat.workspace_size(c),
+                                ctypes.byref(v)) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_view(ctypes.byref(c), ctypes.c_void_p(4096), nat.workspace_size(c),
+                                None) == nat.MOE_ERR_INVALID_ARG

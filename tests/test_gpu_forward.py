@@ -1,12 +1,16 @@
 """GPU parity of the whole layer (moe_forward through the C ABI) against the
 CPU oracle on the same seeded inputs.
 
-Routing (expert ids, counts, capacity drops) must match bit for bit; gates to
-1e-5; the output to max|y - y_ref| / max|y_ref| <= 2e-2 for bf16 layers and
-1e-4 for fp32 layers; the balance loss to 1e-5 relative.  Small cases are
-checked on every token; the five full-size workloads run in the benchmark's
-launch configuration and are checked over all tokens for routing and loss,
-and on sampled tokens (covering every expert that kept a row) for y.
+Routing (expert ids, counts, capacity drops) and the dispatch tables the
+forward pass leaves in its workspace (kept, offsets, row_of, row_token: the
+(expert, token) row order) must match bit for bit; gates to 1e-5; the output
+to max|y - y_ref| / max|y_ref| <= 2e-2 for bf16 layers and 1e-4 for fp32
+layers; the balance loss to 1e-5 relative.  Small cases are checked on every
+token.  The five full-size workloads run in the benchmark's launch
+configuration: routing, dispatch tables and loss over all tokens; y over all
+tokens for the fp32, Switch- and Qwen3-shaped layers and over 2048 sampled
+tokens plus one token of every expert that kept a row for the Mixtral- and
+DeepSeek-shaped layers (whose fp64 oracle costs about 0.7 GFLOP per token).
 """
 import numpy as np
 import pytest
@@ -41,9 +45,25 @@ def check_forward(wl, inp, host, n_sample=None, seed=0):
     dp = oracle.dispatch(dims, r["idx"])
     bal = oracle.balance(dims, dp["counts"], r["pnorm"])
 
-    swapped = check_routing(out.idx.cpu().numpy(), out.gate.cpu().numpy(), r)
+    gpu_idx = out.idx.cpu().numpy()
+    swapped = check_routing(gpu_idx, out.gate.cpu().numpy(), r)
     np.testing.assert_array_equal(out.counts.cpu().numpy(), dp["counts"])
     assert int(out.n_dropped.item()) == dp["n_dropped"]
+    # the forward pass's dispatch tables against the oracle's dispatch of the
+    # same expert ids (slot order may differ from the oracle's only between
+    # tied keys; the tables of a given selection are unique)
+    dpg = dp if swapped == 0 else oracle.dispatch(dims, gpu_idx)
+    tab = nat.workspace_tables(cfg, ws)
+    nrows = int(dpg["offsets"][-1])
+    np.testing.assert_array_equal(tab["kept"].cpu().numpy(), dpg["kept"])
+    np.testing.assert_array_equal(tab["offsets"].cpu().numpy(), dpg["offsets"])
+    np.testing.assert_array_equal(tab["row_of"].cpu().numpy(), dpg["row_of"])
+    np.testing.assert_array_equal(tab["row_token"][:nrows].cpu().numpy(), dpg["row_token"])
+    # each row carries its assignment's gate, bit for bit
+    ro = dpg["row_of"]
+    kept_slots = ro >= 0
+    np.testing.assert_array_equal(tab["row_gate"][:nrows].cpu().numpy()[ro[kept_slots]],
+                                  out.gate.cpu().numpy()[kept_slots])
     assert rel_err(out.logits.cpu().numpy(), r["logits"]) < TOL_LOGIT
     loss = float(out.loss.item())
     assert abs(loss - bal["loss"]) <= TOL_LOSS * abs(bal["loss"])
@@ -90,14 +110,28 @@ def test_forward_small(wl, cuda_device):
     check_forward(wl, inp, host)
 
 
+# y checked on every token (None) or on this many sampled tokens plus one
+# token of every expert that kept a row
+FULL_SIZE_Y_TOKENS = {"tiny_fp32": None, "switch_top1": None, "qwen3_moe": None, "mixtral": 2048,
+                      "deepseek_v3": 2048}
+
+
 @pytest.mark.parametrize("name", ["tiny_fp32", "switch_top1", "mixtral", "qwen3_moe", "deepseek_v3"])
 def test_forward_full_size(name, cuda_device):
     wl = syn.WORKLOADS[name]
     inp, host = make_case(wl, cuda_device, seed=0)
-    n_sample = None if wl.T * wl.d_model * wl.d_ff <= 256 * 128 * 256 else 48
-    res = check_forward(wl, inp, host, n_sample=n_sample)
+    res = check_forward(wl, inp, host, n_sample=FULL_SIZE_Y_TOKENS[name])
     print("%s: max rel err %.3e, loss %.6f (ref %.6f), %d tokens checked, %d tie-swapped slot orders" % (
         name, res["err"], res["loss"], res["loss_ref"], len(res["tokens"]), res["swapped"]))
+
+
+def test_forward_long_sequence(cuda_device):
+    # T = 20000 tokens: 313 dispatch chunks, so the per-expert scan over chunks
+    # takes two passes (256 chunks each); tight capacity drops assignments
+    wl = W("long_T", T=20000, d_model=128, E=16, d_ff=128, top_k=2, capacity_factor=0.9, logit_skew="normal")
+    inp, host = make_case(wl, cuda_device, seed=2)
+    res = check_forward(wl, inp, host)
+    assert res["dp"]["n_dropped"] > 0
 
 
 def test_forward_is_deterministic(cuda_device):
