@@ -226,6 +226,42 @@ typedef struct {
 } moe_ws_view;
 MOE_API moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws_bytes, moe_ws_view *out);
 
+/* ---- Expert parallelism -------------------------------------------------
+ * The experts sharded over R ranks, each rank holding E / R of them ("Fine-
+ * Tuning Mixture of Experts (MoE) Models: Router Optimization Techniques",
+ * Why It Matters 2, token dispatch and gather, and Architecture & Distributed
+ * Execution; "Mixture-of-Experts", Vector Institute post, expert-parallelism
+ * paragraph): every rank routes and permutes its own tokens (moe_router_topk,
+ * moe_permute), so the rows bound for rank j are the contiguous range of j's
+ * experts; the rows travel to their experts' rank (an all-to-all of
+ * variable-size blocks), run through that rank's experts, travel back and are
+ * combined where they came from (moe_combine).  The entry point below is the
+ * middle step: the grouped FFN over the rows a rank received.
+ *
+ * moe_ep_grouped_ffn: cfg describes the local experts: E = experts held by
+ * this rank, d_model, d_ff, dtype, act (T, top_k, score, renorm, capacity and
+ * d_ff_shared are not used; run a shared expert with moe_grouped_ffn).  The
+ * received rows come as n_src blocks (one per source rank), each holding the
+ * source's rows for local expert 0, 1, ..., E-1 in turn, so there are
+ * n_src * E row groups (at most 256): group g = src * E + e holds rows
+ * group_offsets[g] .. group_offsets[g+1] and uses local expert e:
+ *   y_rows[r] = row_gate[r] * expert_e(x_rows[r])   (bf16 or fp32 as in
+ *   moe_grouped_ffn: GELU with b1 / b2, or SwiGLU)
+ *   group_offsets [n_src*E + 1] int32 device, non-decreasing, from 0 to at
+ *       most max_rows;  x_rows, y_rows [max_rows, d_model];  row_gate [max_rows]
+ *   W1, Wu [E, d_ff, d_model]; W2 [E, d_model, d_ff]; b1 [E, d_ff], b2
+ *       [E, d_model] (GELU, may be NULL): the local experts' slices.
+ * Rows past group_offsets[n_src*E] are left untouched.  The workspace (its
+ * first 256 bytes a status word, as for the other entry points) holds the
+ * hidden activation: moe_ep_workspace_size(cfg, n_src, max_rows) bytes (0 on
+ * a bad argument).                                                         */
+MOE_API size_t moe_ep_workspace_size(const moe_config *cfg, int32_t n_src, int64_t max_rows);
+MOE_API moe_status moe_ep_grouped_ffn(const moe_config *cfg, int32_t n_src, const int32_t *group_offsets,
+                                      int64_t max_rows, const void *x_rows, const float *row_gate,
+                                      const void *W1, const float *b1, const void *Wu, const void *W2,
+                                      const float *b2, void *y_rows, void *ws, size_t ws_bytes,
+                                      moe_stream_t stream);
+
 /* ---- FP8 (e4m3) experts -----------------------------------------------
  * Quantized experts for serving ("Fine-tuning and serving MoE models",
  * Serving: throughput does not scale the way you expect, consequences for

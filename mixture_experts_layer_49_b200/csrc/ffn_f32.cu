@@ -39,12 +39,12 @@ __global__ void __launch_bounds__(kThreads) simt_grouped_gemm(FfnArgs a) {
     __shared__ float Bs2[MODE == MODE_SWIGLU ? BK : 1][BN + 4];
 
     const int tid = threadIdx.x;
-    const int G = a.E + (a.S > 0 ? 1 : 0);
+    const int G = a.n_groups + (a.S > 0 ? 1 : 0);
     if (tid == 0) {
         int acc = 0;
         for (int g = 0; g < G; ++g) {
             tab.mt_start[g] = acc;
-            const int rows = g < a.E ? a.offsets[g + 1] - a.offsets[g] : a.T;
+            const int rows = g < a.n_groups ? a.offsets[g + 1] - a.offsets[g] : a.T;
             acc += (rows + BM - 1) / BM;
         }
         tab.mt_start[G] = acc;
@@ -54,8 +54,9 @@ __global__ void __launch_bounds__(kThreads) simt_grouped_gemm(FfnArgs a) {
     if (mt >= tab.mt_start[G]) return;
     int g = 0;
     while (tab.mt_start[g + 1] <= mt) ++g;
-    const bool shared = g >= a.E;
+    const bool shared = g >= a.n_groups;
     const int rows = shared ? a.T : a.offsets[g + 1] - a.offsets[g];
+    const int e = shared ? 0 : (a.n_groups == a.E ? g : g % a.E);     // weight expert of the group
     const int m0 = (mt - tab.mt_start[g]) * BM;
     const int64_t out_row0 = shared ? a.shared_base : (int64_t)a.offsets[g];
 
@@ -68,17 +69,17 @@ __global__ void __launch_bounds__(kThreads) simt_grouped_gemm(FfnArgs a) {
         N = shared ? a.S : a.F;
         A = shared ? static_cast<const float *>(a.x) : static_cast<const float *>(a.x_perm) + out_row0 * a.d;
         lda = a.d;
-        W = shared ? static_cast<const float *>(a.Wsg) : static_cast<const float *>(a.W1) + (size_t)g * a.F * a.d;
+        W = shared ? static_cast<const float *>(a.Wsg) : static_cast<const float *>(a.W1) + (size_t)e * a.F * a.d;
         if (MODE == MODE_SWIGLU)
-            W2nd = shared ? static_cast<const float *>(a.Wsu) : static_cast<const float *>(a.Wu) + (size_t)g * a.F * a.d;
-        if (MODE == MODE_GELU && !shared && a.b1) bias = a.b1 + (size_t)g * a.F;
+            W2nd = shared ? static_cast<const float *>(a.Wsu) : static_cast<const float *>(a.Wu) + (size_t)e * a.F * a.d;
+        if (MODE == MODE_GELU && !shared && a.b1) bias = a.b1 + (size_t)e * a.F;
     } else {
         K = shared ? a.S : a.F;
         N = a.d;
         A = static_cast<const float *>(a.H) + out_row0 * a.hF;
         lda = a.hF;
-        W = shared ? static_cast<const float *>(a.Wsd) : static_cast<const float *>(a.W2) + (size_t)g * a.d * a.F;
-        if (!shared && a.b2) bias = a.b2 + (size_t)g * a.d;
+        W = shared ? static_cast<const float *>(a.Wsd) : static_cast<const float *>(a.W2) + (size_t)e * a.d * a.F;
+        if (!shared && a.b2) bias = a.b2 + (size_t)e * a.d;
     }
     const int n0 = blockIdx.y * BN;
     if (n0 >= N) return;
@@ -154,9 +155,9 @@ __global__ void __launch_bounds__(kThreads) simt_grouped_gemm(FfnArgs a) {
 }  // namespace
 
 cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st) {
-    if (a.T == 0) return cudaSuccess;
-    const int64_t routed = (int64_t)a.T * a.k;
-    int64_t mtiles = (routed + BM - 1) / BM + a.E;
+    if (a.routed_rows == 0 && (a.S == 0 || a.T == 0)) return cudaSuccess;
+    const int64_t routed = a.routed_rows;
+    int64_t mtiles = (routed + BM - 1) / BM + a.n_groups;
     if (a.S > 0) mtiles += (a.T + BM - 1) / BM + 1;
     const int n1 = (a.F > a.S ? a.F : a.S);
     dim3 g1((unsigned)mtiles, (unsigned)((n1 + BN - 1) / BN));

@@ -74,12 +74,13 @@ constexpr uint32_t kIdescF8 = make_idesc_e4m3(BM, BNB);
 template <bool F8> constexpr int bk_elems() { return F8 ? 128 : 64; }
 
 struct GemmParams {
-    const int32_t *offsets;   // [E+1]
+    const int32_t *offsets;   // [E+1]: routed group g holds rows offsets[g] .. offsets[g+1]
     const float *bias;        // [E, N_routed] or null (GELU b1 / b2)
     const float *row_gate;    // [rows] (GM_DOWN) or null
     __nv_bfloat16 *out;       // row stride ldo
     int32_t *status;
-    int E, T;
+    int E, T;                 // E: routed groups (the shared group, if any, is group E)
+    int E_w;                  // experts in the weight tensors: routed group g uses expert g % E_w
     int K_routed, K_shared;
     int N_routed, N_shared;
     int has_shared;
@@ -98,6 +99,12 @@ struct GemmParams {
     const float *sh_col_scale;      // [N_shared]
     const float *sh_col_scale2;     // [N_shared]
 };
+
+// Weight expert of routed group g (groups are the experts themselves, or, for
+// rows gathered from several sources, consecutive runs of all E_w experts).
+__device__ __forceinline__ int group_expert(const GemmParams &p, int g) {
+    return p.E == p.E_w ? g : g % p.E_w;
+}
 
 struct SmemTail {
     uint64_t full[STAGES];
@@ -176,9 +183,9 @@ template <int MODE>
 __device__ __forceinline__ void preload_scales(const GemmParams &p, bool sh, int g, int nt, int half, int N,
                                                bool valid, int64_t arow, float &rscale, float *csv) {
     rscale = valid ? __ldg((sh ? p.shared_row_scale : p.row_scale) + arow) : 0.f;
-    const float *cs = sh ? p.sh_col_scale : p.col_scale + (size_t)g * p.N_routed;
+    const float *cs = sh ? p.sh_col_scale : p.col_scale + (size_t)group_expert(p, g) * p.N_routed;
     if (MODE == GM_SWIGLU) {
-        const float *cs2 = sh ? p.sh_col_scale2 : p.col_scale2 + (size_t)g * p.N_routed;
+        const float *cs2 = sh ? p.sh_col_scale2 : p.col_scale2 + (size_t)group_expert(p, g) * p.N_routed;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = nt * 128 + (half * 2 + cc) * 32;
@@ -364,7 +371,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = sh ? &tmBs : &tmB;
                 const CUtensorMap *mB2 = sh ? &tmBs2 : &tmB2;
-                const int e = sh ? 0 : g;
+                const int e = sh ? 0 : group_expert(p, g);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail(s, p, 1); break; }
                     const uint32_t fb = smem_u32(&s.full[stage]);
@@ -449,7 +456,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
-            const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+            const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
                                    rscale, csv);
             tc_fence_before();
@@ -609,7 +616,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = (MODE == GM_SWIGLU && rank == 1) ? (sh ? &tmBs2 : &tmB2) : (sh ? &tmBs : &tmB);
                 const int b_row = (MODE == GM_SWIGLU) ? nt * 128 : nt * BNB + (int)rank * 128;
-                const int e = sh ? 0 : g;
+                const int e = sh ? 0 : group_expert(p, g);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 21); break; }
                     const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
@@ -682,7 +689,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
-            const float *bias = (!sh && p.bias) ? p.bias + (size_t)g * p.N_routed : nullptr;
+            const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
                                    rscale, csv);
             tc_fence_before();
@@ -810,7 +817,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
     constexpr int es = F8 ? 1 : 2;                 // bytes per A / B element
     const bool swiglu = a.act == MOE_ACT_SWIGLU;
     const bool has_sh = a.S > 0;
-    const uint64_t routed_rows = (uint64_t)a.T * a.k;
+    const uint64_t routed_rows = (uint64_t)a.routed_rows;
     const uint64_t all_rows = routed_rows + (has_sh ? (uint64_t)a.T : 0);
     const int grid = a.num_sms > 0 ? a.num_sms : 148;
     const uint64_t timeout_ns = 2000000000ull;
@@ -842,7 +849,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.row_gate = nullptr;
     p1.out = static_cast<__nv_bfloat16 *>(a.H);
     p1.status = a.status;
-    p1.E = a.E; p1.T = a.T;
+    p1.E = a.n_groups; p1.E_w = a.E; p1.T = a.T;
     p1.K_routed = a.d; p1.K_shared = a.d;
     p1.N_routed = a.F; p1.N_shared = a.S;
     p1.has_shared = has_sh ? 1 : 0;
@@ -894,7 +901,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
         q.rows = (int64_t)routed_rows;
         q.row0 = 0;
         q.cols = a.F;
-        q.rows_limit = a.offsets + a.E;
+        q.rows_limit = a.offsets + a.n_groups;
         q.num_sms = a.num_sms;
         q.pdl = true;
         if ((err = launch_quant_rows(q, st)) != cudaSuccess) return err;
@@ -924,7 +931,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
     p2.row_gate = a.row_gate;
     p2.out = static_cast<__nv_bfloat16 *>(a.y_perm);
     p2.status = a.status;
-    p2.E = a.E; p2.T = a.T;
+    p2.E = a.n_groups; p2.E_w = a.E; p2.T = a.T;
     p2.K_routed = a.F; p2.K_shared = a.S;
     p2.N_routed = a.d; p2.N_shared = a.d;
     p2.has_shared = has_sh ? 1 : 0;
@@ -956,7 +963,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
-    if (a.T == 0) return cudaSuccess;
+    if (a.routed_rows == 0 && (a.S == 0 || a.T == 0)) return cudaSuccess;
     return a.f8 ? run_ffn<true>(a, st) : run_ffn<false>(a, st);
 }
 

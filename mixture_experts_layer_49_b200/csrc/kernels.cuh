@@ -88,11 +88,13 @@ int dispatch_chunks(int T);
 // x_bytes: bytes per element of x and x_perm (4 fp32, 2 bf16, 1 e4m3 codes)
 cudaError_t launch_dispatch(const DispatchArgs &a, int x_bytes, cudaStream_t st);
 
-// Grouped expert FFN.  Group g < E is routed expert g (rows offsets[g] ..
-// offsets[g+1] of x_perm / H / y_perm); group E is the shared expert (rows
-// 0..T-1 of x, rows shared_base.. of H / y_perm).
+// Grouped expert FFN.  Routed group g < n_groups holds rows offsets[g] ..
+// offsets[g+1] of x_perm / H / y_perm and uses weight expert g % E (n_groups
+// = E: group g is expert g; rows gathered from several sources come as
+// n_groups = sources * E runs of all E experts); group n_groups is the shared
+// expert (rows 0..T-1 of x, rows shared_base.. of H / y_perm).
 struct FfnArgs {
-    const void *x_perm;          // [T*k, d]
+    const void *x_perm;          // [routed_rows, d]
     const void *x;               // [T, d] (shared expert) or null
     const int32_t *offsets;      // [E+1]
     const float *row_gate;       // [T*k]
@@ -102,7 +104,9 @@ struct FfnArgs {
     void *H;                     // [T*k (+T), max(F, S)] scratch, row stride hF
     void *y_perm;                // [T*k (+T), d]
     int32_t *status;
-    int T, d, E, k, F, S, act;   // S = d_ff_shared (0: none)
+    int T, d, E, k, F, S, act;   // S = d_ff_shared (0: none); E: experts in the weights
+    int n_groups;                // routed groups (a multiple of E)
+    int64_t routed_rows;         // rows of x_perm / routed rows of H and y_perm
     int hF;                      // row stride of H in elements
     int64_t shared_base;         // = T*k
     int num_sms;

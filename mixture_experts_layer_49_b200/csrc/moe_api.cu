@@ -180,6 +180,8 @@ moe::FfnArgs ffn_args(const moe_config *c, const void *x_perm, const int32_t *of
     a.y_perm = y_perm;
     a.status = status_word(ws);
     a.T = c->T; a.d = c->d_model; a.E = c->E; a.k = c->top_k; a.F = c->d_ff; a.S = c->d_ff_shared;
+    a.n_groups = c->E;
+    a.routed_rows = (int64_t)c->T * c->top_k;
     a.act = c->act;
     a.hF = c->d_ff > c->d_ff_shared ? c->d_ff : c->d_ff_shared;
     a.shared_base = (int64_t)c->T * c->top_k;
@@ -200,6 +202,26 @@ void set_fp8(moe::FfnArgs &a, const moe_config *c, const moe_fp8_experts *w, con
     a.h_scale = at<float>(ws, L.h_scale);
 }
 
+// ---- expert parallelism: the grouped FFN over rows gathered from n_src sources
+moe_status check_ep_cfg(const moe_config *c, int32_t n_src, int64_t max_rows) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL%s");
+    if (c->E < 1) return fail(MOE_ERR_INVALID_ARG, "E (local experts) < 1%s");
+    if (n_src < 1) return fail(MOE_ERR_INVALID_ARG, "n_src < 1%s");
+    if ((int64_t)n_src * c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "n_src * E (row groups) > 256%s");
+    if (c->d_model < 1 || c->d_ff < 1) return fail(MOE_ERR_INVALID_ARG, "non-positive width%s");
+    if (c->d_model % 8 || c->d_ff % 8) return fail(MOE_ERR_UNSUPPORTED, "d_model and d_ff must be multiples of 8%s");
+    if (c->d_model > 65536 || c->d_ff > 65536) return fail(MOE_ERR_UNSUPPORTED, "widths above 65536%s");
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "bad dtype%s");
+    if (c->act != MOE_ACT_GELU_BIAS && c->act != MOE_ACT_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "bad act%s");
+    if (max_rows < 0) return fail(MOE_ERR_INVALID_ARG, "max_rows < 0%s");
+    if (max_rows >= ((int64_t)1 << 31) - 256) return fail(MOE_ERR_UNSUPPORTED, "max_rows too large%s");
+    return MOE_OK;
+}
+size_t ep_h_offset() { return sizeof(moe::WsHeader); }
+size_t ep_ws_bytes(const moe_config *c, int64_t max_rows) {
+    const size_t esz = c->dtype == MOE_BF16 ? 2 : 4;
+    return align256(ep_h_offset() + (size_t)max_rows * c->d_ff * esz);
+}
 }  // namespace
 
 namespace moe {
@@ -389,6 +411,47 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
+}
+
+size_t moe_ep_workspace_size(const moe_config *cfg, int32_t n_src, int64_t max_rows) {
+    if (check_ep_cfg(cfg, n_src, max_rows) != MOE_OK) return 0;
+    return ep_ws_bytes(cfg, max_rows);
+}
+
+moe_status moe_ep_grouped_ffn(const moe_config *cfg, int32_t n_src, const int32_t *group_offsets, int64_t max_rows,
+                              const void *x_rows, const float *row_gate, const void *W1, const float *b1,
+                              const void *Wu, const void *W2, const float *b2, void *y_rows, void *ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_ep_cfg(cfg, n_src, max_rows);
+    if (s != MOE_OK) return s;
+    NEED(group_offsets);
+    if (max_rows > 0) {
+        NEED(x_rows); NEED(row_gate); NEED(y_rows); NEED(W1); NEED(W2);
+        if (cfg->act == MOE_ACT_SWIGLU) NEED(Wu);
+    }
+    ALIGNED(x_rows, 16); ALIGNED(y_rows, 16); ALIGNED(W1, 16); ALIGNED(Wu, 16); ALIGNED(W2, 16);
+    ALIGNED(group_offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4); ALIGNED(b2, 4);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL%s");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    if (ws_bytes < ep_ws_bytes(cfg, max_rows))
+        return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_ep_workspace_size()%s");
+    if (max_rows == 0) return MOE_OK;
+    moe::FfnArgs a{};
+    a.x_perm = x_rows; a.x = nullptr; a.offsets = group_offsets; a.row_gate = row_gate;
+    a.W1 = W1; a.Wu = Wu; a.W2 = W2; a.b1 = b1; a.b2 = b2;
+    a.H = at<char>(ws, ep_h_offset());
+    a.y_perm = y_rows;
+    a.status = status_word(ws);
+    a.T = 0; a.d = cfg->d_model; a.E = cfg->E; a.k = 1; a.F = cfg->d_ff; a.S = 0;
+    a.n_groups = n_src * cfg->E;
+    a.routed_rows = max_rows;
+    a.act = cfg->act;
+    a.hF = cfg->d_ff;
+    a.shared_base = max_rows;
+    a.num_sms = num_sms();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cfg->dtype == MOE_BF16 ? moe::launch_ffn_bf16(a, st) : moe::launch_ffn_f32(a, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ep_grouped_ffn");
 }
 
 moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws_bytes, moe_ws_view *out) {

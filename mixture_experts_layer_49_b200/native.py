@@ -29,7 +29,8 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_combine", "moe_balance_stats", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
-           "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view")
+           "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
+           "moe_ep_workspace_size", "moe_ep_grouped_ffn")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -102,6 +103,11 @@ def lib():
         L.moe_bias_update.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_float, c_vp]
         L.moe_routing_health.restype = ctypes.c_int
         L.moe_routing_health.argtypes = [P(MoeConfig), c_vp, c_vp, c_vp, c_vp]
+        L.moe_ep_workspace_size.restype = ctypes.c_size_t
+        L.moe_ep_workspace_size.argtypes = [P(MoeConfig), c_i32, ctypes.c_int64]
+        L.moe_ep_grouped_ffn.restype = ctypes.c_int
+        L.moe_ep_grouped_ffn.argtypes = [P(MoeConfig), c_i32, c_vp, ctypes.c_int64] + [c_vp] * 9 + [
+            ctypes.c_size_t, c_vp]
         L.moe_workspace_view.restype = ctypes.c_int
         L.moe_workspace_view.argtypes = [P(MoeConfig), c_vp, ctypes.c_size_t, P(MoeWsView)]
         L.moe_check_wait_timeout.restype = ctypes.c_int
@@ -246,6 +252,21 @@ def moe_forward(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh
                              _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g), _p(Wsh_u), _p(Wsh_d), _p(y),
                              _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss), _p(logits_out),
                              _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def ep_workspace_size(cfg, n_src, max_rows) -> int:
+    n = int(lib().moe_ep_workspace_size(ctypes.byref(cfg), int(n_src), int(max_rows)))
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_ep_workspace_size", last_error_detail())
+    return n
+
+
+def moe_ep_grouped_ffn(cfg, n_src, group_offsets, x_rows, row_gate, W1, b1, Wu, W2, b2, y_rows, ws, stream=None):
+    """Grouped FFN over rows received from n_src sources: group src * E + e
+    (rows group_offsets[g] .. group_offsets[g+1]) uses local expert e."""
+    _check(lib().moe_ep_grouped_ffn(ctypes.byref(cfg), int(n_src), _p(group_offsets), int(x_rows.shape[0]),
+                                    _p(x_rows), _p(row_gate), _p(W1), _p(b1), _p(Wu), _p(W2), _p(b2), _p(y_rows),
+                                    _p(ws), ws.numel(), _stream(stream)), "moe_ep_grouped_ffn")
 
 
 def moe_workspace_view(cfg, ws) -> MoeWsView:

@@ -206,3 +206,24 @@ def test_workspace_view_addresses():
                                 ctypes.byref(v)) == nat.MOE_ERR_WORKSPACE
     assert L.moe_workspace_view(ctypes.byref(c), ctypes.c_void_p(4096), nat.workspace_size(c),
                                 None) == nat.MOE_ERR_INVALID_ARG
+
+
+def test_ep_grouped_ffn_host_checks():
+    L = nat.lib()
+    c = nat.make_config(0, 64, 4, 64, 1)
+    assert L.moe_ep_workspace_size(ctypes.byref(c), 3, 100) == 256 + 100 * 64 * 2
+    assert L.moe_ep_workspace_size(ctypes.byref(c), 64, 0) > 0                 # 256 groups
+    assert L.moe_ep_workspace_size(ctypes.byref(c), 65, 0) == 0                 # 260 groups
+    assert L.moe_ep_workspace_size(ctypes.byref(c), 0, 10) == 0
+    assert L.moe_ep_workspace_size(ctypes.byref(nat.make_config(0, 60, 4, 64, 1)), 1, 10) == 0
+    ws = fake(16)
+    n = L.moe_ep_workspace_size(ctypes.byref(c), 2, 10)
+    args = [fake(), 10, fake(), fake(), fake(), None, fake(), fake(), None, fake()]
+    assert L.moe_ep_grouped_ffn(ctypes.byref(c), 2, *args, ws, n - 1, None) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_ep_grouped_ffn(ctypes.byref(c), 2, None, *args[1:], ws, n, None) == nat.MOE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[6] = None                                       # SwiGLU without W_up
+    assert L.moe_ep_grouped_ffn(ctypes.byref(c), 2, *bad, ws, n, None) == nat.MOE_ERR_INVALID_ARG
+    # no rows: nothing to do, nothing launched
+    assert L.moe_ep_grouped_ffn(ctypes.byref(c), 2, fake(), 0, None, None, None, None, None, None, None, None,
+                                ws, 256, None) == nat.MOE_OK
