@@ -315,7 +315,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
     }
-    pdl_wait_then_release();
+    // Last blocks (tail mode) touch only rows the CTA-pair launch before them
+    // leaves alone and read only what the kernel before that wrote (complete
+    // once the pair launch started, which is when this launch can begin), so
+    // they start at once on the SMs the pair launch frees and wait for it
+    // only before exiting: whatever waits for this launch then also sees the
+    // pair launch's results.
+    if (p.tail_mode) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    else pdl_wait_then_release();
     if (tid == 0) s.tile_start[0] = 0;
     // ---- tile table from the device-side offsets
     for (int g = tid; g < G; g += kThreads) {
@@ -474,6 +481,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+    if (p.tail_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 

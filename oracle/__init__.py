@@ -55,7 +55,8 @@ def _load():
         lib.oracle_capacity.argtypes = [ctypes.c_double, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         for name in ("oracle_route", "oracle_dispatch", "oracle_balance",
                      "oracle_expert_apply", "oracle_layer_tokens", "oracle_bias_update",
-                     "oracle_routing_health", "oracle_quantize_rows", "oracle_expert_apply_fp8"):
+                     "oracle_routing_health", "oracle_quantize_rows", "oracle_expert_apply_fp8",
+                     "oracle_layer_backward"):
             getattr(lib, name).restype = ctypes.c_int
         lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -218,6 +219,32 @@ def forward(dims, x, Wr, weights, logit_bias=None, sel_bias=None, tokens=None):
     out.update(bal)
     out["y"] = y
     out["tokens"] = tok
+    return out
+
+
+def layer_backward(dims, x, Wr, weights, dy, alpha=0.0, logit_bias=None, sel_bias=None):
+    """Gradient of sum_t <dy_t, y_t> + alpha * L_aux (all fp64): dict with dx
+    [T,d], dWr [d,E], dbeta [E] (the logit offset), dW1, db1, dWu, dW2, db2,
+    dWsg, dWsu, dWsd (the shapes of the weights; absent weights give None)."""
+    lib = _load()
+    x = _raw(x, "x")
+    Wr = _f32(Wr)
+    lb, sb = _f32(logit_bias), _f32(sel_bias)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    T, d, E, F, S = dims.T, dims.d, dims.E, dims.d_ff, dims.d_ff_shared
+    assert dy.shape == (T, d)
+    out = dict(dx=np.empty((T, d)), dWr=np.empty((d, E)), dbeta=np.empty(E))
+    present = {k for k, v in weights.items() if v is not None}
+    shapes = dict(dW1=("W1", (E, F, d)), db1=("b1", (E, F)), dWu=("Wu", (E, F, d)), dW2=("W2", (E, d, F)),
+                  db2=("b2", (E, d)), dWsg=("Wsg", (S, d)), dWsu=("Wsu", (S, d)), dWsd=("Wsd", (d, S)))
+    for name, (src, shp) in shapes.items():
+        out[name] = np.empty(shp) if src in present else None
+    ws = _weights(weights)
+    rc = lib.oracle_layer_backward(ctypes.byref(dims), _ptr(x), _ptr(Wr), _ptr(lb), _ptr(sb), *[_ptr(a) for a in ws],
+                                   _ptr(dy), ctypes.c_double(alpha), _ptr(out["dx"]), _ptr(out["dWr"]),
+                                   _ptr(out["dbeta"]), *[_ptr(out[n]) for n in shapes])
+    if rc:
+        raise ValueError("oracle_layer_backward rejected its arguments")
     return out
 
 

@@ -637,3 +637,333 @@ int oracle_expert_apply_fp8(const oracle_dims *dm, int64_t nrows, const int32_t 
     parallel_for(nrows, dm->nthreads, apply8_range, &c);
     return 0;
 }
+
+/* ===========================================================================
+ * Backward pass of the layer.
+ *
+ * The layer is trained ([RO] "The Fine-Tuning Router Challenge" and How It
+ * Works 1: the router and experts learn from the task loss plus the
+ * auxiliary balance loss).  For an upstream gradient dy [T, d] of the output
+ * and an aux-loss weight alpha, this computes the gradient of
+ *   ell = sum_t <dy_t, y_t> + alpha * L_aux,   L_aux = E sum_e f_e P_e
+ * with respect to x, W_r, the logit offset beta, every routed expert's
+ * weights and biases and the shared expert's weights.  It is the chain rule
+ * applied to the forward definitions above, in double:
+ *   - the expert selection (a sort of the keys) and the capacity ranks are
+ *     piecewise constant: no gradient flows through which experts are chosen
+ *     or dropped; f_e (counts) is constant in the same way, so L_aux is
+ *     differentiated through P only ([RO] How It Works 1);
+ *   - a kept slot s of token t with expert e adds g_s * E_e(x_t) to y_t, so
+ *     dE_e = g_s dy_t and d g_s = <dy_t, E_e(x_t)>; a dropped slot adds
+ *     nothing and its gate gets no gradient;
+ *   - gate Jacobians: full-softmax gates g_s = p_{e_s}: dh = p (dp - <dp, p>)
+ *     with dp_e the sum of dg over slots choosing e; renormalised softmax
+ *     gates (a softmax over the selected logits): dh_sel = g (dg - <dg, g>);
+ *     sigmoid gates g_s = s_{e_s} / S_sel: ds_sel = (dg - <dg, g>) / S_sel,
+ *     dh = ds s (1 - s);
+ *   - aux loss: dell / dpnorm_e(t) = alpha E f_e / T =: c_e; softmax pnorm = p
+ *     gives dh += p (c - <c, p>); sigmoid pnorm = s / S_all gives
+ *     ds = (c - <c, pnorm>) / S_all, dh += ds s (1 - s);
+ *   - the selection bias never enters y or L_aux: no gradient;
+ *   - GELU' (exact erf form) = Phi(a) + a phi(a); SiLU'(v) = sig(v) (1 + v (1 - sig(v))).
+ * Weight gradients sum over tokens in ascending order; dx_t sums its slots in
+ * slot order, then the shared expert, then the router term.
+ * Outputs (double, any may be NULL except dx): dx [T,d], dWr [d,E], dbeta [E],
+ * dW1 [E,d_ff,d], db1 [E,d_ff], dWu [E,d_ff,d], dW2 [E,d,d_ff], db2 [E,d],
+ * dWsg [S,d], dWsu [S,d], dWsd [d,S].
+ * ======================================================================== */
+typedef struct {
+    expert_weights w;
+    const float *Wr;
+    const int32_t *idx; const double *gate; const int32_t *row_of;
+    const double *h; const double *pnorm; const double *cvec;   /* logits, pnorm, aux weights c_e */
+    const double *dy;
+    double *dx; double *dh;
+    /* pass B */
+    double *dW1, *db1, *dWu, *dW2, *db2, *dWsg, *dWsu, *dWsd;
+} bwd_ctx;
+
+static double gelu_grad(double a)
+{
+    return 0.5 * (1.0 + erf(a / sqrt(2.0))) + a * exp(-0.5 * a * a) / sqrt(2.0 * acos(-1.0));
+}
+
+/* Forward of expert e on token t keeping what the backward needs: pre-
+ * activations a (GELU) or g and u (SwiGLU) in pre1 / pre2, the hidden h and
+ * the output o.                                                            */
+static void expert_fwd_keep(const expert_weights *w, int64_t t, int e, double *pre1, double *pre2, double *hbuf,
+                            double *out)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d, dt = dm->xw_dtype;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const void *Wa = shared ? w->Wsg : w->W1;
+    const void *Wb = shared ? w->Wsu : w->Wu;
+    const void *Wo = shared ? w->Wsd : w->W2;
+    const size_t eb = shared ? 0 : (size_t)e;
+    for (int j = 0; j < dff; ++j) {
+        double a = 0.0;
+        for (int i = 0; i < d; ++i) a += wide(Wa, dt, (eb * dff + j) * d + i) * wide(w->x, dt, (size_t)t * d + i);
+        if (dm->act == 0) {
+            if (!shared && w->b1) a += (double)w->b1[eb * dff + j];
+            pre1[j] = a;
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else {
+            double u = 0.0;
+            for (int i = 0; i < d; ++i) u += wide(Wb, dt, (eb * dff + j) * d + i) * wide(w->x, dt, (size_t)t * d + i);
+            pre1[j] = a;
+            pre2[j] = u;
+            hbuf[j] = a / (1.0 + exp(-a)) * u;
+        }
+    }
+    for (int i = 0; i < d; ++i) {
+        double o = 0.0;
+        for (int j = 0; j < dff; ++j) o += wide(Wo, dt, (eb * d + i) * dff + j) * hbuf[j];
+        if (dm->act == 0 && !shared && w->b2) o += (double)w->b2[eb * d + i];
+        out[i] = o;
+    }
+}
+
+/* Gradient of the expert's pre-activations from dz = dE_e/d(output):
+ * dhid = Wo^T dz, then da (GELU) or dga, dua (SwiGLU) into d1 / d2.        */
+static void expert_bwd_pre(const expert_weights *w, int e, const double *pre1, const double *pre2,
+                           const double *dz, double *dhid, double *d1, double *d2)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d, dt = dm->xw_dtype;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const void *Wo = shared ? w->Wsd : w->W2;
+    const size_t eb = shared ? 0 : (size_t)e;
+    for (int j = 0; j < dff; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += wide(Wo, dt, (eb * d + i) * dff + j) * dz[i];
+        dhid[j] = acc;
+        if (dm->act == 0) {
+            d1[j] = acc * gelu_grad(pre1[j]);
+        } else {
+            const double sg = 1.0 / (1.0 + exp(-pre1[j]));
+            d1[j] = acc * pre2[j] * sg * (1.0 + pre1[j] * (1.0 - sg));
+            d2[j] = acc * pre1[j] * sg;
+        }
+    }
+}
+
+static void bwd_token_range(void *vctx, int64_t lo, int64_t hi)
+{
+    bwd_ctx *c = (bwd_ctx *)vctx;
+    const expert_weights *w = &c->w;
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d, E = dm->E, k = dm->k, dt = dm->xw_dtype;
+    const int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    const size_t hm = (size_t)(hmax > 0 ? hmax : 1);
+    double *pre1 = (double *)malloc(sizeof(double) * hm), *pre2 = (double *)malloc(sizeof(double) * hm);
+    double *hid = (double *)malloc(sizeof(double) * hm), *dhid = (double *)malloc(sizeof(double) * hm);
+    double *d1 = (double *)malloc(sizeof(double) * hm), *d2 = (double *)malloc(sizeof(double) * hm);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d), *dz = (double *)malloc(sizeof(double) * (size_t)d);
+    double *dg = (double *)malloc(sizeof(double) * (size_t)k);
+    for (int64_t t = lo; t < hi; ++t) {
+        const double *dyt = c->dy + (size_t)t * d;
+        double *dxt = c->dx + (size_t)t * d;
+        for (int i = 0; i < d; ++i) dxt[i] = 0.0;
+        /* routed slots (slot order), then the shared expert */
+        for (int s = 0; s <= k; ++s) {
+            int e;
+            double g;
+            if (s < k) {
+                dg[s] = 0.0;
+                if (c->row_of[t * k + s] < 0) continue;
+                e = c->idx[t * k + s];
+                g = c->gate[t * k + s];
+            } else {
+                if (dm->d_ff_shared <= 0) break;
+                e = E;
+                g = 1.0;
+            }
+            const int dff = (e == E) ? dm->d_ff_shared : dm->d_ff;
+            expert_fwd_keep(w, t, e, pre1, pre2, hid, o);
+            if (s < k) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) acc += dyt[i] * o[i];
+                dg[s] = acc;
+            }
+            for (int i = 0; i < d; ++i) dz[i] = g * dyt[i];
+            expert_bwd_pre(w, e, pre1, pre2, dz, dhid, d1, d2);
+            const void *Wa = (e == E) ? w->Wsg : w->W1;
+            const void *Wb = (e == E) ? w->Wsu : w->Wu;
+            const size_t eb = (e == E) ? 0 : (size_t)e;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dff; ++j) {
+                    acc += wide(Wa, dt, (eb * dff + j) * d + i) * d1[j];
+                    if (dm->act == 1) acc += wide(Wb, dt, (eb * dff + j) * d + i) * d2[j];
+                }
+                dxt[i] += acc;
+            }
+        }
+        /* router: gates, then the aux loss, into dh_t */
+        const double *h = c->h + (size_t)t * E;
+        const double *pn = c->pnorm + (size_t)t * E;
+        double *dh = c->dh + (size_t)t * E;
+        for (int e = 0; e < E; ++e) dh[e] = 0.0;
+        if (dm->score == 0) {
+            /* p_e from the logits (pnorm is p for softmax scores) */
+            if (dm->renorm == 0) {
+                double dot = 0.0;
+                for (int s = 0; s < k; ++s) dot += pn[c->idx[t * k + s]] * dg[s];
+                for (int s = 0; s < k; ++s) {
+                    const int e = c->idx[t * k + s];
+                    dh[e] += pn[e] * dg[s];
+                }
+                for (int e = 0; e < E; ++e) dh[e] -= pn[e] * dot;
+            } else {
+                double dot = 0.0;
+                for (int s = 0; s < k; ++s) dot += c->gate[t * k + s] * dg[s];
+                for (int s = 0; s < k; ++s) dh[c->idx[t * k + s]] += c->gate[t * k + s] * (dg[s] - dot);
+            }
+            double cp = 0.0;
+            for (int e = 0; e < E; ++e) cp += c->cvec[e] * pn[e];
+            for (int e = 0; e < E; ++e) dh[e] += pn[e] * (c->cvec[e] - cp);
+        } else {
+            double ssel = 0.0, sall = 0.0, dot = 0.0;
+            for (int s = 0; s < k; ++s) ssel += 1.0 / (1.0 + exp(-h[c->idx[t * k + s]]));
+            for (int e = 0; e < E; ++e) sall += 1.0 / (1.0 + exp(-h[e]));
+            for (int s = 0; s < k; ++s) dot += c->gate[t * k + s] * dg[s];
+            for (int s = 0; s < k; ++s) {
+                const int e = c->idx[t * k + s];
+                const double se = 1.0 / (1.0 + exp(-h[e]));
+                dh[e] += (dg[s] - dot) / ssel * se * (1.0 - se);
+            }
+            double cq = 0.0;
+            for (int e = 0; e < E; ++e) cq += c->cvec[e] * pn[e];
+            for (int e = 0; e < E; ++e) {
+                const double se = 1.0 / (1.0 + exp(-h[e]));
+                dh[e] += (c->cvec[e] - cq) / sall * se * (1.0 - se);
+            }
+        }
+        for (int j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int e = 0; e < E; ++e) acc += (double)c->Wr[(size_t)j * E + e] * dh[e];
+            dxt[j] += acc;
+        }
+    }
+    free(pre1); free(pre2); free(hid); free(dhid); free(d1); free(d2); free(o); free(dz); free(dg);
+}
+
+/* Pass B: weight gradients of expert e (e == E: the shared expert), tokens in
+ * ascending order, one expert per worker.                                   */
+static void bwd_expert_range(void *vctx, int64_t lo, int64_t hi)
+{
+    bwd_ctx *c = (bwd_ctx *)vctx;
+    const expert_weights *w = &c->w;
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d, E = dm->E, k = dm->k, dt = dm->xw_dtype;
+    const int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    const size_t hm = (size_t)(hmax > 0 ? hmax : 1);
+    double *pre1 = (double *)malloc(sizeof(double) * hm), *pre2 = (double *)malloc(sizeof(double) * hm);
+    double *hid = (double *)malloc(sizeof(double) * hm), *dhid = (double *)malloc(sizeof(double) * hm);
+    double *d1 = (double *)malloc(sizeof(double) * hm), *d2 = (double *)malloc(sizeof(double) * hm);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d), *dz = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int64_t e = lo; e < hi; ++e) {
+        const int sh = (e == E);
+        const int dff = sh ? dm->d_ff_shared : dm->d_ff;
+        double *gA = sh ? c->dWsg : (c->dW1 ? c->dW1 + (size_t)e * dff * d : NULL);
+        double *gB = sh ? c->dWsu : (c->dWu ? c->dWu + (size_t)e * dff * d : NULL);
+        double *gO = sh ? c->dWsd : (c->dW2 ? c->dW2 + (size_t)e * d * dff : NULL);
+        double *gb1 = (!sh && c->db1) ? c->db1 + (size_t)e * dff : NULL;
+        double *gb2 = (!sh && c->db2) ? c->db2 + (size_t)e * d : NULL;
+        if (gA) memset(gA, 0, sizeof(double) * (size_t)dff * d);
+        if (gB) memset(gB, 0, sizeof(double) * (size_t)dff * d);
+        if (gO) memset(gO, 0, sizeof(double) * (size_t)d * dff);
+        if (gb1) memset(gb1, 0, sizeof(double) * (size_t)dff);
+        if (gb2) memset(gb2, 0, sizeof(double) * (size_t)d);
+        for (int64_t t = 0; t < dm->T; ++t) {
+            double g = 1.0;
+            if (!sh) {
+                int s = 0;
+                for (; s < k; ++s)
+                    if (c->idx[t * k + s] == (int)e && c->row_of[t * k + s] >= 0) break;
+                if (s == k) continue;
+                g = c->gate[t * k + s];
+            }
+            expert_fwd_keep(w, t, (int)e, pre1, pre2, hid, o);
+            const double *dyt = c->dy + (size_t)t * d;
+            for (int i = 0; i < d; ++i) dz[i] = g * dyt[i];
+            expert_bwd_pre(w, (int)e, pre1, pre2, dz, dhid, d1, d2);
+            for (int i = 0; i < d; ++i) {
+                if (gO) for (int j = 0; j < dff; ++j) gO[(size_t)i * dff + j] += dz[i] * hid[j];
+                if (gb2 && dm->act == 0) gb2[i] += dz[i];
+            }
+            for (int j = 0; j < dff; ++j) {
+                for (int i = 0; i < d; ++i) {
+                    const double xi = wide(w->x, dt, (size_t)t * d + i);
+                    if (gA) gA[(size_t)j * d + i] += d1[j] * xi;
+                    if (gB && dm->act == 1) gB[(size_t)j * d + i] += d2[j] * xi;
+                }
+                if (gb1 && dm->act == 0) gb1[j] += d1[j];
+            }
+        }
+    }
+    free(pre1); free(pre2); free(hid); free(dhid); free(d1); free(d2); free(o); free(dz);
+}
+
+typedef struct { const oracle_dims *dm; const void *x; const double *dh; double *dWr; } dwr_ctx;
+
+static void bwd_router_range(void *vctx, int64_t lo, int64_t hi)
+{
+    dwr_ctx *c = (dwr_ctx *)vctx;
+    const oracle_dims *dm = c->dm;
+    const int E = dm->E, d = dm->d;
+    for (int64_t j = lo; j < hi; ++j)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < dm->T; ++t) acc += wide(c->x, dm->xw_dtype, (size_t)t * d + j) * c->dh[t * E + e];
+            c->dWr[(size_t)j * E + e] = acc;
+        }
+}
+
+int oracle_layer_backward(const oracle_dims *dm, const void *x, const float *Wr, const float *logit_bias,
+                          const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
+                          const float *b2, const void *Wsg, const void *Wsu, const void *Wsd,
+                          const double *dy, double alpha,
+                          double *dx, double *dWr, double *dbeta, double *dW1, double *db1, double *dWu,
+                          double *dW2, double *db2, double *dWsg, double *dWsu, double *dWsd)
+{
+    if (!dm || !dx || dm->T < 0 || dm->k < 1 || dm->k > dm->E) return 1;
+    const int64_t T = dm->T;
+    const int E = dm->E, k = dm->k;
+    const size_t tk = (size_t)(T * k > 0 ? T * k : 1);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * tk);
+    double *gate = (double *)malloc(sizeof(double) * tk);
+    double *h = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * E);
+    double *pn = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * E);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * E);
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *kept = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *offs = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *row_of = (int32_t *)malloc(sizeof(int32_t) * tk);
+    double *cvec = (double *)malloc(sizeof(double) * (size_t)E);
+    int rc = oracle_route(dm, T, NULL, x, Wr, logit_bias, sel_bias, idx, gate, h, pn, NULL, NULL);
+    if (!rc) rc = oracle_dispatch(dm, idx, counts, kept, offs, row_of, NULL, NULL);
+    if (!rc) {
+        for (int e = 0; e < E; ++e)
+            cvec[e] = T > 0 ? alpha * (double)E * ((double)counts[e] / ((double)T * (double)k)) / (double)T : 0.0;
+        bwd_ctx c = { { dm, x, W1, b1, Wu, W2, b2, Wsg, Wsu, Wsd }, Wr, idx, gate, row_of, h, pn, cvec, dy, dx, dh,
+                      dW1, db1, dWu, dW2, db2, dWsg, dWsu, dWsd };
+        parallel_for(T, dm->nthreads, bwd_token_range, &c);
+        parallel_for(E + (dm->d_ff_shared > 0 ? 1 : 0), dm->nthreads, bwd_expert_range, &c);
+        if (dWr) {
+            dwr_ctx r = { dm, x, dh, dWr };
+            parallel_for(dm->d, dm->nthreads, bwd_router_range, &r);
+        }
+        if (dbeta)
+            for (int e = 0; e < E; ++e) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < T; ++t) acc += dh[t * E + e];
+                dbeta[e] = acc;
+            }
+    }
+    free(idx); free(gate); free(h); free(pn); free(dh); free(counts); free(kept); free(offs); free(row_of); free(cvec);
+    return rc;
+}

@@ -173,9 +173,9 @@ def test_entry_points(wl, cuda_device):
     out = nat.Outputs(st.cfg, cuda_device)
     nat.forward(st.cfg, inp, out, st.ws)
     assert torch.equal(out.f, st.f) and torch.equal(out.P, st.P) and torch.equal(out.loss, st.loss)
-    # in bf16 the forward's first expert GEMM gathers its rows from x by token
-    # instead of reading x_perm: the same operands in the same order, so the
-    # same bits as the entry-point chain
+    # the forward pass runs the same kernels on the same operands in the same
+    # order as the entry-point chain (its permute writes x_perm into the
+    # workspace, its grouped FFN reads it from there): the same bits
     assert torch.equal(out.idx, st.idx) and torch.equal(out.y, st.y)
     assert abs(float(st.loss.item()) - bal["loss"]) <= TOL_LOSS * bal["loss"]
     np.testing.assert_allclose(st.f.cpu().numpy(), bal["f"], rtol=1e-6)
