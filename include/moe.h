@@ -226,6 +226,45 @@ typedef struct {
 } moe_ws_view;
 MOE_API moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws_bytes, moe_ws_view *out);
 
+/* ---- Backward pass ------------------------------------------------------
+ * The layer is trained ("Fine-Tuning Mixture of Experts (MoE) Models: Router
+ * Optimization Techniques", The Fine-Tuning Router Challenge and How It Works
+ * 1: the router and the experts learn from the task loss plus the balance
+ * loss).  moe_backward gives the gradient of
+ *     ell = sum_t <dy_t, y_t> + alpha * L_aux
+ * (dy: the gradient of the task loss with respect to the layer output y;
+ * L_aux = E sum_e f_e P_e) with respect to x, W_r, the logit offset and every
+ * expert's weights and biases, shared expert included.  The expert choice,
+ * the capacity ranks and the counts f_e are piecewise constant in the inputs
+ * and carry no gradient; the selection bias gets none.
+ *   - Run it after moe_forward on the same stream with the same cfg, inputs
+ *     and workspace `fwd_ws` (its dispatch tables, packed rows and hidden
+ *     activation are read from there; the expert pre-activations are
+ *     recomputed), passing the forward's outputs idx, gate, counts and its
+ *     router logits (moe_forward's logits_out, required here).
+ *   - bf16 layers with d_model, d_ff and d_ff_shared multiples of 64 (else
+ *     MOE_ERR_UNSUPPORTED).  dy and dx [T, d_model] bf16; every other
+ *     gradient fp32 in the layout of its parameter: dWr [d_model, E],
+ *     dlogit_bias [E] (may be NULL), dW1 / dWu [E, d_ff, d_model], db1 [E,
+ *     d_ff] and db2 [E, d_model] (GELU; may be NULL), dW2 [E, d_model, d_ff],
+ *     dWsh_g / dWsh_u [d_ff_shared, d_model], dWsh_d [d_model, d_ff_shared].
+ *     Gradients are written, not accumulated.
+ *   - Contractions run on the tensor cores with bf16 operands (dy scaled by
+ *     the gates, the recomputed pre-activations, their gradients, dh) and
+ *     fp32 accumulation; the rest in fp32.
+ *   - ws: moe_backward_workspace_size(cfg) bytes of scratch, 256-byte aligned
+ *     (0 on a bad or unsupported config).  Device errors land in fwd_ws's
+ *     status word.                                                          */
+MOE_API size_t moe_backward_workspace_size(const moe_config *cfg);
+MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, const void *W1,
+                                const float *b1, const void *Wu, const void *W2, const float *b2,
+                                const void *Wsh_g, const void *Wsh_u, const void *Wsh_d,
+                                const int32_t *idx, const float *gate, const float *logits, const int32_t *counts,
+                                const void *dy, float alpha, void *dx, float *dWr, float *dlogit_bias,
+                                float *dW1, float *db1, float *dWu, float *dW2, float *db2,
+                                float *dWsh_g, float *dWsh_u, float *dWsh_d,
+                                void *fwd_ws, size_t fwd_ws_bytes, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ---- Expert parallelism -------------------------------------------------
  * The experts sharded over R ranks, each rank holding E / R of them ("Fine-
  * Tuning Mixture of Experts (MoE) Models: Router Optimization Techniques",

@@ -719,6 +719,8 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
 }
 
 // ------------------------------------------------------------------ host side
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (fn == nullptr) {
@@ -736,7 +738,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // maps (A operands) ignore `outer`; rank 3 maps (expert-stacked B operands)
 // are indexed by expert in the third coordinate.
 bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
-              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, int esize = 2) {
+              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, int esize) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     if (outer_stride_elems == 0) outer_stride_elems = mid * mid_stride_elems;
@@ -750,6 +752,8 @@ bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 // Output map for the staged epilogue stores: bf16 [rows][cols] with row
 // stride ld elements, box 32 x 32, 64-byte swizzle.

@@ -122,6 +122,11 @@ struct FfnArgs {
     uint8_t *H8;                 // [T*k (+T), hF] codes
     float *h_scale;              // [T*k (+T)]
 };
+// TMA tile map (128-byte swizzle) of a tensor [outer][mid][inner] (inner
+// contiguous) of bf16 (esize 2) or 8-bit codes (esize 1), box {one 128-byte
+// row of elements, box_mid(, 1)}; rank 2 maps ignore `outer`.  ffn_sm100.cu.
+bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
+              uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, int esize = 2);
 cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st);
 
@@ -167,6 +172,86 @@ cudaError_t launch_bias_update(const int32_t *counts, float *bias, double gamma,
                                cudaStream_t st);
 cudaError_t launch_routing_health(const int32_t *counts, const float *P, double *out, int T, int k, int E,
                                   cudaStream_t st);
+
+// ---- backward pass (bwd_sm100.cu, bwd_aux.cu)
+// One grouped GEMM C = A B^T on the tensor cores, bf16 operands, fp32
+// accumulation.  Group g owns rows offsets[g] .. offsets[g+1]: with kgroup = 0
+// they are rows of A and of C (K fixed), with kgroup = 1 they are the
+// contraction (A and B both indexed by them, M and N fixed, one C per group).
+// Operands are K-major (A rows / B rows of K elements) or MN-major (rows of K
+// index holding the M / N elements); a 3-D B map is indexed by expert g.
+enum { BW_STORE_BF16 = 0, BW_DGRAD2 = 1, BW_STORE_F32 = 2 };
+struct BwdGemmParams {
+    const int32_t *offsets;      // [G+1]
+    int G;
+    int kgroup;
+    int M, N, K;                 // kgroup: M, N fixed; else N, K fixed
+    int b_per_group;             // 1: B is a 3-D map, expert g; 0: a 2-D map
+    int k_split;                 // MN-major B, kgroup 0: K rows >= k_split come from tmB2 (row - k_split)
+    int mode;
+    // BW_STORE_F32 / BW_STORE_BF16: C row r, column c at out[r * ldo + c]
+    // (+ g * out_group_stride when kgroup); BW_STORE_BF16 adds bias[g][c]
+    void *out;
+    int64_t ldo, out_group_stride;
+    const float *bias;
+    int64_t bias_group_stride;
+    // BW_DGRAD2: C = dH (gate applied) of hidden columns; with H (the forward
+    // hidden activation) and GU (pre-activations: G at column c, U at F + c,
+    // or the GELU input) of the same rows: dGU = (dG | dU) or dA, and
+    // part[r][2 nt + half] = sum over the half-tile's columns of H * C
+    float *part;
+    int part_ld;
+    const __nv_bfloat16 *H;
+    int64_t ldh;
+    const __nv_bfloat16 *GU;
+    int64_t ldgu;
+    __nv_bfloat16 *dGU;
+    int F, act;
+    int32_t *status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_bwd_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &B2, bool a_mn, bool b_mn,
+                            const BwdGemmParams &p, int num_sms, cudaStream_t st);
+
+struct BwdAuxArgs {
+    const int32_t *offsets;      // [E+1] forward dispatch tables
+    const int32_t *row_token;
+    const float *row_gate;
+    const int32_t *row_of;       // [T, k]
+    const int32_t *idx;          // [T, k]
+    const float *gate;           // [T, k]
+    const float *logits;         // [T, E] forward router logits (with the logit offset)
+    const int32_t *counts;       // [E]
+    const void *dy;              // [T, d] bf16
+    const float *b2;             // [E, d] GELU output bias or null
+    const float *part;           // [rows, part_ld] partial <H, dH> of the down dgrad
+    int part_ld;
+    __nv_bfloat16 *dZ;           // [rows, d]
+    float *dh;                   // [T, E]
+    __nv_bfloat16 *dh_bf16;      // [T, dh_ld]
+    int dh_ld;
+    const float *dX_rows;        // [rows, d]
+    const float *dX_shared;      // [T, d] or null
+    const float *dX_router;      // [T, d]
+    void *dx;                    // [T, d] bf16
+    float alpha;
+    int T, d, E, k, score, renorm, num_sms;
+};
+cudaError_t launch_scale_rows(const BwdAuxArgs &a, int max_rows, cudaStream_t st);
+cudaError_t launch_router_bwd(const BwdAuxArgs &a, cudaStream_t st);
+cudaError_t launch_dx_combine(const BwdAuxArgs &a, cudaStream_t st);
+// out[g][c] = sum over the rows of group g (offsets, or all `rows` when null) of in[r][c]
+struct ColSumArgs {
+    const void *in;
+    int in_f32;
+    int64_t ld;
+    const int32_t *offsets;
+    int G, rows, cols;
+    float *out;
+};
+cudaError_t launch_column_sums(const ColSumArgs &a, cudaStream_t st);
+cudaError_t launch_to_bf16(const float *in, __nv_bfloat16 *out, int64_t rows, int cols, int64_t ldo, cudaStream_t st);
+cudaError_t launch_set_pair(int32_t *p, int32_t a, int32_t b, cudaStream_t st);     // p[0] = a, p[1] = b
 
 // Host-side helpers shared by the entry points (moe_api.cu).
 moe_status validate_config(const moe_config *cfg);        // sets the error detail

@@ -30,7 +30,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
-           "moe_ep_workspace_size", "moe_ep_grouped_ffn")
+           "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -108,6 +108,11 @@ def lib():
         L.moe_ep_grouped_ffn.restype = ctypes.c_int
         L.moe_ep_grouped_ffn.argtypes = [P(MoeConfig), c_i32, c_vp, ctypes.c_int64] + [c_vp] * 9 + [
             ctypes.c_size_t, c_vp]
+        L.moe_backward_workspace_size.restype = ctypes.c_size_t
+        L.moe_backward_workspace_size.argtypes = [P(MoeConfig)]
+        L.moe_backward.restype = ctypes.c_int
+        L.moe_backward.argtypes = [P(MoeConfig)] + [c_vp] * 15 + [ctypes.c_float] + [c_vp] * 12 + [
+            c_vp, ctypes.c_size_t, c_vp, ctypes.c_size_t, c_vp]
         L.moe_workspace_view.restype = ctypes.c_int
         L.moe_workspace_view.argtypes = [P(MoeConfig), c_vp, ctypes.c_size_t, P(MoeWsView)]
         L.moe_check_wait_timeout.restype = ctypes.c_int
@@ -267,6 +272,47 @@ def moe_ep_grouped_ffn(cfg, n_src, group_offsets, x_rows, row_gate, W1, b1, Wu, 
     _check(lib().moe_ep_grouped_ffn(ctypes.byref(cfg), int(n_src), _p(group_offsets), int(x_rows.shape[0]),
                                     _p(x_rows), _p(row_gate), _p(W1), _p(b1), _p(Wu), _p(W2), _p(b2), _p(y_rows),
                                     _p(ws), ws.numel(), _stream(stream)), "moe_ep_grouped_ffn")
+
+
+def backward_workspace_size(cfg) -> int:
+    n = int(lib().moe_backward_workspace_size(ctypes.byref(cfg)))
+    if n == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_backward_workspace_size", last_error_detail())
+    return n
+
+
+def moe_backward(cfg, x, Wr, W1, b1, Wu, W2, b2, Wsh_g, Wsh_u, Wsh_d, idx, gate, logits, counts, dy, alpha, dx, dWr,
+                 dlogit_bias, dW1, db1, dWu, dW2, db2, dWsh_g, dWsh_u, dWsh_d, fwd_ws, ws, stream=None):
+    _check(lib().moe_backward(ctypes.byref(cfg), _p(x), _p(Wr), _p(W1), _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g),
+                              _p(Wsh_u), _p(Wsh_d), _p(idx), _p(gate), _p(logits), _p(counts), _p(dy), float(alpha),
+                              _p(dx), _p(dWr), _p(dlogit_bias), _p(dW1), _p(db1), _p(dWu), _p(dW2), _p(db2),
+                              _p(dWsh_g), _p(dWsh_u), _p(dWsh_d), _p(fwd_ws), fwd_ws.numel(), _p(ws), ws.numel(),
+                              _stream(stream)), "moe_backward")
+
+
+def backward(cfg, inp, out, fwd_ws, dy, alpha=0.0, ws=None, stream=None) -> dict:
+    """moe_backward after forward(cfg, inp, out, fwd_ws) (out must hold the
+    router logits: Outputs(..., want_logits=True)).  Returns the gradients
+    as fp32 tensors (dx in the layer dtype) keyed like the inputs."""
+    if out.logits is None:
+        raise ValueError("the backward pass needs the forward's router logits (Outputs(want_logits=True))")
+    dev = dy.device
+    T, d, E, F, S = cfg.T, cfg.d_model, cfg.E, cfg.d_ff, cfg.d_ff_shared
+    f32 = dict(dtype=torch.float32, device=dev)
+    swiglu = cfg.act == MOE_ACT_SWIGLU
+    g = dict(dx=torch.empty((T, d), dtype=layer_dtype(cfg), device=dev), dWr=torch.empty((d, E), **f32),
+             dlogit_bias=torch.empty(E, **f32), dW1=torch.empty((E, F, d), **f32),
+             dWu=torch.empty((E, F, d), **f32) if swiglu else None, dW2=torch.empty((E, d, F), **f32),
+             db1=None if swiglu else torch.empty((E, F), **f32), db2=None if swiglu else torch.empty((E, d), **f32),
+             dWsg=torch.empty((S, d), **f32) if S else None, dWsu=torch.empty((S, d), **f32) if S and swiglu else None,
+             dWsd=torch.empty((d, S), **f32) if S else None)
+    if ws is None:
+        ws = torch.empty(backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    moe_backward(cfg, inp["x"], inp["Wr"], inp["W1"], inp.get("b1"), inp.get("Wu"), inp["W2"], inp.get("b2"),
+                 inp.get("Wsg"), inp.get("Wsu"), inp.get("Wsd"), out.idx, out.gate, out.logits, out.counts, dy, alpha,
+                 g["dx"], g["dWr"], g["dlogit_bias"], g["dW1"], g["db1"], g["dWu"], g["dW2"], g["db2"], g["dWsg"],
+                 g["dWsu"], g["dWsd"], fwd_ws, ws, stream)
+    return g
 
 
 def moe_workspace_view(cfg, ws) -> MoeWsView:
