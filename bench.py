@@ -253,8 +253,8 @@ def run_ours(args, wl, dev, world, rank, fp8=None, steps=None, warmup=None, full
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     fp8 = (args.experts == "fp8") if fp8 is None else fp8
-    steps = steps if steps is None else steps
-    warmup = warmup if warmup is None else warmup
+    steps = args.steps if steps is None else steps
+    warmup = args.warmup if warmup is None else warmup
     inp = syn.generate(wl, dev, seed=0, weights=not fp8)
     w8 = None
     if fp8:                                         # e4m3 experts (bf16 layer around them)

@@ -17,8 +17,8 @@
 //                publishes them); the rank of (t, s) among the chunk's
 //                assignments to the same expert comes from __match_any_sync
 //                over flattened (t, s) order, so rows are stable by token id;
-//                then, unless x_perm is null, the kept rows of x are copied
-//                with 16-byte vectors.
+//                then, unless x_perm is null, each token's row of x is read
+//                once and written to each of its kept rows (16-byte vectors).
 #include "balance.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
@@ -209,24 +209,36 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
     }
     if (a.x_perm == nullptr) return;             // row tables only
     __syncthreads();
-    // copy the kept rows of x into x_perm, one warp per row, 16-byte vectors
+    // copy x rows into x_perm: one warp per token, its row read once (eight
+    // 16-byte loads in flight per lane) and written to each of its kept rows
     const int nvec = a.d * (int)sizeof(TX) / 16;
+    const int ntok = min(kChunk, a.T - t0);
     const uint4 *xs = static_cast<const uint4 *>(a.x);
     uint4 *xd = static_cast<uint4 *>(a.x_perm);
-    for (int q = warp; q < npairs; q += kWarps) {
-        const int2 rt = list[q];
-        if (rt.x < 0) continue;
-        const uint4 *__restrict__ src = xs + (size_t)rt.y * nvec;
-        uint4 *__restrict__ dst = xd + (size_t)rt.x * nvec;
+    for (int tl = warp; tl < ntok; tl += kWarps) {
+        const int my_row = lane < k ? list[tl * k + lane].x : -1;
+        if (__ballot_sync(0xffffffffu, my_row >= 0) == 0u) continue;      // every slot dropped
+        const uint4 *__restrict__ src = xs + (size_t)(t0 + tl) * nvec;
         int v = lane;
-        for (; v + 224 < nvec; v += 256) {         // eight 16-byte loads in flight per lane
+        for (; v + 224 < nvec; v += 256) {
             uint4 r[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) r[i] = __ldg(src + v + 32 * i);
+            for (int s = 0; s < k; ++s) {
+                const int row = __shfl_sync(0xffffffffu, my_row, s);
+                if (row < 0) continue;
+                uint4 *__restrict__ dst = xd + (size_t)row * nvec;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[v + 32 * i] = r[i];
+                for (int i = 0; i < 8; ++i) dst[v + 32 * i] = r[i];
+            }
         }
-        for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        for (; v < nvec; v += 32) {
+            const uint4 r = __ldg(src + v);
+            for (int s = 0; s < k; ++s) {
+                const int row = __shfl_sync(0xffffffffu, my_row, s);
+                if (row >= 0) xd[(size_t)row * nvec + v] = r;
+            }
+        }
     }
 }
 

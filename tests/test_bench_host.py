@@ -32,3 +32,26 @@ def test_algorithmic_counts_bf16_and_fp8():
     assert b == xy + wr + 3 * (3 * 32 * 16 * 2)                              # three touched experts
     _, b8, _ = bench.algorithmic_counts(wl, kept, kept, fp8=True)
     assert b8 == xy + wr + 3 * (3 * 32 * 16 * 1) + 3 * 4 * (2 * 16 + 32)
+
+
+def test_tensor_peak_follows_the_runs_clock_record():
+    import bench
+    peaks = {"hbm_gbs": 6557.0, "bf16_tflops": 1667.1, "bf16_tflops_sustained": 1408.6}
+    assert bench.tensor_peak(peaks, {"reasons": []})[0] == 1667.1
+    assert bench.tensor_peak(peaks, {"reasons": ["sw_power_cap"]})[0] == 1408.6
+    assert bench.tensor_peak(peaks, {"reasons": None})[0] == 1667.1
+
+
+def test_roofline_fields_use_the_chosen_peak():
+    import numpy as np
+    import bench
+    peaks = {"hbm_gbs": 6557.0, "bf16_tflops": 1667.1, "bf16_tflops_sustained": 1408.6}
+    r = dict(flops=1.2e12, ms=1.3, bound="tensor", layer_roof_ms=1.2e12 / 1667.1e9, layer_roof_burst_ms=0.72,
+             layer_roof_sust_ms=0.85, alg_bytes=1.3e9, peaks=peaks, peak_src="measured", peak_t=1667.1,
+             peak_which="burst", ffn_tflops=1100.0, traffic=None, stage_avg={"grouped_ffn": 1.0},
+             kept_rows=100, n_dropped=0, loss=1.0, counts=np.array([1, 2]))
+    f = bench.roofline_fields(r, fp8=False)
+    assert abs(f["roofline"]["frac"] - 1100.0 / 1667.1) < 1e-12
+    assert abs(f["roofline"]["frac_sustained"] - 1100.0 / 1408.6) < 1e-12
+    assert f["layer_roofline"]["frac"] == r["layer_roof_ms"] / 1.3
+    assert "of measured" in f["roofline"]["peak_note"]
