@@ -496,7 +496,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: e4m3 experts through moe_forward_fp8 (bf16 layers only; no CPU baseline)")
-    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8",
+    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8,qwen3_moe:backward",
                     help="further workloads (name or name:fp8) timed after the headline one and reported "
                          "under sub_records; '' for none")
     ap.add_argument("--sub-steps", type=int, default=20)
@@ -522,7 +522,10 @@ def main():
         r = run_ours(args, wl, dev, world, rank)
         for spec in [t for t in args.sub.split(",") if t] if args.experts == "bf16" else []:
             torch.cuda.empty_cache()
-            subs[spec] = sub_record(args, spec, dev, world, rank)
+            try:
+                subs[spec] = sub_record(args, spec, dev, world, rank)
+            except Exception as exc:           # a failed sub-record is reported, the headline stands
+                subs[spec] = {"error": "%s: %s" % (type(exc).__name__, exc)}
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
@@ -586,12 +589,66 @@ def roofline_fields(r, fp8):
     }
 
 
+def backward_record(args, wl, dev, world):
+    """The backward pass (moe_backward) after one forward pass: K timed steps,
+    L2 flushed between them.  Algorithmic FLOPs: the expert contractions'
+    input and weight gradients (2 x the forward's expert FLOPs) plus the
+    router's two gradient contractions (2 x 2 T d E); the pre-activation
+    recompute the implementation adds is not counted."""
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inp = syn.generate(wl, dev, seed=0)
+    cfg = nat.config_from_workload(wl)
+    out = nat.Outputs(cfg, dev, want_logits=True)
+    ws = nat.alloc_workspace(cfg, dev)
+    nat.forward(cfg, inp, out, ws, stream)
+    g = torch.Generator(device=dev).manual_seed(1)
+    dy = torch.randn((wl.T, wl.d_model), generator=g, device=dev).to(torch.bfloat16)
+    bws = torch.empty(nat.backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        flush.zero_()
+        nat.backward(cfg, inp, out, ws, dy, 0.01, ws=bws, stream=stream)
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(ws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the backward warm-up")
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.sub_steps)]
+    for i in range(args.sub_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        nat.backward(cfg, inp, out, ws, dy, 0.01, ws=bws, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.sub_steps
+    ms = max_over_ranks([ms], world, dev)[0]
+    counts = out.counts.cpu().numpy()
+    cap = nat.capacity(cfg)
+    kept = np.minimum(counts, cap) if cap >= 0 else counts
+    flops = 2.0 * wl.expert_flops(int(kept.sum())) + 4.0 * wl.T * wl.d_model * wl.E
+    peaks, peak_src = load_peaks()
+    peak_t, which = tensor_peak(peaks, clocks)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": wl.name, "pass": "backward (dx, dW_r, d logit offset, all expert weight gradients)",
+            "steps": args.sub_steps, "warmup": 3, "ms_per_step": ms,
+            "tokens_per_s": job_tokens_per_s(world, wl.T, ms), "tflops": tf,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_t, "unit": "TFLOP/s", "frac": tf / peak_t,
+                         "flops": flops, "peak_note": "%s bf16 peak, %s" % (which, "of measured" if peak_src ==
+                                                                             "measured" else "of fallback")},
+            "clocks": clocks}
+
+
 def sub_record(args, spec, dev, world, rank):
     """One further workload timed like the headline one (device-resident steps
     with the L2 flushed between them, the staged per-stage pass), reported
-    with its own roofline fractions.  spec: "workload" or "workload:fp8"."""
+    with its own roofline fractions.  spec: "workload", "workload:fp8", or
+    "workload:backward" (the backward pass, backward_record)."""
     name, _, experts = spec.partition(":")
     wl = syn.WORKLOADS[name]
+    if experts == "backward":
+        return backward_record(args, wl, dev, world)
     fp8 = experts == "fp8"
     r = run_ours(args, wl, dev, world, rank, fp8=fp8, steps=args.sub_steps, warmup=3, full=False)
     rec = {"workload": name, "experts": "fp8" if fp8 else "bf16", "steps": args.sub_steps, "warmup": 3,

@@ -339,28 +339,57 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const __nv_bfloat16 *hr = p.H + orow * p.ldh + col0;
                     const __nv_bfloat16 *gr = p.GU + orow * p.ldgu + col0;
                     __nv_bfloat16 *dr = p.dGU + orow * p.ldgu + col0;
-                    for (int i = 0; i < ncol; i += 2) {
-                        const int two = (i + 1 < ncol) ? 2 : 1;
-                        float hv[2], gv[2], uv[2], dg_[2], du[2];
-                        for (int j = 0; j < two; ++j) {
-                            hv[j] = __bfloat162float(hr[i + j]);
-                            gv[j] = __bfloat162float(gr[i + j]);
-                            dgp += hv[j] * v[i + j];
-                            if (p.act == MOE_ACT_SWIGLU) {
-                                uv[j] = __bfloat162float(gr[p.F + i + j]);
-                                const float sg = 1.f / (1.f + __expf(-gv[j]));
-                                dg_[j] = v[i + j] * uv[j] * sg * (1.f + gv[j] * (1.f - sg));
-                                du[j] = v[i + j] * gv[j] * sg;
-                            } else {
-                                const float a = gv[j];
-                                const float gp = 0.5f * (1.f + erff(a * 0.70710678118654752f)) +
-                                                 a * 0.39894228040143268f * __expf(-0.5f * a * a);
-                                dg_[j] = v[i + j] * gp;
+                    const bool swiglu = p.act == MOE_ACT_SWIGLU;
+                    if (ncol == 32) {            // whole chunk: 16-byte loads and stores
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint4 h4 = *reinterpret_cast<const uint4 *>(hr + u * 8);
+                            const uint4 g4 = *reinterpret_cast<const uint4 *>(gr + u * 8);
+                            const uint4 u4 = swiglu ? *reinterpret_cast<const uint4 *>(gr + p.F + u * 8)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&h4);
+                            const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g4);
+                            const __nv_bfloat162 *uu2 = reinterpret_cast<const __nv_bfloat162 *>(&u4);
+                            uint4 dg4, du4;
+                            __nv_bfloat162 *dg2 = reinterpret_cast<__nv_bfloat162 *>(&dg4);
+                            __nv_bfloat162 *du2 = reinterpret_cast<__nv_bfloat162 *>(&du4);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 hf = __bfloat1622float2(h2[j]);
+                                const float2 gf = __bfloat1622float2(g2[j]);
+                                const float va = v[u * 8 + 2 * j], vb = v[u * 8 + 2 * j + 1];
+                                dgp += hf.x * va + hf.y * vb;
+                                if (swiglu) {
+                                    const float2 uf = __bfloat1622float2(uu2[j]);
+                                    const float sa = 1.f / (1.f + __expf(-gf.x)), sb = 1.f / (1.f + __expf(-gf.y));
+                                    dg2[j] = __floats2bfloat162_rn(va * uf.x * sa * (1.f + gf.x * (1.f - sa)),
+                                                                   vb * uf.y * sb * (1.f + gf.y * (1.f - sb)));
+                                    du2[j] = __floats2bfloat162_rn(va * gf.x * sa, vb * gf.y * sb);
+                                } else {
+                                    const float pa = 0.5f * (1.f + erff(gf.x * 0.70710678118654752f)) +
+                                                     gf.x * 0.39894228040143268f * __expf(-0.5f * gf.x * gf.x);
+                                    const float pb = 0.5f * (1.f + erff(gf.y * 0.70710678118654752f)) +
+                                                     gf.y * 0.39894228040143268f * __expf(-0.5f * gf.y * gf.y);
+                                    dg2[j] = __floats2bfloat162_rn(va * pa, vb * pb);
+                                }
                             }
+                            *reinterpret_cast<uint4 *>(dr + u * 8) = dg4;
+                            if (swiglu) *reinterpret_cast<uint4 *>(dr + p.F + u * 8) = du4;
                         }
-                        for (int j = 0; j < two; ++j) {
-                            dr[i + j] = __float2bfloat16_rn(dg_[j]);
-                            if (p.act == MOE_ACT_SWIGLU) dr[p.F + i + j] = __float2bfloat16_rn(du[j]);
+                    } else {
+                        for (int i = 0; i < ncol; ++i) {
+                            const float hv = __bfloat162float(hr[i]), gv = __bfloat162float(gr[i]);
+                            dgp += hv * v[i];
+                            if (swiglu) {
+                                const float uv = __bfloat162float(gr[p.F + i]);
+                                const float sg = 1.f / (1.f + __expf(-gv));
+                                dr[i] = __float2bfloat16_rn(v[i] * uv * sg * (1.f + gv * (1.f - sg)));
+                                dr[p.F + i] = __float2bfloat16_rn(v[i] * gv * sg);
+                            } else {
+                                const float gp = 0.5f * (1.f + erff(gv * 0.70710678118654752f)) +
+                                                 gv * 0.39894228040143268f * __expf(-0.5f * gv * gv);
+                                dr[i] = __float2bfloat16_rn(v[i] * gp);
+                            }
                         }
                     }
                 }
