@@ -72,6 +72,7 @@ struct SmemB {
     uint64_t empty[STAGES];
     uint64_t accf[2];
     uint64_t acce[2];
+    uint64_t drain;              // the MMA thread's last commit: every MMA done before TMEM is freed
     uint32_t tmem_base;
     int abort_flag;
     int tile_start[kMaxGroups + 1];
@@ -123,6 +124,7 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             mbar_init(smem_u32(&s.empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 8); }
+        mbar_init(smem_u32(&s.drain), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -162,6 +164,9 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
+            int last_phase[STAGES];                       // phase of each stage's last load, -1: none
+#pragma unroll
+            for (int i = 0; i < STAGES; ++i) last_phase[i] = -1;
             for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
                 int g, mt, nt;
                 decode(s, G, tile, g, mt, nt);
@@ -200,9 +205,17 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     } else {
                         tma_load_3d(b_dst, &tmB, fb, kb * BK, nt * BN, e);
                     }
+#pragma unroll
+                    for (int i = 0; i < STAGES; ++i)
+                        if (i == stage) last_phase[i] = (int)phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
+            // no load may still be writing this CTA's shared memory when it exits
+#pragma unroll
+            for (int i = 0; i < STAGES; ++i)
+                if (last_phase[i] >= 0 && !mbar_wait(smem_u32(&s.full[i]), (uint32_t)last_phase[i], p.timeout_ns))
+                    fail(s, p, 36);
         }
     } else if (warp == 1) {
         // ================= MMA issuer
@@ -238,6 +251,9 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 mma_commit(smem_u32(&s.accf[ab]));
                 if (++ab == 2) { ab = 0; aphase ^= 1u; }
             }
+            // every MMA issued here has completed before the TMEM is freed
+            mma_commit(smem_u32(&s.drain));
+            if (!mbar_wait(smem_u32(&s.drain), 0, p.timeout_ns)) fail(s, p, 37);
         }
     } else if (warp == 10) {
         // ================= K-tail masking (groups that split K)

@@ -219,24 +219,24 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(DispatchArgs a, i
         const int my_row = lane < k ? list[tl * k + lane].x : -1;
         if (__ballot_sync(0xffffffffu, my_row >= 0) == 0u) continue;      // every slot dropped
         const uint4 *__restrict__ src = xs + (size_t)(t0 + tl) * nvec;
-        int v = lane;
-        for (; v + 224 < nvec; v += 256) {
+        // the loop bounds are the same for every lane (the slot rows come by
+        // shuffle); lanes past the row's last vector load and store nothing
+        for (int v0 = 0; v0 < nvec; v0 += 256) {
             uint4 r[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) r[i] = __ldg(src + v + 32 * i);
+            for (int i = 0; i < 8; ++i) {
+                const int v = v0 + 32 * i + lane;
+                if (v < nvec) r[i] = __ldg(src + v);
+            }
             for (int s = 0; s < k; ++s) {
                 const int row = __shfl_sync(0xffffffffu, my_row, s);
-                if (row < 0) continue;
+                if (row < 0) continue;                                      // same row on every lane
                 uint4 *__restrict__ dst = xd + (size_t)row * nvec;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dst[v + 32 * i] = r[i];
-            }
-        }
-        for (; v < nvec; v += 32) {
-            const uint4 r = __ldg(src + v);
-            for (int s = 0; s < k; ++s) {
-                const int row = __shfl_sync(0xffffffffu, my_row, s);
-                if (row >= 0) xd[(size_t)row * nvec + v] = r;
+                for (int i = 0; i < 8; ++i) {
+                    const int v = v0 + 32 * i + lane;
+                    if (v < nvec) dst[v] = r[i];
+                }
             }
         }
     }

@@ -111,7 +111,7 @@ def lib():
         L.moe_backward_workspace_size.restype = ctypes.c_size_t
         L.moe_backward_workspace_size.argtypes = [P(MoeConfig)]
         L.moe_backward.restype = ctypes.c_int
-        L.moe_backward.argtypes = [P(MoeConfig)] + [c_vp] * 15 + [ctypes.c_float] + [c_vp] * 12 + [
+        L.moe_backward.argtypes = [P(MoeConfig)] + [c_vp] * 15 + [ctypes.c_float] + [c_vp] * 11 + [
             c_vp, ctypes.c_size_t, c_vp, ctypes.c_size_t, c_vp]
         L.moe_workspace_view.restype = ctypes.c_int
         L.moe_workspace_view.argtypes = [P(MoeConfig), c_vp, ctypes.c_size_t, P(MoeWsView)]
