@@ -51,7 +51,8 @@ def test_backward_against_oracle(wl, alpha, cuda_device):
     g = torch.Generator(device=cuda_device).manual_seed(9)
     dy = torch.randn((wl.T, wl.d_model), generator=g, device=cuda_device).to(torch.bfloat16)
     grads = nat.backward(cfg, inp, out, ws, dy, alpha)
-    assert nat.moe_get_device_status(ws) == nat.MOE_OK
+    status = nat.moe_get_device_status(ws)
+    assert status == nat.MOE_OK, nat.last_error_detail()
     dims = oracle_dims(wl)
     ref = oracle.layer_backward(dims, host["x"], host["Wr"], weights_host(host), to_f64(dy), alpha,
                                 logit_bias=host["logit_bias"], sel_bias=host["sel_bias"])
