@@ -12,7 +12,7 @@ namespace {
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct BwdLayout {
-    size_t GU, dGU, dZ, dXr, part, dh, dh16, wr16, dXrt, sh_off, GUs, dGUs, dXs, parts;
+    size_t GU, dGU, dZ, dXr, part, dh, dh16, wr16, dXrt, sh_off, GUs, dGUs, dXs, parts, colpart;
     size_t total;
 };
 
@@ -29,7 +29,7 @@ BwdLayout bwd_layout(const moe_config *c) {
     L.GU = o;     o = al256(o + rows * gw * F * 2);
     L.dGU = o;    o = al256(o + rows * gw * F * 2);
     L.dZ = o;     o = al256(o + rows * d * 2);
-    L.dXr = o;    o = al256(o + rows * d * 4);
+    L.dXr = o;    o = al256(o + rows * d * 2);
     L.part = o;   o = al256(o + rows * (size_t)part_cols(c->d_ff) * 4);
     L.dh = o;     o = al256(o + T * (size_t)c->E * 4);
     L.dh16 = o;   o = al256(o + T * E64 * 2);
@@ -40,6 +40,7 @@ BwdLayout bwd_layout(const moe_config *c) {
     L.dGUs = o;   o = al256(o + T * gw * S * 2);
     L.dXs = o;    o = al256(o + (S > 0 ? T * d * 4 : 0));
     L.parts = o;  o = al256(o + (S > 0 ? T * (size_t)part_cols(c->d_ff_shared) * 4 : 0));
+    L.colpart = o; o = al256(o + (T + 255) / 256 * (size_t)c->E * 4);
     L.total = o;
     return L;
 }
@@ -147,7 +148,8 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
     const int E64 = pad64(E);
     __nv_bfloat16 *GU = at<__nv_bfloat16>(ws, L.GU), *dGU = at<__nv_bfloat16>(ws, L.dGU);
     __nv_bfloat16 *dZ = at<__nv_bfloat16>(ws, L.dZ);
-    float *dXr = at<float>(ws, L.dXr), *part = at<float>(ws, L.part), *dh = at<float>(ws, L.dh);
+    __nv_bfloat16 *dXr = at<__nv_bfloat16>(ws, L.dXr);
+    float *part = at<float>(ws, L.part), *dh = at<float>(ws, L.dh);
     __nv_bfloat16 *dh16 = at<__nv_bfloat16>(ws, L.dh16), *wr16 = at<__nv_bfloat16>(ws, L.wr16);
     float *dXrt = at<float>(ws, L.dXrt);
     int32_t *sh_off = at<int32_t>(ws, L.sh_off);
@@ -216,12 +218,12 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
         }
     }
 
-    // ---- 4. up-projection dgrad: dX = dG W_g + dU W_u (or dA W_1), fp32 rows
+    // ---- 4. up-projection dgrad: dX = dG W_g + dU W_u (or dA W_1), bf16 rows
     {
         if (!map2(&mA, dGU, (uint64_t)gw * F, rows, (uint64_t)gw * F, 128) || !map3(&mB, W1, d, F, E, 64) ||
             !map3(&mB2, swiglu ? Wu : W1, d, F, E, 64))
             return cuda(cudaErrorInvalidValue, "maps");
-        moe::BwdGemmParams p = gemm(v.offsets, E, 0, 0, d, gw * F, moe::BW_STORE_F32, status);
+        moe::BwdGemmParams p = gemm(v.offsets, E, 0, 0, d, gw * F, moe::BW_STORE_BF16, status);
         p.k_split = swiglu ? F : 0;
         p.out = dXr; p.ldo = d;
         if ((e = moe::launch_bwd_gemm(mA, mB, mB2, false, true, p, nsm, st)) != cudaSuccess) return cuda(e, "dgrad up");
@@ -290,8 +292,8 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
         if (db1 && (e = moe::launch_column_sums(c1, st)) != cudaSuccess) return cuda(e, "db1");
     }
     if (dlogit_bias) {
-        moe::ColSumArgs cb{dh, 1, E, nullptr, 1, T, E, dlogit_bias};
-        if ((e = moe::launch_column_sums(cb, st)) != cudaSuccess) return cuda(e, "dbeta");
+        if ((e = moe::launch_col_sums_2pass(dh, T, E, E, at<float>(ws, L.colpart), dlogit_bias, st)) != cudaSuccess)
+            return cuda(e, "dbeta");
     }
     return MOE_OK;
 }

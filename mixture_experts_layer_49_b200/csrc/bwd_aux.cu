@@ -215,6 +215,31 @@ __global__ void __launch_bounds__(256) column_sums_kernel(ColSumArgs a) {
     a.out[(int64_t)g * a.cols + c] = acc;
 }
 
+// Column sums of an fp32 [rows][cols] array in two deterministic passes:
+// pass 1, block (rb, cb) sums rows rb*256 .. rb*256+255 of its 256 columns
+// (thread per column, rows in order) into part[rb][c]; pass 2 sums the parts
+// of each column in block order.
+__global__ void __launch_bounds__(256) col_partials_kernel(const float *in, int64_t rows, int cols, int64_t ld,
+                                                           float *part) {
+    pdl_wait_then_release();
+    const int c = blockIdx.y * 256 + threadIdx.x;
+    if (c >= cols) return;
+    const int64_t r0 = (int64_t)blockIdx.x * 256;
+    const int64_t r1 = r0 + 256 < rows ? r0 + 256 : rows;
+    float acc = 0.f;
+    for (int64_t r = r0; r < r1; ++r) acc += in[r * ld + c];
+    part[(int64_t)blockIdx.x * cols + c] = acc;
+}
+
+__global__ void __launch_bounds__(256) col_finish_kernel(const float *part, int nparts, int cols, float *out) {
+    pdl_wait_then_release();
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    if (c >= cols) return;
+    float acc = 0.f;
+    for (int b = 0; b < nparts; ++b) acc += part[(int64_t)b * cols + c];
+    out[c] = acc;
+}
+
 // dx[t] = sum_s dX_rows[row_of[t, s]] (slot order) + dX_shared[t] + dX_router[t]
 __global__ void __launch_bounds__(256) dx_combine_kernel(BwdAuxArgs a) {
     pdl_wait_then_release();
@@ -230,9 +255,11 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(BwdAuxArgs a) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int s = 0; s < a.k; ++s) {
                 const int r = __shfl_sync(0xffffffffu, my_row, s);
-                if (in_row && r >= 0) {
-                    const float4 x = __ldg(reinterpret_cast<const float4 *>(a.dX_rows + (int64_t)r * a.d) + v);
-                    acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                if (in_row && r >= 0) {       // four bf16 values of the packed row
+                    const uint2 x = __ldg(reinterpret_cast<const uint2 *>(a.dX_rows + (int64_t)r * a.d) + v);
+                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
+                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
+                    acc.x += lo.x; acc.y += lo.y; acc.z += hi.x; acc.w += hi.y;
                 }
             }
             if (!in_row) continue;
@@ -297,6 +324,17 @@ cudaError_t launch_dx_combine(const BwdAuxArgs &a, cudaStream_t st) {
 
 cudaError_t launch_set_pair(int32_t *p, int32_t a, int32_t b, cudaStream_t st) {
     return launch_kernel(set_pair_kernel, dim3(1), dim3(32), 0, st, true, p, a, b);
+}
+
+cudaError_t launch_col_sums_2pass(const float *in, int64_t rows, int cols, int64_t ld, float *part, float *out,
+                                  cudaStream_t st) {
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    const int nparts = (int)((rows + 255) / 256);
+    cudaError_t e = launch_kernel(col_partials_kernel, dim3((unsigned)nparts, (unsigned)((cols + 255) / 256)), dim3(256),
+                                  0, st, true, in, rows, cols, ld, part);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(col_finish_kernel, dim3((unsigned)((cols + 255) / 256)), dim3(256), 0, st, true, part, nparts,
+                         cols, out);
 }
 
 cudaError_t launch_to_bf16(const float *in, __nv_bfloat16 *out, int64_t rows, int cols, int64_t ldo, cudaStream_t st) {

@@ -77,6 +77,7 @@ struct SmemB {
     int abort_flag;
     int tile_start[kMaxGroups + 1];
     int mtiles[kMaxGroups];
+    int order[kMaxGroups];       // group of each position in the tile order
 };
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SmemB);
 static_assert(kSmemBytes <= 227 * 1024, "backward GEMM shared memory");
@@ -89,16 +90,18 @@ __device__ __forceinline__ void fail(SmemB &s, const BwdGemmParams &p, int where
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
+// tile_start and mtiles are indexed by position in the tile order; order[]
+// maps a position to its group.
 __device__ __forceinline__ void decode(const SmemB &s, int G, int tile, int &g, int &mt, int &nt) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s.tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    g = lo;
-    const int local = tile - s.tile_start[g];
-    mt = local % s.mtiles[g];
-    nt = local / s.mtiles[g];
+    const int local = tile - s.tile_start[lo];
+    mt = local % s.mtiles[lo];
+    nt = local / s.mtiles[lo];
+    g = s.order[lo];
 }
 
 template <bool A_MN, bool B_MN>
@@ -131,12 +134,29 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), TMEM_COLS);
     pdl_wait_then_release();
     if (tid == 0) s.tile_start[0] = 0;
-    // tile table: groups split M (m-tiles over the group's rows) or K (m-tiles over M)
+    // tile order: groups that split K go largest first (every tile of a group
+    // costs its K, so the longest tiles start first); groups that split M
+    // keep their order.  Position of group g: the number of groups ahead of it.
     for (int g = tid; g < G; g += kThreads) {
+        int pos = g;
+        if (p.kgroup) {
+            const int rg = p.offsets[g + 1] - p.offsets[g];
+            pos = 0;
+            for (int h = 0; h < G; ++h) {
+                const int rh = p.offsets[h + 1] - p.offsets[h];
+                pos += (rh > rg || (rh == rg && h < g)) ? 1 : 0;
+            }
+        }
+        s.order[pos] = g;
+    }
+    __syncthreads();
+    // tile table, by position: groups split M (m-tiles over the group's rows) or K (m-tiles over M)
+    for (int i = tid; i < G; i += kThreads) {
+        const int g = s.order[i];
         const int rows = p.offsets[g + 1] - p.offsets[g];
         const int mt = p.kgroup ? (p.M + BM - 1) / BM : (rows + BM - 1) / BM;
-        s.mtiles[g] = mt > 0 ? mt : 1;
-        s.tile_start[g + 1] = mt * ((p.N + BN - 1) / BN);
+        s.mtiles[i] = mt > 0 ? mt : 1;
+        s.tile_start[i + 1] = mt * ((p.N + BN - 1) / BN);
     }
     __syncthreads();
     if (warp == 0) {

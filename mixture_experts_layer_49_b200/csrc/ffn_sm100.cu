@@ -490,17 +490,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // accumulator with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16).  Each
 // CTA loads its own 128 A rows and half of the B rows (SwiGLU: rank 0 the gate
 // rows, rank 1 the up rows), so a CTA moves 32 KiB per 64-deep K step instead
-// of 48 KiB, and six stages fit in shared memory.  Rank 0 issues the MMAs;
+// of 48 KiB; a stage holds two such K steps (three stages of 64 KiB), so one
+// barrier round trip covers eight MMAs.  Rank 0 issues the MMAs;
 // the full barriers live in rank 0 and collect both CTAs' TMA bytes; rank 0's
 // commits arrive on both CTAs' empty and accumulator-full barriers; both
 // CTAs' epilogue warps arrive on rank 0's accumulator-empty barriers.
 // Pair tiles cover a group's 256-row blocks and a last block of more than 128
 // rows; a last block of 1..128 rows runs in the 1-CTA kernel (tail mode), so
 // row padding never exceeds that of 128-row tiles.
-constexpr int P_STAGES = 6;
+constexpr int P_STAGES = 3;
+constexpr int P_ATOMS = 2;                         // 128-byte K atoms per stage
 constexpr uint32_t P_A_BYTES = BM * BK * 2;         // 16 KiB: this CTA's 128 A rows
 constexpr uint32_t P_B_BYTES = 128 * BK * 2;        // 16 KiB: this CTA's half of B
-constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr uint32_t P_STAGE_BYTES = P_ATOMS * (P_A_BYTES + P_B_BYTES);
 constexpr int PM = 2 * BM;                          // rows per pair tile
 constexpr uint32_t kIdescPair = make_idesc_bf16(PM, BNB);
 constexpr uint32_t kIdescPairF8 = make_idesc_e4m3(PM, BNB);
@@ -554,7 +556,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t *smem = smem_raw + (base - raw_addr);
     PairTail &s = *reinterpret_cast<PairTail *>(smem + P_STAGES * P_STAGE_BYTES);
     const uint32_t smA = base;                           // P_STAGES x 16 KiB
-    const uint32_t smB = base + P_STAGES * P_A_BYTES;    // P_STAGES x 16 KiB
+    const uint32_t smB = base + P_STAGES * P_ATOMS * P_A_BYTES;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -619,7 +621,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 decode_pair(s, G, tile, g, mt, nt);
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
-                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
+                const int nk = (K + P_ATOMS * bk_elems<F8>() - 1) / (P_ATOMS * bk_elems<F8>());
                 const int a_row = (sh ? (int)p.shared_a_row : s.row0[g]) + mt * PM + (int)rank * BM;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA;
                 const CUtensorMap *mB = (MODE == GM_SWIGLU && rank == 1) ? (sh ? &tmBs2 : &tmB2) : (sh ? &tmBs : &tmB);
@@ -629,8 +631,12 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 21); break; }
                     const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * P_STAGE_BYTES);
-                    tma_load_2d_pair(smA + stage * P_A_BYTES, mA, fb, kb * bk_elems<F8>(), a_row);
-                    tma_load_3d_pair(smB + stage * P_B_BYTES, mB, fb, kb * bk_elems<F8>(), b_row, e);
+#pragma unroll
+                    for (int at = 0; at < P_ATOMS; ++at) {
+                        const int kx = (kb * P_ATOMS + at) * bk_elems<F8>();
+                        tma_load_2d_pair(smA + (stage * P_ATOMS + at) * P_A_BYTES, mA, fb, kx, a_row);
+                        tma_load_3d_pair(smB + (stage * P_ATOMS + at) * P_B_BYTES, mB, fb, kx, b_row, e);
+                    }
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -646,7 +652,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 // the shared group, when there is one, is the last: its tiles start
                 // at tile_start[E] (= total without one), so K needs no search
                 const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
-                const int nk = (K + bk_elems<F8>() - 1) / bk_elems<F8>();
+                const int nk = (K + P_ATOMS * bk_elems<F8>() - 1) / (P_ATOMS * bk_elems<F8>());
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 22); break; }
                 tc_fence_after();
                 const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
@@ -654,13 +660,16 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns)) { fail_pair(s, p, 23); ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = smA + stage * P_A_BYTES, b0 = smB + stage * P_B_BYTES;
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
+                    for (int kk = 0; kk < P_ATOMS * (BK / 16); ++kk) {
+                        const int at = kk / (BK / 16), k = kk % (BK / 16);
+                        const uint32_t a0 = smA + (stage * P_ATOMS + at) * P_A_BYTES;
+                        const uint32_t b0 = smB + (stage * P_ATOMS + at) * P_B_BYTES;
                         if (F8)
-                            mma_e4m3_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPairF8, (kb | k) ? 1u : 0u);
+                            mma_e4m3_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPairF8, (kb | kk) ? 1u : 0u);
                         else
-                            mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | k) ? 1u : 0u);
+                            mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | kk) ? 1u : 0u);
+                    }
                     mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
                 }

@@ -230,7 +230,7 @@ struct BwdAuxArgs {
     float *dh;                   // [T, E]
     __nv_bfloat16 *dh_bf16;      // [T, dh_ld]
     int dh_ld;
-    const float *dX_rows;        // [rows, d]
+    const __nv_bfloat16 *dX_rows;  // [rows, d]
     const float *dX_shared;      // [T, d] or null
     const float *dX_router;      // [T, d]
     void *dx;                    // [T, d] bf16
@@ -251,6 +251,10 @@ struct ColSumArgs {
 };
 cudaError_t launch_column_sums(const ColSumArgs &a, cudaStream_t st);
 cudaError_t launch_to_bf16(const float *in, __nv_bfloat16 *out, int64_t rows, int cols, int64_t ldo, cudaStream_t st);
+// out[c] = sum of in[r][c] over r < rows, in two deterministic passes (part:
+// ceil(rows / 256) x cols fp32 scratch)
+cudaError_t launch_col_sums_2pass(const float *in, int64_t rows, int cols, int64_t ld, float *part, float *out,
+                                  cudaStream_t st);
 cudaError_t launch_set_pair(int32_t *p, int32_t a, int32_t b, cudaStream_t st);     // p[0] = a, p[1] = b
 
 // Host-side helpers shared by the entry points (moe_api.cu).
