@@ -186,14 +186,14 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
     // ---- 2. pre-activations again: G | U (SwiGLU) or W1 x + b1 (GELU), routed and shared
     for (int part_i = 0; part_i < gw; ++part_i) {
         const void *Wsrc = part_i == 0 ? W1 : Wu;
-        if (!map2(&mA, v.x_perm, d, rows, d, 128) || !map3(&mB, Wsrc, d, F, E, 256)) return cuda(cudaErrorInvalidValue, "maps");
+        if (!map2(&mA, v.x_perm, d, rows, d, 128) || !map3(&mB, Wsrc, d, F, E, moe::kBwdBoxRowsB)) return cuda(cudaErrorInvalidValue, "maps");
         moe::BwdGemmParams p = gemm(v.offsets, E, 0, 0, F, d, moe::BW_STORE_BF16, status);
         p.out = GU + part_i * F; p.ldo = (int64_t)gw * F;
         p.bias = (!swiglu) ? b1 : nullptr; p.bias_group_stride = F;
         if ((e = moe::launch_bwd_gemm(mA, mB, mB, false, false, p, nsm, st)) != cudaSuccess) return cuda(e, "recompute");
         if (shared) {
             const void *Ws = part_i == 0 ? Wsh_g : Wsh_u;
-            if (!map2(&mA, x, d, T, d, 128) || !map3(&mB, Ws, d, S, 1, 256)) return cuda(cudaErrorInvalidValue, "maps");
+            if (!map2(&mA, x, d, T, d, 128) || !map3(&mB, Ws, d, S, 1, moe::kBwdBoxRowsB)) return cuda(cudaErrorInvalidValue, "maps");
             moe::BwdGemmParams q = gemm(sh_off, 1, 0, 0, S, d, moe::BW_STORE_BF16, status);
             q.out = GUs + part_i * S; q.ldo = (int64_t)gw * S;
             if ((e = moe::launch_bwd_gemm(mA, mB, mB, false, false, q, nsm, st)) != cudaSuccess) return cuda(e, "recompute shared");
@@ -241,7 +241,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
     // ---- 5. router: gate gradients -> logits (+ balance loss); 6. its input gradient
     if ((e = moe::launch_router_bwd(aux, st)) != cudaSuccess) return cuda(e, "router backward");
     {
-        if (!map2(&mA, dh16, E64, T, E64, 128) || !map3(&mB, wr16, E64, d, 1, 256)) return cuda(cudaErrorInvalidValue, "maps");
+        if (!map2(&mA, dh16, E64, T, E64, 128) || !map3(&mB, wr16, E64, d, 1, moe::kBwdBoxRowsB)) return cuda(cudaErrorInvalidValue, "maps");
         moe::BwdGemmParams p = gemm(sh_off, 1, 0, 0, d, E64, moe::BW_STORE_F32, status);
         p.out = dXrt; p.ldo = d;
         if ((e = moe::launch_bwd_gemm(mA, mB, mB, false, false, p, nsm, st)) != cudaSuccess) return cuda(e, "router dgrad");

@@ -210,6 +210,8 @@ struct BwdGemmParams {
     int32_t *status;
     uint64_t timeout_ns;
 };
+// Rows of a K-major B box: each CTA of a pair loads half of a 256-column tile.
+constexpr uint32_t kBwdBoxRowsB = 128;
 cudaError_t launch_bwd_gemm(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &B2, bool a_mn, bool b_mn,
                             const BwdGemmParams &p, int num_sms, cudaStream_t st);
 
