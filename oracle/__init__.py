@@ -14,6 +14,9 @@ uint16 bit patterns; router weights and biases are fp32.
 FP8 experts (``e4m3_value``, ``e4m3_round``, ``quantize_rows``,
 ``expert_apply_fp8``, ``layer_tokens_fp8``): e4m3 codes with per-channel
 weight scales and per-row activation scales, defined in ``moe_oracle.c``.
+Block-scaled (MX) FP8 experts (``quantize_mx``, ``mx_value``,
+``expert_apply_mx``, ``layer_tokens_mx``): e4m3 codes with one power-of-two
+(E8M0) scale per 32 values along the contraction dimension.
 
 Parity pins (tests/test_oracle_pins.py): brute-force top-k on tiny inputs,
 library softmax / sigmoid for the gates, sums of counts, closed-form balance
@@ -56,7 +59,7 @@ def _load():
         for name in ("oracle_route", "oracle_dispatch", "oracle_balance",
                      "oracle_expert_apply", "oracle_layer_tokens", "oracle_bias_update",
                      "oracle_routing_health", "oracle_quantize_rows", "oracle_expert_apply_fp8",
-                     "oracle_layer_backward"):
+                     "oracle_layer_backward", "oracle_quantize_mx", "oracle_expert_apply_mx"):
             getattr(lib, name).restype = ctypes.c_int
         lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -300,6 +303,81 @@ def quantize_rows(v):
     lib.oracle_quantize_rows(_ptr(v), ctypes.c_int64(rows), ctypes.c_int32(cols), ctypes.c_int64(cols),
                              _ptr(codes), _ptr(scale))
     return codes, scale
+
+
+def quantize_mx(v):
+    """MX quantization of a float32 matrix (columns a multiple of 32): (codes
+    uint8 [rows, cols], scale bytes uint8 [rows, cols / 32], E8M0: 2^(s - 127))."""
+    lib = _load()
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, cols = v.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty((rows, cols // 32), np.uint8)
+    if lib.oracle_quantize_mx(_ptr(v), ctypes.c_int64(rows), ctypes.c_int32(cols), ctypes.c_int64(cols),
+                              _ptr(codes), _ptr(scales)):
+        raise ValueError("quantize_mx: columns must be a positive multiple of 32")
+    return codes, scales
+
+
+def mx_value(codes, scales):
+    """float64 values of MX codes with their block scale bytes (last axis of
+    codes = 32 x last axis of scales)."""
+    codes = np.asarray(codes, np.uint8)
+    sc = np.repeat(np.asarray(scales, np.int64), 32, axis=-1)
+    return np.ldexp(e4m3_value(codes.ravel()).reshape(codes.shape), (sc - 127).astype(np.int32))
+
+
+def _mx_weights(w):
+    def u8(a):
+        return None if a is None else np.ascontiguousarray(a, dtype=np.uint8)
+    return (u8(w.get("W1")), u8(w.get("W1_scale")), _f32(w.get("b1")),
+            u8(w.get("Wu")), u8(w.get("Wu_scale")),
+            u8(w.get("W2")), u8(w.get("W2_scale")), _f32(w.get("b2")),
+            u8(w.get("Wsg")), u8(w.get("Wsg_scale")), u8(w.get("Wsu")), u8(w.get("Wsu_scale")),
+            u8(w.get("Wsd")), u8(w.get("Wsd_scale")))
+
+
+def expert_apply_mx(dims, x8, xs, weights, token, expert, scale=None):
+    """out[r] = scale[r] * Emx_{expert[r]}(x8[token[r]]) with MX experts.
+
+    x8: e4m3 codes [T, d] with scale bytes xs [T, d/32]; weights: W1, Wu, W2
+    (and Wsg, Wsu, Wsd) as e4m3 codes with scale bytes "<name>_scale" of shape
+    [..., out, in/32]; biases b1, b2 fp32."""
+    lib = _load()
+    x8 = np.ascontiguousarray(x8, dtype=np.uint8)
+    xs = np.ascontiguousarray(xs, dtype=np.uint8)
+    token = np.ascontiguousarray(token, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.float64)
+    out = np.empty((len(token), dims.d), np.float64)
+    ws = _mx_weights(weights)
+    rc = lib.oracle_expert_apply_mx(ctypes.byref(dims), ctypes.c_int64(len(token)), _ptr(token), _ptr(expert),
+                                    _ptr(sc), _ptr(x8), _ptr(xs), *[_ptr(a) for a in ws], _ptr(out))
+    if rc:
+        raise ValueError("oracle_expert_apply_mx: bad expert id or dimension not a multiple of 32")
+    return out
+
+
+def layer_tokens_mx(dims, x8, xs, weights, idx, gate, row_of, tokens):
+    """y[n] for the listed tokens with MX experts: the gate-weighted sum of
+    the kept experts (+ the shared expert, weight 1), summed in float64."""
+    idx = np.asarray(idx, np.int32)
+    gate = np.asarray(gate, np.float64)
+    tokens = np.asarray(tokens, np.int32)
+    tok, ex, g, owner = [], [], [], []
+    for n, t in enumerate(tokens):
+        for s in range(dims.k):
+            if row_of is not None and row_of[t, s] < 0:
+                continue
+            tok.append(t); ex.append(idx[t, s]); g.append(gate[t, s]); owner.append(n)
+        if dims.d_ff_shared > 0:
+            tok.append(t); ex.append(dims.E); g.append(1.0); owner.append(n)
+    y = np.zeros((len(tokens), dims.d), np.float64)
+    if tok:
+        rows = expert_apply_mx(dims, x8, xs, weights, np.array(tok), np.array(ex), np.array(g))
+        for r, n in enumerate(owner):
+            y[n] += rows[r]
+    return y
 
 
 def _fp8_weights(w):

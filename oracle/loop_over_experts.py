@@ -220,3 +220,82 @@ def layer_fp8(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1,
     if weights.get("Wsg") is not None:
         y += expert_fn_fp8(act, xd, wdeq("Wsg"), wdeq("Wsu"), wdeq("Wsd"))
     return dict(y=y, idx=idx, gate=gate, x8=x8, xs=xs)
+
+
+# ---------------------------------------------------------------- MX experts
+# The same layer with block-scaled (MX) e4m3 experts: 32-value blocks along the
+# contraction dimension share a power-of-two scale, found here by comparing the
+# block maximum against every power of two (no shared code with the C
+# oracle's frexp-based exponent) and applied to the table search above.
+
+def quantize_mx_np(v):
+    """(codes [rows, cols], scale bytes [rows, cols/32]) of a float32 matrix:
+    X is the largest integer in [-127, 127] with 2^(X + 8) <= amax (-127 when
+    no power qualifies or amax = 0); codes are the nearest e4m3 values of v / 2^X."""
+    v = np.asarray(v, np.float32)
+    rows, cols = v.shape
+    blk = v.reshape(rows, cols // 32, 32).astype(np.float64)
+    amax = np.abs(blk).max(axis=2)
+    X = np.full(amax.shape, -127, np.int64)
+    for e in range(-127, 128):
+        X = np.where(amax >= 2.0 ** (e + 8), e, X)
+    q = (blk / np.exp2(X.astype(np.float64))[..., None]).astype(np.float32)
+    codes = e4m3_nearest(q).reshape(rows, cols)
+    return codes, (X + 127).astype(np.uint8)
+
+
+def dequant_mx(codes, scales):
+    codes = np.asarray(codes, np.uint8)
+    sc = np.repeat(np.asarray(scales, np.float64) - 127.0, 32, axis=-1)
+    return E4M3[codes] * np.exp2(sc)
+
+
+def expert_fn_mx(act, xd, Wa, Wb, Wo, b_a=None, b_o=None):
+    """One MX expert on dequantized rows xd with dequantized weights; H is
+    rounded to bf16 and MX-quantized along d_ff before the second product."""
+    a = xd @ Wa.T
+    if act == "gelu":
+        if b_a is not None:
+            a = a + b_a
+        h = a * stats.norm.cdf(a)
+    else:
+        h = a * special.expit(a) * (xd @ Wb.T)
+    hc, hs = quantize_mx_np(bf16_round(h).astype(np.float32))
+    o = dequant_mx(hc, hs) @ Wo.T
+    if b_o is not None:
+        o = o + b_o
+    return o
+
+
+def layer_mx(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1,
+             logit_bias=None, sel_bias=None):
+    """The layer with MX experts.  weights: e4m3 codes W1, Wu, W2 (Wsg, Wsu,
+    Wsd) with scale bytes "<name>_scale" [..., out, in/32], biases b1, b2.
+    Returns dict(y, idx, gate, x8, xs)."""
+    idx, gate, _, _ = route(x, Wr, k, score=score, renorm=renorm, logit_bias=logit_bias, sel_bias=sel_bias)
+    x8, xs = quantize_mx_np(_f64(x).astype(np.float32))
+    xd = dequant_mx(x8, xs)
+    T, d = xd.shape
+    E = np.asarray(Wr).shape[1]
+
+    def wdeq(name):
+        if weights.get(name) is None:
+            return None
+        return dequant_mx(weights[name], weights[name + "_scale"])
+
+    W1, Wu, W2 = wdeq("W1"), wdeq("Wu"), wdeq("W2")
+    b1 = np.asarray(weights["b1"], np.float64) if weights.get("b1") is not None else None
+    b2 = np.asarray(weights["b2"], np.float64) if weights.get("b2") is not None else None
+    y = np.zeros((T, d), np.float64)
+    for e in range(E):
+        tok, slot = np.nonzero(idx == e)
+        if capacity >= 0:
+            tok, slot = tok[:capacity], slot[:capacity]
+        if len(tok) == 0:
+            continue
+        o = expert_fn_mx(act, xd[tok], W1[e], None if Wu is None else Wu[e], W2[e],
+                         None if b1 is None else b1[e], None if b2 is None else b2[e])
+        np.add.at(y, tok, o * gate[tok, slot][:, None])
+    if weights.get("Wsg") is not None:
+        y += expert_fn_mx(act, xd, wdeq("Wsg"), wdeq("Wsu"), wdeq("Wsd"))
+    return dict(y=y, idx=idx, gate=gate, x8=x8, xs=xs)

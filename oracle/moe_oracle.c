@@ -638,6 +638,162 @@ int oracle_expert_apply_fp8(const oracle_dims *dm, int64_t nrows, const int32_t 
     return 0;
 }
 
+/* ---- Block-scaled FP8 (MX) experts ------------------------------------------
+ * [IS] Serving section (quantized experts, FP8 or INT4, once memory binds).
+ * The block-scaled reading follows the OCP microscaling (MX) FP8 layout: along
+ * the contraction dimension of every matrix, each run of 32 consecutive
+ * values shares one power-of-two scale 2^X, stored as the byte X + 127
+ * (E8M0), and every value is stored as an e4m3 code:
+ *   amax = max |v_j| over the block
+ *   X    = floor(log2(amax)) - 8       (8: the exponent of e4m3's largest
+ *                                       normal, 448 = 1.75 * 2^8), clamped to
+ *                                       [-127, 127]; X = -127 for amax = 0
+ *   code = e4m3 nearest to v_j / 2^X (ties to even, saturating at 448, sign
+ *          kept); the division by a power of two is exact
+ * so the block's largest magnitude maps into [256, 512) and values above 448
+ * saturate.  x is quantized per token row along d_model, each weight matrix
+ * per output row along its input dimension, and H (held in bf16 first) per
+ * row along d_ff.  A product of two blocks is
+ *   2^(Xa + Xw) * sum_j e4m3(a_j) e4m3(w_j),
+ * summed over the blocks in double.                                         */
+
+/* X of a block whose largest magnitude is amax > 0.                          */
+static int mx_exponent(float amax)
+{
+    int x;
+    (void)frexp((double)amax, &x);           /* amax = f 2^x, f in [0.5, 1)   */
+    int X = (x - 1) - 8;
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    return X;
+}
+
+/* MX quantization of rows x cols fp32 values (row stride ld, cols a
+ * multiple of 32): codes [rows, cols], scale bytes [rows, cols / 32].       */
+int oracle_quantize_mx(const float *v, int64_t rows, int32_t cols, int64_t ld, uint8_t *codes, uint8_t *scales)
+{
+    if (cols <= 0 || cols % 32 != 0) return 1;
+    const int nb = cols / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = v + r * ld;
+        for (int b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                const float a = fabsf(row[b * 32 + j]);
+                if (a > amax) amax = a;
+            }
+            const int X = amax > 0.0f ? mx_exponent(amax) : -127;
+            scales[r * nb + b] = (uint8_t)(X + 127);
+            for (int j = 0; j < 32; ++j) {
+                const double q = ldexp((double)row[b * 32 + j], -X);
+                codes[r * (int64_t)cols + b * 32 + j] = oracle_e4m3_round((float)q);
+            }
+        }
+    }
+    return 0;
+}
+
+/* sum over the n / 32 blocks of 2^(Xa + Xw) * sum_j e4m3(a_j) e4m3(w_j).      */
+static double mx_dot(const uint8_t *a, const uint8_t *as, const uint8_t *w, const uint8_t *ws, int n)
+{
+    double s = 0.0;
+    for (int b = 0; b < n / 32; ++b) {
+        double blk = 0.0;
+        for (int j = 0; j < 32; ++j) blk += oracle_e4m3_value(a[b * 32 + j]) * oracle_e4m3_value(w[b * 32 + j]);
+        s += ldexp(blk, ((int)as[b] - 127) + ((int)ws[b] - 127));
+    }
+    return s;
+}
+
+typedef struct {
+    const oracle_dims *dm;
+    const uint8_t *x8, *xs;                                  /* [T, d], [T, d/32]             */
+    const uint8_t *W1, *s1; const float *b1;                 /* [E, d_ff, d], [E, d_ff, d/32]  */
+    const uint8_t *Wu, *su;
+    const uint8_t *W2, *s2; const float *b2;                 /* [E, d, d_ff], [E, d, d_ff/32]  */
+    const uint8_t *Wsg, *ssg, *Wsu, *ssu, *Wsd, *ssd;        /* shared expert, same layouts    */
+} mx_experts;
+
+/* One MX expert on token t (e == E: the shared expert).  hbuf: d_ff doubles,
+ * hf: d_ff floats, hc: d_ff bytes, hs: d_ff / 32 bytes of scratch.          */
+static void expert_apply_mx_one(const mx_experts *w, int64_t t, int e, double *hbuf, float *hf, uint8_t *hc,
+                                uint8_t *hs, double *out)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const uint8_t *Wa = shared ? w->Wsg : w->W1, *Wb = shared ? w->Wsu : w->Wu, *Wo = shared ? w->Wsd : w->W2;
+    const uint8_t *sa = shared ? w->ssg : w->s1, *sb = shared ? w->ssu : w->su, *so = shared ? w->ssd : w->s2;
+    const size_t eb = shared ? 0 : (size_t)e;
+    const uint8_t *xr = w->x8 + (size_t)t * d, *xsr = w->xs + (size_t)t * (d / 32);
+    for (int j = 0; j < dff; ++j) {
+        const size_t wr = eb * dff + j;
+        double a = mx_dot(xr, xsr, Wa + wr * d, sa + wr * (d / 32), d);
+        if (dm->act == 0) {
+            if (!shared && w->b1) a += (double)w->b1[eb * dff + j];
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else {
+            const double u = mx_dot(xr, xsr, Wb + wr * d, sb + wr * (d / 32), d);
+            hbuf[j] = a / (1.0 + exp(-a)) * u;
+        }
+        hf[j] = round_bf16(hbuf[j]);
+    }
+    oracle_quantize_mx(hf, 1, dff, dff, hc, hs);
+    for (int i = 0; i < d; ++i) {
+        const size_t orow = eb * d + i;
+        double o = mx_dot(hc, hs, Wo + orow * dff, so + orow * (dff / 32), dff);
+        if (dm->act == 0 && !shared && w->b2) o += (double)w->b2[eb * d + i];
+        out[i] = o;
+    }
+}
+
+typedef struct {
+    mx_experts w;
+    const int32_t *token; const int32_t *expert; const double *scale; double *out;
+} applymx_ctx;
+
+static void applymx_range(void *vctx, int64_t lo, int64_t hi)
+{
+    applymx_ctx *c = (applymx_ctx *)vctx;
+    const oracle_dims *dm = c->w.dm;
+    const int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    const size_t hn = (size_t)(hmax > 0 ? hmax : 32);
+    double *hbuf = (double *)malloc(sizeof(double) * hn);
+    float *hf = (float *)malloc(sizeof(float) * hn);
+    uint8_t *hc = (uint8_t *)malloc(hn);
+    uint8_t *hs = (uint8_t *)malloc(hn / 32 + 1);
+    for (int64_t r = lo; r < hi; ++r) {
+        double *o = c->out + (size_t)r * dm->d;
+        expert_apply_mx_one(&c->w, c->token[r], c->expert[r], hbuf, hf, hc, hs, o);
+        const double sc = c->scale ? c->scale[r] : 1.0;
+        for (int i = 0; i < dm->d; ++i) o[i] *= sc;
+    }
+    free(hbuf); free(hf); free(hc); free(hs);
+}
+
+/* out[r,:] = scale[r] * Emx_{expert[r]}(x8[token[r],:]) for MX experts;
+ * expert == E selects the shared expert.  d, d_ff (and d_ff_shared) must be
+ * multiples of 32.                                                          */
+int oracle_expert_apply_mx(const oracle_dims *dm, int64_t nrows, const int32_t *token, const int32_t *expert,
+                           const double *scale, const uint8_t *x8, const uint8_t *xs,
+                           const uint8_t *W1, const uint8_t *s1, const float *b1,
+                           const uint8_t *Wu, const uint8_t *su,
+                           const uint8_t *W2, const uint8_t *s2, const float *b2,
+                           const uint8_t *Wsg, const uint8_t *ssg, const uint8_t *Wsu, const uint8_t *ssu,
+                           const uint8_t *Wsd, const uint8_t *ssd, double *out)
+{
+    if (dm->d % 32 != 0 || dm->d_ff % 32 != 0 || (dm->d_ff_shared > 0 && dm->d_ff_shared % 32 != 0)) return 2;
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (expert[r] < 0 || expert[r] > dm->E) return 1;
+        if (expert[r] == dm->E && dm->d_ff_shared <= 0) return 1;
+    }
+    applymx_ctx c = { { dm, x8, xs, W1, s1, b1, Wu, su, W2, s2, b2, Wsg, ssg, Wsu, ssu, Wsd, ssd },
+                      token, expert, scale, out };
+    parallel_for(nrows, dm->nthreads, applymx_range, &c);
+    return 0;
+}
+
 /* ===========================================================================
  * Backward pass of the layer.
  *
