@@ -359,6 +359,65 @@ MOE_API moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const f
                                    int32_t *counts, float *f, float *P, double *loss, float *logits_out,
                                    int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- Block-scaled (MX) FP8 experts --------------------------------------
+ * The block-scaled form of quantized experts ("Fine-tuning and serving MoE
+ * models", Serving: quantize the experts since memory binds), laid out as OCP
+ * microscaling (MX) FP8: along the contraction dimension of every matrix,
+ * each run of 32 values shares one power-of-two scale 2^X stored as the byte
+ * X + 127 (E8M0), each value one e4m3 code.  The expert GEMMs run as
+ * tcgen05.mma.kind::mxf8f6f4.block_scale (the hardware applies both
+ * operands' block scales; fp32 accumulation).
+ *   quantization (moe_quantize_rows_mx, and H on the device): per block of
+ *     32 values, amax = max |v|, X = floor(log2 amax) - 8 clamped to
+ *     [-127, 127] (-127 for a zero or subnormal amax), code = e4m3(v * 2^-X),
+ *     round to nearest even, saturating at 448 (values in (448, 512) * 2^X
+ *     saturate).
+ *   weights: codes in the nn.Linear [out, in] layout stacked over experts,
+ *     scale bytes [.., out, in / 32] with rows of sld bytes.
+ *   activations: x per token row along d_model; H (formed in bf16 first, as
+ *     in the bf16 layer) per row along d_ff.
+ * Every scale array (x, weights) has rows of sld bytes: sld a multiple of 16
+ * and at least d_model / 32, d_ff / 32 and d_ff_shared / 32.  Only bf16
+ * layers with d_model, d_ff and d_ff_shared multiples of 128 and E <= 256
+ * (else MOE_ERR_UNSUPPORTED).  All pointers in the struct are device
+ * pointers, codes and scale arrays 16-byte aligned; the struct is read
+ * during the call.                                                          */
+typedef struct {
+    const uint8_t *W1;    const uint8_t *W1_scale;      /* [E, d_ff, d_model], [E, d_ff, sld]     */
+    const uint8_t *Wu;    const uint8_t *Wu_scale;      /* SwiGLU W_up (same shapes), else NULL   */
+    const uint8_t *W2;    const uint8_t *W2_scale;      /* [E, d_model, d_ff], [E, d_model, sld]  */
+    const uint8_t *Wsh_g; const uint8_t *Wsh_g_scale;   /* shared expert [d_ff_shared, d_model],
+                                                           [d_ff_shared, sld], or NULL            */
+    const uint8_t *Wsh_u; const uint8_t *Wsh_u_scale;   /* SwiGLU shared W_up, or NULL            */
+    const uint8_t *Wsh_d; const uint8_t *Wsh_d_scale;   /* [d_model, d_ff_shared], [d_model, sld] */
+    int32_t sld;                                        /* scale row stride in bytes             */
+} moe_mx_experts;
+
+/* MX quantization of a bf16 matrix: `rows` rows of `cols` values (row stride
+ * ld_in elements, cols a multiple of 32) -> codes [rows, ld_out bytes] and
+ * one scale byte per 32 values, scales [rows, ld_scale bytes] (ld_scale >=
+ * cols / 32).  ld_in, ld_out multiples of 8; in 16-byte, codes 8-byte
+ * aligned.  The codes are a function of the bf16 values alone (the scaling
+ * by 2^-X is exact).                                                        */
+MOE_API moe_status moe_quantize_rows_mx(const void *in, int64_t rows, int32_t cols, int64_t ld_in,
+                                        uint8_t *codes, int64_t ld_out, uint8_t *scales, int64_t ld_scale,
+                                        moe_stream_t stream);
+
+/* moe_grouped_ffn with MX experts: x8_perm [T*top_k, d_model] codes of the
+ * packed rows with their scales xs_perm [T*top_k, sld]; x8 / xs the codes and
+ * scales of x [T, d_model] (the shared expert's input; NULL without one); b1,
+ * b2 fp32 as in moe_grouped_ffn.  Output y_perm [moe_perm_rows(cfg), d_model]
+ * bf16 as in moe_grouped_ffn (routed rows past offsets[E] untouched, the
+ * shared expert's rows from T*top_k on).  The workspace (its first 256 bytes
+ * a status word) holds H in bf16, its MX codes and scales:
+ * moe_grouped_ffn_mx_workspace_size(cfg, sld) bytes, 256-byte aligned (0 on
+ * a bad or unsupported configuration).                                      */
+MOE_API size_t moe_grouped_ffn_mx_workspace_size(const moe_config *cfg, int32_t sld);
+MOE_API moe_status moe_grouped_ffn_mx(const moe_config *cfg, const uint8_t *x8_perm, const uint8_t *xs_perm,
+                                      const int32_t *offsets, const float *row_gate, const moe_mx_experts *w,
+                                      const float *b1, const float *b2, const uint8_t *x8, const uint8_t *xs,
+                                      void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Auxiliary-loss-free bias update, to run after a training step on the
  * counts that step's routing produced ("Fine-Tuning Mixture of Experts (MoE)
  * Models: Router Optimization Techniques", How It Works 2, and its router

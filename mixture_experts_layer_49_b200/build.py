@@ -13,7 +13,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["moe_api.cu", "router_topk.cu", "dispatch.cu", "ffn_f32.cu", "ffn_sm100.cu",
            "combine_balance.cu", "permute_noalloc.cu", "router_sm100.cu", "quant_fp8.cu",
-           "bwd_sm100.cu", "bwd_aux.cu", "bwd_api.cu"]
+           "bwd_sm100.cu", "bwd_aux.cu", "bwd_api.cu", "mx_sm100.cu"]
 HEADERS = ["balance.cuh", "common.cuh", "kernels.cuh", "sm100.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

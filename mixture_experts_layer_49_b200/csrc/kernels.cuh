@@ -130,6 +130,50 @@ bool make_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64
 cudaError_t launch_ffn_f32(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st);
 
+// Block-scaled (MX) e4m3 quantization of bf16 rows (row0 + r for r < rows,
+// or fewer when rows_limit points at a smaller device count): codes [.., ld_out]
+// and one E8M0 scale byte per 32 values [.., ld_scale].  cols % 32 == 0,
+// ld_out % 8 == 0.  mx_sm100.cu.
+struct QuantMxArgs {
+    const __nv_bfloat16 *in;
+    int64_t ld_in;
+    uint8_t *out;
+    int64_t ld_out;
+    uint8_t *scale;
+    int64_t ld_scale;
+    int64_t rows, row0;
+    int cols;
+    const int32_t *rows_limit;
+    int num_sms;
+    bool pdl;
+};
+cudaError_t launch_quant_mx(const QuantMxArgs &a, cudaStream_t st);
+
+// The grouped FFN with MX experts (mx_sm100.cu).  Every scale array has rows
+// of sld bytes (sld % 16 == 0, at least its K / 32); K dimensions (d, F, S)
+// are multiples of 128.
+struct FfnMxArgs {
+    const uint8_t *x_perm; const uint8_t *xs_perm;    // [routed_rows, d] codes, [routed_rows, sld] scales
+    const uint8_t *x; const uint8_t *xs;              // [T, d], [T, sld] (shared expert) or null
+    const int32_t *offsets;                           // [E+1]
+    const float *row_gate;                            // [routed_rows]
+    const uint8_t *W1, *W1s, *Wu, *Wus;               // [E, F, d] codes, [E, F, sld] scales
+    const uint8_t *W2, *W2s;                          // [E, d, F], [E, d, sld]
+    const float *b1, *b2;                             // GELU biases or null
+    const uint8_t *Wsg, *Wsgs, *Wsu, *Wsus, *Wsd, *Wsds;
+    __nv_bfloat16 *H;                                 // [routed_rows (+T), hF]
+    uint8_t *H8, *Hs;                                 // codes [.., hF], scales [.., sld]
+    __nv_bfloat16 *y_perm;                            // [routed_rows (+T), d]
+    int32_t *status;
+    int T, d, E, F, S, act;
+    int64_t routed_rows;
+    int hF;
+    int64_t shared_base;                              // first shared row of H / y_perm
+    int sld;
+    int num_sms;
+};
+cudaError_t launch_ffn_mx(const FfnMxArgs &a, cudaStream_t st);
+
 // Per-row e4m3 quantization of bf16 rows (row0 + r for r < rows, or fewer
 // when rows_limit points at a smaller device count): in [.., ld_in] bf16,
 // out [.., ld_out] e4m3 codes, scale [..] fp32.  cols % 8 == 0.

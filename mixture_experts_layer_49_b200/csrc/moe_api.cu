@@ -1,6 +1,8 @@
 // moe_api.cu -- the extern "C" boundary of libmoe: argument checks, workspace
 // layout and the launch sequence.  See include/moe.h for the contract.
 #include <math.h>
+
+#include <algorithm>
 #include <stdio.h>
 #include <string.h>
 
@@ -121,6 +123,35 @@ moe_status check_fp8_cfg(const moe_config *c) {
     if (c->d_model % 16 || c->d_ff % 16 || c->d_ff_shared % 16)
         return fail(MOE_ERR_UNSUPPORTED, "FP8 experts need d_model, d_ff, d_ff_shared multiples of 16%s");
     return MOE_OK;
+}
+
+// MX experts: bf16 layers, K dimensions in whole 128-value stages, at most
+// 256 routed groups, scale rows of sld bytes (a multiple of 16 that holds
+// d_model / 32, d_ff / 32 and d_ff_shared / 32 bytes).
+moe_status check_mx_cfg(const moe_config *c, int32_t sld) {
+    if (c->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "MX experts need a bf16 layer%s");
+    if (c->d_model % 128 || c->d_ff % 128 || c->d_ff_shared % 128)
+        return fail(MOE_ERR_UNSUPPORTED, "MX experts need d_model, d_ff, d_ff_shared multiples of 128%s");
+    if (c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "MX experts: at most 256 experts%s");
+    const int need = std::max(c->d_model, std::max(c->d_ff, c->d_ff_shared)) / 32;
+    if (sld < need || sld % 16) return fail(MOE_ERR_INVALID_ARG, "sld below the widest K / 32 or not a multiple of 16%s");
+    return MOE_OK;
+}
+
+struct MxLayout {
+    size_t H, H8, Hs, total;
+    int hF;
+};
+MxLayout mx_layout(const moe_config *c, int32_t sld) {
+    MxLayout L{};
+    const size_t rows = (size_t)c->T * c->top_k + (c->d_ff_shared > 0 ? (size_t)c->T : 0);
+    L.hF = std::max(c->d_ff, c->d_ff_shared);
+    size_t o = sizeof(moe::WsHeader);
+    L.H = o;   o = align256(o + rows * L.hF * 2);
+    L.H8 = o;  o = align256(o + rows * L.hF);
+    L.Hs = o;  o = align256(o + rows * (size_t)sld);
+    L.total = o;
+    return L;
 }
 
 moe_status check_fp8_weights(const moe_config *c, const moe_fp8_experts *w) {
@@ -641,6 +672,88 @@ moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
     if ((e = moe::launch_combine(ca, true, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
+}
+
+// ---- block-scaled (MX) e4m3 experts
+
+moe_status moe_quantize_rows_mx(const void *in, int64_t rows, int32_t cols, int64_t ld_in, uint8_t *codes,
+                                int64_t ld_out, uint8_t *scales, int64_t ld_scale, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return fail(MOE_ERR_INVALID_ARG, "negative rows or cols%s");
+    if (rows == 0 || cols == 0) return MOE_OK;
+    NEED(in); NEED(codes); NEED(scales);
+    if (cols % 32) return fail(MOE_ERR_UNSUPPORTED, "cols must be a multiple of 32%s");
+    if (ld_in < cols || ld_in % 8) return fail(MOE_ERR_INVALID_ARG, "ld_in < cols or not a multiple of 8%s");
+    if (ld_out < cols || ld_out % 8) return fail(MOE_ERR_INVALID_ARG, "ld_out < cols or not a multiple of 8%s");
+    if (ld_scale < cols / 32) return fail(MOE_ERR_INVALID_ARG, "ld_scale < cols / 32%s");
+    ALIGNED(in, 16); ALIGNED(codes, 8);
+    moe::QuantMxArgs q{};
+    q.in = static_cast<const __nv_bfloat16 *>(in);
+    q.ld_in = ld_in;
+    q.out = codes;
+    q.ld_out = ld_out;
+    q.scale = scales;
+    q.ld_scale = ld_scale;
+    q.rows = rows;
+    q.cols = cols;
+    q.num_sms = num_sms();
+    cudaError_t e = moe::launch_quant_mx(q, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "quantize_rows_mx");
+}
+
+size_t moe_grouped_ffn_mx_workspace_size(const moe_config *cfg, int32_t sld) {
+    if (check_cfg(cfg) != MOE_OK || check_mx_cfg(cfg, sld) != MOE_OK) return 0;
+    return mx_layout(cfg, sld).total;
+}
+
+moe_status moe_grouped_ffn_mx(const moe_config *cfg, const uint8_t *x8_perm, const uint8_t *xs_perm,
+                              const int32_t *offsets, const float *row_gate, const moe_mx_experts *w, const float *b1,
+                              const float *b2, const uint8_t *x8, const uint8_t *xs, void *y_perm, void *ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(w);
+    if ((s = check_mx_cfg(cfg, w->sld)) != MOE_OK) return s;
+    const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+    const bool shared = cfg->d_ff_shared > 0;
+    if (cfg->T > 0) {
+        NEED(x8_perm); NEED(xs_perm); NEED(offsets); NEED(row_gate); NEED(y_perm);
+        NEED(w->W1); NEED(w->W1_scale); NEED(w->W2); NEED(w->W2_scale);
+        if (swiglu) { NEED(w->Wu); NEED(w->Wu_scale); }
+        if (shared) {
+            NEED(x8); NEED(xs); NEED(w->Wsh_g); NEED(w->Wsh_g_scale); NEED(w->Wsh_d); NEED(w->Wsh_d_scale);
+            if (swiglu) { NEED(w->Wsh_u); NEED(w->Wsh_u_scale); }
+        }
+    }
+    ALIGNED(x8_perm, 16); ALIGNED(xs_perm, 16); ALIGNED(x8, 16); ALIGNED(xs, 16); ALIGNED(y_perm, 16);
+    ALIGNED(offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4); ALIGNED(b2, 4);
+    ALIGNED(w->W1, 16); ALIGNED(w->Wu, 16); ALIGNED(w->W2, 16); ALIGNED(w->Wsh_g, 16); ALIGNED(w->Wsh_u, 16);
+    ALIGNED(w->Wsh_d, 16); ALIGNED(w->W1_scale, 16); ALIGNED(w->Wu_scale, 16); ALIGNED(w->W2_scale, 16);
+    ALIGNED(w->Wsh_g_scale, 16); ALIGNED(w->Wsh_u_scale, 16); ALIGNED(w->Wsh_d_scale, 16);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL%s");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    const MxLayout L = mx_layout(cfg, w->sld);
+    if (ws_bytes < L.total) return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_grouped_ffn_mx_workspace_size()%s");
+    if (cfg->T == 0) return MOE_OK;
+    moe::FfnMxArgs a{};
+    a.x_perm = x8_perm; a.xs_perm = xs_perm; a.x = x8; a.xs = xs;
+    a.offsets = offsets; a.row_gate = row_gate;
+    a.W1 = w->W1; a.W1s = w->W1_scale; a.Wu = w->Wu; a.Wus = w->Wu_scale; a.W2 = w->W2; a.W2s = w->W2_scale;
+    a.b1 = b1; a.b2 = b2;
+    a.Wsg = w->Wsh_g; a.Wsgs = w->Wsh_g_scale; a.Wsu = w->Wsh_u; a.Wsus = w->Wsh_u_scale;
+    a.Wsd = w->Wsh_d; a.Wsds = w->Wsh_d_scale;
+    a.H = at<__nv_bfloat16>(ws, L.H);
+    a.H8 = at<uint8_t>(ws, L.H8);
+    a.Hs = at<uint8_t>(ws, L.Hs);
+    a.y_perm = static_cast<__nv_bfloat16 *>(y_perm);
+    a.status = status_word(ws);
+    a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.F = cfg->d_ff; a.S = cfg->d_ff_shared; a.act = cfg->act;
+    a.routed_rows = (int64_t)cfg->T * cfg->top_k;
+    a.hF = L.hF;
+    a.shared_base = (int64_t)cfg->T * cfg->top_k;
+    a.sld = w->sld;
+    a.num_sms = num_sms();
+    cudaError_t e = moe::launch_ffn_mx(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "grouped_ffn_mx");
 }
 
 const char *moe_status_string(moe_status s) {

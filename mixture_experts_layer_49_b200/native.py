@@ -30,7 +30,8 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_status_string", "moe_last_error_detail", "moe_permute_noalloc",
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
-           "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward")
+           "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward",
+           "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -39,6 +40,14 @@ class MoeFp8Experts(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
         "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")]
+
+
+class MoeMxExperts(ctypes.Structure):
+    """moe_mx_experts: block-scaled e4m3 expert weights (device pointers),
+    their E8M0 scale bytes and the scale row stride sld."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
+        "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")] + [("sld", ctypes.c_int32)]
 
 
 class MoeWsView(ctypes.Structure):
@@ -124,6 +133,14 @@ def lib():
                                              c_vp, c_vp]
         L.moe_grouped_ffn_fp8.restype = ctypes.c_int
         L.moe_grouped_ffn_fp8.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeFp8Experts)] + [c_vp] * 6 + [
+            ctypes.c_size_t, c_vp]
+        L.moe_quantize_rows_mx.restype = ctypes.c_int
+        L.moe_quantize_rows_mx.argtypes = [c_vp, ctypes.c_int64, c_i32, ctypes.c_int64, c_vp, ctypes.c_int64,
+                                           c_vp, ctypes.c_int64, c_vp]
+        L.moe_grouped_ffn_mx_workspace_size.restype = ctypes.c_size_t
+        L.moe_grouped_ffn_mx_workspace_size.argtypes = [P(MoeConfig), c_i32]
+        L.moe_grouped_ffn_mx.restype = ctypes.c_int
+        L.moe_grouped_ffn_mx.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeMxExperts)] + [c_vp] * 6 + [
             ctypes.c_size_t, c_vp]
         L.moe_forward_fp8.restype = ctypes.c_int
         L.moe_forward_fp8.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeFp8Experts)] + [c_vp] * 12 + [
@@ -441,6 +458,50 @@ def moe_forward_fp8(cfg, x, Wr, logit_bias, sel_bias, w, b1, b2, y, idx, gate, c
                                  _p(b1), _p(b2), _p(y), _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss),
                                  _p(logits_out), _p(n_dropped), _p(ws), ws.numel(), _stream(stream)),
            "moe_forward_fp8")
+
+
+# ---------------------------------------------------------------- MX experts
+def mx_sld(cfg) -> int:
+    """Smallest valid scale row stride (bytes) for a configuration."""
+    need = max(cfg.d_model, cfg.d_ff, cfg.d_ff_shared) // 32
+    return (need + 15) // 16 * 16
+
+
+def mx_experts(w, sld) -> MoeMxExperts:
+    """moe_mx_experts from a dict of device tensors: e4m3 codes (uint8) under
+    W1, Wu, W2, Wsg, Wsu, Wsd and scale bytes (uint8, rows of sld bytes) under
+    "<name>_scale"."""
+    s = MoeMxExperts()
+    for name in FP8_WEIGHTS:
+        field = _FP8_FIELD[name]
+        setattr(s, field, _p(w.get(name)))
+        setattr(s, field + "_scale", _p(w.get(name + "_scale")))
+    s.sld = int(sld)
+    return s
+
+
+def moe_quantize_rows_mx(x, codes, scales, rows=None, cols=None, ld_in=None, ld_out=None, ld_scale=None,
+                         stream=None):
+    """MX quantization of a bf16 [rows, cols] tensor into codes (uint8) and
+    scale bytes (uint8 [rows, ld_scale])."""
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld_in = x.shape[1] if ld_in is None else ld_in
+    ld_out = codes.shape[1] if ld_out is None else ld_out
+    ld_scale = scales.shape[1] if ld_scale is None else ld_scale
+    _check(lib().moe_quantize_rows_mx(_p(x), rows, cols, ld_in, _p(codes), ld_out, _p(scales), ld_scale,
+                                      _stream(stream)), "moe_quantize_rows_mx")
+
+
+def grouped_ffn_mx_workspace_size(cfg, sld) -> int:
+    return int(lib().moe_grouped_ffn_mx_workspace_size(ctypes.byref(cfg), int(sld)))
+
+
+def moe_grouped_ffn_mx(cfg, x8_perm, xs_perm, offsets, row_gate, w, sld, b1, b2, x8, xs, y_perm, ws, stream=None):
+    ex = mx_experts(w, sld)
+    _check(lib().moe_grouped_ffn_mx(ctypes.byref(cfg), _p(x8_perm), _p(xs_perm), _p(offsets), _p(row_gate),
+                                    ctypes.byref(ex), _p(b1), _p(b2), _p(x8), _p(xs), _p(y_perm), _p(ws),
+                                    ws.numel(), _stream(stream)), "moe_grouped_ffn_mx")
 
 
 def forward_fp8(cfg, inp, w8, out: Outputs, ws, stream=None):

@@ -25,6 +25,8 @@ from __future__ import annotations
 import dataclasses
 import zlib
 
+import math
+
 import torch
 
 
@@ -183,6 +185,53 @@ def _fp8_stack(wl, name, E, rows, cols, device, seed):
                        .view(torch.uint8))
         scale[e].copy_((torch.rand((rows,), generator=g, device=device) + 0.5) * cols ** -0.5)
     return codes, scale
+
+
+def _mx_stack(wl, name, E, rows, cols, sld, device, seed):
+    """E x rows x cols e4m3 codes of N(0, 1) draws (torch's float8_e4m3fn
+    cast) and E x rows x sld scale bytes: one per 32 inputs, uniform over the
+    three powers of two around 1/sqrt(cols), bytes past cols / 32 zero."""
+    codes = torch.empty((E, rows, cols), dtype=torch.uint8, device=device)
+    scale = torch.zeros((E, rows, sld), dtype=torch.uint8, device=device)
+    base = 127 - int(math.ceil(math.log2(math.sqrt(cols))))
+    for e in range(E):
+        g = _gen(device, seed, wl, name + "_mx", e)
+        codes[e].copy_(torch.randn((rows, cols), generator=g, device=device).to(torch.float8_e4m3fn)
+                       .view(torch.uint8))
+        scale[e, :, :cols // 32].copy_(torch.randint(base - 1, base + 2, (rows, cols // 32), generator=g,
+                                                     device=device).to(torch.uint8))
+    return codes, scale
+
+
+def generate_mx_experts(wl: Workload, sld: int, device="cpu", seed: int = 0) -> dict:
+    """Block-scaled (MX) expert weights for a bf16 workload: e4m3 codes
+    (uint8, nn.Linear [out, in] layout) and E8M0 scale bytes, one per 32
+    inputs, in rows of sld bytes.  Keys W1, Wu, W2, Wsg, Wsu, Wsd and
+    "<key>_scale" (absent ones None), and for GELU experts the fp32 biases b1,
+    b2 (the same draws as generate()'s)."""
+    dev = torch.device(device)
+    d, E, F = wl.d_model, wl.E, wl.d_ff
+    w = {k: None for k in ("W1", "Wu", "W2", "Wsg", "Wsu", "Wsd")}
+    w.update({k + "_scale": None for k in list(w)})
+    w["W1"], w["W1_scale"] = _mx_stack(wl, "W1", E, F, d, sld, dev, seed)
+    w["W2"], w["W2_scale"] = _mx_stack(wl, "W2", E, d, F, sld, dev, seed)
+    if wl.act == "swiglu":
+        w["Wu"], w["Wu_scale"] = _mx_stack(wl, "Wu", E, F, d, sld, dev, seed)
+    if wl.act == "gelu":
+        g = _gen(dev, seed, wl, "b1")
+        w["b1"] = (torch.rand((E, F), generator=g, device=dev) * 0.02 - 0.01)
+        g = _gen(dev, seed, wl, "b2")
+        w["b2"] = (torch.rand((E, d), generator=g, device=dev) * 0.02 - 0.01)
+    if wl.d_ff_shared:
+        S = wl.d_ff_shared
+        c, s = _mx_stack(wl, "Wsg", 1, S, d, sld, dev, seed)
+        w["Wsg"], w["Wsg_scale"] = c[0], s[0]
+        c, s = _mx_stack(wl, "Wsd", 1, d, S, sld, dev, seed)
+        w["Wsd"], w["Wsd_scale"] = c[0], s[0]
+        if wl.act == "swiglu":
+            c, s = _mx_stack(wl, "Wsu", 1, S, d, sld, dev, seed)
+            w["Wsu"], w["Wsu_scale"] = c[0], s[0]
+    return w
 
 
 def generate_fp8_experts(wl: Workload, device="cpu", seed: int = 0) -> dict:

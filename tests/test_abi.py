@@ -178,6 +178,48 @@ def test_fp8_entry_points_check_arguments():
     assert L.moe_quantize_rows_e4m3(None, 0, 16, 16, None, 16, None, None) == nat.MOE_OK
 
 
+def test_mx_entry_points_check_arguments():
+    L = nat.lib()
+    # configuration: bf16, K dimensions multiples of 128, sld a multiple of 16 holding every K / 32
+    assert nat.grouped_ffn_mx_workspace_size(cfg(), 16) > 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(dtype="f32"), 16) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(d_model=192), 16) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(d_ff=320), 16) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(d_ff_shared=64), 16) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(d_ff=768), 16) == 0       # 768 / 32 = 24 bytes > 16
+    assert nat.grouped_ffn_mx_workspace_size(cfg(d_ff=768), 32) > 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(), 8) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(), 24) == 0
+    assert nat.grouped_ffn_mx_workspace_size(cfg(E=300), 16) == 0
+    assert nat.mx_sld(cfg(d_ff=768)) == 32 and nat.mx_sld(cfg()) == 16
+    c = cfg()
+    n = nat.grouped_ffn_mx_workspace_size(c, 16)
+
+    def raw(w, **null):
+        args = dict(x8p=fake(), xsp=fake(), off=fake(), rg=fake())
+        rest = dict(b1=None, b2=None, x8=None, xs=None, y=fake())
+        for k in null:
+            (args if k in args else rest)[k] = None
+        return L.moe_grouped_ffn_mx(ctypes.byref(c), *args.values(), ctypes.byref(w) if w is not None else None,
+                                    *rest.values(), fake(16), n, None)
+
+    full = dict(W1=4096, W1_scale=4096, Wu=4096, Wu_scale=4096, W2=4096, W2_scale=4096, sld=16)
+    assert raw(None) == nat.MOE_ERR_INVALID_ARG
+    assert raw(nat.MoeMxExperts(**dict(full, Wu_scale=None))) == nat.MOE_ERR_INVALID_ARG    # SwiGLU W_up scales
+    assert "Wu_scale" in nat.last_error_detail()
+    assert raw(nat.MoeMxExperts(**full), xsp=None) == nat.MOE_ERR_INVALID_ARG
+    assert raw(nat.MoeMxExperts(**dict(full, W2_scale=4096 + 8))) == nat.MOE_ERR_INVALID_ARG  # misaligned
+    assert raw(nat.MoeMxExperts(**dict(full, sld=8))) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_grouped_ffn_mx(ctypes.byref(c), fake(), fake(), fake(), fake(), ctypes.byref(nat.MoeMxExperts(**full)),
+                                None, None, None, None, fake(), fake(16), n - 256, None) == nat.MOE_ERR_WORKSPACE
+    # the MX row quantizer
+    assert L.moe_quantize_rows_mx(fake(), 4, 48, 48, fake(), 48, fake(), 2, None) == nat.MOE_ERR_UNSUPPORTED
+    assert L.moe_quantize_rows_mx(fake(), 4, 64, 64, fake(), 64, fake(), 1, None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_mx(fake(), 4, 64, 60, fake(), 64, fake(), 2, None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_mx(None, 4, 64, 64, fake(), 64, fake(), 2, None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_mx(None, 0, 64, 64, None, 64, None, 2, None) == nat.MOE_OK
+
+
 def test_workspace_view_addresses():
     # a host-only call: addresses inside the workspace, in increasing order,
     # aligned for their element type, every region inside ws_bytes
