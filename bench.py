@@ -496,7 +496,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: e4m3 experts through moe_forward_fp8 (bf16 layers only; no CPU baseline)")
-    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8,qwen3_moe:backward",
+    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8,qwen3_moe:mx,qwen3_moe:backward",
                     help="further workloads (name or name:fp8) timed after the headline one and reported "
                          "under sub_records; '' for none")
     ap.add_argument("--sub-steps", type=int, default=20)
@@ -640,15 +640,95 @@ def backward_record(args, wl, dev, world):
             "clocks": clocks}
 
 
+def mx_record(args, wl, dev, world):
+    """The grouped FFN with block-scaled (MX) e4m3 experts (moe_grouped_ffn_mx:
+    GEMM 1, the MX quantization of H, GEMM 2) on the workload's routed rows:
+    routing, permutation and the MX codes and scale rows of the packed rows
+    are produced once before the timed region; K timed steps, L2 flushed
+    between them.  Roofline: the expert FLOPs of the kept rows against the
+    e4m3 tensor peak (2 x the measured bf16 figure)."""
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inp = syn.generate(wl, dev, seed=0, weights=False)
+    cfg = nat.config_from_workload(wl)
+    T, k, E, d = wl.T, wl.top_k, wl.E, wl.d_model
+    sld = nat.mx_sld(cfg)
+    w = syn.generate_mx_experts(wl, sld, dev, seed=0)
+    ws = nat.alloc_workspace(cfg, dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    psum = torch.empty((nat.router_blocks(cfg), E), dtype=torch.float32, device=dev)
+    nat.moe_router_topk(cfg, inp["x"], inp["Wr"], inp["logit_bias"], inp["sel_bias"], idx, gate, None, psum, ws)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    row_token = torch.zeros(T * k, dtype=torch.int32, device=dev)
+    row_gate = torch.zeros(T * k, dtype=torch.float32, device=dev)
+    nat.moe_permute(cfg, inp["x"], idx, gate, counts, kept, offsets, row_of, row_token, row_gate, None, None, ws)
+    x8 = torch.empty((T, d), dtype=torch.uint8, device=dev)
+    xs = torch.zeros((T, sld), dtype=torch.uint8, device=dev)
+    nat.moe_quantize_rows_mx(inp["x"], x8, xs)
+    torch.cuda.synchronize(dev)
+    n = int(offsets[-1].item())
+    rt = row_token[:n].long()
+    x8p = torch.zeros((T * k, d), dtype=torch.uint8, device=dev)
+    x8p[:n] = x8[rt]
+    xsp = torch.zeros((T * k, sld), dtype=torch.uint8, device=dev)
+    xsp[:n] = xs[rt]
+    y_perm = torch.empty((nat.perm_rows(cfg), d), dtype=torch.bfloat16, device=dev)
+    mws = torch.zeros(nat.grouped_ffn_mx_workspace_size(cfg, sld), dtype=torch.uint8, device=dev)
+
+    def step():
+        nat.moe_grouped_ffn_mx(cfg, x8p, xsp, offsets, row_gate, w, sld, w.get("b1"), w.get("b2"), x8, xs, y_perm,
+                               mws, stream)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(mws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the MX warm-up")
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.sub_steps)]
+    for i in range(args.sub_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.sub_steps
+    ms = max_over_ranks([ms], world, dev)[0]
+    flops = float(wl.expert_flops(n))
+    peaks, peak_src = load_peaks()
+    peak_t, which = tensor_peak(peaks, clocks)
+    peak_t *= 2.0
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": wl.name, "experts": "mx_e4m3 (32-value E8M0 blocks, tcgen05 block-scaled MMA)",
+            "pass": "grouped FFN stage (GEMM 1, H quantization, GEMM 2) on the packed rows",
+            "steps": args.sub_steps, "warmup": 3, "ms_per_step": ms, "tflops": tf,
+            "gpu_launches": (4 if wl.d_ff_shared else 3) * args.sub_steps,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_t, "unit": "TFLOP/s", "frac": tf / peak_t,
+                         "flops": flops, "peak_note": "e4m3: 2 x the %s bf16 peak (the nominal fp8 : bf16 ratio), %s"
+                         % (which, "of measured" if peak_src == "measured" else "of fallback")},
+            "clocks": clocks}
+
+
 def sub_record(args, spec, dev, world, rank):
     """One further workload timed like the headline one (device-resident steps
     with the L2 flushed between them, the staged per-stage pass), reported
-    with its own roofline fractions.  spec: "workload", "workload:fp8", or
-    "workload:backward" (the backward pass, backward_record)."""
+    with its own roofline fractions.  spec: "workload", "workload:fp8",
+    "workload:backward" (the backward pass, backward_record) or "workload:mx"
+    (the MX grouped FFN stage, mx_record)."""
     name, _, experts = spec.partition(":")
     wl = syn.WORKLOADS[name]
     if experts == "backward":
         return backward_record(args, wl, dev, world)
+    if experts == "mx":
+        return mx_record(args, wl, dev, world)
     fp8 = experts == "fp8"
     r = run_ours(args, wl, dev, world, rank, fp8=fp8, steps=args.sub_steps, warmup=3, full=False)
     rec = {"workload": name, "experts": "fp8" if fp8 else "bf16", "steps": args.sub_steps, "warmup": 3,

@@ -59,7 +59,7 @@ class Workload:
         mats = 3 if self.act == "swiglu" else 2
         f = 2.0 * kept_rows * self.d_model * self.d_ff * mats
         if self.d_ff_shared:
-            f += 2.0 * self.T * self.d_model * self.d_ff_shared * 3
+            f += 2.0 * self.T * self.d_model * self.d_ff_shared * mats
         return f
 
 
