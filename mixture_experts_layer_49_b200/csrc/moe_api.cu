@@ -3,6 +3,8 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 #include <stdio.h>
 #include <string.h>
 
@@ -154,6 +156,40 @@ MxLayout mx_layout(const moe_config *c, int32_t sld) {
     return L;
 }
 
+// Frozen routers (moe_router_freeze): the workspace whose router scratch
+// holds the split of a given W_r (pointer, d_model, E).  Router launches on
+// that workspace with the same W_r skip the split; a launch with other
+// weights re-splits and drops the entry; moe_workspace_init drops it too.
+struct FrozenRouter {
+    const void *ws;
+    const float *Wr;
+    int d, E;
+};
+std::mutex g_frozen_mu;
+std::vector<FrozenRouter> g_frozen;
+
+bool router_split_ready(const void *ws, const float *Wr, int d, int E) {
+    std::lock_guard<std::mutex> lock(g_frozen_mu);
+    for (size_t i = 0; i < g_frozen.size(); ++i) {
+        if (g_frozen[i].ws != ws) continue;
+        if (g_frozen[i].Wr == Wr && g_frozen[i].d == d && g_frozen[i].E == E) return true;
+        g_frozen.erase(g_frozen.begin() + (long)i);     // this launch overwrites the split
+        return false;
+    }
+    return false;
+}
+void set_frozen(const void *ws, const float *Wr, int d, int E) {
+    std::lock_guard<std::mutex> lock(g_frozen_mu);
+    for (auto &f : g_frozen)
+        if (f.ws == ws) { f.Wr = Wr; f.d = d; f.E = E; return; }
+    g_frozen.push_back(FrozenRouter{ws, Wr, d, E});
+}
+void forget_frozen(const void *ws) {
+    std::lock_guard<std::mutex> lock(g_frozen_mu);
+    for (size_t i = 0; i < g_frozen.size(); ++i)
+        if (g_frozen[i].ws == ws) { g_frozen.erase(g_frozen.begin() + (long)i); return; }
+}
+
 moe_status check_fp8_weights(const moe_config *c, const moe_fp8_experts *w) {
     NEED(w);
     NEED(w->W1); NEED(w->W1_scale); NEED(w->W2); NEED(w->W2_scale);
@@ -291,8 +327,27 @@ const char *moe_last_error_detail(void) { return g_detail; }
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
     if (!ws || ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace missing or < 256 bytes%s");
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
+    forget_frozen(ws);
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(moe::WsHeader), reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
+}
+
+moe_status moe_router_freeze(const moe_config *cfg, const float *Wr, void *ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(Wr);
+    ALIGNED(Wr, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    if (cfg->dtype != MOE_BF16) return MOE_OK;      // fp32 layers keep every product in fp32: nothing to split
+    moe::RouterArgs a{};
+    a.Wr = Wr; a.d = cfg->d_model; a.E = cfg->E;
+    a.wsplit = at<char>(ws, layout(cfg).router_w);
+    a.pdl = false;
+    cudaError_t e = moe::launch_router_split(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "router_freeze");
+    set_frozen(ws, Wr, cfg->d_model, cfg->E);
+    return MOE_OK;
 }
 
 moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
@@ -308,6 +363,7 @@ moe_status moe_router_topk(const moe_config *cfg, const void *x, const float *Wr
                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
                       at<char>(ws, layout(cfg).router_w), at<float>(ws, layout(cfg).logits), status_word(ws),
                       num_sms()};
+    a.split_ready = cfg->dtype == MOE_BF16 && router_split_ready(ws, Wr, cfg->d_model, cfg->E);
     cudaError_t e = moe::launch_router(a, cfg->dtype == MOE_BF16, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router");
 }
@@ -412,6 +468,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                        cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
                        at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
+    ra.split_ready = bf16 && router_split_ready(ws, Wr, cfg->d_model, cfg->E);
     if ((e = moe::launch_router(ra, bf16, st)) != cudaSuccess) return cuda_fail(e, "router");
 
     moe::DispatchArgs da{};
@@ -629,6 +686,7 @@ moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr
     moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
                        cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
                        at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
+    ra.split_ready = router_split_ready(ws, Wr, cfg->d_model, cfg->E);
     if ((e = moe::launch_router(ra, true, st)) != cudaSuccess) return cuda_fail(e, "router");
 
     moe::QuantArgs q{};                           // x -> e4m3 codes + row scales

@@ -329,13 +329,17 @@ int router_logit_splits(int T, int d, int num_sms) {
 size_t router_split_bytes(int d, int E) { return (size_t)3 * E * d * 2; }
 
 // Logits h = x W_r (+ logit offset) into `out`: [splits][T][E] partial sums.
+cudaError_t launch_router_split(const RouterArgs &a, cudaStream_t st) {
+    dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
+    return launch_kernel(split_router_weights, sg, dim3(256), 0, st, a.pdl, a.Wr, a.d, a.E,
+                         static_cast<__nv_bfloat16 *>(a.wsplit));
+}
+
 cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits, cudaStream_t st) {
     void *wsplit = a.wsplit;
     if (a.T == 0) return cudaSuccess;
-    dim3 sg((a.d + 31) / 32, (a.E + 31) / 32);
-    cudaError_t e = launch_kernel(split_router_weights, sg, dim3(256), 0, st, a.pdl, a.Wr, a.d, a.E,
-                                  static_cast<__nv_bfloat16 *>(wsplit));
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!a.split_ready && (e = launch_router_split(a, st)) != cudaSuccess) return e;
 
     TcRouterParams p{};
     p.logit_bias = a.logit_bias; p.out = out; p.status = a.status;
@@ -387,7 +391,8 @@ cudaError_t launch_router_logits_tc(const RouterArgs &a, float *out, int splits,
         attr = true;
     }
     const int grid = 2 * pair_blocks(a.T) * splits;
-    return launch_kernel(router_tc_kernel, dim3(grid), dim3(kThreads), smem, st, true, mx, mw, p);
+    return launch_kernel(router_tc_kernel, dim3(grid), dim3(kThreads), smem, st, a.split_ready ? a.pdl : true, mx, mw,
+                         p);
 }
 
 }  // namespace moe

@@ -31,7 +31,8 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
            "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward",
-           "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx")
+           "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx",
+           "moe_router_freeze")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -134,6 +135,8 @@ def lib():
         L.moe_grouped_ffn_fp8.restype = ctypes.c_int
         L.moe_grouped_ffn_fp8.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeFp8Experts)] + [c_vp] * 6 + [
             ctypes.c_size_t, c_vp]
+        L.moe_router_freeze.restype = ctypes.c_int
+        L.moe_router_freeze.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_size_t, c_vp]
         L.moe_quantize_rows_mx.restype = ctypes.c_int
         L.moe_quantize_rows_mx.argtypes = [c_vp, ctypes.c_int64, c_i32, ctypes.c_int64, c_vp, ctypes.c_int64,
                                            c_vp, ctypes.c_int64, c_vp]
@@ -458,6 +461,13 @@ def moe_forward_fp8(cfg, x, Wr, logit_bias, sel_bias, w, b1, b2, y, idx, gate, c
                                  _p(b1), _p(b2), _p(y), _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss),
                                  _p(logits_out), _p(n_dropped), _p(ws), ws.numel(), _stream(stream)),
            "moe_forward_fp8")
+
+
+def moe_router_freeze(cfg, Wr, ws, stream=None):
+    """Split W_r into the workspace once; later router calls on ws with the
+    same W_r pointer skip the split (see include/moe.h)."""
+    _check(lib().moe_router_freeze(ctypes.byref(cfg), _p(Wr), _p(ws), ws.numel(), _stream(stream)),
+           "moe_router_freeze")
 
 
 # ---------------------------------------------------------------- MX experts

@@ -220,6 +220,17 @@ def test_mx_entry_points_check_arguments():
     assert L.moe_quantize_rows_mx(None, 0, 64, 64, None, 64, None, 2, None) == nat.MOE_OK
 
 
+def test_router_freeze_checks_arguments():
+    L = nat.lib()
+    c = cfg()
+    n = nat.workspace_size(c)
+    assert L.moe_router_freeze(ctypes.byref(c), None, fake(16), n, None) == nat.MOE_ERR_INVALID_ARG
+    assert L.moe_router_freeze(ctypes.byref(c), fake(), None, n, None) == nat.MOE_ERR_WORKSPACE
+    assert L.moe_router_freeze(ctypes.byref(c), fake(), fake(16), n - 1, None) == nat.MOE_ERR_WORKSPACE
+    c32 = cfg(dtype="f32")                                   # nothing to split for fp32 layers
+    assert L.moe_router_freeze(ctypes.byref(c32), fake(), fake(16), nat.workspace_size(c32), None) == nat.MOE_OK
+
+
 def test_workspace_view_addresses():
     # a host-only call: addresses inside the workspace, in increasing order,
     # aligned for their element type, every region inside ws_bytes

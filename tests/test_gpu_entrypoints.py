@@ -203,3 +203,45 @@ def test_combine_flags_bad_row(cuda_device):
     st.row_of[3, 0] = 10_000
     st.combine()
     assert st.status() == nat.MOE_ERR_DEVICE_BOUNDS
+
+
+def test_frozen_router_matches_the_per_call_split(cuda_device):
+    """moe_router_freeze: a forward pass on a frozen workspace gives the same
+    bits as one that splits W_r itself; new router weights (another tensor,
+    or new values refrozen in place) are picked up; moe_workspace_init drops
+    the freeze."""
+    wl = W("frozen_router", T=300, d_model=256, E=16, d_ff=128, top_k=2, logit_skew="normal")
+    dev = cuda_device
+    inp = syn.generate(wl, dev, seed=5)
+    cfg = nat.config_from_workload(wl)
+
+    def run(ws, Wr):
+        out = nat.Outputs(cfg, dev, want_logits=True)
+        nat.forward(cfg, dict(inp, Wr=Wr), out, ws)
+        torch.cuda.synchronize(dev)
+        return out
+
+    def same(a, b):
+        return (torch.equal(a.y, b.y) and torch.equal(a.idx, b.idx) and torch.equal(a.gate, b.gate)
+                and torch.equal(a.logits, b.logits))
+
+    Wr = inp["Wr"]
+    ref = run(nat.alloc_workspace(cfg, dev), Wr)
+    ws = nat.alloc_workspace(cfg, dev)
+    nat.moe_router_freeze(cfg, Wr, ws)
+    assert same(run(ws, Wr), ref)
+    assert same(run(ws, Wr), ref)                              # still frozen on the next call
+    # other router weights: re-split, and the freeze is dropped
+    Wr2 = Wr * 1.5
+    ref2 = run(nat.alloc_workspace(cfg, dev), Wr2)
+    assert same(run(ws, Wr2), ref2)
+    assert same(run(ws, Wr), ref)                              # back to W_r: split again
+    # new values in place need a new freeze
+    nat.moe_router_freeze(cfg, Wr, ws)
+    Wr.mul_(0.5)
+    nat.moe_router_freeze(cfg, Wr, ws)
+    ref3 = run(nat.alloc_workspace(cfg, dev), Wr)
+    assert same(run(ws, Wr), ref3)
+    nat.moe_workspace_init(ws)
+    assert same(run(ws, Wr), ref3)
+    assert nat.moe_get_device_status(ws) == nat.MOE_OK
