@@ -712,9 +712,30 @@ def mx_record(args, wl, dev, world):
     peak_t, which = tensor_peak(peaks, clocks)
     peak_t *= 2.0
     tf = flops / (ms * 1e-3) / 1e12
+
+    # the whole layer with MX experts (moe_forward_mx), timed the same way
+    out = nat.Outputs(cfg, dev)
+    nat.moe_router_freeze(cfg, inp["Wr"], ws, stream)
+    for _ in range(3):
+        flush.zero_()
+        nat.forward_mx(cfg, inp, w, sld, out, ws, mws, stream)
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(ws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the MX layer warm-up")
+    for i in range(args.sub_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        nat.forward_mx(cfg, inp, w, sld, out, ws, mws, stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    layer_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in ev) / args.sub_steps], world, dev)[0]
     return {"workload": wl.name, "experts": "mx_e4m3 (32-value E8M0 blocks, tcgen05 block-scaled MMA)",
             "pass": "grouped FFN stage (GEMM 1, H quantization, GEMM 2) on the packed rows",
             "steps": args.sub_steps, "warmup": 3, "ms_per_step": ms, "tflops": tf,
+            "layer": {"entry": "moe_forward_mx (router, x quantization, permute, scale-row gather, grouped FFN, "
+                               "combine)", "ms_per_step": layer_ms,
+                      "tokens_per_s": job_tokens_per_s(world, wl.T, layer_ms),
+                      "tflops": flops / (layer_ms * 1e-3) / 1e12},
             "gpu_launches": (4 if wl.d_ff_shared else 3) * args.sub_steps,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_t, "unit": "TFLOP/s", "frac": tf / peak_t,
                          "flops": flops, "peak_note": "e4m3: 2 x the %s bf16 peak (the nominal fp8 : bf16 ratio), %s"

@@ -417,7 +417,8 @@ MOE_API moe_status moe_quantize_rows_mx(const void *in, int64_t rows, int32_t co
                                         uint8_t *codes, int64_t ld_out, uint8_t *scales, int64_t ld_scale,
                                         moe_stream_t stream);
 
-/* moe_grouped_ffn with MX experts: x8_perm [T*top_k, d_model] codes of the
+/* moe_grouped_ffn with MX experts (moe_forward_mx below runs the whole layer):
+ * x8_perm [T*top_k, d_model] codes of the
  * packed rows with their scales xs_perm [T*top_k, sld]; x8 / xs the codes and
  * scales of x [T, d_model] (the shared expert's input; NULL without one); b1,
  * b2 fp32 as in moe_grouped_ffn.  Output y_perm [moe_perm_rows(cfg), d_model]
@@ -427,6 +428,19 @@ MOE_API moe_status moe_quantize_rows_mx(const void *in, int64_t rows, int32_t co
  * moe_grouped_ffn_mx_workspace_size(cfg, sld) bytes, 256-byte aligned (0 on
  * a bad or unsupported configuration).                                      */
 MOE_API size_t moe_grouped_ffn_mx_workspace_size(const moe_config *cfg, int32_t sld);
+/* moe_forward with MX experts: router on the bf16 x, x quantized to MX codes
+ * per token (the codes permuted with the rows, the scale rows gathered after
+ * them), the MX grouped FFN, combine, statistics.  Arguments and outputs as
+ * in moe_forward, the expert weights in *w; ws is the layer's workspace
+ * (moe_workspace_size) and mx_ws a second one of
+ * moe_grouped_ffn_mx_workspace_size(cfg, w->sld) bytes, 256-byte aligned,
+ * for x's and H's codes and scale rows.  Device status goes to ws.          */
+MOE_API moe_status moe_forward_mx(const moe_config *cfg, const void *x, const float *Wr,
+                                  const float *logit_bias, const float *sel_bias, const moe_mx_experts *w,
+                                  const float *b1, const float *b2, void *y, int32_t *idx, float *gate,
+                                  int32_t *counts, float *f, float *P, double *loss, float *logits_out,
+                                  int32_t *n_dropped, void *ws, size_t ws_bytes, void *mx_ws, size_t mx_ws_bytes,
+                                  moe_stream_t stream);
 MOE_API moe_status moe_grouped_ffn_mx(const moe_config *cfg, const uint8_t *x8_perm, const uint8_t *xs_perm,
                                       const int32_t *offsets, const float *row_gate, const moe_mx_experts *w,
                                       const float *b1, const float *b2, const uint8_t *x8, const uint8_t *xs,

@@ -151,6 +151,10 @@ struct QuantMxArgs {
     bool pdl;
 };
 cudaError_t launch_quant_mx(const QuantMxArgs &a, cudaStream_t st);
+// dst[r] = src[row_token[r]] for r < min(*count, max_rows), rows of ld bytes
+// (ld % 16 == 0): the MX scale rows of the packed rows.  mx_sm100.cu.
+cudaError_t launch_mx_gather_rows(const uint8_t *src, uint8_t *dst, int64_t ld, const int32_t *row_token,
+                                  const int32_t *count, int64_t max_rows, int num_sms, cudaStream_t st);
 
 // The grouped FFN with MX experts (mx_sm100.cu).  Every scale array has rows
 // of sld bytes (sld % 16 == 0, at least its K / 32); K dimensions (d, F, S)

@@ -140,18 +140,24 @@ moe_status check_mx_cfg(const moe_config *c, int32_t sld) {
     return MOE_OK;
 }
 
+// MX workspace: H in bf16, its codes and scale rows (the grouped FFN), then
+// x's codes and scale rows and the packed rows' scale rows (moe_forward_mx).
 struct MxLayout {
-    size_t H, H8, Hs, total;
+    size_t H, H8, Hs, x8, xs, xs_perm, total;
     int hF;
 };
 MxLayout mx_layout(const moe_config *c, int32_t sld) {
     MxLayout L{};
-    const size_t rows = (size_t)c->T * c->top_k + (c->d_ff_shared > 0 ? (size_t)c->T : 0);
+    const size_t Tk = (size_t)c->T * c->top_k;
+    const size_t rows = Tk + (c->d_ff_shared > 0 ? (size_t)c->T : 0);
     L.hF = std::max(c->d_ff, c->d_ff_shared);
     size_t o = sizeof(moe::WsHeader);
-    L.H = o;   o = align256(o + rows * L.hF * 2);
-    L.H8 = o;  o = align256(o + rows * L.hF);
-    L.Hs = o;  o = align256(o + rows * (size_t)sld);
+    L.H = o;        o = align256(o + rows * L.hF * 2);
+    L.H8 = o;       o = align256(o + rows * L.hF);
+    L.Hs = o;       o = align256(o + rows * (size_t)sld);
+    L.x8 = o;       o = align256(o + (size_t)c->T * c->d_model);
+    L.xs = o;       o = align256(o + (size_t)c->T * (size_t)sld);
+    L.xs_perm = o;  o = align256(o + Tk * (size_t)sld);
     L.total = o;
     return L;
 }
@@ -812,6 +818,119 @@ moe_status moe_grouped_ffn_mx(const moe_config *cfg, const uint8_t *x8_perm, con
     a.num_sms = num_sms();
     cudaError_t e = moe::launch_ffn_mx(a, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "grouped_ffn_mx");
+}
+
+moe_status moe_forward_mx(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                          const float *sel_bias, const moe_mx_experts *w, const float *b1, const float *b2, void *y,
+                          int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                          float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, void *mx_ws,
+                          size_t mx_ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(w);
+    if ((s = check_mx_cfg(cfg, w->sld)) != MOE_OK) return s;
+    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+    const bool shared = cfg->d_ff_shared > 0;
+    if (cfg->T > 0) {
+        NEED(x); NEED(Wr); NEED(y); NEED(idx); NEED(gate);
+        NEED(w->W1); NEED(w->W1_scale); NEED(w->W2); NEED(w->W2_scale);
+        if (swiglu) { NEED(w->Wu); NEED(w->Wu_scale); }
+        if (shared) {
+            NEED(w->Wsh_g); NEED(w->Wsh_g_scale); NEED(w->Wsh_d); NEED(w->Wsh_d_scale);
+            if (swiglu) { NEED(w->Wsh_u); NEED(w->Wsh_u_scale); }
+        }
+    }
+    ALIGNED(x, 16); ALIGNED(y, 16); ALIGNED(Wr, 4); ALIGNED(logit_bias, 4); ALIGNED(sel_bias, 4);
+    ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
+    ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
+    ALIGNED(w->W1, 16); ALIGNED(w->Wu, 16); ALIGNED(w->W2, 16); ALIGNED(w->Wsh_g, 16); ALIGNED(w->Wsh_u, 16);
+    ALIGNED(w->Wsh_d, 16); ALIGNED(w->W1_scale, 16); ALIGNED(w->Wu_scale, 16); ALIGNED(w->W2_scale, 16);
+    ALIGNED(w->Wsh_g_scale, 16); ALIGNED(w->Wsh_u_scale, 16); ALIGNED(w->Wsh_d_scale, 16);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    if (!mx_ws) return fail(MOE_ERR_WORKSPACE, "MX workspace is NULL%s");
+    if (reinterpret_cast<uintptr_t>(mx_ws) & 255u) return fail(MOE_ERR_WORKSPACE, "MX workspace not 256-byte aligned%s");
+    const MxLayout M = mx_layout(cfg, w->sld);
+    if (mx_ws_bytes < M.total) return fail(MOE_ERR_WORKSPACE, "MX workspace smaller than moe_grouped_ffn_mx_workspace_size()%s");
+    const Layout L = layout(cfg);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *psum = at<float>(ws, L.psum);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *row_of = at<int32_t>(ws, L.row_of);
+    int32_t *row_token = at<int32_t>(ws, L.row_token);
+    float *row_gate = at<float>(ws, L.row_gate);
+    void *y_perm = at<char>(ws, L.y_perm);
+    uint8_t *x8 = at<uint8_t>(mx_ws, M.x8);
+    uint8_t *xs = at<uint8_t>(mx_ws, M.xs);
+    uint8_t *xs_perm = at<uint8_t>(mx_ws, M.xs_perm);
+    cudaError_t e;
+
+    moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
+                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
+                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
+    ra.split_ready = router_split_ready(ws, Wr, cfg->d_model, cfg->E);
+    if ((e = moe::launch_router(ra, true, st)) != cudaSuccess) return cuda_fail(e, "router");
+
+    moe::QuantMxArgs q{};                         // x -> MX codes + scale rows
+    q.in = static_cast<const __nv_bfloat16 *>(x);
+    q.ld_in = cfg->d_model;
+    q.out = x8;
+    q.ld_out = cfg->d_model;
+    q.scale = xs;
+    q.ld_scale = w->sld;
+    q.rows = cfg->T;
+    q.cols = cfg->d_model;
+    q.num_sms = num_sms();
+    q.pdl = true;
+    if ((e = moe::launch_quant_mx(q, st)) != cudaSuccess) return cuda_fail(e, "quantize_x_mx");
+
+    moe::DispatchArgs da{};
+    da.x = x8; da.idx = idx; da.gate = gate;
+    da.chunk_cnt = at<int32_t>(ws, L.chunk_cnt);
+    da.chunk_base = at<int32_t>(ws, L.chunk_base);
+    da.counts = counts; da.kept = at<int32_t>(ws, L.kept); da.offsets = offsets;
+    da.row_of = row_of; da.row_token = row_token; da.row_gate = row_gate;
+    da.x_perm = at<char>(ws, L.x_perm);
+    da.n_dropped = n_dropped;
+    da.status = status_word(ws);
+    da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
+    da.capacity = moe_capacity(cfg);
+    da.psum = psum; da.f = f; da.P = P; da.loss = loss;
+    da.contrib = at<double>(ws, L.contrib);
+    da.nblk = moe::router_blocks(cfg->T, true);
+    da.pdl = true;
+    if ((e = moe::launch_dispatch(da, 1, st)) != cudaSuccess) return cuda_fail(e, "permute");
+    if (cfg->T > 0 &&
+        (e = moe::launch_mx_gather_rows(xs, xs_perm, w->sld, row_token, offsets + cfg->E,
+                                        (int64_t)cfg->T * cfg->top_k, num_sms(), st)) != cudaSuccess)
+        return cuda_fail(e, "gather_scales_mx");
+
+    if (cfg->T > 0) {
+        moe::FfnMxArgs a{};
+        a.x_perm = at<uint8_t>(ws, L.x_perm); a.xs_perm = xs_perm; a.x = x8; a.xs = xs;
+        a.offsets = offsets; a.row_gate = row_gate;
+        a.W1 = w->W1; a.W1s = w->W1_scale; a.Wu = w->Wu; a.Wus = w->Wu_scale; a.W2 = w->W2; a.W2s = w->W2_scale;
+        a.b1 = b1; a.b2 = b2;
+        a.Wsg = w->Wsh_g; a.Wsgs = w->Wsh_g_scale; a.Wsu = w->Wsh_u; a.Wsus = w->Wsh_u_scale;
+        a.Wsd = w->Wsh_d; a.Wsds = w->Wsh_d_scale;
+        a.H = at<__nv_bfloat16>(mx_ws, M.H);
+        a.H8 = at<uint8_t>(mx_ws, M.H8);
+        a.Hs = at<uint8_t>(mx_ws, M.Hs);
+        a.y_perm = static_cast<__nv_bfloat16 *>(y_perm);
+        a.status = status_word(ws);
+        a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.F = cfg->d_ff; a.S = cfg->d_ff_shared; a.act = cfg->act;
+        a.routed_rows = (int64_t)cfg->T * cfg->top_k;
+        a.hF = M.hF;
+        a.shared_base = (int64_t)cfg->T * cfg->top_k;
+        a.sld = w->sld;
+        a.num_sms = num_sms();
+        if ((e = moe::launch_ffn_mx(a, st)) != cudaSuccess) return cuda_fail(e, "grouped_ffn_mx");
+    }
+
+    moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
+                        shared ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
+    if ((e = moe::launch_combine(ca, true, st)) != cudaSuccess) return cuda_fail(e, "combine");
+    return MOE_OK;
 }
 
 const char *moe_status_string(moe_status s) {

@@ -101,6 +101,24 @@ __global__ void __launch_bounds__(kMxQuantThreads) mx_quant_kernel(QuantMxArgs a
     }
 }
 
+// dst[r, :] = src[row_token[r], :] for r < *count: the scale rows of the
+// packed rows (bytes per row a multiple of 16).  One warp per row.
+__global__ void __launch_bounds__(256) mx_gather_rows_kernel(const uint8_t *src, uint8_t *dst, int64_t ld,
+                                                             const int32_t *row_token, const int32_t *count,
+                                                             int64_t max_rows) {
+    pdl_wait_then_release();
+    const int lane = threadIdx.x & 31;
+    int64_t n = *count;
+    n = n < 0 ? 0 : (n < max_rows ? n : max_rows);
+    const int nvec = (int)(ld / 16);
+    const int64_t nw = (int64_t)gridDim.x * 8;
+    for (int64_t r = blockIdx.x * 8 + (threadIdx.x >> 5); r < n; r += nw) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(src + (int64_t)row_token[r] * ld);
+        uint4 *d = reinterpret_cast<uint4 *>(dst + r * ld);
+        for (int v = lane; v < nvec; v += 32) d[v] = __ldg(s + v);
+    }
+}
+
 // ------------------------------------------------------------------ grouped GEMM
 constexpr int MX_BM = 128, MX_BN = 128, MX_BK = 128;   // K per stage: one 128-byte row of e4m3 codes
 constexpr int MX_STAGES = 5;
@@ -522,6 +540,17 @@ cudaError_t launch_mx_gemm(const MxMaps &m, const MxParams &p, int num_sms, cuda
 }
 
 }  // namespace
+
+cudaError_t launch_mx_gather_rows(const uint8_t *src, uint8_t *dst, int64_t ld, const int32_t *row_token,
+                                  const int32_t *count, int64_t max_rows, int num_sms, cudaStream_t st) {
+    if (max_rows <= 0) return cudaSuccess;
+    if (ld % 16) return cudaErrorInvalidValue;
+    const int sms = num_sms > 0 ? num_sms : 148;
+    const int64_t want = (max_rows + 7) / 8;
+    const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+    return launch_kernel(mx_gather_rows_kernel, dim3(grid), dim3(256), 0, st, true, src, dst, ld, row_token, count,
+                         max_rows);
+}
 
 cudaError_t launch_quant_mx(const QuantMxArgs &a, cudaStream_t st) {
     if (a.rows <= 0 || a.cols <= 0) return cudaSuccess;

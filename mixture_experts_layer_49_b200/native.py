@@ -32,7 +32,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
            "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward",
            "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx",
-           "moe_router_freeze")
+           "moe_router_freeze", "moe_forward_mx")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -137,6 +137,9 @@ def lib():
             ctypes.c_size_t, c_vp]
         L.moe_router_freeze.restype = ctypes.c_int
         L.moe_router_freeze.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_size_t, c_vp]
+        L.moe_forward_mx.restype = ctypes.c_int
+        L.moe_forward_mx.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeMxExperts)] + [c_vp] * 12 + [
+            ctypes.c_size_t, c_vp, ctypes.c_size_t, c_vp]
         L.moe_quantize_rows_mx.restype = ctypes.c_int
         L.moe_quantize_rows_mx.argtypes = [c_vp, ctypes.c_int64, c_i32, ctypes.c_int64, c_vp, ctypes.c_int64,
                                            c_vp, ctypes.c_int64, c_vp]
@@ -512,6 +515,30 @@ def moe_grouped_ffn_mx(cfg, x8_perm, xs_perm, offsets, row_gate, w, sld, b1, b2,
     _check(lib().moe_grouped_ffn_mx(ctypes.byref(cfg), _p(x8_perm), _p(xs_perm), _p(offsets), _p(row_gate),
                                     ctypes.byref(ex), _p(b1), _p(b2), _p(x8), _p(xs), _p(y_perm), _p(ws),
                                     ws.numel(), _stream(stream)), "moe_grouped_ffn_mx")
+
+
+def moe_forward_mx(cfg, x, Wr, logit_bias, sel_bias, w, sld, b1, b2, y, idx, gate, counts, f, P, loss, logits_out,
+                   n_dropped, ws, mx_ws, stream=None):
+    ex = mx_experts(w, sld)
+    _check(lib().moe_forward_mx(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias), ctypes.byref(ex),
+                                _p(b1), _p(b2), _p(y), _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss),
+                                _p(logits_out), _p(n_dropped), _p(ws), ws.numel(), _p(mx_ws), mx_ws.numel(),
+                                _stream(stream)), "moe_forward_mx")
+
+
+def alloc_mx_workspace(cfg, sld, device="cuda") -> torch.Tensor:
+    """A zeroed MX workspace (moe_grouped_ffn_mx_workspace_size bytes)."""
+    n = grouped_ffn_mx_workspace_size(cfg, sld)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_mx_workspace_size", last_error_detail())
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def forward_mx(cfg, inp, wmx, sld, out: Outputs, ws, mx_ws, stream=None):
+    """moe_forward_mx on a dict of device inputs and a dict of MX experts."""
+    moe_forward_mx(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"), wmx, sld,
+                   wmx.get("b1"), wmx.get("b2"), out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss,
+                   out.logits, out.n_dropped, ws, mx_ws, stream)
 
 
 def forward_fp8(cfg, inp, w8, out: Outputs, ws, stream=None):
