@@ -16,7 +16,10 @@ FP8 experts (``e4m3_value``, ``e4m3_round``, ``quantize_rows``,
 weight scales and per-row activation scales, defined in ``moe_oracle.c``.
 Block-scaled (MX) FP8 experts (``quantize_mx``, ``mx_value``,
 ``expert_apply_mx``, ``layer_tokens_mx``): e4m3 codes with one power-of-two
-(E8M0) scale per 32 values along the contraction dimension.
+(E8M0) scale per 32 values along the contraction dimension.  INT4
+weight-only experts (``w4_dequant``, ``expert_apply_w4``, ``layer_tokens_w4``):
+signed 4-bit weights, two per byte, one bf16 scale per 128 inputs of a row,
+bf16 activations.
 
 Parity pins (tests/test_oracle_pins.py): brute-force top-k on tiny inputs,
 library softmax / sigmoid for the gates, sums of counts, closed-form balance
@@ -59,7 +62,8 @@ def _load():
         for name in ("oracle_route", "oracle_dispatch", "oracle_balance",
                      "oracle_expert_apply", "oracle_layer_tokens", "oracle_bias_update",
                      "oracle_routing_health", "oracle_quantize_rows", "oracle_expert_apply_fp8",
-                     "oracle_layer_backward", "oracle_quantize_mx", "oracle_expert_apply_mx"):
+                     "oracle_layer_backward", "oracle_quantize_mx", "oracle_expert_apply_mx",
+                     "oracle_expert_apply_w4", "oracle_w4_dequant"):
             getattr(lib, name).restype = ctypes.c_int
         lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -375,6 +379,73 @@ def layer_tokens_mx(dims, x8, xs, weights, idx, gate, row_of, tokens):
     y = np.zeros((len(tokens), dims.d), np.float64)
     if tok:
         rows = expert_apply_mx(dims, x8, xs, weights, np.array(tok), np.array(ex), np.array(g))
+        for r, n in enumerate(owner):
+            y[n] += rows[r]
+    return y
+
+
+def w4_dequant(codes, scales):
+    """float64 values of INT4 weights: codes uint8 [rows, cols/2] (low nibble
+    = even input, nibble = q + 8), scales bf16 bits uint16 [rows, cols/128]."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    rows, half = codes.shape
+    out = np.empty((rows, half * 2), np.float64)
+    if lib.oracle_w4_dequant(_ptr(codes), _ptr(scales), ctypes.c_int64(rows), ctypes.c_int32(half * 2), _ptr(out)):
+        raise ValueError("w4_dequant: columns must be a positive multiple of 128")
+    return out
+
+
+def _w4_weights(w):
+    def u8(a):
+        return None if a is None else np.ascontiguousarray(a, dtype=np.uint8)
+
+    def u16(a):
+        return None if a is None else np.ascontiguousarray(a, dtype=np.uint16)
+    return (u8(w.get("W1")), u16(w.get("W1_scale")), _f32(w.get("b1")),
+            u8(w.get("Wu")), u16(w.get("Wu_scale")),
+            u8(w.get("W2")), u16(w.get("W2_scale")), _f32(w.get("b2")),
+            u8(w.get("Wsg")), u16(w.get("Wsg_scale")), u8(w.get("Wsu")), u16(w.get("Wsu_scale")),
+            u8(w.get("Wsd")), u16(w.get("Wsd_scale")))
+
+
+def expert_apply_w4(dims, x, weights, token, expert, scale=None):
+    """out[r] = scale[r] * Ew4_{expert[r]}(x[token[r]]) with INT4 weight-only
+    experts.  x: bf16 bits [T, d]; weights: W1, Wu, W2 (and Wsg, Wsu, Wsd) as
+    packed codes [..., out, in/2] with bf16-bit scales "<name>_scale"
+    [..., out, in/128]; biases b1, b2 fp32."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    token = np.ascontiguousarray(token, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.float64)
+    out = np.empty((len(token), dims.d), np.float64)
+    ws = _w4_weights(weights)
+    rc = lib.oracle_expert_apply_w4(ctypes.byref(dims), ctypes.c_int64(len(token)), _ptr(token), _ptr(expert),
+                                    _ptr(sc), _ptr(x), *[_ptr(a) for a in ws], _ptr(out))
+    if rc:
+        raise ValueError("oracle_expert_apply_w4: bad expert id or dimension not a multiple of 128")
+    return out
+
+
+def layer_tokens_w4(dims, x, weights, idx, gate, row_of, tokens):
+    """y[n] for the listed tokens with INT4 weight-only experts: the
+    gate-weighted sum of the kept experts (+ the shared expert, weight 1)."""
+    idx = np.asarray(idx, np.int32)
+    gate = np.asarray(gate, np.float64)
+    tokens = np.asarray(tokens, np.int32)
+    tok, ex, g, owner = [], [], [], []
+    for n, t in enumerate(tokens):
+        for s in range(dims.k):
+            if row_of is not None and row_of[t, s] < 0:
+                continue
+            tok.append(t); ex.append(idx[t, s]); g.append(gate[t, s]); owner.append(n)
+        if dims.d_ff_shared > 0:
+            tok.append(t); ex.append(dims.E); g.append(1.0); owner.append(n)
+    y = np.zeros((len(tokens), dims.d), np.float64)
+    if tok:
+        rows = expert_apply_w4(dims, x, weights, np.array(tok), np.array(ex), np.array(g))
         for r, n in enumerate(owner):
             y[n] += rows[r]
     return y

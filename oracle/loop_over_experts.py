@@ -299,3 +299,31 @@ def layer_mx(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1,
     if weights.get("Wsg") is not None:
         y += expert_fn_mx(act, xd, wdeq("Wsg"), wdeq("Wsu"), wdeq("Wsd"))
     return dict(y=y, idx=idx, gate=gate, x8=x8, xs=xs)
+
+
+# ---------------------------------------------------------------- INT4 weight-only experts
+# The layer with INT4 weight-only experts: nibbles unpacked with numpy bit
+# operations, each weight rounded to bf16 from q * s, then the bf16 layer's
+# dense expert on the dequantized matrices.
+
+def w4_dequant_np(codes, scales):
+    codes = np.asarray(codes, np.uint8)
+    lo = (codes & 15).astype(np.int64) - 8
+    hi = (codes >> 4).astype(np.int64) - 8
+    q = np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (codes.shape[-1] * 2,))
+    s = np.repeat(_f64(np.asarray(scales, np.uint16)), 128, axis=-1)
+    return bf16_round(q.astype(np.float64) * s)
+
+
+def layer_w4(x, Wr, weights, k, *, act, score="softmax", renorm=1, capacity=-1, logit_bias=None, sel_bias=None):
+    """The layer with INT4 weight-only experts (weights: packed codes W1, Wu,
+    W2 (Wsg, Wsu, Wsd) with bf16-bit scales "<name>_scale", biases b1, b2)."""
+    dq = {}
+    for name in ("W1", "Wu", "W2", "Wsg", "Wsu", "Wsd"):
+        if weights.get(name) is not None:
+            dq[name] = w4_dequant_np(weights[name], weights[name + "_scale"])
+    for name in ("b1", "b2"):
+        if weights.get(name) is not None:
+            dq[name] = np.asarray(weights[name], np.float64)
+    return layer(x, Wr, dq, k, act=act, score=score, renorm=renorm, capacity=capacity, logit_bias=logit_bias,
+                 sel_bias=sel_bias)

@@ -794,6 +794,128 @@ int oracle_expert_apply_mx(const oracle_dims *dm, int64_t nrows, const int32_t *
     return 0;
 }
 
+/* ---- INT4 weight-only experts -----------------------------------------------
+ * [IS] Serving: weight-only INT4 experts (torchao's INT4 weight-only path) once
+ * memory binds.  The reading written out here: every expert weight matrix
+ * [out, in] is stored as signed 4-bit integers q in [-8, 7], two per byte
+ * (the low nibble holds the even input index; a nibble stores q + 8), with one
+ * bf16 scale per output row and group of 128 consecutive inputs; a weight's
+ * value is the bf16 nearest to q * s (ties to even).  Everything else is the
+ * bf16 layer's expert (bf16 x, H exact), in double on the exact weight
+ * values.                                                                    */
+
+static double bf16_bits_value(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Value of input j of weight row `row` (cols inputs per row).                */
+static double w4_value(const uint8_t *codes, const uint16_t *scales, size_t row, int cols, int j)
+{
+    const uint8_t byte = codes[row * (size_t)(cols / 2) + (size_t)(j / 2)];
+    const int q = ((j & 1) ? (byte >> 4) : (byte & 15)) - 8;
+    const double sc = bf16_bits_value(scales[row * (size_t)(cols / 128) + (size_t)(j / 128)]);
+    return (double)round_bf16((double)q * sc);
+}
+
+typedef struct {
+    const oracle_dims *dm;
+    const uint16_t *x;                                       /* [T, d] bf16 bits              */
+    const uint8_t *W1; const uint16_t *s1; const float *b1;  /* [E, d_ff, d/2], [E, d_ff, d/128] */
+    const uint8_t *Wu; const uint16_t *su;
+    const uint8_t *W2; const uint16_t *s2; const float *b2;  /* [E, d, d_ff/2], [E, d, d_ff/128] */
+    const uint8_t *Wsg; const uint16_t *ssg; const uint8_t *Wsu; const uint16_t *ssu;
+    const uint8_t *Wsd; const uint16_t *ssd;
+} w4_experts;
+
+/* One INT4 expert on token t (e == E: the shared expert); hbuf: d_ff doubles of scratch. */
+static void expert_apply_w4_one(const w4_experts *w, int64_t t, int e, double *hbuf, double *out)
+{
+    const oracle_dims *dm = w->dm;
+    const int d = dm->d;
+    const int shared = (e == dm->E);
+    const int dff = shared ? dm->d_ff_shared : dm->d_ff;
+    const uint8_t *Wa = shared ? w->Wsg : w->W1, *Wb = shared ? w->Wsu : w->Wu, *Wo = shared ? w->Wsd : w->W2;
+    const uint16_t *sa = shared ? w->ssg : w->s1, *sb = shared ? w->ssu : w->su, *so = shared ? w->ssd : w->s2;
+    const size_t eb = shared ? 0 : (size_t)e;
+    const uint16_t *xr = w->x + (size_t)t * d;
+    for (int j = 0; j < dff; ++j) {
+        const size_t wr = eb * dff + j;
+        double a = 0.0;
+        for (int i = 0; i < d; ++i) a += w4_value(Wa, sa, wr, d, i) * bf16_bits_value(xr[i]);
+        if (dm->act == 0) {
+            if (!shared && w->b1) a += (double)w->b1[eb * dff + j];
+            hbuf[j] = 0.5 * a * (1.0 + erf(a / sqrt(2.0)));
+        } else {
+            double u = 0.0;
+            for (int i = 0; i < d; ++i) u += w4_value(Wb, sb, wr, d, i) * bf16_bits_value(xr[i]);
+            hbuf[j] = a / (1.0 + exp(-a)) * u;
+        }
+    }
+    for (int i = 0; i < d; ++i) {
+        const size_t orow = eb * d + i;
+        double o = 0.0;
+        for (int j = 0; j < dff; ++j) o += w4_value(Wo, so, orow, dff, j) * hbuf[j];
+        if (dm->act == 0 && !shared && w->b2) o += (double)w->b2[eb * d + i];
+        out[i] = o;
+    }
+}
+
+typedef struct {
+    w4_experts w;
+    const int32_t *token; const int32_t *expert; const double *scale; double *out;
+} applyw4_ctx;
+
+static void applyw4_range(void *vctx, int64_t lo, int64_t hi)
+{
+    applyw4_ctx *c = (applyw4_ctx *)vctx;
+    const oracle_dims *dm = c->w.dm;
+    const int hmax = dm->d_ff > dm->d_ff_shared ? dm->d_ff : dm->d_ff_shared;
+    const size_t hn = (size_t)(hmax > 0 ? hmax : 1);
+    double *hbuf = (double *)malloc(sizeof(double) * hn);
+    for (int64_t r = lo; r < hi; ++r) {
+        double *o = c->out + (size_t)r * dm->d;
+        expert_apply_w4_one(&c->w, c->token[r], c->expert[r], hbuf, o);
+        const double sc = c->scale ? c->scale[r] : 1.0;
+        for (int i = 0; i < dm->d; ++i) o[i] *= sc;
+    }
+    free(hbuf);
+}
+
+/* out[r,:] = scale[r] * Ew4_{expert[r]}(x[token[r],:]) for INT4 weight-only
+ * experts (expert == E: the shared expert).  d, d_ff (and d_ff_shared) must
+ * be multiples of 128; x is bf16 bits.                                       */
+int oracle_expert_apply_w4(const oracle_dims *dm, int64_t nrows, const int32_t *token, const int32_t *expert,
+                           const double *scale, const uint16_t *x,
+                           const uint8_t *W1, const uint16_t *s1, const float *b1,
+                           const uint8_t *Wu, const uint16_t *su,
+                           const uint8_t *W2, const uint16_t *s2, const float *b2,
+                           const uint8_t *Wsg, const uint16_t *ssg, const uint8_t *Wsu, const uint16_t *ssu,
+                           const uint8_t *Wsd, const uint16_t *ssd, double *out)
+{
+    if (dm->d % 128 != 0 || dm->d_ff % 128 != 0 || (dm->d_ff_shared > 0 && dm->d_ff_shared % 128 != 0)) return 2;
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (expert[r] < 0 || expert[r] > dm->E) return 1;
+        if (expert[r] == dm->E && dm->d_ff_shared <= 0) return 1;
+    }
+    applyw4_ctx c = { { dm, x, W1, s1, b1, Wu, su, W2, s2, b2, Wsg, ssg, Wsu, ssu, Wsd, ssd },
+                      token, expert, scale, out };
+    parallel_for(nrows, dm->nthreads, applyw4_range, &c);
+    return 0;
+}
+
+/* Value of every input of `rows` weight rows (the dequantized matrix, double). */
+int oracle_w4_dequant(const uint8_t *codes, const uint16_t *scales, int64_t rows, int32_t cols, double *out)
+{
+    if (cols <= 0 || cols % 128 != 0) return 1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int j = 0; j < cols; ++j) out[r * cols + j] = w4_value(codes, scales, (size_t)r, cols, j);
+    return 0;
+}
+
 /* ===========================================================================
  * Backward pass of the layer.
  *
