@@ -501,7 +501,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: e4m3 experts through moe_forward_fp8 (bf16 layers only; no CPU baseline)")
-    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8,qwen3_moe:mx,qwen3_moe:backward",
+    ap.add_argument("--sub", default="mixtral,deepseek_v3,qwen3_moe:fp8,qwen3_moe:mx,qwen3_moe:w4,qwen3_moe:backward",
                     help="further workloads (name or name:fp8) timed after the headline one and reported "
                          "under sub_records; '' for none")
     ap.add_argument("--sub-steps", type=int, default=20)
@@ -743,18 +743,110 @@ def mx_record(args, wl, dev, world):
             "clocks": clocks}
 
 
+def w4_record(args, wl, dev, world):
+    """The grouped FFN with INT4 weight-only experts (moe_grouped_ffn_w4: the
+    two GEMMs with the weights decoded to bf16 in shared memory each stage)
+    on the workload's routed rows, then the whole layer (moe_forward_w4),
+    timed like the MX record.  Roofline: the expert FLOPs of the kept rows
+    against the bf16 tensor peak, and the packed weight bytes per step."""
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inp = syn.generate(wl, dev, seed=0, weights=False)
+    cfg = nat.config_from_workload(wl)
+    T, k, E, d = wl.T, wl.top_k, wl.E, wl.d_model
+    sld = nat.w4_sld(cfg)
+    w = syn.generate_w4_experts(wl, sld, dev, seed=0)
+    ws = nat.alloc_workspace(cfg, dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    psum = torch.empty((nat.router_blocks(cfg), E), dtype=torch.float32, device=dev)
+    nat.moe_router_topk(cfg, inp["x"], inp["Wr"], inp["logit_bias"], inp["sel_bias"], idx, gate, None, psum, ws)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    row_token = torch.zeros(T * k, dtype=torch.int32, device=dev)
+    row_gate = torch.zeros(T * k, dtype=torch.float32, device=dev)
+    x_perm = torch.zeros((nat.perm_rows(cfg), d), dtype=torch.bfloat16, device=dev)
+    nat.moe_permute(cfg, inp["x"], idx, gate, counts, kept, offsets, row_of, row_token, row_gate, x_perm, None, ws)
+    torch.cuda.synchronize(dev)
+    n = int(offsets[-1].item())
+    y_perm = torch.empty((nat.perm_rows(cfg), d), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        nat.moe_grouped_ffn_w4(cfg, x_perm, offsets, row_gate, w, sld, w.get("b1"), w.get("b2"), inp["x"], y_perm,
+                               ws, stream)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(ws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the INT4 warm-up")
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.sub_steps)]
+    for i in range(args.sub_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.sub_steps
+    ms = max_over_ranks([ms], world, dev)[0]
+    flops = float(wl.expert_flops(n))
+    peaks, peak_src = load_peaks()
+    peak_t, which = tensor_peak(peaks, clocks)
+    tf = flops / (ms * 1e-3) / 1e12
+    wbytes = sum(int(v.numel()) for key, v in w.items() if v is not None and key[0] == "W")
+
+    out = nat.Outputs(cfg, dev)
+    nat.moe_router_freeze(cfg, inp["Wr"], ws, stream)
+    for _ in range(3):
+        flush.zero_()
+        nat.forward_w4(cfg, inp, w, sld, out, ws, stream)
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(ws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the INT4 layer warm-up")
+    for i in range(args.sub_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        nat.forward_w4(cfg, inp, w, sld, out, ws, stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    layer_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in ev) / args.sub_steps], world, dev)[0]
+    return {"workload": wl.name, "experts": "int4 weight-only (bf16 scale per 128 inputs, decoded to bf16 in "
+                                            "shared memory, tcgen05 kind::f16)",
+            "pass": "grouped FFN stage (GEMM 1, GEMM 2) on the packed rows",
+            "steps": args.sub_steps, "warmup": 3, "ms_per_step": ms, "tflops": tf,
+            "weight_bytes": wbytes,
+            "layer": {"entry": "moe_forward_w4 (router, permute, grouped FFN, combine)", "ms_per_step": layer_ms,
+                      "tokens_per_s": job_tokens_per_s(world, wl.T, layer_ms),
+                      "tflops": flops / (layer_ms * 1e-3) / 1e12},
+            "gpu_launches": 2 * args.sub_steps,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_t, "unit": "TFLOP/s", "frac": tf / peak_t,
+                         "flops": flops, "peak_note": "bf16 (the MMA's operand type), %s %s"
+                         % (which, "of measured" if peak_src == "measured" else "of fallback")},
+            "clocks": clocks}
+
+
 def sub_record(args, spec, dev, world, rank):
     """One further workload timed like the headline one (device-resident steps
     with the L2 flushed between them, the staged per-stage pass), reported
     with its own roofline fractions.  spec: "workload", "workload:fp8",
-    "workload:backward" (the backward pass, backward_record) or "workload:mx"
-    (the MX grouped FFN stage, mx_record)."""
+    "workload:backward" (the backward pass, backward_record), "workload:mx"
+    (the MX grouped FFN stage, mx_record) or "workload:w4" (the INT4
+    weight-only grouped FFN stage, w4_record)."""
     name, _, experts = spec.partition(":")
     wl = syn.WORKLOADS[name]
     if experts == "backward":
         return backward_record(args, wl, dev, world)
     if experts == "mx":
         return mx_record(args, wl, dev, world)
+    if experts == "w4":
+        return w4_record(args, wl, dev, world)
     fp8 = experts == "fp8"
     r = run_ours(args, wl, dev, world, rank, fp8=fp8, steps=args.sub_steps, warmup=3, full=False)
     rec = {"workload": name, "experts": "fp8" if fp8 else "bf16", "steps": args.sub_steps, "warmup": 3,

@@ -446,6 +446,47 @@ MOE_API moe_status moe_grouped_ffn_mx(const moe_config *cfg, const uint8_t *x8_p
                                       const float *b1, const float *b2, const uint8_t *x8, const uint8_t *xs,
                                       void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- INT4 weight-only experts --------------------------------------------
+ * Weight-only INT4 experts ("Fine-tuning and serving MoE models", Serving:
+ * weight-only INT4 / FP8 experts, torchao's INT4 weight-only path, once
+ * memory binds): every expert weight matrix [out, in] holds signed 4-bit
+ * integers q in [-8, 7], two per byte (the low nibble the even input; a
+ * nibble stores q + 8), with one bf16 scale per output row and group of 128
+ * consecutive inputs; a weight's value is bf16(q * s) (nearest, ties to
+ * even).  Activations stay bf16 (the bf16 layer's x and H); the tensor cores
+ * run bf16 x bf16 products with fp32 accumulation on weights decoded into
+ * shared memory stage by stage.
+ * Scale arrays have rows of sld bytes: sld a multiple of 16 and at least
+ * 2 * d_model / 128, 2 * d_ff / 128 and 2 * d_ff_shared / 128.  Only bf16
+ * layers with d_model, d_ff and d_ff_shared multiples of 128 and E <= 256
+ * (else MOE_ERR_UNSUPPORTED).  All pointers in the struct are device
+ * pointers, 16-byte aligned; the struct is read during the call.            */
+typedef struct {
+    const uint8_t *W1;    const uint8_t *W1_scale;      /* [E, d_ff, d_model / 2], [E, d_ff, sld] */
+    const uint8_t *Wu;    const uint8_t *Wu_scale;      /* SwiGLU W_up (same shapes), else NULL   */
+    const uint8_t *W2;    const uint8_t *W2_scale;      /* [E, d_model, d_ff / 2], [E, d_model, sld] */
+    const uint8_t *Wsh_g; const uint8_t *Wsh_g_scale;   /* shared expert, same layouts, or NULL   */
+    const uint8_t *Wsh_u; const uint8_t *Wsh_u_scale;
+    const uint8_t *Wsh_d; const uint8_t *Wsh_d_scale;
+    int32_t sld;                                        /* scale row stride in bytes             */
+} moe_w4_experts;
+
+/* moe_grouped_ffn with INT4 weight-only experts: arguments and output as in
+ * moe_grouped_ffn (x_perm, x bf16), the experts in *w; ws is the layer's
+ * workspace (moe_workspace_size: its hidden-activation region holds H).      */
+MOE_API moe_status moe_grouped_ffn_w4(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                                      const float *row_gate, const moe_w4_experts *w, const float *b1,
+                                      const float *b2, const void *x, void *y_perm, void *ws, size_t ws_bytes,
+                                      moe_stream_t stream);
+/* moe_forward with INT4 weight-only experts: the bf16 layer (router,
+ * permute, combine, statistics) around the INT4 grouped FFN.  Arguments and
+ * outputs as in moe_forward, the expert weights in *w.                      */
+MOE_API moe_status moe_forward_w4(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                                  const float *sel_bias, const moe_w4_experts *w, const float *b1, const float *b2,
+                                  void *y, int32_t *idx, float *gate, int32_t *counts, float *f, float *P,
+                                  double *loss, float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
 /* Auxiliary-loss-free bias update, to run after a training step on the
  * counts that step's routing produced ("Fine-Tuning Mixture of Experts (MoE)
  * Models: Router Optimization Techniques", How It Works 2, and its router

@@ -180,6 +180,11 @@ struct FfnMxArgs {
     int num_sms;
 };
 cudaError_t launch_ffn_mx(const FfnMxArgs &a, cudaStream_t st);
+// INT4 weight-only experts through the same arguments: x_perm / x hold bf16
+// rows, W* packed INT4 codes [.., N, K/2] (low nibble = even input, nibble =
+// q + 8), W*s bf16 scale bytes [.., N, sld] (one scale per 128 inputs); H
+// stays bf16 between the GEMMs.  mx_sm100.cu.
+cudaError_t launch_ffn_w4(const FfnMxArgs &a, cudaStream_t st);
 
 // Per-row e4m3 quantization of bf16 rows (row0 + r for r < rows, or fewer
 // when rows_limit points at a smaller device count): in [.., ld_in] bf16,

@@ -142,6 +142,32 @@ moe_status check_mx_cfg(const moe_config *c, int32_t sld) {
 
 // MX workspace: H in bf16, its codes and scale rows (the grouped FFN), then
 // x's codes and scale rows and the packed rows' scale rows (moe_forward_mx).
+// INT4 experts: bf16 layers, K dimensions in whole 128-input groups, at most
+// 256 routed groups, bf16 scale rows of sld bytes (a multiple of 16 that holds
+// 2 * K / 128 bytes for every K).
+moe_status check_w4_cfg(const moe_config *c, int32_t sld) {
+    if (c->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "INT4 experts need a bf16 layer%s");
+    if (c->d_model % 128 || c->d_ff % 128 || c->d_ff_shared % 128)
+        return fail(MOE_ERR_UNSUPPORTED, "INT4 experts need d_model, d_ff, d_ff_shared multiples of 128%s");
+    if (c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "INT4 experts: at most 256 experts%s");
+    const int need = std::max(c->d_model, std::max(c->d_ff, c->d_ff_shared)) / 64;
+    if (sld < need || sld % 16) return fail(MOE_ERR_INVALID_ARG, "sld below 2 * K / 128 or not a multiple of 16%s");
+    return MOE_OK;
+}
+
+moe_status check_w4_weights(const moe_config *c, const moe_w4_experts *w) {
+    NEED(w->W1); NEED(w->W1_scale); NEED(w->W2); NEED(w->W2_scale);
+    if (c->act == MOE_ACT_SWIGLU) { NEED(w->Wu); NEED(w->Wu_scale); }
+    if (c->d_ff_shared > 0) {
+        NEED(w->Wsh_g); NEED(w->Wsh_g_scale); NEED(w->Wsh_d); NEED(w->Wsh_d_scale);
+        if (c->act == MOE_ACT_SWIGLU) { NEED(w->Wsh_u); NEED(w->Wsh_u_scale); }
+    }
+    ALIGNED(w->W1, 16); ALIGNED(w->Wu, 16); ALIGNED(w->W2, 16); ALIGNED(w->Wsh_g, 16); ALIGNED(w->Wsh_u, 16);
+    ALIGNED(w->Wsh_d, 16); ALIGNED(w->W1_scale, 16); ALIGNED(w->Wu_scale, 16); ALIGNED(w->W2_scale, 16);
+    ALIGNED(w->Wsh_g_scale, 16); ALIGNED(w->Wsh_u_scale, 16); ALIGNED(w->Wsh_d_scale, 16);
+    return MOE_OK;
+}
+
 struct MxLayout {
     size_t H, H8, Hs, x8, xs, xs_perm, total;
     int hF;
@@ -295,6 +321,29 @@ size_t ep_ws_bytes(const moe_config *c, int64_t max_rows) {
     const size_t esz = c->dtype == MOE_BF16 ? 2 : 4;
     return align256(ep_h_offset() + (size_t)max_rows * c->d_ff * esz);
 }
+moe::FfnMxArgs w4_args(const moe_config *cfg, const void *x_perm, const int32_t *offsets, const float *row_gate,
+                       const moe_w4_experts *w, const float *b1, const float *b2, const void *x, void *y_perm,
+                       void *ws) {
+    const Layout L = layout(cfg);
+    moe::FfnMxArgs a{};
+    a.x_perm = static_cast<const uint8_t *>(x_perm); a.x = static_cast<const uint8_t *>(x);
+    a.offsets = offsets; a.row_gate = row_gate;
+    a.W1 = w->W1; a.W1s = w->W1_scale; a.Wu = w->Wu; a.Wus = w->Wu_scale; a.W2 = w->W2; a.W2s = w->W2_scale;
+    a.b1 = b1; a.b2 = b2;
+    a.Wsg = w->Wsh_g; a.Wsgs = w->Wsh_g_scale; a.Wsu = w->Wsh_u; a.Wsus = w->Wsh_u_scale;
+    a.Wsd = w->Wsh_d; a.Wsds = w->Wsh_d_scale;
+    a.H = at<__nv_bfloat16>(ws, L.H);
+    a.y_perm = static_cast<__nv_bfloat16 *>(y_perm);
+    a.status = status_word(ws);
+    a.T = cfg->T; a.d = cfg->d_model; a.E = cfg->E; a.F = cfg->d_ff; a.S = cfg->d_ff_shared; a.act = cfg->act;
+    a.routed_rows = (int64_t)cfg->T * cfg->top_k;
+    a.hF = std::max(cfg->d_ff, cfg->d_ff_shared);
+    a.shared_base = (int64_t)cfg->T * cfg->top_k;
+    a.sld = w->sld;
+    a.num_sms = num_sms();
+    return a;
+}
+
 }  // namespace
 
 namespace moe {
@@ -929,6 +978,87 @@ moe_status moe_forward_mx(const moe_config *cfg, const void *x, const float *Wr,
 
     moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
                         shared ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
+    if ((e = moe::launch_combine(ca, true, st)) != cudaSuccess) return cuda_fail(e, "combine");
+    return MOE_OK;
+}
+
+
+moe_status moe_grouped_ffn_w4(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                              const float *row_gate, const moe_w4_experts *w, const float *b1, const float *b2,
+                              const void *x, void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(w);
+    if ((s = check_w4_cfg(cfg, w->sld)) != MOE_OK) return s;
+    if (cfg->T > 0) {
+        NEED(x_perm); NEED(offsets); NEED(row_gate); NEED(y_perm);
+        if ((s = check_w4_weights(cfg, w)) != MOE_OK) return s;
+        if (cfg->d_ff_shared > 0) NEED(x);
+    }
+    ALIGNED(x_perm, 16); ALIGNED(x, 16); ALIGNED(y_perm, 16); ALIGNED(offsets, 4); ALIGNED(row_gate, 4);
+    ALIGNED(b1, 4); ALIGNED(b2, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    if (cfg->T == 0) return MOE_OK;
+    moe::FfnMxArgs a = w4_args(cfg, x_perm, offsets, row_gate, w, b1, b2, x, y_perm, ws);
+    cudaError_t e = moe::launch_ffn_w4(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "grouped_ffn_w4");
+}
+
+moe_status moe_forward_w4(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                          const float *sel_bias, const moe_w4_experts *w, const float *b1, const float *b2, void *y,
+                          int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                          float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    NEED(w);
+    if ((s = check_w4_cfg(cfg, w->sld)) != MOE_OK) return s;
+    NEED(counts); NEED(f); NEED(P); NEED(loss);
+    if (cfg->T > 0) {
+        NEED(x); NEED(Wr); NEED(y); NEED(idx); NEED(gate);
+        if ((s = check_w4_weights(cfg, w)) != MOE_OK) return s;
+    }
+    ALIGNED(x, 16); ALIGNED(y, 16); ALIGNED(Wr, 4); ALIGNED(logit_bias, 4); ALIGNED(sel_bias, 4);
+    ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
+    ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
+    if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    const Layout L = layout(cfg);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *psum = at<float>(ws, L.psum);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *row_of = at<int32_t>(ws, L.row_of);
+    float *row_gate = at<float>(ws, L.row_gate);
+    void *y_perm = at<char>(ws, L.y_perm);
+    cudaError_t e;
+
+    moe::RouterArgs ra{x, Wr, logit_bias, sel_bias, idx, gate, logits_out, psum,
+                       cfg->T, cfg->d_model, cfg->E, cfg->top_k, cfg->score, cfg->renorm,
+                       at<char>(ws, L.router_w), at<float>(ws, L.logits), status_word(ws), num_sms()};
+    ra.split_ready = router_split_ready(ws, Wr, cfg->d_model, cfg->E);
+    if ((e = moe::launch_router(ra, true, st)) != cudaSuccess) return cuda_fail(e, "router");
+
+    moe::DispatchArgs da{};
+    da.x = x; da.idx = idx; da.gate = gate;
+    da.chunk_cnt = at<int32_t>(ws, L.chunk_cnt);
+    da.chunk_base = at<int32_t>(ws, L.chunk_base);
+    da.counts = counts; da.kept = at<int32_t>(ws, L.kept); da.offsets = offsets;
+    da.row_of = row_of; da.row_token = at<int32_t>(ws, L.row_token); da.row_gate = row_gate;
+    da.x_perm = at<char>(ws, L.x_perm);
+    da.n_dropped = n_dropped;
+    da.status = status_word(ws);
+    da.T = cfg->T; da.d = cfg->d_model; da.E = cfg->E; da.k = cfg->top_k;
+    da.capacity = moe_capacity(cfg);
+    da.psum = psum; da.f = f; da.P = P; da.loss = loss;
+    da.contrib = at<double>(ws, L.contrib);
+    da.nblk = moe::router_blocks(cfg->T, true);
+    da.pdl = true;
+    if ((e = moe::launch_dispatch(da, 2, st)) != cudaSuccess) return cuda_fail(e, "permute");
+
+    if (cfg->T > 0) {
+        moe::FfnMxArgs a = w4_args(cfg, da.x_perm, offsets, row_gate, w, b1, b2, x, y_perm, ws);
+        if ((e = moe::launch_ffn_w4(a, st)) != cudaSuccess) return cuda_fail(e, "grouped_ffn_w4");
+    }
+    moe::CombineArgs ca{y_perm, row_of, y, status_word(ws), cfg->T, cfg->d_model, cfg->top_k,
+                        cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
     if ((e = moe::launch_combine(ca, true, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
 }

@@ -120,14 +120,26 @@ __global__ void __launch_bounds__(256) mx_gather_rows_kernel(const uint8_t *src,
 }
 
 // ------------------------------------------------------------------ grouped GEMM
-constexpr int MX_BM = 128, MX_BN = 128, MX_BK = 128;   // K per stage: one 128-byte row of e4m3 codes
+// Two kinds share the kernel: MX (e4m3 A and B with E8M0 block scales, K =
+// 128 per stage, one 128-byte row of codes) and W4 (bf16 A, INT4 weight-only
+// B: K = 64 per stage, one 128-byte row of bf16; the B codes, 32 bytes per
+// row, and their bf16 scales arrive by TMA and four warps decode them into the
+// stage's bf16 B tile).
+enum { KIND_MX = 0, KIND_W4 = 1 };
+constexpr int MX_BM = 128, MX_BN = 128;
 constexpr int MX_STAGES = 5;
 constexpr int kMxThreads = 320;
-constexpr uint32_t MX_A_BYTES = MX_BM * MX_BK;          // 16 KiB
-constexpr uint32_t MX_B_BYTES = MX_BN * MX_BK;          // 16 KiB
-constexpr uint32_t MX_SA_BYTES = MX_BM * 16;            // 128 rows x 16 scale bytes
-constexpr uint32_t MX_SB_BYTES = MX_BN * 16;
+constexpr uint32_t MX_A_BYTES = MX_BM * 128;            // 16 KiB: 128 rows x 128 bytes
+constexpr uint32_t MX_B_BYTES = MX_BN * 128;            // 16 KiB
+constexpr uint32_t MX_SA_BYTES = MX_BM * 16;            // MX: 128 rows x 16 scale bytes
+constexpr uint32_t MX_SB_BYTES = MX_BN * 16;            // MX: B scale rows; W4: B bf16 scale rows
+constexpr uint32_t W4_CODE_BYTES = MX_BN * 32;          // W4: 128 rows x 64 nibbles
+template <int KIND> constexpr int kind_bk() { return KIND == KIND_MX ? 128 : 64; }
+// Per stage: A | B | (MX) A scales, B scales | (W4) B codes, B scales; the same size for both kinds.
 constexpr uint32_t MX_STAGE_BYTES = MX_A_BYTES + MX_B_BYTES + MX_SA_BYTES + MX_SB_BYTES;   // 36 KiB
+static_assert(MX_SA_BYTES + MX_SB_BYTES <= W4_CODE_BYTES + MX_SB_BYTES, "W4 stage layout");
+constexpr uint32_t W4_STAGE_BYTES = MX_A_BYTES + MX_B_BYTES + W4_CODE_BYTES + MX_SB_BYTES;  // 38 KiB
+constexpr uint32_t STAGE_STRIDE = W4_STAGE_BYTES;       // both kinds use the larger stride
 constexpr uint32_t MX_TMEM_COLS = 512;
 constexpr uint32_t MX_SF_COL0 = 2 * MX_BN;              // scale slots after the two accumulators
 constexpr int kMxMaxGroups = 257;
@@ -184,7 +196,7 @@ struct MxSmem {
     int rows[kMxMaxGroups];
     int row0[kMxMaxGroups];
 };
-constexpr size_t kMxStgOff = ((size_t)MX_STAGES * MX_STAGE_BYTES + sizeof(MxSmem) + 1023) / 1024 * 1024;
+constexpr size_t kMxStgOff = ((size_t)MX_STAGES * STAGE_STRIDE + sizeof(MxSmem) + 1023) / 1024 * 1024;
 constexpr size_t kMxSmemBytes = 1024 + kMxStgOff + 4 * MX_STG_BYTES;
 static_assert(kMxSmemBytes <= 227 * 1024, "MX GEMM shared memory");
 
@@ -243,7 +255,7 @@ __device__ __forceinline__ void mx_store32(uint32_t stg, const float *h, __nv_bf
     }
 }
 
-template <int MODE>
+template <int MODE, int KIND>
 __global__ void __launch_bounds__(kMxThreads, 1)
 tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
            const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSAs,
@@ -256,8 +268,9 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_addr);
-    MxSmem &s = *reinterpret_cast<MxSmem *>(smem + MX_STAGES * MX_STAGE_BYTES);
+    MxSmem &s = *reinterpret_cast<MxSmem *>(smem + MX_STAGES * STAGE_STRIDE);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int BK = kind_bk<KIND>();
     const int G = p.E + (p.has_shared ? 1 : 0);
     constexpr int OUT_COLS = (MODE == MX_SWIGLU) ? MX_BN / 2 : MX_BN;   // output columns per tile
 
@@ -320,7 +333,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 mx_decode(s, G, tile, g, mt, nt);
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
-                const int nk = K / MX_BK;
+                const int nk = K / BK;
                 const int a_row = sh ? (int)p.shared_a_row + mt * MX_BM : s.row0[g] + mt * MX_BM;
                 const int e = sh ? 0 : g;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA, *mSA = sh ? &tmSAs : &tmSA;
@@ -329,12 +342,37 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { mx_fail(s, p, 41); break; }
                     const uint32_t fb = smem_u32(&s.full[stage]);
-                    mbar_arrive_expect_tx(fb, MX_STAGE_BYTES);
-                    const uint32_t a_dst = base + stage * MX_STAGE_BYTES;
+                    const uint32_t a_dst = base + stage * STAGE_STRIDE;
                     const uint32_t b_dst = a_dst + MX_A_BYTES;
+                    if (KIND == KIND_W4) {
+                        // A (bf16, 64 of K), the B codes (32 bytes of each of 128 rows) and the
+                        // 16-byte box of B scale bytes holding the stage's group scale
+                        mbar_arrive_expect_tx(fb, MX_A_BYTES + W4_CODE_BYTES + MX_SB_BYTES);
+                        const uint32_t c_dst = b_dst + MX_B_BYTES;
+                        const uint32_t s_dst = c_dst + W4_CODE_BYTES;
+                        const int cx = kb * 32;                       // code bytes: 64 nibbles per stage
+                        const int gx = ((kb >> 1) * 2) & ~15;         // scale bytes: group kb / 2, bf16
+                        tma_load_2d(a_dst, mA, fb, kb * BK, a_row);
+                        if (MODE == MX_SWIGLU) {
+                            const int j0 = nt * OUT_COLS;
+                            tma_load_3d(c_dst, mB, fb, cx, j0, e);
+                            tma_load_3d(c_dst + W4_CODE_BYTES / 2, mB2, fb, cx, j0, e);
+                            tma_load_3d(s_dst, mSB, fb, gx, j0, e);
+                            tma_load_3d(s_dst + MX_SB_BYTES / 2, mSB2, fb, gx, j0, e);
+                        } else {
+                            tma_load_3d(c_dst, mB, fb, cx, nt * MX_BN, e);
+                            tma_load_3d(s_dst, mSB, fb, gx, nt * MX_BN, e);
+                        }
+#pragma unroll
+                        for (int i = 0; i < MX_STAGES; ++i)
+                            if (i == stage) last_phase[i] = (int)phase;
+                        if (++stage == MX_STAGES) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
+                    mbar_arrive_expect_tx(fb, MX_STAGE_BYTES);
                     const uint32_t sa_dst = b_dst + MX_B_BYTES;
                     const uint32_t sb_dst = sa_dst + MX_SA_BYTES;
-                    const int kx = kb * MX_BK;
+                    const int kx = kb * BK;
                     const int sx = (kb * 4) & ~15;          // 16-byte box holding the stage's 4 scale bytes
                     tma_load_2d(a_dst, mA, fb, kx, a_row);
                     tma_load_2d(sa_dst, mSA, fb, sx, a_row);
@@ -369,7 +407,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             uint32_t aphase = 0;
             for (int tile = blockIdx.x; tile < total && !mx_aborted(s); tile += gridDim.x) {
                 const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
-                const int nk = K / MX_BK;
+                const int nk = K / BK;
                 if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { mx_fail(s, p, 42); break; }
                 tc_fence_after();
                 const uint32_t dtm = tmem_base + (uint32_t)(ab * MX_BN);
@@ -377,12 +415,19 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&s.sf_full[stage]), phase, p.timeout_ns)) { mx_fail(s, p, 43); ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = base + stage * MX_STAGE_BYTES, b0 = a0 + MX_A_BYTES;
-                    const uint32_t sfa = tmem_base + MX_SF_COL0 + (uint32_t)stage * 8, sfb = sfa + 4;
+                    const uint32_t a0 = base + stage * STAGE_STRIDE, b0 = a0 + MX_A_BYTES;
+                    if (KIND == KIND_W4) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mma_mx(dtm, sdesc(a0 + j * 32), sdesc(b0 + j * 32), mx_idesc(MX_BM, MX_BN, (uint32_t)j),
-                               sfa | ((uint32_t)j << 30), sfb | ((uint32_t)j << 30), (kb | j) ? 1u : 0u);
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16(dtm, sdesc(a0 + j * 32), sdesc(b0 + j * 32), make_idesc_bf16(MX_BM, MX_BN),
+                                     (kb | j) ? 1u : 0u);
+                    } else {
+                        const uint32_t sfa = tmem_base + MX_SF_COL0 + (uint32_t)stage * 8, sfb = sfa + 4;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_mx(dtm, sdesc(a0 + j * 32), sdesc(b0 + j * 32), mx_idesc(MX_BM, MX_BN, (uint32_t)j),
+                                   sfa | ((uint32_t)j << 30), sfb | ((uint32_t)j << 30), (kb | j) ? 1u : 0u);
+                    }
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == MX_STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -402,14 +447,50 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             if (__shfl_sync(0xffffffffu, mx_aborted(s) ? 1 : 0, 0)) break;       // uniform over the warp
             const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
-            const int nk = K / MX_BK;
+            const int nk = K / BK;
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
                 int okw = 1;
                 if (lane == 0) okw = mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns) ? 1 : 0;
                 okw = __shfl_sync(0xffffffffu, okw, 0);
                 if (!okw) { if (lane == 0) mx_fail(s, p, 44); ok = false; break; }
-                const uint32_t sa = base + stage * MX_STAGE_BYTES + MX_A_BYTES + MX_B_BYTES;
+                if (KIND == KIND_W4) {
+                    // row n of the B tile: 64 nibbles -> bf16(q * s) into the 128-byte swizzled row
+                    const int n = (warp - 2) * 32 + lane;
+                    const uint32_t b_dst = base + stage * STAGE_STRIDE + MX_A_BYTES;
+                    const uint32_t c_src = b_dst + MX_B_BYTES + (uint32_t)n * 32;
+                    const uint32_t s_src = b_dst + MX_B_BYTES + W4_CODE_BYTES + (uint32_t)n * 16 +
+                                           (uint32_t)(((kb >> 1) * 2) & 15);
+                    uint32_t c[8];
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3]) : "r"(c_src));
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(c[4]), "=r"(c[5]), "=r"(c[6]), "=r"(c[7]) : "r"(c_src + 16));
+                    unsigned short sb;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sb) : "r"(s_src));
+                    const float sc = __uint_as_float((uint32_t)sb << 16);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {            // 8 bf16 values per 16-byte chunk
+                        const uint32_t word = c[ch];
+                        uint32_t o[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float lo = (float)((int)((word >> (8 * t)) & 15u) - 8) * sc;
+                            const float hi = (float)((int)((word >> (8 * t + 4)) & 15u) - 8) * sc;
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+                            o[t] = *reinterpret_cast<const uint32_t *>(&b2);
+                        }
+                        const uint32_t a = b_dst + (uint32_t)n * 128 + ((uint32_t)(ch ^ (n & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                     ::"r"(a), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&s.sf_full[stage]));
+                    if (++stage == MX_STAGES) { stage = 0; phase ^= 1u; }
+                    continue;
+                }
+                const uint32_t sa = base + stage * STAGE_STRIDE + MX_A_BYTES + MX_B_BYTES;
                 const uint32_t sb = sa + MX_SA_BYTES;
                 const uint32_t byte = (uint32_t)((kb * 4) & 15);
                 uint32_t wa[4], wb[4];
@@ -506,36 +587,43 @@ bool mx_code_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uin
                  uint32_t box_rows) {
     return make_map(m, rank, base, inner, mid, outer, ld, mid * ld, box_rows, 1);
 }
-// Scale map: bytes [outer][mid][inner] (inner = K / 32 scale bytes, rows of
-// sld bytes), box {16 bytes, box_rows(, 1)}, no swizzle.
-bool mx_scale_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
-                  uint64_t sld, uint32_t box_rows) {
+// Byte map: bytes [outer][mid][inner] (rows of ld bytes), box {box_inner
+// bytes, box_rows(, 1)}, no swizzle: MX scale rows (box 16), INT4 code rows
+// (box 32) and INT4 bf16 scale rows (box 16).
+bool byte_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer, uint64_t ld,
+              uint32_t box_inner, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {inner, mid, outer};
-    cuuint64_t strides[2] = {sld, mid * sld};
-    cuuint32_t box[3] = {16, box_rows, 1};
+    cuuint64_t strides[2] = {ld, mid * ld};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+// Scale map: bytes [outer][mid][inner] (inner = K / 32 scale bytes, rows of
+// sld bytes), box {16 bytes, box_rows(, 1)}.
+bool mx_scale_map(CUtensorMap *m, int rank, const void *base, uint64_t inner, uint64_t mid, uint64_t outer,
+                  uint64_t sld, uint32_t box_rows) {
+    return byte_map(m, rank, base, inner, mid, outer, sld, 16, box_rows);
+}
 
 struct MxMaps {
     CUtensorMap A, As, SA, SAs, B, B2, Bs, Bs2, SB, SB2, SBs, SBs2;
 };
 
-template <int MODE>
+template <int MODE, int KIND = KIND_MX>
 cudaError_t launch_mx_gemm(const MxMaps &m, const MxParams &p, int num_sms, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_mx_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(tc_mx_gemm<MODE, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kMxSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_kernel(tc_mx_gemm<MODE>, dim3(num_sms > 0 ? num_sms : 148), dim3(kMxThreads), kMxSmemBytes, st, true,
+    return launch_kernel(tc_mx_gemm<MODE, KIND>, dim3(num_sms > 0 ? num_sms : 148), dim3(kMxThreads), kMxSmemBytes, st, true,
                          m.A, m.As, m.SA, m.SAs, m.B, m.B2, m.Bs, m.Bs2, m.SB, m.SB2, m.SBs, m.SBs2, p);
 }
 
@@ -677,6 +765,102 @@ cudaError_t launch_ffn_mx(const FfnMxArgs &a, cudaStream_t st) {
     p2.shared_a_row = a.shared_base;
     p2.shared_out_row = a.shared_base;
     return launch_mx_gemm<MX_DOWN>(m2, p2, nsm, st);
+}
+
+// INT4 weight-only experts: GEMM 1 (H = act(x W1^T [+ b1]) in bf16 from bf16
+// rows and INT4 weights), GEMM 2 (y_perm = gate * (H W2^T [+ b2])).  The
+// FfnMxArgs fields carry: x_perm / x bf16 rows, W* packed codes [.., N, K/2],
+// W*s bf16 scale bytes [.., N, sld] (one scale per 128 inputs); xs_perm, xs,
+// H8 and Hs are unused.
+cudaError_t launch_ffn_w4(const FfnMxArgs &a, cudaStream_t st) {
+    if (a.routed_rows == 0 && (a.S == 0 || a.T == 0)) return cudaSuccess;
+    if (a.E + 1 > kMxMaxGroups) return cudaErrorInvalidValue;
+    const bool swiglu = a.act == MOE_ACT_SWIGLU;
+    const bool has_sh = a.S > 0 && a.T > 0;
+    const uint64_t routed_rows = (uint64_t)a.routed_rows;
+    const uint64_t all_rows = routed_rows + (has_sh ? (uint64_t)a.T : 0);
+    const int nsm = a.num_sms > 0 ? a.num_sms : 148;
+    const uint64_t sld = (uint64_t)a.sld;
+    const uint32_t bbox = swiglu ? 64 : 128;
+    cudaError_t err;
+
+    // ---- GEMM 1
+    MxMaps m1;
+    const uint64_t ar = routed_rows > 0 ? routed_rows : 1;
+    if (!make_map(&m1.A, 2, a.x_perm, a.d, ar, 1, a.d, 0, 128, 2) ||
+        !byte_map(&m1.B, 3, a.W1, a.d / 2, a.F, a.E, a.d / 2, 32, bbox) ||
+        !byte_map(&m1.SB, 3, a.W1s, a.d / 64, a.F, a.E, sld, 16, bbox))
+        return cudaErrorInvalidValue;
+    m1.SA = m1.SB; m1.SAs = m1.SB;                      // no activation scales
+    if (swiglu) {
+        if (!byte_map(&m1.B2, 3, a.Wu, a.d / 2, a.F, a.E, a.d / 2, 32, bbox) ||
+            !byte_map(&m1.SB2, 3, a.Wus, a.d / 64, a.F, a.E, sld, 16, bbox))
+            return cudaErrorInvalidValue;
+    } else {
+        m1.B2 = m1.B; m1.SB2 = m1.SB;
+    }
+    if (has_sh) {
+        if (!make_map(&m1.As, 2, a.x, a.d, a.T, 1, a.d, 0, 128, 2) ||
+            !byte_map(&m1.Bs, 3, a.Wsg, a.d / 2, a.S, 1, a.d / 2, 32, bbox) ||
+            !byte_map(&m1.SBs, 3, a.Wsgs, a.d / 64, a.S, 1, sld, 16, bbox))
+            return cudaErrorInvalidValue;
+        if (swiglu) {
+            if (!byte_map(&m1.Bs2, 3, a.Wsu, a.d / 2, a.S, 1, a.d / 2, 32, bbox) ||
+                !byte_map(&m1.SBs2, 3, a.Wsus, a.d / 64, a.S, 1, sld, 16, bbox))
+                return cudaErrorInvalidValue;
+        } else {
+            m1.Bs2 = m1.Bs; m1.SBs2 = m1.SBs;
+        }
+    } else {
+        m1.As = m1.A; m1.Bs = m1.B; m1.Bs2 = m1.B2; m1.SBs = m1.SB; m1.SBs2 = m1.SB2;
+    }
+    MxParams p1{};
+    p1.offsets = a.offsets;
+    p1.bias = swiglu ? nullptr : a.b1;
+    p1.out = a.H;
+    p1.ldo = a.hF;
+    p1.status = a.status;
+    p1.timeout_ns = 2000000000ull;
+    p1.E = a.E; p1.T = a.T; p1.has_shared = has_sh ? 1 : 0;
+    p1.K_routed = a.d; p1.K_shared = a.d;
+    p1.N_routed = a.F; p1.N_shared = a.S;
+    p1.shared_a_row = 0;
+    p1.shared_out_row = a.shared_base;
+    err = swiglu ? launch_mx_gemm<MX_SWIGLU, KIND_W4>(m1, p1, nsm, st)
+                 : launch_mx_gemm<MX_GELU, KIND_W4>(m1, p1, nsm, st);
+    if (err != cudaSuccess) return err;
+
+    // ---- GEMM 2 (A: H in bf16)
+    MxMaps m2;
+    const uint64_t hr = all_rows > 0 ? all_rows : 1;
+    if (!make_map(&m2.A, 2, a.H, a.F, hr, 1, a.hF, 0, 128, 2) ||
+        !byte_map(&m2.B, 3, a.W2, a.F / 2, a.d, a.E, a.F / 2, 32, 128) ||
+        !byte_map(&m2.SB, 3, a.W2s, a.F / 64, a.d, a.E, sld, 16, 128))
+        return cudaErrorInvalidValue;
+    m2.SA = m2.SB; m2.SAs = m2.SB; m2.B2 = m2.B; m2.SB2 = m2.SB;
+    if (has_sh) {
+        if (!make_map(&m2.As, 2, a.H, a.S, hr, 1, a.hF, 0, 128, 2) ||
+            !byte_map(&m2.Bs, 3, a.Wsd, a.S / 2, a.d, 1, a.S / 2, 32, 128) ||
+            !byte_map(&m2.SBs, 3, a.Wsds, a.S / 64, a.d, 1, sld, 16, 128))
+            return cudaErrorInvalidValue;
+    } else {
+        m2.As = m2.A; m2.Bs = m2.B; m2.SBs = m2.SB;
+    }
+    m2.Bs2 = m2.Bs; m2.SBs2 = m2.SBs;
+    MxParams p2{};
+    p2.offsets = a.offsets;
+    p2.bias = swiglu ? nullptr : a.b2;
+    p2.row_gate = a.row_gate;
+    p2.out = a.y_perm;
+    p2.ldo = a.d;
+    p2.status = a.status;
+    p2.timeout_ns = 2000000000ull;
+    p2.E = a.E; p2.T = a.T; p2.has_shared = has_sh ? 1 : 0;
+    p2.K_routed = a.F; p2.K_shared = a.S;
+    p2.N_routed = a.d; p2.N_shared = a.d;
+    p2.shared_a_row = a.shared_base;
+    p2.shared_out_row = a.shared_base;
+    return launch_mx_gemm<MX_DOWN, KIND_W4>(m2, p2, nsm, st);
 }
 
 }  // namespace moe

@@ -32,7 +32,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
            "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward",
            "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx",
-           "moe_router_freeze", "moe_forward_mx")
+           "moe_router_freeze", "moe_forward_mx", "moe_grouped_ffn_w4", "moe_forward_w4")
 
 
 class MoeFp8Experts(ctypes.Structure):
@@ -46,6 +46,14 @@ class MoeFp8Experts(ctypes.Structure):
 class MoeMxExperts(ctypes.Structure):
     """moe_mx_experts: block-scaled e4m3 expert weights (device pointers),
     their E8M0 scale bytes and the scale row stride sld."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
+        "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")] + [("sld", ctypes.c_int32)]
+
+
+class MoeW4Experts(ctypes.Structure):
+    """moe_w4_experts: INT4 weight-only expert weights (packed codes), their
+    bf16 group scales (as bytes) and the scale row stride sld."""
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "W1", "W1_scale", "Wu", "Wu_scale", "W2", "W2_scale",
         "Wsh_g", "Wsh_g_scale", "Wsh_u", "Wsh_u_scale", "Wsh_d", "Wsh_d_scale")] + [("sld", ctypes.c_int32)]
@@ -137,6 +145,12 @@ def lib():
             ctypes.c_size_t, c_vp]
         L.moe_router_freeze.restype = ctypes.c_int
         L.moe_router_freeze.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_size_t, c_vp]
+        L.moe_grouped_ffn_w4.restype = ctypes.c_int
+        L.moe_grouped_ffn_w4.argtypes = [P(MoeConfig)] + [c_vp] * 3 + [P(MoeW4Experts)] + [c_vp] * 5 + [
+            ctypes.c_size_t, c_vp]
+        L.moe_forward_w4.restype = ctypes.c_int
+        L.moe_forward_w4.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeW4Experts)] + [c_vp] * 12 + [
+            ctypes.c_size_t, c_vp]
         L.moe_forward_mx.restype = ctypes.c_int
         L.moe_forward_mx.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [P(MoeMxExperts)] + [c_vp] * 12 + [
             ctypes.c_size_t, c_vp, ctypes.c_size_t, c_vp]
@@ -539,6 +553,49 @@ def forward_mx(cfg, inp, wmx, sld, out: Outputs, ws, mx_ws, stream=None):
     moe_forward_mx(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"), wmx, sld,
                    wmx.get("b1"), wmx.get("b2"), out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss,
                    out.logits, out.n_dropped, ws, mx_ws, stream)
+
+
+# ---------------------------------------------------------------- INT4 weight-only experts
+def w4_sld(cfg) -> int:
+    """Smallest valid bf16 scale row stride (bytes) for a configuration."""
+    need = max(cfg.d_model, cfg.d_ff, cfg.d_ff_shared) // 64
+    return (need + 15) // 16 * 16
+
+
+def w4_experts(w, sld) -> MoeW4Experts:
+    """moe_w4_experts from a dict of device tensors: packed codes (uint8) under
+    W1, Wu, W2, Wsg, Wsu, Wsd and bf16 scales as bytes (uint8, rows of sld
+    bytes) under "<name>_scale"."""
+    s = MoeW4Experts()
+    for name in FP8_WEIGHTS:
+        field = _FP8_FIELD[name]
+        setattr(s, field, _p(w.get(name)))
+        setattr(s, field + "_scale", _p(w.get(name + "_scale")))
+    s.sld = int(sld)
+    return s
+
+
+def moe_grouped_ffn_w4(cfg, x_perm, offsets, row_gate, w, sld, b1, b2, x, y_perm, ws, stream=None):
+    ex = w4_experts(w, sld)
+    _check(lib().moe_grouped_ffn_w4(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(row_gate), ctypes.byref(ex),
+                                    _p(b1), _p(b2), _p(x), _p(y_perm), _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_w4")
+
+
+def moe_forward_w4(cfg, x, Wr, logit_bias, sel_bias, w, sld, b1, b2, y, idx, gate, counts, f, P, loss, logits_out,
+                   n_dropped, ws, stream=None):
+    ex = w4_experts(w, sld)
+    _check(lib().moe_forward_w4(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias), ctypes.byref(ex),
+                                _p(b1), _p(b2), _p(y), _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss),
+                                _p(logits_out), _p(n_dropped), _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward_w4")
+
+
+def forward_w4(cfg, inp, w4, sld, out: Outputs, ws, stream=None):
+    """moe_forward_w4 on a dict of device inputs and a dict of INT4 experts."""
+    moe_forward_w4(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"), w4, sld,
+                   w4.get("b1"), w4.get("b2"), out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss,
+                   out.logits, out.n_dropped, ws, stream)
 
 
 def forward_fp8(cfg, inp, w8, out: Outputs, ws, stream=None):

@@ -234,6 +234,53 @@ def generate_mx_experts(wl: Workload, sld: int, device="cpu", seed: int = 0) -> 
     return w
 
 
+def _w4_stack(wl, name, E, rows, cols, sld, device, seed):
+    """E x rows x cols/2 packed INT4 codes (uniform bytes: every nibble uniform
+    over -8..7) and E x rows x sld scale bytes: one bf16 scale per 128 inputs,
+    U(0.5, 1.5) / (3 sqrt(cols)) (so the weights spread like N(0, 1/cols)),
+    bytes past the scales zero."""
+    codes = torch.empty((E, rows, cols // 2), dtype=torch.uint8, device=device)
+    scale = torch.zeros((E, rows, sld), dtype=torch.uint8, device=device)
+    ng = cols // 128
+    for e in range(E):
+        g = _gen(device, seed, wl, name + "_w4", e)
+        codes[e].copy_(torch.randint(0, 256, (rows, cols // 2), generator=g, device=device).to(torch.uint8))
+        s = (torch.rand((rows, ng), generator=g, device=device) + 0.5) / (3.0 * math.sqrt(cols))
+        scale[e, :, :2 * ng].copy_(s.to(torch.bfloat16).view(torch.uint8).reshape(rows, 2 * ng))
+    return codes, scale
+
+
+def generate_w4_experts(wl: Workload, sld: int, device="cpu", seed: int = 0) -> dict:
+    """INT4 weight-only expert weights for a bf16 workload: packed codes
+    (uint8, nn.Linear [out, in/2] layout, low nibble = even input) and bf16
+    group scales as bytes, one per 128 inputs, in rows of sld bytes.  Keys
+    W1, Wu, W2, Wsg, Wsu, Wsd and "<key>_scale" (absent ones None), and for
+    GELU experts the fp32 biases b1, b2 (the same draws as generate()'s)."""
+    dev = torch.device(device)
+    d, E, F = wl.d_model, wl.E, wl.d_ff
+    w = {k: None for k in ("W1", "Wu", "W2", "Wsg", "Wsu", "Wsd")}
+    w.update({k + "_scale": None for k in list(w)})
+    w["W1"], w["W1_scale"] = _w4_stack(wl, "W1", E, F, d, sld, dev, seed)
+    w["W2"], w["W2_scale"] = _w4_stack(wl, "W2", E, d, F, sld, dev, seed)
+    if wl.act == "swiglu":
+        w["Wu"], w["Wu_scale"] = _w4_stack(wl, "Wu", E, F, d, sld, dev, seed)
+    if wl.act == "gelu":
+        g = _gen(dev, seed, wl, "b1")
+        w["b1"] = (torch.rand((E, F), generator=g, device=dev) * 0.02 - 0.01)
+        g = _gen(dev, seed, wl, "b2")
+        w["b2"] = (torch.rand((E, d), generator=g, device=dev) * 0.02 - 0.01)
+    if wl.d_ff_shared:
+        S = wl.d_ff_shared
+        c, s = _w4_stack(wl, "Wsg", 1, S, d, sld, dev, seed)
+        w["Wsg"], w["Wsg_scale"] = c[0], s[0]
+        c, s = _w4_stack(wl, "Wsd", 1, d, S, sld, dev, seed)
+        w["Wsd"], w["Wsd_scale"] = c[0], s[0]
+        if wl.act == "swiglu":
+            c, s = _w4_stack(wl, "Wsu", 1, S, d, sld, dev, seed)
+            w["Wsu"], w["Wsu_scale"] = c[0], s[0]
+    return w
+
+
 def generate_fp8_experts(wl: Workload, device="cpu", seed: int = 0) -> dict:
     """FP8 expert weights for a bf16 workload: e4m3 codes (uint8, nn.Linear
     [out, in] layout) with one fp32 scale per output channel, spread like the
