@@ -40,7 +40,9 @@
 // elements of K); the epilogue multiplies each fp32 accumulator by its row's
 // activation scale and its column's weight scale before the activation or
 // gate (the scales are loaded before the accumulator wait; a column's scale
-// reaches the warp's rows by shuffle).
+// reaches the warp's rows by shuffle in the SwiGLU GEMM, and through a
+// per-warp shared-memory slot read as float4 broadcasts in the others, whose
+// down projection also folds the row's gate into its row scale).
 //
 // Every mbarrier wait is bounded (a global-timer limit); a wait that runs out
 // records MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds,
@@ -121,10 +123,12 @@ struct SmemTail {
 };
 
 // Epilogue staging: one 2 KiB buffer per epilogue warp (32 rows x 32 bf16),
-// 1024-byte aligned after the tail.
+// 1024-byte aligned after the tail, then a 512-byte column-scale slot per
+// epilogue warp (e4m3 tiles).
 constexpr uint32_t STG_BYTES = 32 * 32 * 2;
 constexpr size_t kStgOff = (STAGES * STAGE_BYTES + sizeof(SmemTail) + 1023) / 1024 * 1024;
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStgOff + 8 * STG_BYTES;
+constexpr uint32_t SCL_BYTES = 512;        // e4m3: a warp's 128 column scales
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStgOff + 8 * STG_BYTES + 8 * SCL_BYTES;
 static_assert(kSmemBytes <= 227 * 1024, "1-CTA kernel shared memory");
 
 __device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.f + erff(v * 0.70710678118654752f)); }
@@ -169,7 +173,7 @@ __device__ __forceinline__ void stage_store32(uint32_t stg, const CUtensorMap *t
 
 // The scale of column col0 + lane (0 past N): one coalesced load per warp
 // and 32-column chunk; the epilogue hands each column's scale to every row
-// (lane) with a shuffle.
+// (lane) with a shuffle (SwiGLU) or through the warp's shared-memory slot.
 __device__ __forceinline__ float col_scale_lane(const float *cs, int col0, int N) {
     const int c = col0 + (int)(threadIdx.x & 31);
     return c < N ? __ldg(cs + c) : 0.f;
@@ -209,7 +213,7 @@ template <int MODE, bool F8>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
                                              __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
                                              const CUtensorMap *tmO, uint32_t stg, int row0, float rscale,
-                                             const float *csv) {
+                                             const float *csv, float *scl) {
     float v[128];
     const bool staged = __all_sync(0xffffffffu, valid);
     if (MODE == GM_SWIGLU) {
@@ -239,20 +243,38 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
     } else {
         const int c0 = half * 4;
         tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + (c0 + 2) * 32, taddr + (c0 + 3) * 32, v);
+        if (F8) {
+            const int lane = threadIdx.x & 31;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) scl[j * 32 + lane] = csv[j];
+            __syncwarp();
+        }
+        // no bias: the down projection's gate joins the row scale
+        const float rs = (F8 && MODE == GM_DOWN && bias == nullptr) ? rscale * gscale : rscale;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             const int col0 = nt * BNB + (c0 + cc) * 32;
             if (col0 >= N) continue;                  // uniform over the warp
             float *h = v + cc * 32;                  // in place
             if (F8) {
+                const float4 *c4 = reinterpret_cast<const float4 *>(scl + cc * 32);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) h[i] *= rscale * __shfl_sync(0xffffffffu, csv[cc], i);
+                for (int i = 0; i < 8; ++i) {
+                    const float4 a = c4[i];
+                    h[4 * i] *= a.x * rs; h[4 * i + 1] *= a.y * rs;
+                    h[4 * i + 2] *= a.z * rs; h[4 * i + 3] *= a.w * rs;
+                }
             }
+            if (!F8 || bias != nullptr) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
-                h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
-            }
+                for (int i = 0; i < 32; ++i) {
+                    const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
+                    h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
+                }
+            } else if (MODE == GM_GELU) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] = gelu_erf(h[i]);
+            }                                         // e4m3 down, no bias: the gate is in rs
             if (staged) {
                 stage_store32(stg, tmO, col0, row0, h);
             } else if (valid) {
@@ -435,6 +457,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int half = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
         const uint32_t stg = base + (uint32_t)kStgOff + (uint32_t)(warp - 2) * STG_BYTES;
+        float *scl = reinterpret_cast<float *>(smem + kStgOff + 8 * STG_BYTES + (warp - 2) * SCL_BYTES);
         int ab = 0;
         uint32_t aphase = 0;
         for (int tile = blockIdx.x; tile < total && !aborted(s); tile += gridDim.x) {
@@ -465,7 +488,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, csv);
+                                   rscale, csv, scl);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
@@ -521,10 +544,11 @@ struct PairTail {
 };
 
 constexpr size_t kPairStgOff = (P_STAGES * P_STAGE_BYTES + sizeof(PairTail) + 1023) / 1024 * 1024;
-constexpr size_t kPairSmemBytes = 1024 + kPairStgOff + 8 * STG_BYTES;
+constexpr size_t kPairSmemBytes = 1024 + kPairStgOff + 8 * STG_BYTES + 8 * SCL_BYTES;
 static_assert(kPairSmemBytes <= 227 * 1024, "pair kernel shared memory");
 
-__device__ __forceinline__ void decode_pair(const PairTail &s, int G, int tile, int &g, int &mt, int &nt) {
+template <class Tail>
+__device__ __forceinline__ void decode_pair(const Tail &s, int G, int tile, int &g, int &mt, int &nt) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -536,10 +560,12 @@ __device__ __forceinline__ void decode_pair(const PairTail &s, int G, int tile, 
     nt = local / s.mtiles[g];
 }
 
-__device__ __forceinline__ bool aborted_pair(const PairTail &s) {
+template <class Tail>
+__device__ __forceinline__ bool aborted_pair(const Tail &s) {
     return *reinterpret_cast<const volatile int *>(&s.abort_flag) != 0;
 }
-__device__ __forceinline__ void fail_pair(PairTail &s, const GemmParams &p, int where) {
+template <class Tail>
+__device__ __forceinline__ void fail_pair(Tail &s, const GemmParams &p, int where) {
     record_error(p.status, MOE_ERR_TIMEOUT, where);
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
@@ -684,6 +710,7 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int half = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
         const uint32_t stg = base + (uint32_t)kPairStgOff + (uint32_t)(warp - 2) * STG_BYTES;
+        float *scl = reinterpret_cast<float *>(smem + kPairStgOff + 8 * STG_BYTES + (warp - 2) * SCL_BYTES);
         int ab = 0;
         uint32_t aphase = 0;
         for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
@@ -708,7 +735,381 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
             epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, csv);
+                                   rscale, csv, scl);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
+            if (++ab == 2) { ab = 0; aphase ^= 1u; }
+        }
+        if (lane == 0) tma_store_wait_all();            // the staged stores have landed
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                  // no CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+
+// The bf16 epilogue of one accumulator row with fewer registers than
+// epilogue_row: SwiGLU takes gate and up chunk cc under one TMEM wait, the
+// other modes one 32-column chunk per wait.
+template <int MODE>
+__device__ __forceinline__ void epilogue_row_lean(uint32_t taddr, int half, int nt, bool valid, int N,
+                                               __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
+                                               const CUtensorMap *tmO, uint32_t stg, int row0) {
+    const bool staged = __all_sync(0xffffffffu, valid);
+    if (MODE == GM_SWIGLU) {
+        const int c0 = half * 2;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            float v[64];
+            tmem_ld32x2(taddr + (c0 + cc) * 32, taddr + 128 + (c0 + cc) * 32, v);   // gate, up
+            const int col0 = nt * 128 + (c0 + cc) * 32;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * v[32 + i];
+            if (staged) {
+                if (col0 < N) stage_store32(stg, tmO, col0, row0, v);
+            } else if (valid) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, v + u * 8);
+            }
+        }
+    } else {
+        const int c0 = half * 4;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(taddr + (c0 + cc) * 32, v);
+            {
+                const int col0 = nt * BNB + (c0 + cc) * 32;
+                if (col0 >= N) continue;                  // uniform over the warp
+                float *h = v;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
+                    h[i] = (MODE == GM_GELU) ? gelu_erf(z) : gscale * z;
+                }
+                if (staged) {
+                    stage_store32(stg, tmO, col0, row0, h);
+                } else if (valid) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (col0 + u * 8 < N) store8(orow_ptr + col0 + u * 8, h + u * 8);
+                }
+            }
+        }
+    }
+}
+
+// ============================================================================
+// INT4 weight-only experts on CTA pairs: the pair kernel above with its B
+// operand decoded on the chip.  The TMA producer brings only A (this CTA's
+// 128 rows, two 64-deep bf16 atoms per stage, on the first CTA's barrier as in
+// the bf16 pair kernel).  The decode warps of each CTA (four: warp w owns B
+// rows 32w .. 32w + 31 of the CTA's half) read their rows' packed codes (64
+// bytes a row per stage) and bf16 group scale straight from global memory one
+// stage ahead into registers; once the MMA has freed a stage they write its
+// two bf16 B atoms in the 128-byte swizzled layout -- bf16(q * s), rounded
+// once --, fence them for the tensor core and report to the first CTA, whose
+// MMA thread starts once the stage's A has landed and every decode warp of
+// the pair has reported.  The decode thus overlaps the A loads instead of
+// following them.  Roles: warp 0 TMA, warp 1 MMA (first CTA), warps 2-9
+// epilogue (the bf16 pair kernel's with fewer registers, so that 14 warps
+// fit), warps 10-13 decode (one per SM sub-partition).
+constexpr int W4P_STAGES = 3;
+constexpr int W4P_DEC_WARPS = 4;                                // decode warps per CTA: 4 or 8
+constexpr int W4P_DEC_ATOMS = P_ATOMS * 4 / W4P_DEC_WARPS;      // B atoms a decode warp writes per stage
+constexpr int kW4Threads = (10 + W4P_DEC_WARPS) * 32;
+constexpr uint32_t W4P_A_STAGE = P_ATOMS * P_A_BYTES;           // 32 KiB: two A atoms
+constexpr uint32_t W4P_B_STAGE = P_ATOMS * P_B_BYTES;           // 32 KiB: two decoded B atoms
+
+// Packed INT4 weights of one GEMM: codes [.., N, K/2] bytes (low nibble = even
+// input, nibble = q + 8), scales [.., N, sld] bytes (one bf16 per 128 inputs).
+struct W4Ptrs {
+    const uint8_t *c, *c2, *cs, *cs2;      // codes: routed, routed SwiGLU up, shared, shared up
+    const uint8_t *sc, *sc2, *scs, *scs2;  // scale rows, the same four
+    int64_t sld;
+};
+
+struct W4PairTail {
+    uint64_t full[W4P_STAGES];        // first CTA's: both CTAs' A landed
+    uint64_t ready[W4P_STAGES];       // first CTA's: the pair's decode warps wrote B
+    uint64_t empty[W4P_STAGES];
+    uint64_t accf[2];
+    uint64_t acce[2];                 // first CTA's: 8 warps x 2 CTAs
+    uint32_t tmem_base;
+    int abort_flag;
+    int tile_start[kMaxGroups + 1];
+    int mtiles[kMaxGroups];
+    int rows[kMaxGroups];
+    int row0[kMaxGroups];
+};
+constexpr size_t kW4TailOff = (size_t)W4P_STAGES * (W4P_A_STAGE + W4P_B_STAGE);
+constexpr size_t kW4StgOff = (kW4TailOff + sizeof(W4PairTail) + 1023) / 1024 * 1024;
+constexpr size_t kW4SmemBytes = 1024 + kW4StgOff + 8 * STG_BYTES;
+static_assert(kW4SmemBytes <= 227 * 1024, "INT4 pair kernel shared memory");
+
+// One decode warp's view of a tile: where its row's codes and scales start.
+struct W4Row {
+    const uint8_t *code;     // this thread's row, stage 0 (null past the weight's rows)
+    const uint8_t *scale;
+    int nk;                  // stages of the tile
+};
+
+template <int MODE>
+__device__ __forceinline__ W4Row w4_row(const W4PairTail &s, const GemmParams &p, const W4Ptrs &w, int G, int tile,
+                                        uint32_t rank, int n) {
+    int g, mt, nt;
+    decode_pair(s, G, tile, g, mt, nt);
+    const bool sh = g >= p.E;
+    const bool up = MODE == GM_SWIGLU && rank == 1;
+    const int K = sh ? p.K_shared : p.K_routed;
+    const int N = sh ? p.N_shared : p.N_routed;
+    const int e = sh ? 0 : group_expert(p, g);
+    const int row = ((MODE == GM_SWIGLU) ? nt * 128 : nt * BNB + (int)rank * 128) + n;
+    W4Row r;
+    r.nk = K / (P_ATOMS * BK);
+    if (row < N) {
+        const int64_t er = (int64_t)e * N + row;
+        r.code = (sh ? (up ? w.cs2 : w.cs) : (up ? w.c2 : w.c)) + er * (K / 2);
+        r.scale = (sh ? (up ? w.scs2 : w.scs) : (up ? w.sc2 : w.sc)) + er * w.sld;
+    } else {
+        r.code = nullptr;
+        r.scale = nullptr;
+    }
+    return r;
+}
+
+// Stage kb of a row, atoms atom0 .. atom0 + W4P_DEC_ATOMS - 1: 32 code bytes
+// (64 inputs) per atom and the stage's group scale; zeros past the weight's
+// rows (decoding to zeros).
+__device__ __forceinline__ void w4_fetch(const W4Row &r, int kb, int atom0, uint4 *c, uint32_t &s2) {
+    if (r.code) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(r.code + (int64_t)kb * 64 + atom0 * 32);
+#pragma unroll
+        for (int j = 0; j < 2 * W4P_DEC_ATOMS; ++j) c[j] = __ldg(src + j);
+        s2 = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(r.scale) + kb) * 0x10001u;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 2 * W4P_DEC_ATOMS; ++j) c[j] = make_uint4(0u, 0u, 0u, 0u);
+        s2 = 0u;
+    }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kW4Threads, 1)
+tc_w4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                const __grid_constant__ CUtensorMap tmO, const GemmParams p, const W4Ptrs w) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    W4PairTail &s = *reinterpret_cast<W4PairTail *>(smem + kW4TailOff);
+    const uint32_t smA = base;                                      // stages x 32 KiB
+    const uint32_t smB = base + W4P_STAGES * W4P_A_STAGE;           // stages x 32 KiB
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = (int)cluster_id_x(), npairs = (int)ncluster_x();
+    constexpr int BNO = (MODE == GM_SWIGLU) ? 128 : 256;
+    constexpr int BKS = P_ATOMS * BK;                               // 128 of K per stage
+    const int G = p.E + (p.has_shared ? 1 : 0);
+
+    if (tid == 0) {
+        s.abort_flag = 0;
+        for (int i = 0; i < W4P_STAGES; ++i) {
+            mbar_init(smem_u32(&s.full[i]), 1);
+            mbar_init(smem_u32(&s.ready[i]), 2 * W4P_DEC_WARPS);
+            mbar_init(smem_u32(&s.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&s.accf[i]), 1); mbar_init(smem_u32(&s.acce[i]), 16); }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(&s.tmem_base), TMEM_COLS);
+    if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+    pdl_wait_then_release();
+    if (tid == 0) s.tile_start[0] = 0;
+    for (int g = tid; g < G; g += kW4Threads) {
+        const bool sh = g >= p.E;
+        const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        const int n = sh ? p.N_shared : p.N_routed;
+        const int mt = rows / PM + ((rows % PM) > BM ? 1 : 0);
+        s.rows[g] = rows;
+        s.row0[g] = sh ? 0 : p.offsets[g];
+        s.mtiles[g] = mt > 0 ? mt : 1;
+        s.tile_start[g + 1] = mt * ((n + BNO - 1) / BNO);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            int v = g < G ? s.tile_start[g + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (g < G) s.tile_start[g + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    tc_fence_before();
+    cluster_sync();                                  // barriers of both CTAs initialised
+    tc_fence_after();
+    const int total = s.tile_start[G];
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == 0) {
+        // ================= TMA producer of A (both CTAs, bytes on the first CTA's barrier)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+                int g, mt, nt;
+                decode_pair(s, G, tile, g, mt, nt);
+                const bool sh = g >= p.E;
+                const int nk = (sh ? p.K_shared : p.K_routed) / BKS;
+                const int a_row = (sh ? (int)p.shared_a_row : s.row0[g]) + mt * PM + (int)rank * BM;
+                const CUtensorMap *mA = sh ? &tmAs : &tmA;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 61); break; }
+                    const uint32_t fb = mapa_shared(smem_u32(&s.full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * W4P_A_STAGE);
+#pragma unroll
+                    for (int at = 0; at < P_ATOMS; ++at)
+                        tma_load_2d_pair(smA + stage * W4P_A_STAGE + at * P_A_BYTES, mA, fb, kb * BKS + at * BK, a_row);
+                    if (++stage == W4P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer (first CTA only): the stage's A landed and its B decoded
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int ab = 0;
+            uint32_t aphase = 0;
+            for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+                const int K = tile >= s.tile_start[p.E] ? p.K_shared : p.K_routed;
+                const int nk = K / BKS;
+                if (!mbar_wait(smem_u32(&s.acce[ab]), aphase ^ 1u, p.timeout_ns)) { fail_pair(s, p, 62); break; }
+                tc_fence_after();
+                const uint32_t dtm = tmem_base + (uint32_t)(ab * BNB);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, p.timeout_ns) ||
+                        !mbar_wait(smem_u32(&s.ready[stage]), phase, p.timeout_ns)) {
+                        fail_pair(s, p, 63);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < P_ATOMS * (BK / 16); ++kk) {
+                        const int at = kk / (BK / 16), k = kk % (BK / 16);
+                        const uint32_t a0 = smA + stage * W4P_A_STAGE + at * P_A_BYTES;
+                        const uint32_t b0 = smB + stage * W4P_B_STAGE + at * P_B_BYTES;
+                        mma_bf16_pair(dtm, sdesc(a0 + k * 32), sdesc(b0 + k * 32), kIdescPair, (kb | kk) ? 1u : 0u);
+                    }
+                    mma_commit_pair(smem_u32(&s.empty[stage]), (uint16_t)0x3);
+                    if (++stage == W4P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit_pair(smem_u32(&s.accf[ab]), (uint16_t)0x3);
+                if (++ab == 2) { ab = 0; aphase ^= 1u; }
+            }
+        }
+    } else if (warp >= 10) {
+        // ================= decode (both CTAs): warp 10 + w owns B rows 32 (w % 4) .. + 31 and
+        // atoms (w / 4) W4P_DEC_ATOMS .. + W4P_DEC_ATOMS - 1 of each stage
+        const int dw = warp - 10;
+        const int n = (dw & 3) * 32 + lane;
+        const int atom0 = (dw >> 2) * W4P_DEC_ATOMS;
+        int stage = 0;
+        uint32_t phase = 0;
+        int tile = pair, kb = 0;
+        if (tile < total) {
+            W4Row row = w4_row<MODE>(s, p, w, G, tile, rank, n);
+            uint4 c[2 * W4P_DEC_ATOMS];
+            uint32_t s2;
+            w4_fetch(row, 0, atom0, c, s2);
+            while (true) {
+                // the next stage's codes travel while this one is decoded
+                int tile_n = tile, kb_n = kb + 1;
+                W4Row row_n = row;
+                if (kb_n == row.nk) {
+                    tile_n = tile + npairs;
+                    kb_n = 0;
+                    if (tile_n < total) row_n = w4_row<MODE>(s, p, w, G, tile_n, rank, n);
+                }
+                uint4 cn[2 * W4P_DEC_ATOMS];
+                uint32_t s2n = 0u;
+                if (tile_n < total) w4_fetch(row_n, kb_n, atom0, cn, s2n);
+                int okw = 1;
+                if (lane == 0)
+                    okw = (!aborted_pair(s) && mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1u, p.timeout_ns)) ? 1 : 0;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) { if (lane == 0 && !aborted_pair(s)) fail_pair(s, p, 64); break; }
+                const uint32_t bst = smB + stage * W4P_B_STAGE;
+                const uint32_t *cw = reinterpret_cast<const uint32_t *>(c);
+#pragma unroll
+                for (int q = 0; q < 8 * W4P_DEC_ATOMS; ++q) {   // word q: inputs 8q .. of the warp's atoms
+                    uint32_t o[4];
+                    w4_decode8(cw[q], s2, o);
+                    const uint32_t a = bst + (uint32_t)(atom0 + (q >> 3)) * P_B_BYTES + (uint32_t)n * 128 +
+                                       ((uint32_t)((q & 7) ^ (n & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 ::"r"(a), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.ready[stage]), 0));
+                if (++stage == W4P_STAGES) { stage = 0; phase ^= 1u; }
+                if (tile_n >= total) break;
+                tile = tile_n;
+                kb = kb_n;
+                row = row_n;
+#pragma unroll
+                for (int j = 0; j < 2 * W4P_DEC_ATOMS; ++j) c[j] = cn[j];
+                s2 = s2n;
+            }
+        }
+    } else {
+        // ================= epilogue (both CTAs), warps 2..9 as in the bf16 pair kernel
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int r_in_tile = q * 32 + lane;
+        const uint32_t stg = base + (uint32_t)kW4StgOff + (uint32_t)(warp - 2) * STG_BYTES;
+        int ab = 0;
+        uint32_t aphase = 0;
+        for (int tile = pair; tile < total && !aborted_pair(s); tile += npairs) {
+            int g, mt, nt;
+            decode_pair(s, G, tile, g, mt, nt);
+            const bool sh = g >= p.E;
+            const int grow = mt * PM + (int)rank * BM + r_in_tile;
+            const bool valid = grow < s.rows[g];
+            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            float gscale = 1.f;
+            if (MODE == GM_DOWN && !sh && valid) gscale = __ldg(p.row_gate + orow);
+            const int N = sh ? p.N_shared : p.N_routed;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(smem_u32(&s.accf[ab]), aphase, p.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { if (lane == 0) fail_pair(s, p, 67); break; }
+            __syncwarp();
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
+            __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
+            const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
+            epilogue_row_lean<MODE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
@@ -982,6 +1383,69 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
 }
 
 }  // namespace
+
+namespace {
+
+template <int MODE>
+cudaError_t launch_w4_pair_mode(const W4PairArgs &a, const CUtensorMap &O, const GemmParams &p, cudaStream_t st) {
+    static int grid = 0;
+    if (grid == 0) {
+        cudaError_t e = cudaFuncSetAttribute(tc_w4_gemm_pair<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kW4SmemBytes);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (a.num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(kW4Threads, 1, 1);
+        cfg.dynamicSmemBytes = kW4SmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_w4_gemm_pair<MODE>, &cfg);
+        if (e != cudaSuccess || nclusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        grid = 2 * nclusters;
+    }
+    W4Ptrs w{};
+    w.c = a.c; w.c2 = a.c2; w.cs = a.cs; w.cs2 = a.cs2;
+    w.sc = a.sc; w.sc2 = a.sc2; w.scs = a.scs; w.scs2 = a.scs2;
+    w.sld = a.sld;
+    return launch_kernel(tc_w4_gemm_pair<MODE>, dim3(grid), dim3(kW4Threads), kW4SmemBytes, st, a.pdl, a.A, a.As, O,
+                         p, w);
+}
+
+}  // namespace
+
+cudaError_t launch_w4_gemm_pair(const W4PairArgs &a, cudaStream_t st) {
+    if (a.K_routed % 128 != 0 || (a.has_shared && a.K_shared % 128 != 0) || a.E + 1 > kMaxGroups)
+        return cudaErrorInvalidValue;
+    CUtensorMap O;
+    if (!make_store_map(&O, a.out, a.out_cols, a.out_rows > 0 ? a.out_rows : 1, (uint64_t)a.ldo))
+        return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.offsets = a.offsets;
+    p.bias = a.bias;
+    p.row_gate = a.row_gate;
+    p.out = a.out;
+    p.status = a.status;
+    p.E = a.E; p.E_w = a.E; p.T = a.T;
+    p.K_routed = a.K_routed; p.K_shared = a.K_shared;
+    p.N_routed = a.N_routed; p.N_shared = a.N_shared;
+    p.has_shared = a.has_shared;
+    p.ldo = a.ldo;
+    p.shared_a_row = a.shared_a_row;
+    p.shared_out_row = a.shared_out_row;
+    p.timeout_ns = 2000000000ull;
+    switch (a.mode) {
+        case GM_SWIGLU: return launch_w4_pair_mode<GM_SWIGLU>(a, O, p, st);
+        case GM_GELU: return launch_w4_pair_mode<GM_GELU>(a, O, p, st);
+        case GM_DOWN: return launch_w4_pair_mode<GM_DOWN>(a, O, p, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_ffn_bf16(const FfnArgs &a, cudaStream_t st) {
     if (a.routed_rows == 0 && (a.S == 0 || a.T == 0)) return cudaSuccess;

@@ -186,6 +186,33 @@ cudaError_t launch_ffn_mx(const FfnMxArgs &a, cudaStream_t st);
 // stays bf16 between the GEMMs.  mx_sm100.cu.
 cudaError_t launch_ffn_w4(const FfnMxArgs &a, cudaStream_t st);
 
+// One GEMM of the INT4 weight-only grouped FFN on CTA pairs (M = 256, N =
+// 256): every group's 256-row blocks and a last block of more than 128 rows
+// (a last block of 1..128 rows is left to the 1-CTA kernel).  A / As: TMA
+// maps of the bf16 activations (128-byte swizzle, box 64 x 128).  Packed
+// weights: codes [.., N, K/2] bytes and bf16 scale bytes [.., N, sld], read by
+// the kernel's decode warps: c / sc routed (SwiGLU: the gate projection),
+// c2 / sc2 the SwiGLU up projection, cs* the shared expert's.  out: bf16
+// [out_rows, out_cols] with row stride ldo.  mode: 0 SwiGLU, 1 GELU (+ bias),
+// 2 down (+ bias, times row_gate).  ffn_sm100.cu.
+struct W4PairArgs {
+    CUtensorMap A, As;
+    const uint8_t *c, *c2, *cs, *cs2;
+    const uint8_t *sc, *sc2, *scs, *scs2;
+    int64_t sld;
+    const int32_t *offsets;
+    const float *bias;           // [E, N_routed] or null
+    const float *row_gate;       // mode 2: [rows]
+    __nv_bfloat16 *out;
+    uint64_t out_cols, out_rows;
+    int32_t *status;
+    int mode, E, T, has_shared, K_routed, K_shared, N_routed, N_shared, ldo;
+    int64_t shared_a_row, shared_out_row;
+    int num_sms;
+    bool pdl;
+};
+cudaError_t launch_w4_gemm_pair(const W4PairArgs &a, cudaStream_t st);
+
 // Per-row e4m3 quantization of bf16 rows (row0 + r for r < rows, or fewer
 // when rows_limit points at a smaller device count): in [.., ld_in] bf16,
 // out [.., ld_out] e4m3 codes, scale [..] fp32.  cols % 8 == 0.

@@ -180,6 +180,8 @@ struct MxParams {
     int N_routed, N_shared;      // output columns
     int64_t shared_a_row;        // first A row of the shared group in the shared maps
     int64_t shared_out_row;      // first output row of the shared group
+    int tail_mode;               // 1: only a group's last rows when rows % 256 is in 1..128
+                                 // (the CTA-pair INT4 kernel runs the rest)
 };
 
 struct MxSmem {
@@ -287,15 +289,25 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) tmem_alloc(smem_u32(&s.tmem_base), MX_TMEM_COLS);
-    pdl_wait_then_release();
+    // Last blocks (tail mode) touch only rows the CTA-pair launch before them
+    // leaves alone and read only what the kernel before that wrote, so they
+    // start at once and wait for the pair launch only before exiting.
+    if (p.tail_mode) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    else pdl_wait_then_release();
     if (tid == 0) s.tile_start[0] = 0;
     for (int g = tid; g < G; g += kMxThreads) {
         const bool sh = g >= p.E;
-        const int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        int rows = sh ? p.T : p.offsets[g + 1] - p.offsets[g];
+        int start = 0;
+        if (p.tail_mode) {
+            const int rem = rows % (2 * MX_BM);
+            start = rows - rem;
+            rows = (rem > 0 && rem <= MX_BM) ? rem : 0;
+        }
         const int n = sh ? p.N_shared : p.N_routed;
         const int mt = (rows + MX_BM - 1) / MX_BM;
         s.rows[g] = rows;
-        s.row0[g] = sh ? 0 : p.offsets[g];
+        s.row0[g] = sh ? start : p.offsets[g] + start;      // the shared group: offset past shared_*_row
         s.mtiles[g] = mt > 0 ? mt : 1;
         s.tile_start[g + 1] = mt * ((n + OUT_COLS - 1) / OUT_COLS);
     }
@@ -334,7 +346,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 const bool sh = g >= p.E;
                 const int K = sh ? p.K_shared : p.K_routed;
                 const int nk = K / BK;
-                const int a_row = sh ? (int)p.shared_a_row + mt * MX_BM : s.row0[g] + mt * MX_BM;
+                const int a_row = sh ? (int)p.shared_a_row + s.row0[g] + mt * MX_BM : s.row0[g] + mt * MX_BM;
                 const int e = sh ? 0 : g;
                 const CUtensorMap *mA = sh ? &tmAs : &tmA, *mSA = sh ? &tmSAs : &tmSA;
                 const CUtensorMap *mB = sh ? &tmBs : &tmB, *mB2 = sh ? &tmBs2 : &tmB2;
@@ -468,18 +480,13 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                                  : "=r"(c[4]), "=r"(c[5]), "=r"(c[6]), "=r"(c[7]) : "r"(c_src + 16));
                     unsigned short sb;
                     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sb) : "r"(s_src));
-                    const float sc = __uint_as_float((uint32_t)sb << 16);
+                    const uint32_t s2 = (uint32_t)sb * 0x10001u;   // the scale in both bf16 halves
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {            // 8 bf16 values per 16-byte chunk
+                        // word = inputs 8ch .. 8ch+7, input i in bits 4i .. 4i+3
                         const uint32_t word = c[ch];
                         uint32_t o[4];
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const float lo = (float)((int)((word >> (8 * t)) & 15u) - 8) * sc;
-                            const float hi = (float)((int)((word >> (8 * t + 4)) & 15u) - 8) * sc;
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
-                            o[t] = *reinterpret_cast<const uint32_t *>(&b2);
-                        }
+                        w4_decode8(word, s2, o);
                         const uint32_t a = b_dst + (uint32_t)n * 128 + ((uint32_t)(ch ^ (n & 7)) << 4);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
                                      ::"r"(a), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
@@ -525,7 +532,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             const int grow = mt * MX_BM + q * 32 + lane;
             const bool valid = grow < s.rows[g];
             const int nrows = __popc(__ballot_sync(0xffffffffu, valid));
-            const int64_t orow = sh ? p.shared_out_row + grow : (int64_t)s.row0[g] + grow;
+            const int64_t orow = sh ? p.shared_out_row + s.row0[g] + grow : (int64_t)s.row0[g] + grow;
             const int64_t orow0 = orow - lane;
             float gscale = 1.f;
             if (MODE == MX_DOWN && !sh && valid && p.row_gate) gscale = __ldg(p.row_gate + orow);
@@ -578,6 +585,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         tc_fence_after();
         tmem_dealloc(tmem_base, MX_TMEM_COLS);
     }
+    if (p.tail_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ host side
@@ -826,6 +834,33 @@ cudaError_t launch_ffn_w4(const FfnMxArgs &a, cudaStream_t st) {
     p1.N_routed = a.F; p1.N_shared = a.S;
     p1.shared_a_row = 0;
     p1.shared_out_row = a.shared_base;
+    // CTA pairs over the 256-row blocks (and a last block of > 128 rows) ...
+    W4PairArgs w1{};
+    w1.A = m1.A; w1.As = m1.As;
+    w1.c = a.W1; w1.sc = a.W1s;
+    w1.c2 = swiglu ? a.Wu : a.W1; w1.sc2 = swiglu ? a.Wus : a.W1s;
+    w1.cs = has_sh ? a.Wsg : a.W1; w1.scs = has_sh ? a.Wsgs : a.W1s;
+    w1.cs2 = has_sh && swiglu ? a.Wsu : w1.cs; w1.scs2 = has_sh && swiglu ? a.Wsus : w1.scs;
+    w1.sld = (int64_t)sld;
+    w1.offsets = a.offsets;
+    w1.bias = p1.bias;
+    w1.row_gate = nullptr;
+    w1.out = a.H;
+    w1.out_cols = (uint64_t)a.hF;
+    w1.out_rows = all_rows;
+    w1.status = a.status;
+    w1.mode = swiglu ? 0 : 1;
+    w1.E = a.E; w1.T = a.T; w1.has_shared = p1.has_shared;
+    w1.K_routed = a.d; w1.K_shared = a.d;
+    w1.N_routed = a.F; w1.N_shared = a.S;
+    w1.ldo = a.hF;
+    w1.shared_a_row = 0;
+    w1.shared_out_row = a.shared_base;
+    w1.num_sms = nsm;
+    w1.pdl = true;
+    if ((err = launch_w4_gemm_pair(w1, st)) != cudaSuccess) return err;
+    // ... then one CTA per SM over the last blocks of 1..128 rows
+    p1.tail_mode = 1;
     err = swiglu ? launch_mx_gemm<MX_SWIGLU, KIND_W4>(m1, p1, nsm, st)
                  : launch_mx_gemm<MX_GELU, KIND_W4>(m1, p1, nsm, st);
     if (err != cudaSuccess) return err;
@@ -860,6 +895,30 @@ cudaError_t launch_ffn_w4(const FfnMxArgs &a, cudaStream_t st) {
     p2.N_routed = a.d; p2.N_shared = a.d;
     p2.shared_a_row = a.shared_base;
     p2.shared_out_row = a.shared_base;
+    W4PairArgs w2{};
+    w2.A = m2.A; w2.As = m2.As;
+    w2.c = a.W2; w2.sc = a.W2s;
+    w2.cs = has_sh ? a.Wsd : a.W2; w2.scs = has_sh ? a.Wsds : a.W2s;
+    w2.c2 = w2.c; w2.sc2 = w2.sc; w2.cs2 = w2.cs; w2.scs2 = w2.scs;
+    w2.sld = (int64_t)sld;
+    w2.offsets = a.offsets;
+    w2.bias = p2.bias;
+    w2.row_gate = a.row_gate;
+    w2.out = a.y_perm;
+    w2.out_cols = (uint64_t)a.d;
+    w2.out_rows = all_rows;
+    w2.status = a.status;
+    w2.mode = 2;
+    w2.E = a.E; w2.T = a.T; w2.has_shared = p2.has_shared;
+    w2.K_routed = a.F; w2.K_shared = a.S;
+    w2.N_routed = a.d; w2.N_shared = a.d;
+    w2.ldo = a.d;
+    w2.shared_a_row = a.shared_base;
+    w2.shared_out_row = a.shared_base;
+    w2.num_sms = nsm;
+    w2.pdl = true;
+    if ((err = launch_w4_gemm_pair(w2, st)) != cudaSuccess) return err;
+    p2.tail_mode = 1;
     return launch_mx_gemm<MX_DOWN, KIND_W4>(m2, p2, nsm, st);
 }
 

@@ -207,6 +207,12 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Arrive on a barrier of this cluster with release semantics at cluster
+// scope: this thread's earlier shared-memory writes are visible to whoever
+// acquires the barrier's phase in the other CTA.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 
 // ---------------------------------------------------------------- TMA stores
 // Shared -> global tensor store of one box (bulk-group completion).
@@ -221,5 +227,28 @@ __device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.b
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Order this thread's shared-memory writes before later async-proxy (TMA) reads.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---------------------------------------------------------------- INT4 weights
+// Eight INT4 weights (one 32-bit code word, nibble i = input i, stored as
+// q + 8) -> four bf16x2 words bf16(q * s), inputs (0,1) (2,3) (4,5) (6,7).
+// A nibble u placed in the low mantissa bits of bf16 128 (0x4300) reads as
+// 128 + u; subtracting 136 leaves q exactly, and one bf16 multiply by the
+// scale rounds q * s once to nearest even.  Masking the word shifted by 4j
+// with 0x000F000F yields inputs (j, j + 4) in one bf16x2; byte permutes pair
+// the neighbours.
+__device__ __forceinline__ void w4_decode8(uint32_t word, uint32_t s2, uint32_t *o) {
+    uint32_t t[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t x = ((word >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+        uint32_t q;
+        asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(x), "r"(0x43084308u));       // 136 in both halves
+        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t[j]) : "r"(q), "r"(s2));
+    }
+    o[0] = __byte_perm(t[0], t[1], 0x5410);
+    o[1] = __byte_perm(t[2], t[3], 0x5410);
+    o[2] = __byte_perm(t[0], t[1], 0x7632);
+    o[3] = __byte_perm(t[2], t[3], 0x7632);
+}
 
 }  // namespace moe
