@@ -59,6 +59,10 @@ struct Vec16<float> {
 constexpr int kCombThreads = 256;
 
 // One warp per token (grid-stride); lanes stride over 16-byte column vectors.
+// The row is taken in blocks of 256 vectors (4 KiB of bf16): for each block,
+// each slot's part arrives in one burst of eight 16-byte loads per lane and
+// joins the fp32 sums in slot order (then the shared expert's row), so the
+// sum order -- and the result -- is that of a plain per-element loop.
 template <typename TY>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     pdl_wait_then_release();
@@ -80,20 +84,31 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
         const int64_t shared_row = a.rows_routed + t;
         // every lane runs the column loop (the row indices come by shuffle
         // from lanes 0..k-1); lanes past the row's last vector only idle
-        for (int v0 = 0; v0 < nvec; v0 += 32) {
-            const int v = v0 + lane;
-            const bool in_row = v < nvec;
-            float acc[V::N];
+        for (int vb = 0; vb < nvec; vb += 256) {
+            float acc[8][V::N];
 #pragma unroll
-            for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
-#pragma unroll 4
-            for (int s = 0; s < a.k; ++s) {
-                const int r = __shfl_sync(0xffffffffu, my_row, s);
-                if (in_row && r >= 0) V::add(__ldg(yp + (size_t)r * nvec + v), acc);
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int i = 0; i < V::N; ++i) acc[j][i] = 0.f;
+            for (int s = 0; s <= a.k; ++s) {
+                int64_t r;
+                if (s < a.k) r = __shfl_sync(0xffffffffu, my_row, s);
+                else r = a.has_shared ? shared_row : -1;
+                if (r < 0) continue;                                    // the same on every lane
+                uint4 q[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int v = vb + 32 * j + lane;
+                    if (v < nvec) q[j] = __ldg(yp + (size_t)r * nvec + v);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (vb + 32 * j + lane < nvec) V::add(q[j], acc[j]);
             }
-            if (in_row) {
-                if (a.has_shared) V::add(__ldg(yp + (size_t)shared_row * nvec + v), acc);
-                y[(size_t)t * nvec + v] = V::pack(acc);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int v = vb + 32 * j + lane;
+                if (v < nvec) y[(size_t)t * nvec + v] = V::pack(acc[j]);
             }
         }
     }
