@@ -599,7 +599,9 @@ def backward_record(args, wl, dev, world):
     L2 flushed between them.  Algorithmic FLOPs: the expert contractions'
     input and weight gradients (2 x the forward's expert FLOPs) plus the
     router's two gradient contractions (2 x 2 T d E); the pre-activation
-    recompute the implementation adds is not counted."""
+    recompute the implementation adds is not counted.  Then K training steps
+    (moe_forward_train + moe_backward, the forward handing its expert
+    pre-activations to the backward), timed per half."""
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     inp = syn.generate(wl, dev, seed=0)
@@ -636,9 +638,37 @@ def backward_record(args, wl, dev, world):
     peaks, peak_src = load_peaks()
     peak_t, which = tensor_peak(peaks, clocks)
     tf = flops / (ms * 1e-3) / 1e12
+
+    # a training step: moe_forward_train (the forward that also leaves the
+    # expert pre-activations in the backward workspace) and moe_backward
+    def train_step(evs):
+        evs[0].record(stream)
+        nat.forward_train(cfg, inp, out, ws, bws, stream)
+        evs[1].record(stream)
+        nat.backward(cfg, inp, out, ws, dy, 0.01, ws=bws, stream=stream)
+        evs[2].record(stream)
+
+    ev3 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.sub_steps)]
+    for _ in range(3):
+        flush.zero_()
+        train_step(ev3[0])
+    torch.cuda.synchronize(dev)
+    if nat.moe_get_device_status(ws, stream) != nat.MOE_OK:
+        raise RuntimeError("device status after the training-step warm-up")
+    for i in range(args.sub_steps):
+        flush.zero_()
+        train_step(ev3[i])
+    torch.cuda.synchronize(dev)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev3) / args.sub_steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev3) / args.sub_steps
+    fwd_ms, bwd_ms = max_over_ranks([fwd_ms, bwd_ms], world, dev)
     return {"workload": wl.name, "pass": "backward (dx, dW_r, d logit offset, all expert weight gradients)",
             "steps": args.sub_steps, "warmup": 3, "ms_per_step": ms,
             "tokens_per_s": job_tokens_per_s(world, wl.T, ms), "tflops": tf,
+            "training_step": {"entry": "moe_forward_train + moe_backward (pre-activations handed over, no recompute)",
+                              "ms_per_step": fwd_ms + bwd_ms, "forward_ms": fwd_ms, "backward_ms": bwd_ms,
+                              "backward_tflops": flops / (bwd_ms * 1e-3) / 1e12,
+                              "backward_frac": flops / (bwd_ms * 1e-3) / 1e12 / peak_t},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_t, "unit": "TFLOP/s", "frac": tf / peak_t,
                          "flops": flops, "peak_note": "%s bf16 peak, %s" % (which, "of measured" if peak_src ==
                                                                              "measured" else "of fallback")},

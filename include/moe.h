@@ -254,8 +254,9 @@ MOE_API moe_status moe_workspace_view(const moe_config *cfg, void *ws, size_t ws
  *   - Run it after moe_forward on the same stream with the same cfg, inputs
  *     and workspace `fwd_ws` (its dispatch tables, packed rows and hidden
  *     activation are read from there; the expert pre-activations are
- *     recomputed), passing the forward's outputs idx, gate, counts and its
- *     router logits (moe_forward's logits_out, required here).
+ *     recomputed, unless the forward pass was moe_forward_train with this
+ *     backward workspace), passing the forward's outputs idx, gate, counts
+ *     and its router logits (moe_forward's logits_out, required here).
  *   - bf16 layers with d_model, d_ff and d_ff_shared multiples of 64 (else
  *     MOE_ERR_UNSUPPORTED).  dy and dx [T, d_model] bf16; every other
  *     gradient fp32 in the layout of its parameter: dWr [d_model, E],
@@ -278,6 +279,28 @@ MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const floa
                                 float *dW1, float *db1, float *dWu, float *dW2, float *db2,
                                 float *dWsh_g, float *dWsh_u, float *dWsh_d,
                                 void *fwd_ws, size_t fwd_ws_bytes, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Training forward pass: moe_forward (same arguments, same results) that
+ * also leaves the expert pre-activations -- G and U of the SwiGLU experts,
+ * W_1 x + b_1 of the GELU experts, shared expert included, in bf16 as the
+ * first GEMM computed them -- inside `bwd_ws`, the workspace the following
+ * moe_backward will use, so that call skips their recomputation (two grouped
+ * GEMMs, about a sixth of its time on a Qwen3-shaped layer).
+ *   - bwd_ws: moe_backward_workspace_size(cfg) bytes, 256-byte aligned; the
+ *     layer must be one moe_backward supports (else MOE_ERR_UNSUPPORTED).
+ *   - The hand-over is recorded on the host: the next moe_backward with
+ *     workspace bwd_ws, forward workspace ws and an identical cfg uses the
+ *     saved values; any call that rewrites ws's packed rows or hidden
+ *     activation (moe_forward*, moe_grouped_ffn*, moe_permute) or
+ *     reinitialises ws or bwd_ws (moe_workspace_init) cancels the record, and
+ *     moe_backward recomputes.  Calls are taken in host order, as the
+ *     stream runs them.                                                     */
+MOE_API moe_status moe_forward_train(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                                     const float *sel_bias, const void *W1, const float *b1, const void *Wu,
+                                     const void *W2, const float *b2, const void *Wsh_g, const void *Wsh_u,
+                                     const void *Wsh_d, void *y, int32_t *idx, float *gate, int32_t *counts, float *f,
+                                     float *P, double *loss, float *logits_out, int32_t *n_dropped, void *ws,
+                                     size_t ws_bytes, void *bwd_ws, size_t bwd_ws_bytes, moe_stream_t stream);
 
 /* ---- Expert parallelism -------------------------------------------------
  * The experts sharded over R ranks, each rank holding E / R of them ("Fine-

@@ -84,6 +84,21 @@ moe::BwdGemmParams gemm(const int32_t *offsets, int G, int kgroup, int M, int N,
 
 }  // namespace
 
+namespace moe {
+
+// Where moe_backward keeps the expert pre-activations inside its workspace
+// (G | U rows [T*k, 2F] or W_1 x + b_1 rows [T*k, F]; the shared expert's
+// [T, 2S] or [T, S]); false on an unsupported config.
+bool bwd_preact_buffers(const moe_config *cfg, void *ws, void **GU, void **GUs) {
+    if (check_bwd_cfg(cfg) != MOE_OK) return false;
+    const BwdLayout L = bwd_layout(cfg);
+    *GU = static_cast<char *>(ws) + L.GU;
+    *GUs = static_cast<char *>(ws) + L.GUs;
+    return true;
+}
+
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_backward_workspace_size(const moe_config *cfg) {
@@ -183,8 +198,10 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const float *Wr, c
     // ---- 1. dZ = gate * dy[token] for every packed row
     if ((e = moe::launch_scale_rows(aux, rows, st)) != cudaSuccess) return cuda(e, "scale rows");
 
-    // ---- 2. pre-activations again: G | U (SwiGLU) or W1 x + b1 (GELU), routed and shared
-    for (int part_i = 0; part_i < gw; ++part_i) {
+    // ---- 2. pre-activations again: G | U (SwiGLU) or W1 x + b1 (GELU), routed and shared --
+    // unless moe_forward_train on fwd_ws already left them in this workspace
+    const bool saved = moe::take_saved_preacts(ws, fwd_ws, *cfg);
+    for (int part_i = 0; part_i < (saved ? 0 : gw); ++part_i) {
         const void *Wsrc = part_i == 0 ? W1 : Wu;
         if (!map2(&mA, v.x_perm, d, rows, d, 128) || !map3(&mB, Wsrc, d, F, E, moe::kBwdBoxRowsB)) return cuda(cudaErrorInvalidValue, "maps");
         moe::BwdGemmParams p = gemm(v.offsets, E, 0, 0, F, d, moe::BW_STORE_BF16, status);

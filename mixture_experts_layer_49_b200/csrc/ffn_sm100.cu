@@ -89,6 +89,12 @@ struct GemmParams {
     int ldo;
     int64_t shared_a_row;     // first A row of the shared group
     int64_t shared_out_row;   // first output row of the shared group
+    // training forward (SAVE instantiations of the first GEMM): the
+    // pre-activations as bf16 -- SwiGLU: G in columns 0..N-1 and U in N..2N-1
+    // of each row, GELU: W_1 x + b_1 -- routed row r at pre + r * pre_ld,
+    // shared row t at pre_s + t * pre_ld_s
+    __nv_bfloat16 *pre, *pre_s;
+    int64_t pre_ld, pre_ld_s;
     int tail_mode;            // 1-CTA kernel: 0 all rows; 1 only a group's last rows
                               // when rows % 256 is in 1..128 (the rest runs in pair tiles)
     uint64_t timeout_ns;
@@ -209,16 +215,34 @@ __device__ __forceinline__ void preload_scales(const GemmParams &p, bool sh, int
 // all 32 rows of the warp are valid, each 32-column chunk leaves through the
 // staging buffer and a TMA store (row0: the warp's first output row);
 // otherwise each valid row stores its columns below N with 16-byte stores.
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool SAVE = false>
 __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, bool valid, int N,
                                              __nv_bfloat16 *orow_ptr, const float *bias, float gscale,
                                              const CUtensorMap *tmO, uint32_t stg, int row0, float rscale,
-                                             const float *csv, float *scl) {
+                                             const float *csv, float *scl, const CUtensorMap *tmP = nullptr,
+                                             int prow0 = 0, __nv_bfloat16 *prow_ptr = nullptr) {
     float v[128];
     const bool staged = __all_sync(0xffffffffu, valid);
     if (MODE == GM_SWIGLU) {
         const int c0 = half * 2;
         tmem_ld32x4(taddr + c0 * 32, taddr + (c0 + 1) * 32, taddr + 128 + c0 * 32, taddr + 128 + (c0 + 1) * 32, v);
+        if (SAVE) {                                   // G and U as computed, before the activation
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int col0 = nt * 128 + (c0 + cc) * 32;
+                if (col0 >= N) continue;                  // uniform over the warp
+                if (staged) {
+                    stage_store32(stg, tmP, col0, prow0, v + cc * 32);
+                    stage_store32(stg, tmP, N + col0, prow0, v + 64 + cc * 32);
+                } else if (valid) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        store8(prow_ptr + col0 + u * 8, v + cc * 32 + u * 8);
+                        store8(prow_ptr + N + col0 + u * 8, v + 64 + cc * 32 + u * 8);
+                    }
+                }
+            }
+        }
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = nt * 128 + (c0 + cc) * 32;
@@ -265,7 +289,19 @@ __device__ __forceinline__ void epilogue_row(uint32_t taddr, int half, int nt, b
                     h[4 * i + 2] *= a.z * rs; h[4 * i + 3] *= a.w * rs;
                 }
             }
-            if (!F8 || bias != nullptr) {
+            if (SAVE && MODE == GM_GELU) {                // the pre-activation W_1 x + b_1, then GELU
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] += (bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f;
+                if (staged) {
+                    stage_store32(stg, tmP, col0, prow0, h);
+                } else if (valid) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (col0 + u * 8 < N) store8(prow_ptr + col0 + u * 8, h + u * 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] = gelu_erf(h[i]);
+            } else if (!F8 || bias != nullptr) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float z = h[i] + ((bias && col0 + i < N) ? __ldg(bias + col0 + i) : 0.f);
@@ -306,12 +342,13 @@ __device__ __forceinline__ void fail(SmemTail &s, const GemmParams &p, int where
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool SAVE = false>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                 const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                 const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
-                const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP,
+                const __grid_constant__ CUtensorMap tmPs, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -487,8 +524,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
-            epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, csv, scl);
+            const int64_t prow = sh ? orow - p.shared_out_row : orow;   // row in the pre-activation buffer
+            epilogue_row<MODE, F8, SAVE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg,
+                                         (int)(orow - lane), rscale, csv, scl, sh ? &tmPs : &tmP,
+                                         (int)(prow - lane),
+                                         SAVE ? (sh ? p.pre_s + prow * p.pre_ld_s : p.pre + prow * p.pre_ld)
+                                              : nullptr);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.acce[ab]));
@@ -570,12 +611,13 @@ __device__ __forceinline__ void fail_pair(Tail &s, const GemmParams &p, int wher
     *reinterpret_cast<volatile int *>(&s.abort_flag) = 1;
 }
 
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool SAVE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
-                     const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP,
+                     const __grid_constant__ CUtensorMap tmPs, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -734,8 +776,12 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint32_t taddr = tmem_base + (uint32_t)(ab * BNB) + ((uint32_t)(q * 32) << 16);
             __nv_bfloat16 *orow_ptr = p.out + orow * p.ldo;
             const float *bias = (!sh && p.bias) ? p.bias + (size_t)group_expert(p, g) * p.N_routed : nullptr;
-            epilogue_row<MODE, F8>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg, (int)(orow - lane),
-                                   rscale, csv, scl);
+            const int64_t prow = sh ? orow - p.shared_out_row : orow;   // row in the pre-activation buffer
+            epilogue_row<MODE, F8, SAVE>(taddr, half, nt, valid, N, orow_ptr, bias, gscale, &tmO, stg,
+                                         (int)(orow - lane), rscale, csv, scl, sh ? &tmPs : &tmP,
+                                         (int)(prow - lane),
+                                         SAVE ? (sh ? p.pre_s + prow * p.pre_ld_s : p.pre + prow * p.pre_ld)
+                                              : nullptr);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.acce[ab]), 0));
@@ -1180,29 +1226,30 @@ bool make_store_map(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool SAVE = false>
 cudaError_t launch_gemm(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B, const CUtensorMap &B2,
-                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const CUtensorMap &O, const GemmParams &p,
-                        int grid, cudaStream_t st, bool pdl) {
+                        const CUtensorMap &Bs, const CUtensorMap &Bs2, const CUtensorMap &O, const CUtensorMap &P,
+                        const CUtensorMap &Ps, const GemmParams &p, int grid, cudaStream_t st, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, F8, SAVE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_kernel(tc_grouped_gemm<MODE, F8>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B, B2, Bs,
-                         Bs2, O, p);
+    return launch_kernel(tc_grouped_gemm<MODE, F8, SAVE>, dim3(grid), dim3(kThreads), kSmemBytes, st, pdl, A, As, B,
+                         B2, Bs, Bs2, O, P, Ps, p);
 }
 
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool SAVE = false>
 cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const CUtensorMap &B,
                              const CUtensorMap &B2, const CUtensorMap &Bs, const CUtensorMap &Bs2,
-                             const CUtensorMap &O, const GemmParams &p, int num_sms, cudaStream_t st, bool pdl) {
+                             const CUtensorMap &O, const CUtensorMap &P, const CUtensorMap &Ps, const GemmParams &p,
+                             int num_sms, cudaStream_t st, bool pdl) {
     static int grid = 0;
     if (grid == 0) {
-        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kPairSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm_pair<MODE, F8, SAVE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmemBytes);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
@@ -1216,12 +1263,12 @@ cudaError_t launch_gemm_pair(const CUtensorMap &A, const CUtensorMap &As, const 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_grouped_gemm_pair<MODE, F8>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&nclusters, tc_grouped_gemm_pair<MODE, F8, SAVE>, &cfg);
         if (e != cudaSuccess || nclusters < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
         grid = 2 * nclusters;
     }
-    return launch_kernel(tc_grouped_gemm_pair<MODE, F8>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A, As, B, B2,
-                         Bs, Bs2, O, p);
+    return launch_kernel(tc_grouped_gemm_pair<MODE, F8, SAVE>, dim3(grid), dim3(kThreads), kPairSmemBytes, st, pdl, A,
+                         As, B, B2, Bs, Bs2, O, P, Ps, p);
 }
 
 }  // namespace
@@ -1304,13 +1351,41 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
     // the first GEMM's output: H [all rows, hF], stored in 32 x 32 blocks
     CUtensorMap O1;
     if (!make_store_map(&O1, a.H, a.hF, all_rows, a.hF)) return cudaErrorInvalidValue;
-    cudaError_t err = swiglu ? launch_gemm_pair<GM_SWIGLU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl)
-                             : launch_gemm_pair<GM_GELU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, p1, grid, st, a.pdl);
-    if (err != cudaSuccess) return err;
-    p1.tail_mode = 1;
-    err = swiglu ? launch_gemm<GM_SWIGLU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true)
-                 : launch_gemm<GM_GELU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, p1, grid, st, true);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
+    if (!F8 && a.pre) {
+        // training forward: the pre-activations too (routed rows, then the shared rows' own buffer)
+        const int gw = swiglu ? 2 : 1;
+        CUtensorMap Q1, Q1s;
+        if (!make_store_map(&Q1, a.pre, (uint64_t)gw * a.F, routed_rows > 0 ? routed_rows : 1, (uint64_t)gw * a.F))
+            return cudaErrorInvalidValue;
+        if (has_sh) {
+            if (!make_store_map(&Q1s, a.pre_s, (uint64_t)gw * a.S, (uint64_t)a.T, (uint64_t)gw * a.S))
+                return cudaErrorInvalidValue;
+        } else {
+            Q1s = Q1;
+        }
+        p1.pre = static_cast<__nv_bfloat16 *>(a.pre);
+        p1.pre_s = static_cast<__nv_bfloat16 *>(a.pre_s);
+        p1.pre_ld = (int64_t)gw * a.F;
+        p1.pre_ld_s = (int64_t)gw * a.S;
+        err = swiglu ? launch_gemm_pair<GM_SWIGLU, false, true>(A1, A1s, P1, P1u, P1s, P1su, O1, Q1, Q1s, p1, grid, st,
+                                                                a.pdl)
+                     : launch_gemm_pair<GM_GELU, false, true>(A1, A1s, P1, P1u, P1s, P1su, O1, Q1, Q1s, p1, grid, st,
+                                                              a.pdl);
+        if (err != cudaSuccess) return err;
+        p1.tail_mode = 1;
+        err = swiglu ? launch_gemm<GM_SWIGLU, false, true>(A1, A1s, B1, B1u, B1s, B1su, O1, Q1, Q1s, p1, grid, st, true)
+                     : launch_gemm<GM_GELU, false, true>(A1, A1s, B1, B1u, B1s, B1su, O1, Q1, Q1s, p1, grid, st, true);
+        if (err != cudaSuccess) return err;
+    } else {
+        err = swiglu ? launch_gemm_pair<GM_SWIGLU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, O1, O1, p1, grid, st, a.pdl)
+                     : launch_gemm_pair<GM_GELU, F8>(A1, A1s, P1, P1u, P1s, P1su, O1, O1, O1, p1, grid, st, a.pdl);
+        if (err != cudaSuccess) return err;
+        p1.tail_mode = 1;
+        err = swiglu ? launch_gemm<GM_SWIGLU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, O1, O1, p1, grid, st, true)
+                     : launch_gemm<GM_GELU, F8>(A1, A1s, B1, B1u, B1s, B1su, O1, O1, O1, p1, grid, st, true);
+        if (err != cudaSuccess) return err;
+    }
 
     // ---- e4m3: quantize H per row (kept routed rows, then the shared rows)
     if (F8) {
@@ -1376,10 +1451,10 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t st) {
     }
     CUtensorMap O2;                               // y_perm [all rows, d_model]
     if (!make_store_map(&O2, a.y_perm, a.d, all_rows, a.d)) return cudaErrorInvalidValue;
-    err = launch_gemm_pair<GM_DOWN, F8>(A2, A2s, P2, P2, P2s, P2s, O2, p2, grid, st, true);
+    err = launch_gemm_pair<GM_DOWN, F8>(A2, A2s, P2, P2, P2s, P2s, O2, O2, O2, p2, grid, st, true);
     if (err != cudaSuccess) return err;
     p2.tail_mode = 1;
-    return launch_gemm<GM_DOWN, F8>(A2, A2s, B2m, B2m, B2s, B2s, O2, p2, grid, st, true);
+    return launch_gemm<GM_DOWN, F8>(A2, A2s, B2m, B2m, B2s, B2s, O2, O2, O2, p2, grid, st, true);
 }
 
 }  // namespace

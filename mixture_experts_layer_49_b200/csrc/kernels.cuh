@@ -124,6 +124,11 @@ struct FfnArgs {
     const float *Wsgs, *Wsus, *Wsds;   // [S], [S], [d]
     uint8_t *H8;                 // [T*k (+T), hF] codes
     float *h_scale;              // [T*k (+T)]
+    // training forward (bf16 experts): the first GEMM also stores the
+    // pre-activations in bf16 -- SwiGLU [rows, 2F] (G | U), GELU [rows, F]
+    // (W_1 x + b_1) -- routed rows in pre, the shared expert's T rows in
+    // pre_s ([T, 2S] or [T, S]); null for inference
+    void *pre, *pre_s;
 };
 // TMA tile map (128-byte swizzle) of a tensor [outer][mid][inner] (inner
 // contiguous) of bf16 (esize 2) or 8-bit codes (esize 1), box {one 128-byte
@@ -212,6 +217,18 @@ struct W4PairArgs {
     bool pdl;
 };
 cudaError_t launch_w4_gemm_pair(const W4PairArgs &a, cudaStream_t st);
+
+// Training forward -> backward hand-over of the expert pre-activations
+// (moe_api.cu): moe_forward_train records that it left them in a backward
+// workspace for a forward workspace and config; moe_backward takes the record
+// (true: skip the recompute) and drops any other for its workspace; every
+// call that rewrites a forward workspace's packed rows or hidden activation,
+// or reinitialises a workspace, forgets the records that involve it.
+void note_saved_preacts(const void *bwd_ws, const void *fwd_ws, const moe_config &cfg);
+bool take_saved_preacts(const void *bwd_ws, const void *fwd_ws, const moe_config &cfg);
+void forget_saved_preacts(const void *ws);
+// Where moe_backward keeps the pre-activations in its workspace (bwd_api.cu).
+bool bwd_preact_buffers(const moe_config *cfg, void *ws, void **GU, void **GUs);
 
 // Per-row e4m3 quantization of bf16 rows (row0 + r for r < rows, or fewer
 // when rows_limit points at a smaller device count): in [.., ld_in] bf16,

@@ -348,6 +348,43 @@ moe::FfnMxArgs w4_args(const moe_config *cfg, const void *x_perm, const int32_t 
 
 namespace moe {
 moe_status validate_config(const moe_config *cfg) { return check_cfg(cfg); }
+
+namespace {
+struct SavedPreacts {
+    const void *bwd_ws;
+    const void *fwd_ws;
+    moe_config cfg;
+};
+std::mutex g_pre_mu;
+std::vector<SavedPreacts> g_pre;
+bool same_cfg(const moe_config &a, const moe_config &b) { return memcmp(&a, &b, sizeof(moe_config)) == 0; }
+}  // namespace
+
+void note_saved_preacts(const void *bwd_ws, const void *fwd_ws, const moe_config &cfg) {
+    std::lock_guard<std::mutex> lock(g_pre_mu);
+    g_pre.push_back(SavedPreacts{bwd_ws, fwd_ws, cfg});
+}
+bool take_saved_preacts(const void *bwd_ws, const void *fwd_ws, const moe_config &cfg) {
+    std::lock_guard<std::mutex> lock(g_pre_mu);
+    bool hit = false;
+    for (size_t i = 0; i < g_pre.size();) {
+        if (g_pre[i].bwd_ws == bwd_ws) {
+            hit = hit || (g_pre[i].fwd_ws == fwd_ws && same_cfg(g_pre[i].cfg, cfg));
+            g_pre.erase(g_pre.begin() + (long)i);
+        } else {
+            ++i;
+        }
+    }
+    return hit;
+}
+void forget_saved_preacts(const void *ws) {
+    std::lock_guard<std::mutex> lock(g_pre_mu);
+    for (size_t i = 0; i < g_pre.size();) {
+        if (g_pre[i].bwd_ws == ws || g_pre[i].fwd_ws == ws) g_pre.erase(g_pre.begin() + (long)i);
+        else ++i;
+    }
+}
+
 void set_error_detail(const char *where, const char *what) {
     snprintf(g_detail, sizeof g_detail, "%s: %s", where, what);
 }
@@ -383,6 +420,7 @@ moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
     if (!ws || ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace missing or < 256 bytes%s");
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned%s");
     forget_frozen(ws);
+    moe::forget_saved_preacts(ws);
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(moe::WsHeader), reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
 }
@@ -434,6 +472,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *idx,
     ALIGNED(x, 16); ALIGNED(x_perm, 16); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(kept, 4);
     ALIGNED(offsets, 4); ALIGNED(row_of, 4); ALIGNED(row_token, 4); ALIGNED(row_gate, 4); ALIGNED(n_dropped, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     const Layout L = layout(cfg);
     moe::DispatchArgs a{};
     a.x = x; a.idx = idx; a.gate = gate;
@@ -462,6 +501,7 @@ moe_status moe_grouped_ffn(const moe_config *cfg, const void *x_perm, const int3
     ALIGNED(x_perm, 16); ALIGNED(y_perm, 16); ALIGNED(offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4);
     ALIGNED(b2, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     moe::FfnArgs a = ffn_args(cfg, x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d, y_perm, ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cfg->dtype == MOE_BF16 ? moe::launch_ffn_bf16(a, st) : moe::launch_ffn_f32(a, st);
@@ -494,11 +534,14 @@ moe_status moe_balance_stats(const moe_config *cfg, const int32_t *counts, const
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "balance");
 }
 
-moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
-                       const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
-                       const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y,
-                       int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
-                       float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+// The layer's forward pass; pre / pre_s non-null: the training form, which
+// also leaves the expert pre-activations there (bf16 layers).
+static moe_status forward_impl(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                               const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
+                               const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y,
+                               int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                               float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream,
+                               void *pre, void *pre_s) {
     moe_status s = check_cfg(cfg);
     if (s != MOE_OK) return s;
     NEED(counts); NEED(f); NEED(P); NEED(loss);
@@ -510,6 +553,7 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
     ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     const Layout L = layout(cfg);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = cfg->dtype == MOE_BF16;
@@ -547,6 +591,8 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
     moe::FfnArgs fa = ffn_args(cfg, da.x_perm, offsets, row_gate, W1, b1, Wu, W2, b2, x, Wsh_g, Wsh_u, Wsh_d,
                                y_perm, ws);
     fa.pdl = true;
+    fa.pre = pre;
+    fa.pre_s = pre_s;
     e = bf16 ? moe::launch_ffn_bf16(fa, st) : moe::launch_ffn_f32(fa, st);
     if (e != cudaSuccess) return cuda_fail(e, "grouped_ffn");
 
@@ -554,6 +600,38 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, co
                         cfg->d_ff_shared > 0 ? 1 : 0, (int64_t)cfg->T * cfg->top_k, num_sms(), true};
     if ((e = moe::launch_combine(ca, bf16, st)) != cudaSuccess) return cuda_fail(e, "combine");
     return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                       const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
+                       const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y,
+                       int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                       float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    return forward_impl(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh_u, Wsh_d, y, idx, gate,
+                        counts, f, P, loss, logits_out, n_dropped, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+moe_status moe_forward_train(const moe_config *cfg, const void *x, const float *Wr, const float *logit_bias,
+                             const float *sel_bias, const void *W1, const float *b1, const void *Wu, const void *W2,
+                             const float *b2, const void *Wsh_g, const void *Wsh_u, const void *Wsh_d, void *y,
+                             int32_t *idx, float *gate, int32_t *counts, float *f, float *P, double *loss,
+                             float *logits_out, int32_t *n_dropped, void *ws, size_t ws_bytes, void *bwd_ws,
+                             size_t bwd_ws_bytes, moe_stream_t stream) {
+    moe_status s = check_cfg(cfg);
+    if (s != MOE_OK) return s;
+    const size_t need = moe_backward_workspace_size(cfg);
+    if (need == 0) return fail(MOE_ERR_UNSUPPORTED, "training forward: the layer has no backward pass%s");
+    if (!bwd_ws || (reinterpret_cast<uintptr_t>(bwd_ws) & 255u))
+        return fail(MOE_ERR_WORKSPACE, "backward workspace NULL or not 256-byte aligned%s");
+    if (bwd_ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "backward workspace smaller than moe_backward_workspace_size()%s");
+    void *GU = nullptr, *GUs = nullptr;
+    if (!moe::bwd_preact_buffers(cfg, bwd_ws, &GU, &GUs))
+        return fail(MOE_ERR_UNSUPPORTED, "training forward: the layer has no backward pass%s");
+    moe::forget_saved_preacts(bwd_ws);
+    s = forward_impl(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh_u, Wsh_d, y, idx, gate, counts,
+                     f, P, loss, logits_out, n_dropped, ws, ws_bytes, stream, GU, GUs);
+    if (s == MOE_OK) moe::note_saved_preacts(bwd_ws, ws, *cfg);
+    return s;
 }
 
 size_t moe_ep_workspace_size(const moe_config *cfg, int32_t n_src, int64_t max_rows) {
@@ -702,6 +780,7 @@ moe_status moe_grouped_ffn_fp8(const moe_config *cfg, const uint8_t *x8_perm, co
     ALIGNED(x8_perm, 16); ALIGNED(x8, 16); ALIGNED(y_perm, 16); ALIGNED(x8_perm_scale, 4); ALIGNED(x8_scale, 4);
     ALIGNED(offsets, 4); ALIGNED(row_gate, 4); ALIGNED(b1, 4); ALIGNED(b2, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     if (cfg->T == 0) return MOE_OK;
     moe::FfnArgs a = ffn_args(cfg, x8_perm, offsets, row_gate, w->W1, b1, w->Wu, w->W2, b2, x8, w->Wsh_g, w->Wsh_u,
                               w->Wsh_d, y_perm, ws);
@@ -726,6 +805,7 @@ moe_status moe_forward_fp8(const moe_config *cfg, const void *x, const float *Wr
     ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
     ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     const Layout L = layout(cfg);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float *psum = at<float>(ws, L.psum);
@@ -897,6 +977,7 @@ moe_status moe_forward_mx(const moe_config *cfg, const void *x, const float *Wr,
     ALIGNED(w->Wsh_d, 16); ALIGNED(w->W1_scale, 16); ALIGNED(w->Wu_scale, 16); ALIGNED(w->W2_scale, 16);
     ALIGNED(w->Wsh_g_scale, 16); ALIGNED(w->Wsh_u_scale, 16); ALIGNED(w->Wsh_d_scale, 16);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     if (!mx_ws) return fail(MOE_ERR_WORKSPACE, "MX workspace is NULL%s");
     if (reinterpret_cast<uintptr_t>(mx_ws) & 255u) return fail(MOE_ERR_WORKSPACE, "MX workspace not 256-byte aligned%s");
     const MxLayout M = mx_layout(cfg, w->sld);
@@ -998,6 +1079,7 @@ moe_status moe_grouped_ffn_w4(const moe_config *cfg, const void *x_perm, const i
     ALIGNED(x_perm, 16); ALIGNED(x, 16); ALIGNED(y_perm, 16); ALIGNED(offsets, 4); ALIGNED(row_gate, 4);
     ALIGNED(b1, 4); ALIGNED(b2, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     if (cfg->T == 0) return MOE_OK;
     moe::FfnMxArgs a = w4_args(cfg, x_perm, offsets, row_gate, w, b1, b2, x, y_perm, ws);
     cudaError_t e = moe::launch_ffn_w4(a, reinterpret_cast<cudaStream_t>(stream));
@@ -1021,6 +1103,7 @@ moe_status moe_forward_w4(const moe_config *cfg, const void *x, const float *Wr,
     ALIGNED(b1, 4); ALIGNED(b2, 4); ALIGNED(idx, 4); ALIGNED(gate, 4); ALIGNED(counts, 4); ALIGNED(f, 4);
     ALIGNED(P, 4); ALIGNED(loss, 8); ALIGNED(logits_out, 4); ALIGNED(n_dropped, 4);
     if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+    moe::forget_saved_preacts(ws);        // the packed rows / hidden activation change
     const Layout L = layout(cfg);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float *psum = at<float>(ws, L.psum);

@@ -31,6 +31,7 @@ EXPORTS = ("moe_workspace_size", "moe_capacity", "moe_router_blocks", "moe_perm_
            "moe_bias_update", "moe_routing_health", "moe_check_wait_timeout",
            "moe_quantize_rows_e4m3", "moe_grouped_ffn_fp8", "moe_forward_fp8", "moe_workspace_view",
            "moe_ep_workspace_size", "moe_ep_grouped_ffn", "moe_backward_workspace_size", "moe_backward",
+           "moe_forward_train",
            "moe_quantize_rows_mx", "moe_grouped_ffn_mx_workspace_size", "moe_grouped_ffn_mx",
            "moe_router_freeze", "moe_forward_mx", "moe_grouped_ffn_w4", "moe_forward_w4")
 
@@ -116,6 +117,8 @@ def lib():
         L.moe_combine.argtypes = [P(MoeConfig)] + [c_vp] * 4 + [ctypes.c_size_t, c_vp]
         L.moe_balance_stats.argtypes = [P(MoeConfig)] + [c_vp] * 6
         L.moe_forward.argtypes = [P(MoeConfig)] + [c_vp] * 22 + [ctypes.c_size_t, c_vp]
+        L.moe_forward_train.restype = ctypes.c_int
+        L.moe_forward_train.argtypes = [P(MoeConfig)] + [c_vp] * 22 + [ctypes.c_size_t, c_vp, ctypes.c_size_t, c_vp]
         L.moe_get_device_status.argtypes = [c_vp, c_vp, P(c_i32)]
         L.moe_bias_update.restype = ctypes.c_int
         L.moe_bias_update.argtypes = [P(MoeConfig), c_vp, c_vp, ctypes.c_float, c_vp]
@@ -296,6 +299,15 @@ def moe_forward(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh
                              _p(n_dropped), _p(ws), ws.numel(), _stream(stream)), "moe_forward")
 
 
+def moe_forward_train(cfg, x, Wr, logit_bias, sel_bias, W1, b1, Wu, W2, b2, Wsh_g, Wsh_u, Wsh_d,
+                      y, idx, gate, counts, f, P, loss, logits_out, n_dropped, ws, bwd_ws, stream=None):
+    _check(lib().moe_forward_train(ctypes.byref(cfg), _p(x), _p(Wr), _p(logit_bias), _p(sel_bias), _p(W1),
+                                   _p(b1), _p(Wu), _p(W2), _p(b2), _p(Wsh_g), _p(Wsh_u), _p(Wsh_d), _p(y),
+                                   _p(idx), _p(gate), _p(counts), _p(f), _p(P), _p(loss), _p(logits_out),
+                                   _p(n_dropped), _p(ws), ws.numel(), _p(bwd_ws), bwd_ws.numel(), _stream(stream)),
+           "moe_forward_train")
+
+
 def ep_workspace_size(cfg, n_src, max_rows) -> int:
     n = int(lib().moe_ep_workspace_size(ctypes.byref(cfg), int(n_src), int(max_rows)))
     if n == 0:
@@ -434,6 +446,20 @@ def forward(cfg, inp, out: Outputs, ws, stream=None):
                 inp.get("Wsg"), inp.get("Wsu"), inp.get("Wsd"),
                 out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss, out.logits,
                 out.n_dropped, ws, stream)
+
+
+def alloc_backward_workspace(cfg, device="cuda") -> torch.Tensor:
+    return torch.empty(backward_workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def forward_train(cfg, inp, out: Outputs, ws, bwd_ws, stream=None):
+    """moe_forward_train: forward(...) that also leaves the expert
+    pre-activations in bwd_ws for the following backward(..., ws=bwd_ws)."""
+    moe_forward_train(cfg, inp["x"], inp["Wr"], inp.get("logit_bias"), inp.get("sel_bias"),
+                      inp["W1"], inp.get("b1"), inp.get("Wu"), inp["W2"], inp.get("b2"),
+                      inp.get("Wsg"), inp.get("Wsu"), inp.get("Wsd"),
+                      out.y, out.idx, out.gate, out.counts, out.f, out.P, out.loss, out.logits,
+                      out.n_dropped, ws, bwd_ws, stream)
 
 
 # ---------------------------------------------------------------- FP8 experts

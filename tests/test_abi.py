@@ -280,3 +280,21 @@ def test_ep_grouped_ffn_host_checks():
     # no rows: nothing to do, nothing launched
     assert L.moe_ep_grouped_ffn(ctypes.byref(c), 2, fake(), 0, None, None, None, None, None, None, None, None,
                                 ws, 256, None) == nat.MOE_OK
+
+
+def test_forward_train_checks_arguments():
+    # the backward workspace is checked before anything runs
+    L = nat.lib()
+    c = cfg(d_model=128, d_ff=256)
+    n = nat.workspace_size(c)
+    nb = nat.backward_workspace_size(c)
+    args = [fake(), fake(), None, None, fake(), None, fake(), fake(), None, None, None, None, fake(), fake(), fake(),
+            fake(), fake(), fake(), fake(), None, None]
+    call = lambda cc, bws, bn: L.moe_forward_train(ctypes.byref(cc), *args, fake(16), n, bws, bn, None)
+    assert call(c, None, nb) == nat.MOE_ERR_WORKSPACE
+    assert call(c, ctypes.c_void_p(4096 + 64), nb) == nat.MOE_ERR_WORKSPACE     # not 256-byte aligned
+    assert call(c, fake(32), nb - 1) == nat.MOE_ERR_WORKSPACE
+    c32 = cfg(dtype="f32")                                   # no backward pass for fp32 layers
+    assert call(c32, fake(32), nb) == nat.MOE_ERR_UNSUPPORTED
+    c96 = cfg(d_model=96)                                    # d_model not a multiple of 64
+    assert call(c96, fake(32), nb) == nat.MOE_ERR_UNSUPPORTED
