@@ -138,7 +138,10 @@ constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStgOff + 8 * STG_BYTES + 8
 static_assert(kSmemBytes <= 227 * 1024, "1-CTA kernel shared memory");
 
 __device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.f + erff(v * 0.70710678118654752f)); }
-__device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
+// SiLU with the fast reciprocal division: its few-ulp fp32 error sits far
+// below the bf16 rounding of H; a large negative v gives exp overflow, a
+// quotient of 0 and silu = -0.
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 __device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *v) {
     uint4 pk;

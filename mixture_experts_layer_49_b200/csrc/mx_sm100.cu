@@ -221,7 +221,7 @@ __device__ __forceinline__ void mx_decode(const MxSmem &s, int G, int tile, int 
     nt = local / s.mtiles[g];
 }
 
-__device__ __forceinline__ float mx_silu(float v) { return v / (1.f + __expf(-v)); }
+__device__ __forceinline__ float mx_silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 __device__ __forceinline__ float mx_gelu(float v) { return 0.5f * v * (1.f + erff(v * 0.70710678118654752f)); }
 
 // 32 rows x 32 bf16 columns of the warp (this lane's row in h) to global
