@@ -44,6 +44,14 @@
 // per-warp shared-memory slot read as float4 broadcasts in the others, whose
 // down projection also folds the row's gate into its row scale).
 //
+// Training forward (the SAVE instantiations of the first GEMM): the epilogue
+// also stores the pre-activations -- G and U before the SwiGLU, W_1 x + b_1
+// before the GELU -- in bf16 through the same staging buffer, for the
+// backward pass to read instead of recomputing them.
+//
+// INT4 weight-only experts (tc_w4_gemm_pair, further below): the pair kernel
+// with its B operand decoded on the chip by four extra warps per CTA.
+//
 // Every mbarrier wait is bounded (a global-timer limit); a wait that runs out
 // records MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds,
 // freeing its TMEM.  No TMA multicast is used.
